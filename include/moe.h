@@ -1,0 +1,177 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) int4 routed-expert MoE decode layer.
+ *
+ * The layer (one decode step of a GLM-5.2 / DeepSeek-V3 style MoE block):
+ *   1. router GEMV:   logit[e] = sum_h W_g[e][h] * x[h]
+ *   2. noaux_tc:      s = sigmoid(logit), s' = s + e_score_correction_bias;
+ *                     group score = sum of the two largest s' of each of
+ *                     n_group groups; keep topk_group groups; top_k largest
+ *                     s' inside them (ties to the lower index);
+ *                     w_j = routed_scaling_factor * s_j / sum_j s_j
+ *   3. gather:        the top_k selected int4 experts
+ *   4. expert FFN:    h = silu(W_gate x) * (W_up x); y_e = W_down h
+ *   5. combine:       y = sum_j w_j * y_{e_j} + y_shared
+ * Sources: "LightLX" page, section "How it works" (256 experts per layer, a
+ * router picks 8 per token, noaux_tc sigmoid router, resident shared
+ * experts); colibri summary ("Show HN: run GLM 5.2 on a slow computer"),
+ * section "Principales fonctionnalites implementees" (DeepSeek-V3 sigmoid
+ * router with noaux_tc, routed_scaling_factor, shared expert; int4
+ * dequant-on-use kernels; batch-union MoE; per-layer LRU expert cache).
+ *
+ * int4 format (the layer's spec): symmetric two's-complement codes in
+ * [-8, 7], two per byte, byte j of a row holding input 2j in its low nibble
+ * and 2j+1 in its high nibble; one fp16 scale per group_size (= 32)
+ * consecutive inputs of a row.  Weight value = code * scale.
+ *
+ * Conventions for every call:
+ *  - Pointers named *_dev are device memory; *_host are host memory.
+ *    Sizes are element counts unless named *_bytes.
+ *  - All compute calls are asynchronous on the given stream (a cudaStream_t
+ *    passed as void*; NULL = the legacy default stream).  The returned status
+ *    covers argument checks and launch errors only; faults of the kernels
+ *    themselves surface at the next synchronising call (moe_ws_check).
+ *  - No call throws; moe_last_error() gives a text for the last failure of
+ *    the calling thread.
+ *  - The caller owns x, y, idx, w and the workspace; the library owns what
+ *    moe_layer_create / moe_cache_create allocate.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer */
+  MOE_ERR_CUDA = 2,         /* a CUDA runtime call failed */
+  MOE_ERR_OOM = 3,          /* an allocation failed or would not fit */
+  MOE_ERR_TIMEOUT = 4,      /* a bounded wait ran out (host or device) */
+  MOE_ERR_UNSUPPORTED = 5,  /* shape outside what the kernels handle */
+  MOE_ERR_DEVICE = 6        /* a kernel reported an error in the workspace */
+} moe_status;
+
+/* Layer shape.  Supported: hidden / 32 and inter / 32 each 2, 4, 8, 16 or a
+ * multiple of 32 up to 256 (GLM-5.2: hidden 6144, inter 2048); group_size
+ * 32; n_experts <= 1024 divisible by n_group; n_experts / n_group <= 32;
+ * n_group <= 32; top_k <= 32; topk_group * (n_experts / n_group) >= top_k;
+ * n_shared 0 or 1.  Other shapes return MOE_ERR_UNSUPPORTED. */
+typedef struct {
+  int32_t hidden;
+  int32_t inter;
+  int32_t n_experts;
+  int32_t n_shared;
+  int32_t top_k;
+  int32_t n_group;
+  int32_t topk_group;
+  int32_t group_size;
+  float routed_scaling_factor;
+} moe_config;
+
+/* One expert in the canonical layout, every pointer 16-byte aligned:
+ *   q_gate, q_up  uint8 [inter][hidden/2]       packed int4 codes
+ *   s_gate, s_up  fp16  [inter][hidden/32]      scales
+ *   q_down        uint8 [hidden][inter/2]
+ *   s_down        fp16  [hidden][inter/32]
+ * Bytes per expert: 3*hidden*inter/2 + 3*hidden*inter/16. */
+typedef struct {
+  const uint8_t* q_gate;
+  const uint8_t* q_up;
+  const uint16_t* s_gate;
+  const uint16_t* s_up;
+  const uint8_t* q_down;
+  const uint16_t* s_down;
+} moe_expert;
+
+typedef struct moe_layer moe_layer;
+
+/* ---- layers ---------------------------------------------------------- */
+
+/* Create a layer VIEW over caller-owned device tensors (nothing is copied):
+ *   w_router_dev fp32 [n_experts][hidden], bias_dev fp32 [n_experts],
+ *   experts_host[n_experts] (host array of device pointers), shared_host
+ *   (host pointer to one moe_expert of device pointers; NULL iff
+ *   n_shared == 0).
+ * The device tensors must stay alive and unchanged until moe_layer_destroy.
+ * Allocates a small device pointer table (about 48 bytes per expert) on the
+ * current device.  Errors: INVALID_ARG (null / misaligned / host memory where
+ * device memory is required), UNSUPPORTED (shape), OOM, CUDA. */
+moe_status moe_layer_create(const moe_config* cfg, const float* w_router_dev,
+                            const float* bias_dev,
+                            const moe_expert* experts_host,
+                            const moe_expert* shared_host, moe_layer** out);
+void moe_layer_destroy(moe_layer* layer);
+
+/* Repoint routed expert e of a layer at other device tensors (used by the
+ * expert cache).  Enqueued on stream, so kernels already enqueued on that
+ * stream still see the old pointers. */
+moe_status moe_layer_set_expert(moe_layer* layer, int e,
+                                const moe_expert* expert_host, void* stream);
+
+/* ---- workspace --------------------------------------------------------- */
+
+/* Bytes of device workspace a call with T tokens needs.  The workspace must
+ * be 256-byte aligned and zero-filled before its first use; every call that
+ * returns MOE_OK leaves its control words zero again.  One workspace must not
+ * be used by two calls that can run at the same time. */
+size_t moe_workspace_bytes(const moe_config* cfg, int T);
+
+/* Synchronise the stream, then read the device error word of a workspace.
+ * Returns MOE_OK, or MOE_ERR_DEVICE / MOE_ERR_TIMEOUT when a kernel reported
+ * a problem (the error word is then cleared), or MOE_ERR_CUDA. */
+moe_status moe_ws_check(void* ws_dev, size_t ws_bytes, void* stream);
+
+/* ---- the hot path ------------------------------------------------------ */
+
+/* Steps 1-2 for T tokens.  x_dev bf16 [T][hidden]; idx_dev int32 [T][top_k]
+ * (ascending expert ids); w_dev fp32 [T][top_k]; scores_dev fp32
+ * [T][n_experts] = sigmoid scores s (nullable, for inspection).
+ * 1 <= T <= 64. */
+moe_status moe_route(const moe_layer* layer, const void* x_dev, int T,
+                     int32_t* idx_dev, float* w_dev, float* scores_dev,
+                     void* ws_dev, size_t ws_bytes, void* stream);
+
+/* Steps 3-5 for T tokens with given routes: y_dev fp32 [T][hidden] =
+ * sum_j w[t][j] * FFN_{idx[t][j]}(x_t) + FFN_shared(x_t).  Expert ids must be
+ * in [0, n_experts); an out-of-range id sets the workspace error word and its
+ * term is skipped.  1 <= T <= 64. */
+moe_status moe_expert_ffn(const moe_layer* layer, const void* x_dev, int T,
+                          const int32_t* idx_dev, const float* w_dev,
+                          float* y_dev, void* ws_dev, size_t ws_bytes,
+                          void* stream);
+
+/* Steps 1-5 for T tokens.  idx_out_dev / w_out_dev nullable.  T == 1 runs the
+ * single fused persistent decode kernel; T > 1 runs the batched path, which
+ * reads every distinct selected expert once for all tokens routed to it.
+ * 1 <= T <= 64. */
+moe_status moe_layer_forward(const moe_layer* layer, const void* x_dev, int T,
+                             float* y_dev, int32_t* idx_out_dev,
+                             float* w_out_dev, void* ws_dev, size_t ws_bytes,
+                             void* stream);
+
+/* ---- diagnostics ------------------------------------------------------- */
+
+/* One dequantising int4 GEMV with the layer kernels' group dot product:
+ * y_dev[r] = sum_c q[r][c] * fp16(s[r][c / 32]) * x_dev[c] for r < rows.
+ * q_dev uint8 [rows][cols/2] (16-byte aligned, packing as in moe_expert),
+ * s_dev fp16 [rows][cols/32], x_dev fp32 [cols] (16-byte aligned), y_dev
+ * fp32 [rows].  cols follows the rule for hidden in moe_config.  For checks
+ * of the packing and the scale indexing (x = a unit vector returns one
+ * dequantised column). */
+moe_status moe_debug_gemv_int4(const uint8_t* q_dev, const uint16_t* s_dev,
+                               int rows, int cols, const float* x_dev,
+                               float* y_dev, void* stream);
+
+const char* moe_status_string(moe_status s);
+/* Text of the last failure on the calling thread ("" if none). */
+const char* moe_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

@@ -1,0 +1,185 @@
+"""Thin Python binding of libmoe.so, the C ABI of include/moe.h (int4
+routed-expert MoE decode layer for B200 / sm_100a).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch provides device memory and streams.  There is no CPU
+fallback: loading fails loudly when libmoe.so is missing.
+"""
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe.so")
+
+MOE_OK = 0
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_CUDA", 3: "MOE_ERR_OOM",
+                4: "MOE_ERR_TIMEOUT", 5: "MOE_ERR_UNSUPPORTED", 6: "MOE_ERR_DEVICE"}
+
+EXPERT_FIELDS = ("q_gate", "q_up", "s_gate", "s_up", "q_down", "s_down")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status, where, detail):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {detail}")
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int32), ("inter", ctypes.c_int32),
+                ("n_experts", ctypes.c_int32), ("n_shared", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("n_group", ctypes.c_int32),
+                ("topk_group", ctypes.c_int32), ("group_size", ctypes.c_int32),
+                ("routed_scaling_factor", ctypes.c_float)]
+
+    @classmethod
+    def from_shape(cls, s):
+        return cls(s.hidden, s.inter, s.n_experts, s.n_shared, s.top_k, s.n_group,
+                   s.topk_group, s.group_size, float(s.rsf))
+
+
+class Expert(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in EXPERT_FIELDS]
+
+    @classmethod
+    def from_ptrs(cls, d):
+        return cls(*[int(d[n]) for n in EXPERT_FIELDS])
+
+
+_lib = None
+
+
+def lib():
+    """Load libmoe.so (built in-tree by build.py); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "python -m int4_routed_expert_noaux_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        p, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        st = ctypes.c_int
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_status_string.argtypes = [st]
+        L.moe_last_error.restype = ctypes.c_char_p
+        L.moe_last_error.argtypes = []
+        L.moe_layer_create.restype = st
+        L.moe_layer_create.argtypes = [p, p, p, p, p, ctypes.POINTER(p)]
+        L.moe_layer_destroy.restype = None
+        L.moe_layer_destroy.argtypes = [p]
+        L.moe_layer_set_expert.restype = st
+        L.moe_layer_set_expert.argtypes = [p, i, p, p]
+        L.moe_workspace_bytes.restype = sz
+        L.moe_workspace_bytes.argtypes = [p, i]
+        L.moe_ws_check.restype = st
+        L.moe_ws_check.argtypes = [p, sz, p]
+        L.moe_route.restype = st
+        L.moe_route.argtypes = [p, p, i, p, p, p, p, sz, p]
+        L.moe_expert_ffn.restype = st
+        L.moe_expert_ffn.argtypes = [p, p, i, p, p, p, p, sz, p]
+        L.moe_layer_forward.restype = st
+        L.moe_layer_forward.argtypes = [p, p, i, p, p, p, p, sz, p]
+        L.moe_debug_gemv_int4.restype = st
+        L.moe_debug_gemv_int4.argtypes = [p, p, i, i, p, p, p]
+        _lib = L
+    return _lib
+
+
+def check(status, where):
+    if status != MOE_OK:
+        raise MoeError(status, where, lib().moe_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def workspace_bytes(cfg, T):
+    return int(lib().moe_workspace_bytes(ctypes.byref(cfg), int(T)))
+
+
+def alloc_workspace(cfg, T, device="cuda"):
+    """Zero-filled workspace tensor (torch allocations are 512-byte aligned)."""
+    import torch
+    n = workspace_bytes(cfg, T)
+    if n == 0:
+        raise MoeError(1, "workspace_bytes", "unsupported config or T")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+class Layer:
+    """A layer view over caller-owned device tensors (see moe_layer_create).
+
+    experts: list of n_experts dicts name -> device address (int) or tensor;
+    shared: one such dict or None.  The tensors must outlive the Layer."""
+
+    def __init__(self, cfg, w_router, bias, experts, shared):
+        self.cfg = cfg
+        arr = (Expert * cfg.n_experts)()
+        for e, d in enumerate(experts):
+            arr[e] = Expert.from_ptrs({k: _addr(v) for k, v in d.items()})
+        sh = Expert.from_ptrs({k: _addr(v) for k, v in shared.items()}) if shared else None
+        out = ctypes.c_void_p()
+        check(lib().moe_layer_create(ctypes.byref(cfg), _addr(w_router), _addr(bias), arr,
+                                     ctypes.byref(sh) if sh is not None else None,
+                                     ctypes.byref(out)), "moe_layer_create")
+        self.handle = out
+        self._keep = (w_router, bias, experts, shared)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib().moe_layer_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def set_expert(self, e, ptrs, stream=None):
+        ex = Expert.from_ptrs({k: _addr(v) for k, v in ptrs.items()})
+        check(lib().moe_layer_set_expert(self.handle, int(e), ctypes.byref(ex), _stream(stream)),
+              "moe_layer_set_expert")
+
+    def route(self, x, idx, w, ws, scores=None, stream=None):
+        T = x.shape[0]
+        check(lib().moe_route(self.handle, _ptr(x), T, _ptr(idx), _ptr(w), _ptr(scores),
+                              _ptr(ws), ws.numel(), _stream(stream)), "moe_route")
+
+    def expert_ffn(self, x, idx, w, y, ws, stream=None):
+        T = x.shape[0]
+        check(lib().moe_expert_ffn(self.handle, _ptr(x), T, _ptr(idx), _ptr(w), _ptr(y),
+                                   _ptr(ws), ws.numel(), _stream(stream)), "moe_expert_ffn")
+
+    def forward(self, x, y, ws, idx=None, w=None, stream=None):
+        T = x.shape[0]
+        check(lib().moe_layer_forward(self.handle, _ptr(x), T, _ptr(y), _ptr(idx), _ptr(w),
+                                      _ptr(ws), ws.numel(), _stream(stream)),
+              "moe_layer_forward")
+
+
+def gemv_int4(q, s, rows, cols, x, y, stream=None):
+    """y = dequant(q, s) @ x through the library's int4 group dot product."""
+    check(lib().moe_debug_gemv_int4(_ptr(q), _ptr(s), int(rows), int(cols), _ptr(x), _ptr(y),
+                                    _stream(stream)), "moe_debug_gemv_int4")
+
+
+def ws_check(ws, stream=None):
+    check(lib().moe_ws_check(_ptr(ws), ws.numel(), _stream(stream)), "moe_ws_check")
+
+
+def _addr(v):
+    if v is None:
+        return None
+    if isinstance(v, int):
+        return v
+    return v.data_ptr()

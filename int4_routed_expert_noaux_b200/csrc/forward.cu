@@ -1,0 +1,43 @@
+// forward.cu -- launch sequences of the hot path.
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "layer.h"
+
+namespace moe {
+
+moe_status route_impl(const moe_layer* l, const uint16_t* x, int T, int32_t* idx, float* w,
+                      float* scores, uint8_t* ws, const WsLayout& L, cudaStream_t st) {
+  const moe_config& c = l->cfg;
+  float* logits = reinterpret_cast<float*>(ws + L.logits);
+  cudaError_t e = launch_router_logits(l->w_router, x, T, c.hidden, c.n_experts, logits, st);
+  if (e == cudaSuccess)
+    e = launch_select(logits, l->bias, T, c.n_experts, c.n_group, c.topk_group, c.top_k,
+                      c.routed_scaling_factor, idx, w, scores, st);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "route launch");
+}
+
+moe_status ffn_impl(const moe_layer* l, const uint16_t* x, int T, const int32_t* idx,
+                    const float* w, float* y, uint8_t* ws, const WsLayout& L, cudaStream_t st) {
+  const moe_config& c = l->cfg;
+  const int slots = c.top_k + c.n_shared;
+  float* hbuf = reinterpret_cast<float*>(ws + L.hbuf);
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws + L.ctrl);
+  cudaError_t e = launch_gate_up(l->table, idx, c.n_experts, c.top_k, slots, x, T, c.hidden,
+                                 c.inter, hbuf, err, st);
+  if (e == cudaSuccess)
+    e = launch_down_combine(l->table, idx, w, c.n_experts, c.top_k, slots, hbuf, T, c.hidden,
+                            c.inter, y, err, st);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "expert launch");
+}
+
+moe_status forward_impl(const moe_layer* l, const uint16_t* x, int T, float* y, int32_t* idx_out,
+                        float* w_out, uint8_t* ws, const WsLayout& L, cudaStream_t st) {
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
+  float* w = w_out ? w_out : reinterpret_cast<float*>(ws + L.w);
+  moe_status s = route_impl(l, x, T, idx, w, nullptr, ws, L, st);
+  if (s != MOE_OK) return s;
+  return ffn_impl(l, x, T, idx, w, y, ws, L, st);
+}
+
+}  // namespace moe

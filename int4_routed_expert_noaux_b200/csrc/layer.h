@@ -1,0 +1,45 @@
+// layer.h -- host-side layer view, workspace layout and the launch
+// sequences shared by the C ABI entry points.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "moe.h"
+
+struct moe_layer {
+  moe_config cfg;
+  const float* w_router = nullptr;   // device fp32 [E][H]
+  const float* bias = nullptr;       // device fp32 [E]
+  moe::ExpertPtrs* table = nullptr;  // device [E + 1]; entry E = shared
+  moe::ExpertPtrs* host_table = nullptr;
+  int device = 0;
+};
+
+namespace moe {
+
+constexpr int kMaxTokens = 64;
+constexpr size_t kCtrlBytes = 256;  // error word + counters of fused kernels
+
+// Byte offsets inside a workspace.
+struct WsLayout {
+  size_t ctrl, logits, idx, w, hbuf, total;
+};
+
+WsLayout ws_layout(const moe_config* c, int T);
+moe_status fail(moe_status s, const char* fmt, ...);
+moe_status cuda_fail(cudaError_t e, const char* what);
+moe_status check_config(const moe_config* c);
+moe_status check_expert(const moe_expert* e, const char* what);
+ExpertPtrs to_ptrs(const moe_expert& e);
+
+moe_status route_impl(const moe_layer* l, const uint16_t* x, int T, int32_t* idx, float* w,
+                      float* scores, uint8_t* ws, const WsLayout& L, cudaStream_t st);
+moe_status ffn_impl(const moe_layer* l, const uint16_t* x, int T, const int32_t* idx,
+                    const float* w, float* y, uint8_t* ws, const WsLayout& L, cudaStream_t st);
+moe_status forward_impl(const moe_layer* l, const uint16_t* x, int T, float* y, int32_t* idx_out,
+                        float* w_out, uint8_t* ws, const WsLayout& L, cudaStream_t st);
+
+}  // namespace moe

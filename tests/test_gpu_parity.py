@@ -1,0 +1,209 @@
+"""GPU parity of the hot path against the fp64 oracle, through the C ABI.
+
+Bars: expert ids bit-exact (ties to the lower index); weights within fp32
+rounding; outputs max |dy| <= 2e-3 * rms(y_oracle) per token.  Routing
+decisions are also checked in the kernel's own precision: the oracle's
+selection applied to the GPU's fp32 scores must give the GPU's ids for every
+token.  Tokens whose fp64 decision margin is below FLAG_MARGIN are reported
+and checked that way only (fp32 logits carry errors of order 1e-6 to 1e-5,
+so a smaller gap may legitimately flip)."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from synth.layers import DeviceLayer
+
+torch = pytest.importorskip("torch")
+import int4_routed_expert_noaux_b200 as moe  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+MEDIUM = synth.Shape(hidden=3072, inter=1024, n_experts=36, n_shared=1, top_k=5, n_group=4,
+                     topk_group=2)
+FLAG_MARGIN = 1e-5
+Y_TOL = 2e-3
+
+
+def needs_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+_LAYERS = {}
+
+
+def get_layer(shape, seed=0, layer=0):
+    needs_gpu()
+    key = (shape, seed, layer)
+    if key not in _LAYERS:
+        dl = DeviceLayer(shape, seed, layer)
+        L = moe.Layer(moe.Config.from_shape(shape), dl.w_router, dl.bias, dl.routed, dl.shared)
+        _LAYERS[key] = (dl, L)
+    return _LAYERS[key]
+
+
+def to_dev_bf16(x_bits):
+    return torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).cuda()
+
+
+def oracle_y(shape, dl, x_bits, idx, w):
+    needed = sorted(set(int(e) for e in np.ravel(idx)))
+    ex = {e: dl.host_expert(e) for e in needed}
+    sh = dl.host_expert(shape.n_experts) if shape.n_shared else None
+    xd = synth.bf16_to_f32(x_bits).astype(np.float64)
+    return oracle.experts_combine(shape, ex, sh, xd, idx, np.asarray(w, dtype=np.float64))
+
+
+def assert_y_close(y_gpu, y_ref):
+    for t in range(y_ref.shape[0]):
+        rms = np.sqrt(np.mean(y_ref[t] ** 2))
+        err = np.max(np.abs(y_gpu[t].astype(np.float64) - y_ref[t]))
+        assert err <= Y_TOL * rms, (t, err, rms, err / rms)
+
+
+def run_route(shape, L, x_bits):
+    T = x_bits.shape[0]
+    cfg = moe.Config.from_shape(shape)
+    x = to_dev_bf16(x_bits)
+    idx = torch.empty((T, shape.top_k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, shape.top_k), dtype=torch.float32, device="cuda")
+    sc = torch.empty((T, shape.n_experts), dtype=torch.float32, device="cuda")
+    ws = moe.alloc_workspace(cfg, T)
+    L.route(x, idx, w, ws, scores=sc)
+    moe.ws_check(ws)
+    return idx.cpu().numpy(), w.cpu().numpy(), sc.cpu().numpy()
+
+
+def check_route(shape, dl, x_bits, gidx, gw, gsc):
+    W, b = dl.host_router()
+    lg = oracle.router_logits(shape, W, x_bits)
+    oidx, ow, margin, osc = oracle.route(shape, lg, b)
+    # (a) sigmoid scores
+    assert np.max(np.abs(gsc.astype(np.float64) - osc)) <= 1e-5
+    # (b) the decision in the kernel's precision: oracle selection on the
+    # GPU's fp32 scores and fp32 bias-corrected scores
+    sp32 = (gsc + b[None, :]).astype(np.float32)
+    didx, dw, _ = oracle.select_scores(shape, gsc.astype(np.float64), sp32.astype(np.float64),
+                                       round_group_f32=True)
+    assert np.array_equal(gidx, didx)
+    assert np.allclose(gw, dw, rtol=2e-6, atol=1e-7)
+    # (c) bit-exact against the fp64 oracle where the decision is not a near tie
+    ok = margin > FLAG_MARGIN
+    assert np.array_equal(gidx[ok], oidx[ok])
+    assert np.allclose(gw[ok], ow[ok], rtol=2e-5, atol=1e-6)
+    # invariants
+    per = shape.n_experts // shape.n_group
+    for t in range(gidx.shape[0]):
+        assert np.all(np.diff(gidx[t]) > 0)
+        assert len(set((gidx[t] // per).tolist())) <= shape.topk_group
+        assert abs(float(gw[t].sum()) - shape.rsf) <= 1e-5 * shape.rsf
+    return int((~ok).sum())
+
+
+@pytest.mark.parametrize("shape,T", [(synth.TINY, 1), (synth.TINY, 13), (MEDIUM, 7),
+                                     (synth.GLM, 64)], ids=["tiny1", "tiny13", "medium7", "glm64"])
+def test_route_parity(shape, T):
+    dl, L = get_layer(shape)
+    x_bits = synth.tokens(shape, 0, 100, T)
+    gidx, gw, gsc = run_route(shape, L, x_bits)
+    check_route(shape, dl, x_bits, gidx, gw, gsc)
+
+
+@pytest.mark.parametrize("shape,T", [(synth.TINY, 4), (MEDIUM, 3), (synth.GLM, 2)],
+                         ids=["tiny", "medium", "glm"])
+def test_expert_ffn_parity(shape, T):
+    dl, L = get_layer(shape)
+    cfg = moe.Config.from_shape(shape)
+    x_bits = synth.tokens(shape, 0, 200, T)
+    rng = np.random.default_rng(T)
+    idx = np.stack([np.sort(rng.choice(shape.n_experts, shape.top_k, replace=False))
+                    for _ in range(T)]).astype(np.int32)
+    w = rng.uniform(0.1, 1.0, size=(T, shape.top_k)).astype(np.float32)
+    y = torch.empty((T, shape.hidden), dtype=torch.float32, device="cuda")
+    ws = moe.alloc_workspace(cfg, T)
+    L.expert_ffn(to_dev_bf16(x_bits), torch.from_numpy(idx).cuda(), torch.from_numpy(w).cuda(),
+                 y, ws)
+    moe.ws_check(ws)
+    assert_y_close(y.cpu().numpy(), oracle_y(shape, dl, x_bits, idx, w))
+
+
+def run_forward(shape, L, x_bits):
+    T = x_bits.shape[0]
+    cfg = moe.Config.from_shape(shape)
+    y = torch.empty((T, shape.hidden), dtype=torch.float32, device="cuda")
+    idx = torch.empty((T, shape.top_k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, shape.top_k), dtype=torch.float32, device="cuda")
+    ws = moe.alloc_workspace(cfg, T)
+    L.forward(to_dev_bf16(x_bits), y, ws, idx=idx, w=w)
+    moe.ws_check(ws)
+    return y.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy()
+
+
+def check_forward(shape, dl, x_bits, y, gidx, gw):
+    W, b = dl.host_router()
+    lg = oracle.router_logits(shape, W, x_bits)
+    oidx, ow, margin, _ = oracle.route(shape, lg, b)
+    same = np.all(gidx == oidx, axis=1)
+    assert np.all(same | (margin <= FLAG_MARGIN))
+    # outputs: against the oracle's own routes where they agree, and against
+    # the oracle FFN on the GPU's routes everywhere
+    if same.any():
+        assert_y_close(y[same], oracle_y(shape, dl, x_bits[same], oidx[same], ow[same]))
+    assert_y_close(y, oracle_y(shape, dl, x_bits, gidx, gw))
+
+
+@pytest.mark.parametrize("shape,T,first", [(synth.TINY, 1, 0), (synth.TINY, 1, 1),
+                                           (synth.TINY, 5, 7), (MEDIUM, 1, 0), (MEDIUM, 6, 3),
+                                           (synth.GLM, 1, 0), (synth.GLM, 1, 1),
+                                           (synth.GLM, 3, 10)],
+                         ids=["tiny-a", "tiny-b", "tiny-T5", "medium-1", "medium-T6",
+                              "glm-a", "glm-b", "glm-T3"])
+def test_layer_forward_parity(shape, T, first):
+    dl, L = get_layer(shape)
+    x_bits = synth.tokens(shape, 0, first, T)
+    y, gidx, gw = run_forward(shape, L, x_bits)
+    check_forward(shape, dl, x_bits, y, gidx, gw)
+
+
+def test_forward_deterministic():
+    dl, L = get_layer(synth.GLM)
+    x_bits = synth.tokens(synth.GLM, 0, 5, 1)
+    y1, i1, w1 = run_forward(synth.GLM, L, x_bits)
+    y2, i2, w2 = run_forward(synth.GLM, L, x_bits)
+    assert np.array_equal(y1, y2) and np.array_equal(i1, i2) and np.array_equal(w1, w2)
+
+
+def test_gemv_one_hot_columns():
+    needs_gpu()
+    rows, cols = 64, 256
+    rng = np.random.default_rng(9)
+    codes = rng.integers(-8, 8, size=(rows, cols))
+    u = (codes & 0xF).astype(np.uint8)
+    q = (u[:, 0::2] | (u[:, 1::2] << 4)).astype(np.uint8)
+    sc = rng.uniform(0.005, 0.02, size=(rows, cols // 32)).astype(np.float16)
+    qd = torch.from_numpy(q).cuda()
+    sd = torch.from_numpy(sc.view(np.int16)).cuda()
+    y = torch.empty(rows, dtype=torch.float32, device="cuda")
+    for c in range(cols):
+        x = torch.zeros(cols, dtype=torch.float32, device="cuda")
+        x[c] = 1.0
+        moe.gemv_int4(qd, sd, rows, cols, x, y)
+        expect = (codes[:, c] * sc[:, c // 32].astype(np.float64)).astype(np.float32)
+        assert np.array_equal(y.cpu().numpy(), expect), c
+
+
+def test_bad_expert_id_reported():
+    shape = synth.TINY
+    dl, L = get_layer(shape)
+    cfg = moe.Config.from_shape(shape)
+    x_bits = synth.tokens(shape, 0, 0, 1)
+    idx = torch.tensor([[3, 99]], dtype=torch.int32, device="cuda")
+    w = torch.tensor([[1.0, 1.0]], dtype=torch.float32, device="cuda")
+    y = torch.empty((1, shape.hidden), dtype=torch.float32, device="cuda")
+    ws = moe.alloc_workspace(cfg, 1)
+    L.expert_ffn(to_dev_bf16(x_bits), idx, w, y, ws)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.ws_check(ws)
+    assert ei.value.status == 6
+    moe.ws_check(ws)  # cleared

@@ -73,6 +73,8 @@ def test_correlated_tokens_overlap():
 @pytest.mark.gpu
 def test_device_generator_matches_host():
     import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
     sh = synth.GLM
     ptrs, bufs = {}, {}
     for name, dt, shp, tag in synth.expert_layout(sh):
