@@ -151,26 +151,30 @@ __device__ __forceinline__ float dot_group(const uint4 w, const XGroup& g) {
 // Butterfly reduce-scatter of NV values across SEG lanes (SEG a power of two
 // <= 32, NV a power of two <= SEG).  On return v[0] of each lane holds the
 // sum over the lane's SEG-lane segment of value index reduce_index<NV,SEG>.
+template <int NV, int O, int N>
+__device__ __forceinline__ void reduce_scatter_stage(float (&v)[NV], int lane) {
+  if constexpr (O >= 1) {
+    if constexpr (N > 1) {
+      constexpr int half = N / 2;
+      const bool upper = (lane & O) != 0;
+#pragma unroll
+      for (int i = 0; i < half; ++i) {
+        const float send = upper ? v[i] : v[i + half];
+        const float keep = upper ? v[i + half] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+      }
+      reduce_scatter_stage<NV, O / 2, half>(v, lane);
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
+      reduce_scatter_stage<NV, O / 2, 1>(v, lane);
+    }
+  }
+}
+
 template <int NV, int SEG>
 __device__ __forceinline__ void reduce_scatter(float (&v)[NV]) {
   static_assert(NV <= SEG && SEG <= 32, "bad reduce shape");
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int o = SEG / 2, n = NV; o >= 1; o >>= 1) {
-    if (n > 1) {
-      const int half = n >> 1;
-      const bool upper = (lane & o) != 0;
-#pragma unroll
-      for (int i = 0; i < half; ++i) {
-        float send = upper ? v[i] : v[i + half];
-        float keep = upper ? v[i + half] : v[i];
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-      }
-      n = half;
-    } else {
-      v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
-    }
-  }
+  reduce_scatter_stage<NV, SEG / 2, NV>(v, threadIdx.x & 31);
 }
 
 template <int NV, int SEG>
@@ -209,10 +213,9 @@ struct ColMap {
   int wir;    // this warp's index inside its row (0..wpr-1)
 };
 
-__device__ __forceinline__ ColMap col_map(int G) {
+__device__ __forceinline__ ColMap col_map_n(int G, int NW) {
   ColMap m;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int NW = blockDim.x >> 5;
   if (G >= 32) {
     m.wpr = G >> 5;
     m.P = NW / m.wpr;
@@ -231,5 +234,7 @@ __device__ __forceinline__ ColMap col_map(int G) {
   }
   return m;
 }
+
+__device__ __forceinline__ ColMap col_map(int G) { return col_map_n(G, blockDim.x >> 5); }
 
 }  // namespace moe

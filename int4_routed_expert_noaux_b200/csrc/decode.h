@@ -1,0 +1,54 @@
+// decode.h -- the fused persistent decode kernel (one launch per token).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "moe.h"
+
+namespace moe {
+
+// Control words at the start of a workspace (uint32 indices).  Word 0 is the
+// error word the host reads; the rest are counters of the fused kernel,
+// zero between calls.
+constexpr size_t kCtrlBytes = 4096;
+enum : int {
+  kCtrlErr = 0,
+  kCtrlTicket = 1,
+  kCtrlRouterDone = 2,
+  kCtrlSelReady = 3,
+  kCtrlExit = 4,
+  kCtrlAbort = 5,
+  kCtrlGuDone = 16,  // [slots]
+  kCtrlRbDone = 64,  // [row blocks of hidden]
+};
+
+struct DecodeParams {
+  const ExpertPtrs* table;
+  const float* w_router;
+  const float* bias;
+  const uint16_t* x;  // bf16 [H]
+  float* y;           // fp32 [H]
+  int32_t* idx_out;   // nullable
+  float* w_out;       // nullable
+  uint32_t* ctrl;
+  float* logits;      // [E]
+  int32_t* idx_ws;    // [k]
+  float* w_ws;        // [k]
+  float* hbuf;        // [slots][I]
+  float* ypart;       // [slots][H]
+  int H, I, E, k, n_group, topk_group, has_shared;
+  float rsf;
+  int RR, RG, RD;     // rows per router / gate-up / down item
+  int nR, nG, nD, n_items;
+};
+
+// Fill the shape part of p; false if the fused kernel does not cover the
+// shape (the step kernels are used instead).
+bool decode_plan(const moe_config& c, DecodeParams& p);
+size_t decode_smem_bytes();
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t st);
+
+}  // namespace moe

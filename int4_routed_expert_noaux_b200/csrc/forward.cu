@@ -1,6 +1,7 @@
 // forward.cu -- launch sequences of the hot path.
 #include <cuda_runtime.h>
 
+#include "decode.h"
 #include "kernels.h"
 #include "layer.h"
 
@@ -33,6 +34,24 @@ moe_status ffn_impl(const moe_layer* l, const uint16_t* x, int T, const int32_t*
 
 moe_status forward_impl(const moe_layer* l, const uint16_t* x, int T, float* y, int32_t* idx_out,
                         float* w_out, uint8_t* ws, const WsLayout& L, cudaStream_t st) {
+  DecodeParams p;
+  if (T == 1 && decode_plan(l->cfg, p)) {
+    p.table = l->table;
+    p.w_router = l->w_router;
+    p.bias = l->bias;
+    p.x = x;
+    p.y = y;
+    p.idx_out = idx_out;
+    p.w_out = w_out;
+    p.ctrl = reinterpret_cast<uint32_t*>(ws + L.ctrl);
+    p.logits = reinterpret_cast<float*>(ws + L.logits);
+    p.idx_ws = reinterpret_cast<int32_t*>(ws + L.idx);
+    p.w_ws = reinterpret_cast<float*>(ws + L.w);
+    p.hbuf = reinterpret_cast<float*>(ws + L.hbuf);
+    p.ypart = reinterpret_cast<float*>(ws + L.ypart);
+    cudaError_t e = launch_decode(p, st);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "decode launch");
+  }
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
   float* w = w_out ? w_out : reinterpret_cast<float*>(ws + L.w);
   moe_status s = route_impl(l, x, T, idx, w, nullptr, ws, L, st);

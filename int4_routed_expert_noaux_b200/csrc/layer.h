@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "decode.h"
 #include "moe.h"
 
 struct moe_layer {
@@ -21,11 +22,10 @@ struct moe_layer {
 namespace moe {
 
 constexpr int kMaxTokens = 64;
-constexpr size_t kCtrlBytes = 256;  // error word + counters of fused kernels
 
 // Byte offsets inside a workspace.
 struct WsLayout {
-  size_t ctrl, logits, idx, w, hbuf, total;
+  size_t ctrl, logits, idx, w, hbuf, ypart, total;
 };
 
 WsLayout ws_layout(const moe_config* c, int T);

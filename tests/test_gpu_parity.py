@@ -207,3 +207,39 @@ def test_bad_expert_id_reported():
         moe.ws_check(ws)
     assert ei.value.status == 6
     moe.ws_check(ws)  # cleared
+
+
+@pytest.mark.parametrize("shape,n", [(synth.TINY, 24), (MEDIUM, 8), (synth.GLM, 6)],
+                         ids=["tiny", "medium", "glm"])
+def test_many_decode_calls_one_workspace(shape, n):
+    # back-to-back single-token calls with no host sync in between: the fused
+    # kernel's control counters must come back to zero after every call
+    dl, L = get_layer(shape)
+    cfg = moe.Config.from_shape(shape)
+    x_bits = synth.tokens(shape, 0, 300, n)
+    x = to_dev_bf16(x_bits)
+    ys = torch.empty((n, shape.hidden), dtype=torch.float32, device="cuda")
+    idx = torch.empty((n, shape.top_k), dtype=torch.int32, device="cuda")
+    w = torch.empty((n, shape.top_k), dtype=torch.float32, device="cuda")
+    ws = moe.alloc_workspace(cfg, 1)
+    for t in range(n):
+        L.forward(x[t:t + 1], ys[t:t + 1], ws, idx=idx[t:t + 1], w=w[t:t + 1])
+    moe.ws_check(ws)
+    assert int(ws[4:4096].count_nonzero().item()) == 0  # counters reset
+    check_forward(shape, dl, x_bits, ys.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy())
+
+
+def test_fused_decode_matches_step_kernels():
+    shape = synth.GLM
+    dl, L = get_layer(shape)
+    cfg = moe.Config.from_shape(shape)
+    x_bits = synth.tokens(shape, 0, 42, 1)
+    y_f, idx, w = run_forward(shape, L, x_bits)
+    y_s = torch.empty((1, shape.hidden), dtype=torch.float32, device="cuda")
+    ws = moe.alloc_workspace(cfg, 1)
+    L.expert_ffn(to_dev_bf16(x_bits), torch.from_numpy(idx).cuda(), torch.from_numpy(w).cuda(),
+                 y_s, ws)
+    moe.ws_check(ws)
+    y_s = y_s.cpu().numpy()
+    rms = np.sqrt(np.mean(y_s.astype(np.float64) ** 2))
+    assert np.max(np.abs(y_f - y_s)) <= 1e-4 * rms
