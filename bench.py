@@ -48,6 +48,8 @@ def parse():
     p.add_argument("--cpu-sample", type=int, default=6, help="tokens in the CPU-baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--small", action="store_true", help="tiny layer (smoke/profiling only)")
+    p.add_argument("--experts", type=int, default=0,
+                   help="routed experts per layer (profiling only; default: the shape's 256)")
     return p.parse_args()
 
 
@@ -202,6 +204,9 @@ def main():
     args = parse()
     import synth
     shape = synth.TINY if args.small else synth.GLM
+    if args.experts:
+        import dataclasses
+        shape = dataclasses.replace(shape, n_experts=args.experts)
     if args.impl == "reference":
         run_reference(args, shape)
         return
@@ -362,7 +367,7 @@ def main():
 
 
 def launches_per_forward():
-    return 4
+    return 1
 
 
 if __name__ == "__main__":

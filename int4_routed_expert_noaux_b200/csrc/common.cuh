@@ -82,67 +82,88 @@ __device__ __forceinline__ uint32_t lop3_sel_xor(uint32_t a, uint32_t c1, uint32
 }
 
 // ---------------------------------------------------------------------------
-// int4 x fp32 dot product of one 32-input scale group (16 packed bytes).
+// int4 dot product of one 32-input scale group (16 packed bytes), exact in
+// integers.
 //
-// A nibble n (two's complement code q) placed in bits [12,16) of the
-// mantissa of 1.0f, with its top bit flipped, is the float 1 + (q+8) 2^-11;
-// placed in bits [16,20) it is 1 + (q+8) 2^-7.  One LOP3 builds either
-// float from a shifted copy of the packed word.  Inputs are paired so that
-// each shifted word yields (odd element in [12,16), even element in
-// [16,20)); a packed FMA accumulates acc = {accB, accA} over the 16 pairs of
-// the group, with
-//     accB0 = -(1 + 8 * 2^-11) * sum_odd x,   accA0 = -(1 + 8 * 2^-7) * sum_even x
-// so that at the end  sum_k q_k x_k = 2048 * accB + 128 * accA.
+// The group's 32 inputs x_k are held as int16 X_k = round(x_k * 2^e) with
+// one power-of-two exponent e per group, chosen so that max |X_k| <= 2^14
+// (exact for every input within 2^6 of the group's largest; otherwise the
+// representation error is below 2^-14 of the group's largest input).
+// A packed word w holds codes q_{8i..8i+7} (nibble j = element 8i + j,
+// two's complement).  The bytes of (w & 0xF0F0F0F0), read as signed int8,
+// are exactly 16 * q of the odd elements; those of ((w << 4) & 0xF0F0F0F0)
+// are 16 * q of the even elements.  dp2a multiplies two int16 by two int8
+// and accumulates in int32, so four dp2a per word give 16 * sum q_k X_k with
+// no rounding (|sum| < 2^27 and a multiple of 16: the int32 -> fp32
+// conversion is exact too).  sum_k q_k x_k = that * 2^-e / 16.
 //
-// XGroup holds the group's 32 inputs as 16 packed pairs in the order
-//   p[0] = {x31, x0},  p[m] = {x(2m-1), x(2m)} for m = 1..15,
-// and init = {accB0, accA0}.
-struct XGroup {
-  unsigned long long p[16];
-  unsigned long long init;
+// XQ holds the int16 pairs in dp2a order: for word i,
+//   ev[2i] = (X_{8i}, X_{8i+2})    ev[2i+1] = (X_{8i+4}, X_{8i+6})
+//   od[2i] = (X_{8i+1}, X_{8i+3})  od[2i+1] = (X_{8i+5}, X_{8i+7})
+// and f = 2^-e / 16.
+struct XQ {
+  uint32_t ev[8];
+  uint32_t od[8];
+  float f;
 };
 
-// Build the XGroup of inputs x[0..31] (given as floats).
-__device__ __forceinline__ void xgroup_from_floats(const float* x, XGroup& g) {
-  float so = 0.f, se = 0.f;
-#pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    se += x[i];
-    so += x[i + 1];
-  }
-  g.p[0] = pack_f2(x[31], x[0]);
-#pragma unroll
-  for (int m = 1; m < 16; ++m) g.p[m] = pack_f2(x[2 * m - 1], x[2 * m]);
-  g.init = pack_f2(-1.00390625f * so, -1.0625f * se);
+__device__ __forceinline__ uint32_t pack_i16x2(int lo, int hi) {
+  return (uint32_t)(lo & 0xFFFF) | ((uint32_t)hi << 16);
 }
 
-// sum_k q_k x_k for the 32 codes of one 16-byte chunk (words w0..w3).
-__device__ __forceinline__ float dot_group(const uint4 w, const XGroup& g) {
-  const uint32_t MB = 0x0000F000u, CB = 0x3F808000u;  // window [12,16)
-  const uint32_t MA = 0x000F0000u, CA = 0x3F880000u;  // window [16,20)
-  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-  unsigned long long acc = g.init;
+// Quantise 32 floats to an XQ (shared power-of-two exponent, RNE).
+__device__ __forceinline__ void xq_from_floats(const float* x, XQ& g) {
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(x[i]));
+  int ex = 0;
+  if (m > 0.f) frexpf(m, &ex);  // m = fr * 2^ex, fr in [0.5, 1)
+  const int e = 14 - ex;        // m * 2^e < 2^14
+  const float sc = (m > 0.f) ? ldexpf(1.0f, e) : 0.f;
+  g.f = (m > 0.f) ? ldexpf(1.0f, -e - 4) : 0.f;
+  int X[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) X[i] = __float2int_rn(x[i] * sc);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint32_t wi = ws[i];
-    const uint32_t wn = ws[(i + 1) & 3];
-    uint32_t s;
-    // pair m = 4i+1: nibbles 1 (B) and 2 (A) of word i
-    s = wi << 8;
-    acc = ffma2(pack_u2(lop3_sel_xor(s, MB, CB), lop3_sel_xor(s, MA, CA)), g.p[4 * i + 1], acc);
-    // pair m = 4i+2: nibbles 3 (B) and 4 (A)
-    s = wi;
-    acc = ffma2(pack_u2(lop3_sel_xor(s, MB, CB), lop3_sel_xor(s, MA, CA)), g.p[4 * i + 2], acc);
-    // pair m = 4i+3: nibbles 5 (B) and 6 (A)
-    s = wi >> 8;
-    acc = ffma2(pack_u2(lop3_sel_xor(s, MB, CB), lop3_sel_xor(s, MA, CA)), g.p[4 * i + 3], acc);
-    // pair m = 4i+4 (mod 16): nibble 7 of word i (B), nibble 0 of word i+1 (A)
-    s = __funnelshift_r(wi, wn, 16);
-    acc = ffma2(pack_u2(lop3_sel_xor(s, MB, CB), lop3_sel_xor(s, MA, CA)), g.p[(4 * i + 4) & 15], acc);
+    g.ev[2 * i] = pack_i16x2(X[8 * i + 0], X[8 * i + 2]);
+    g.ev[2 * i + 1] = pack_i16x2(X[8 * i + 4], X[8 * i + 6]);
+    g.od[2 * i] = pack_i16x2(X[8 * i + 1], X[8 * i + 3]);
+    g.od[2 * i + 1] = pack_i16x2(X[8 * i + 5], X[8 * i + 7]);
   }
-  float accB, accA;
-  unpack_f2(acc, accB, accA);
-  return fmaf(accB, 2048.f, accA * 128.f);
+}
+
+__device__ __forceinline__ int dp2a_lo(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.lo.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ int dp2a_hi(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.hi.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// 16 * sum_k q_k X_k over the 32 codes of one 16-byte chunk.
+__device__ __forceinline__ int dotq_group(const uint4 w, const XQ& g) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  int ae = 0, ao = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t odd = ws[i] & 0xF0F0F0F0u;
+    const uint32_t even = (ws[i] << 4) & 0xF0F0F0F0u;
+    ae = dp2a_lo(g.ev[2 * i], even, ae);
+    ae = dp2a_hi(g.ev[2 * i + 1], even, ae);
+    ao = dp2a_lo(g.od[2 * i], odd, ao);
+    ao = dp2a_hi(g.od[2 * i + 1], odd, ao);
+  }
+  return ae + ao;
+}
+
+// sum_k (q_k * scale) x_k for one chunk: exact group sum, one rounding.
+__device__ __forceinline__ float dot_scaled(const uint4 w, const XQ& g, float scale) {
+  return (float)dotq_group(w, g) * (scale * g.f);
 }
 
 // ---------------------------------------------------------------------------

@@ -3,29 +3,33 @@
 // int4 expert FFNs, weighted combine) in ONE launch.
 //
 // Design (sm_100a):
-//  * one CTA per SM; warp 6 is the producer, warps 0-5 (192 threads) consume;
+//  * one CTA per SM: a producer warp and two consumer groups of 6 warps;
 //  * the producer claims work items from a global ticket counter, in a fixed
 //    order, and moves each item's weights HBM -> shared memory with 1-D bulk
-//    async copies (the TMA engine) into a 3-stage ring of 56 KB stages,
-//    completion tracked by mbarriers (transaction bytes);
+//    async copies (the TMA engine) into a 4-stage ring of 54 KB stages,
+//    completion tracked by mbarriers (transaction bytes).  Fill n goes to
+//    stage n % 4 and is consumed by group n % 2, so one group reduces and
+//    publishes while the other computes and two stages stay in flight;
 //  * consumers are column-stationary: each thread owns one 16-byte chunk
-//    column of the rows it visits, keeps its 32 inputs in registers and runs
-//    the LOP3 + packed-FMA int4 group dot product; one butterfly
-//    reduce-scatter plus a cross-warp sum finishes each row;
+//    column of the rows it visits and keeps its 32 inputs in registers as
+//    int16 fixed point with one exponent per group; the int4 group dot
+//    product is exact in integers (dp2a); one butterfly reduce-scatter plus
+//    a cross-warp sum finishes each row; one named barrier per item;
 //  * item order: router rows, shared-expert gate/up, shared-expert down,
 //    routed gate/up of slot 0, then (gate/up of slot j, down of slot j-1)
 //    for j = 1..k-1, then down of slot k-1.  Every dependency points to an
-//    earlier ticket (router -> selection -> routed items; gate/up of a slot
-//    -> its down items), so in-order claiming always makes progress;
-//  * the CTA that finishes the last router item runs the selection and
+//    earlier ticket, so in-order claiming always makes progress;
+//  * the warp that finishes the last router item runs the selection and
 //    publishes idx / w with a release flag; the producer acquires it before
 //    loading routed weights;
-//  * down items write per-slot partial rows; the CTA that completes the last
-//    slot of a row block sums the partials in slot order (deterministic,
-//    no atomics on data) into y;
+//  * the warp that finishes the last gate/up item of a slot converts that
+//    slot's h to int16 groups once and flags it ready for the down items;
+//  * down items write per-slot partial rows; the warp that completes the
+//    last slot of a row block sums the partials in slot order
+//    (deterministic, no atomics on data) into y;
 //  * every wait is bounded (1 s); a wait that runs out sets the workspace
-//    error word, and all threads leave in step; the last CTA to exit resets
-//    the control counters so the next call starts clean.
+//    error word and the kernel winds down; the last CTA to exit resets the
+//    control counters so the next call starts clean.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -37,13 +41,16 @@ namespace moe {
 
 namespace {
 
-constexpr int kCW = 6;                  // consumer warps
-constexpr int kCT = kCW * 32;           // consumer threads
-constexpr int kThreads = kCT + 32;      // + producer warp
-constexpr int kStages = 3;
-constexpr uint32_t kStageBytes = 57344;
-constexpr int kRouterChunks = 8;        // 16-byte W chunks per consumer per row
-constexpr int kMaxRR = 8;               // router rows per item
+constexpr int kGW = 6;                   // warps per consumer group
+constexpr int kGT = kGW * 32;            // threads per consumer group
+constexpr int kGroups = 2;
+constexpr int kThreads = kGroups * kGT + 32;
+constexpr int kProducerWarp = kGroups * kGW;
+constexpr int kStages = 4;
+constexpr uint32_t kStageBytes = 55296;
+constexpr int kRouterChunks = 8;         // 16-byte W chunks per thread per row
+constexpr int kMaxRR = 8;                // router rows per item
+constexpr int kMaxE = 256;
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 enum ItemType : int { kRouter = 0, kGateUp = 1, kDown = 2, kDone = 3 };
@@ -56,12 +63,10 @@ struct Smem {
   uint64_t full[kStages];
   uint64_t empty[kStages];
   ItemDesc desc[kStages];
-  float red[kCW][32];
-  int status;        // consumer broadcast: 1 = go on, 0 = stop
-  int flag;          // consumer broadcast: run select / combine
-  float gscore[32];
-  float sc[1024];
-  float sp[1024];
+  float red[kGroups][2][kGW][32];
+  int abort_flag[kGroups];
+  float sc[kMaxE];
+  float sp[kMaxE];
 };
 
 __device__ __forceinline__ ItemDesc make_item(int type, int slot, int row0, int nrows) {
@@ -117,7 +122,7 @@ __device__ bool wait_counter(uint32_t* ctrl, const uint32_t* p, uint32_t target)
   const uint64_t deadline = global_timer_ns() + kWaitNs;
   for (uint32_t it = 0;; ++it) {
     if (ld_acquire(p) >= target) return true;
-    __nanosleep(64);
+    __nanosleep(32);
     if ((it & 15) == 15) {
       if (aborted(ctrl) || global_timer_ns() > deadline) return false;
     }
@@ -147,76 +152,117 @@ __device__ __forceinline__ ArgMaxF am_warp(ArgMaxF a) {
   return a;
 }
 
-// noaux_tc selection over the logits (all consumer threads of one CTA).
+// noaux_tc selection over the E logits, by one warp ("LightLX", "How it
+// works": the noaux_tc sigmoid router; colibri summary, "Principales
+// fonctionnalites implementees": routed_scaling_factor).
 __device__ void run_select(const DecodeParams& p, Smem& S) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31;
   const int per = p.E / p.n_group;
-  for (int g = warp; g < p.n_group; g += kCW) {
-    ArgMaxF a{0.f, -1};
-    if (lane < per) {
-      const int e = g * per + lane;
-      const float s = 1.0f / (1.0f + expf(-__ldcg(p.logits + e)));
-      const float sp = s + __ldg(p.bias + e);
-      S.sc[e] = s;
-      S.sp[e] = sp;
-      a = ArgMaxF{sp, e};
-    }
-    const ArgMaxF t1 = am_warp(a);
-    ArgMaxF b = a;
-    if (b.i == t1.i) b.i = -1;
-    const ArgMaxF t2 = am_warp(b);
-    if (lane == 0) S.gscore[g] = (t2.i >= 0) ? t1.v + t2.v : t1.v;
+  for (int e = lane; e < p.E; e += 32) {
+    const float s = 1.0f / (1.0f + expf(-__ldcg(p.logits + e)));
+    S.sc[e] = s;
+    S.sp[e] = s + __ldg(p.bias + e);
   }
-  named_bar(1, kCT);
-  if (warp != 0) return;
-  bool kept = false;
-  {
-    const ArgMaxF g{lane < p.n_group ? S.gscore[lane] : 0.f, lane < p.n_group ? lane : -1};
-    for (int r = 0; r < p.topk_group; ++r) {
-      const ArgMaxF best = am_warp(kept ? ArgMaxF{0.f, -1} : g);
-      if (best.i == lane) kept = true;
+  __syncwarp();
+  // group score: sum of the two largest bias-corrected scores (lane = group)
+  float gs = 0.f;
+  if (lane < p.n_group) {
+    float b1 = 0.f, b2 = 0.f;
+    int i1 = -1, i2 = -1;
+    for (int e = lane * per; e < (lane + 1) * per; ++e) {
+      const float v = S.sp[e];
+      if (i1 < 0 || v > b1) {
+        b2 = b1;
+        i2 = i1;
+        b1 = v;
+        i1 = e;
+      } else if (i2 < 0 || v > b2) {
+        b2 = v;
+        i2 = e;
+      }
     }
+    gs = (i2 >= 0) ? b1 + b2 : b1;
   }
-  const unsigned kept_mask = __ballot_sync(0xffffffffu, kept);
+  // keep topk_group groups: rank by (score desc, index asc)
+  int rank = 0;
+  for (int h = 0; h < p.n_group; ++h) {
+    const float o = __shfl_sync(0xffffffffu, gs, h);
+    if (lane < p.n_group && (o > gs || (o == gs && h < lane))) ++rank;
+  }
+  const unsigned kept_mask = __ballot_sync(0xffffffffu, lane < p.n_group && rank < p.topk_group);
+  // top_k of sp over kept experts; lane owns experts lane + 32 m
   const int nper = (p.E + 31) >> 5;
   unsigned taken = 0;
+  ArgMaxF local{0.f, -1};
+  for (int m = 0; m < nper; ++m) {
+    const int e = lane + 32 * m;
+    if (e < p.E && ((kept_mask >> (e / per)) & 1u)) local = am_merge(local, ArgMaxF{S.sp[e], e});
+  }
   int my_sel = -1;
   for (int r = 0; r < p.k; ++r) {
-    ArgMaxF a{0.f, -1};
-    for (int m = 0; m < nper; ++m) {
-      const int e = lane + 32 * m;
-      if (e < p.E && ((kept_mask >> (e / per)) & 1u) && !((taken >> m) & 1u))
-        a = am_merge(a, ArgMaxF{S.sp[e], e});
-    }
-    const ArgMaxF best = am_warp(a);
-    if (best.i >= 0 && (best.i & 31) == lane) taken |= 1u << (best.i >> 5);
+    const ArgMaxF best = am_warp(local);
     if (lane == r) my_sel = best.i;
+    if (best.i >= 0 && (best.i & 31) == lane) {
+      taken |= 1u << (best.i >> 5);
+      local = ArgMaxF{0.f, -1};
+      for (int m = 0; m < nper; ++m) {
+        const int e = lane + 32 * m;
+        if (e < p.E && ((kept_mask >> (e / per)) & 1u) && !((taken >> m) & 1u))
+          local = am_merge(local, ArgMaxF{S.sp[e], e});
+      }
+    }
   }
-  int rank = 0;
+  int pos = 0;
   for (int j = 0; j < p.k; ++j) {
     const int other = __shfl_sync(0xffffffffu, my_sel, j);
-    if (lane < p.k && other < my_sel) ++rank;
+    if (lane < p.k && other < my_sel) ++pos;
   }
   const float s_mine = (lane < p.k && my_sel >= 0) ? S.sc[my_sel] : 0.f;
-  const float denom = [&] {
-    float v = s_mine;
+  float denom = s_mine;
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-  }() + 1e-20f;
+  for (int o = 16; o >= 1; o >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, o);
+  denom += 1e-20f;
   if (lane < p.k) {
     const float wv = p.rsf * s_mine / denom;
-    p.idx_ws[rank] = my_sel;
-    p.w_ws[rank] = wv;
-    if (p.idx_out) p.idx_out[rank] = my_sel;
-    if (p.w_out) p.w_out[rank] = wv;
+    p.idx_ws[pos] = my_sel;
+    p.w_ws[pos] = wv;
+    if (p.idx_out) p.idx_out[pos] = my_sel;
+    if (p.w_out) p.w_out[pos] = wv;
   }
-  __threadfence();
   __syncwarp();
   if (lane == 0) st_release(p.ctrl + kCtrlSelReady, 1u);
 }
 
-// Index of the lane holding reduce-scatter value `vi` for row-phase `ph`.
+// Convert h of one slot (fp32 [I], complete) to int16 groups, by one warp.
+__device__ void quantize_slot(const DecodeParams& p, int slot) {
+  const int lane = threadIdx.x & 31;
+  const int ngroups = p.I >> 5;
+  const float* h = p.hbuf + (size_t)slot * p.I;
+  for (int gi = lane; gi < ngroups; gi += 32) {
+    float v[32];
+    const float4* hp = reinterpret_cast<const float4*>(h + gi * 32);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 t = __ldcg(hp + i);
+      v[4 * i] = t.x;
+      v[4 * i + 1] = t.y;
+      v[4 * i + 2] = t.z;
+      v[4 * i + 3] = t.w;
+    }
+    XQ q;
+    xq_from_floats(v, q);
+    uint4* dst = reinterpret_cast<uint4*>(p.hq + ((size_t)slot * ngroups + gi) * 16);
+    dst[0] = make_uint4(q.ev[0], q.ev[1], q.ev[2], q.ev[3]);
+    dst[1] = make_uint4(q.ev[4], q.ev[5], q.ev[6], q.ev[7]);
+    dst[2] = make_uint4(q.od[0], q.od[1], q.od[2], q.od[3]);
+    dst[3] = make_uint4(q.od[4], q.od[5], q.od[6], q.od[7]);
+    p.hq_f[(size_t)slot * ngroups + gi] = q.f;
+  }
+  __syncwarp();
+  if (lane == 0) st_release(p.ctrl + kCtrlHqReady + slot, 1u);
+}
+
+// Lane holding reduce-scatter value `vi` of row phase `ph` (group-local warp).
 template <int NV, int SEG>
 __device__ __forceinline__ void owner_of(int ph, int vi, int wpr, int& warp0, int& lane) {
   if (SEG == 32) {
@@ -227,6 +273,27 @@ __device__ __forceinline__ void owner_of(int ph, int vi, int wpr, int& warp0, in
     warp0 = ph / rpw;
     lane = (ph % rpw) * SEG + vi * (SEG / NV);
   }
+}
+
+__device__ __forceinline__ ColMap group_col_map(int Gc, int gw, int lane) {
+  ColMap m;
+  if (Gc >= 32) {
+    m.wpr = Gc >> 5;
+    m.P = kGW / m.wpr;
+    m.col = (gw % m.wpr) * 32 + lane;
+    m.phase = gw / m.wpr;
+    m.seg = 32;
+    m.wir = gw % m.wpr;
+  } else {
+    const int rpw = 32 / Gc;
+    m.wpr = 1;
+    m.P = kGW * rpw;
+    m.col = lane % Gc;
+    m.phase = gw * rpw + lane / Gc;
+    m.seg = Gc;
+    m.wir = 0;
+  }
+  return m;
 }
 
 template <int SEG_G, int SEG_D>
@@ -243,51 +310,58 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&S.full[s], 1);
-      mbar_init(&S.empty[s], kCW);
+      mbar_init(&S.empty[s], kGW);
     }
+    S.abort_flag[0] = S.abort_flag[1] = 0;
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == kCW) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t policy = l2_policy_evict_first();
       bool sel_seen = false;
-      uint32_t filled = 0;    // bit s: stage s has been filled at least once
-      uint32_t last_par = 0;  // bit s: parity of the latest fill of stage s
-      int stage = 0;
+      int dones = 0;
       int t = (int)atomicAdd(p.ctrl + kCtrlTicket, 1u);
-      bool stop = false;
-      while (!stop) {
-        ItemDesc d = decode_ticket(p, t);
-        if (d.type != kDone && d.type != kRouter) {
-          if (d.slot < p.k) {
-            if (!sel_seen) {
-              if (!wait_counter(p.ctrl, p.ctrl + kCtrlSelReady, 1u)) {
-                set_error(p.ctrl, kErrTimeout);
-                d = make_item(kDone, 0, 0, 0);
-              } else {
-                sel_seen = true;
+      for (uint32_t n = 0;; ++n) {
+        const int stage = (int)(n % kStages);
+        ItemDesc d = make_item(kDone, 0, 0, 0);
+        if (dones == 0) {
+          d = decode_ticket(p, t);
+          if (d.type == kGateUp || d.type == kDown) {
+            if (d.slot < p.k) {
+              if (!sel_seen) {
+                if (wait_counter(p.ctrl, p.ctrl + kCtrlSelReady, 1u)) {
+                  sel_seen = true;
+                } else {
+                  set_error(p.ctrl, kErrTimeout);
+                  d = make_item(kDone, 0, 0, 0);
+                }
               }
-            }
-            if (d.type != kDone) {
-              d.eid = __ldcg(p.idx_ws + d.slot);
-              if (d.eid < 0 || d.eid >= p.E) {
-                set_error(p.ctrl, kErrBadExpertId);
-                d = make_item(kDone, 0, 0, 0);
+              if (d.type != kDone) {
+                d.eid = __ldcg(p.idx_ws + d.slot);
+                if (d.eid < 0 || d.eid >= p.E) {
+                  set_error(p.ctrl, kErrBadExpertId);
+                  d = make_item(kDone, 0, 0, 0);
+                }
               }
+            } else {
+              d.eid = p.E;  // shared expert
             }
-          } else {
-            d.eid = p.E;  // shared expert
           }
         }
         // wait until the consumers released this stage's previous contents
-        if (filled & (1u << stage)) {
+        if (n >= (uint32_t)kStages) {
           const uint64_t deadline = global_timer_ns() + kWaitNs;
-          if (!mbar_wait(&S.empty[stage], (last_par >> stage) & 1u, deadline)) {
+          if (!mbar_wait(&S.empty[stage], ((n / kStages) - 1) & 1u, deadline)) {
             set_error(p.ctrl, kErrTimeout);
-            break;  // consumers time out on their own full-barrier waits
+            // stop issuing; wait (bounded) for the fills already issued
+            for (uint32_t m = n - kStages; m < n; ++m) {
+              const uint64_t dl = global_timer_ns() + kWaitNs;
+              mbar_wait(&S.full[m % kStages], (m / kStages) & 1u, dl);
+            }
+            break;
           }
         }
         S.desc[stage] = d;
@@ -314,31 +388,34 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           bulk_g2s(dst + p.RD * (p.I / 2), ep.s_down + (size_t)d.row0 * (p.I / 32), sb,
                    &S.full[stage], policy);
         } else {
-          mbar_arrive(&S.full[stage]);
-          stop = true;
+          mbar_arrive(&S.full[stage]);  // a DONE fill: one per consumer group
+          if (++dones == kGroups) {
+            // leave no bulk copy in flight
+            for (uint32_t m = (n >= (uint32_t)kStages ? n - kStages + 1 : 0); m < n; ++m) {
+              const uint64_t dl = global_timer_ns() + kWaitNs;
+              mbar_wait(&S.full[m % kStages], (m / kStages) & 1u, dl);
+            }
+            break;
+          }
+          continue;
         }
-        // this fill's parity: 0 for the first fill, then alternating
-        last_par = (filled & (1u << stage)) ? (last_par ^ (1u << stage)) : (last_par & ~(1u << stage));
-        filled |= 1u << stage;
-        stage = (stage + 1 == kStages) ? 0 : stage + 1;
-        if (!stop) t = (int)atomicAdd(p.ctrl + kCtrlTicket, 1u);
-      }
-      // leave no bulk copy in flight: wait (bounded) for every issued fill
-      for (int s = 0; s < kStages; ++s) {
-        if (filled & (1u << s)) {
-          const uint64_t deadline = global_timer_ns() + kWaitNs;
-          mbar_wait(&S.full[s], (last_par >> s) & 1u, deadline);
-        }
+        t = (int)atomicAdd(p.ctrl + kCtrlTicket, 1u);
       }
     }
   } else {
     // ------------------------------------------------------------ consumers
+    const int grp = warp / kGW;
+    const int gw = warp % kGW;                 // warp index inside the group
+    const int tg = gw * 32 + lane;             // thread index inside the group
+    const int bar_id = 1 + grp;
     const int G = p.H >> 5, GD = p.I >> 5;
-    const ColMap cg = col_map_n(G, kCW);
-    const ColMap cd = col_map_n(GD, kCW);
-    const int tid = threadIdx.x;
+    const ColMap cg = group_col_map(G, gw, lane);
+    const ColMap cd = group_col_map(GD, gw, lane);
+    const int fw_g = (cg.P * NR_G + 31) / 32;  // finalizer warps of a gate/up item
+    const int fw_d = (cd.P * NR_D + 31) / 32;  // finalizer warps of a down item
 
-    XGroup xg;
+    // this thread's gate/up inputs (int16 groups) and router inputs (bf16)
+    XQ xq;
     {
       float xf[32];
       const uint4* xp = reinterpret_cast<const uint4*>(p.x + cg.col * 32);
@@ -352,43 +429,50 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           xf[8 * i + 2 * j + 1] = bf16_bits_to_f32(u[j] >> 16);
         }
       }
-      xgroup_from_floats(xf, xg);
+      xq_from_floats(xf, xq);
     }
-    float4 xr[kRouterChunks];
+    uint2 xr[kRouterChunks];
     const int rchunks = p.H >> 2;
 #pragma unroll
     for (int i = 0; i < kRouterChunks; ++i) {
-      const int c = tid + kCT * i;
-      if (c < rchunks) {
-        const uint2 v = __ldg(reinterpret_cast<const uint2*>(p.x) + c);
-        xr[i] = make_float4(bf16_bits_to_f32(v.x & 0xFFFFu), bf16_bits_to_f32(v.x >> 16),
-                            bf16_bits_to_f32(v.y & 0xFFFFu), bf16_bits_to_f32(v.y >> 16));
-      } else {
-        xr[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+      const int c = tg + kGT * i;
+      xr[i] = (c < rchunks) ? __ldg(reinterpret_cast<const uint2*>(p.x) + c) : make_uint2(0, 0);
     }
 
-    int stage = 0;
-    uint32_t cons_par = 0;  // bit s: parity of the next consumption of stage s
-    for (;;) {
-      const uint32_t par = (cons_par >> stage) & 1u;
-      if (tid == 0) {
-        const uint64_t deadline = global_timer_ns() + kWaitNs;
-        int go = mbar_wait(&S.full[stage], par, deadline) ? 1 : 0;
-        if (!go) set_error(p.ctrl, kErrTimeout);
-        if (go && S.desc[stage].type == kDown) {
-          if (!wait_counter(p.ctrl, p.ctrl + kCtrlGuDone + S.desc[stage].slot, (uint32_t)p.nG)) {
-            set_error(p.ctrl, kErrTimeout);
-            go = 0;
-          }
-        }
-        S.status = go;
+    int& gabort = S.abort_flag[grp];
+    for (uint32_t c = 0;; ++c) {
+      const uint32_t n = 2 * c + grp;  // fill number consumed
+      const int stage = (int)(n % kStages);
+      const uint32_t par = (n / kStages) & 1u;
+      const int rbuf = c & 1;
+      // Every path through this loop body passes the group barrier exactly
+      // once, and wait results are uniform per warp, so a wait that runs out
+      // in one warp can never leave a barrier or a shuffle half-joined.
+      int okw = 0;
+      if (lane == 0) okw = mbar_wait(&S.full[stage], par, global_timer_ns() + kWaitNs) ? 1 : 0;
+      bool ok = __shfl_sync(0xffffffffu, okw, 0) != 0;
+      if (ok) {
+        mbar_test(&S.full[stage], par);  // acquire the bulk-copied bytes in every lane
+      } else {
+        if (lane == 0) set_error(p.ctrl, kErrTimeout);
+        gabort = 1;
       }
-      named_bar(1, kCT);
-      if (!S.status) break;
-      mbar_test(&S.full[stage], par);  // acquire the bulk-copied bytes
       const ItemDesc d = S.desc[stage];
-      if (d.type == kDone) break;
+      if (!ok || d.type == kDone) {
+        named_bar(bar_id, kGT);
+        break;
+      }
+      if (d.type == kDown) {
+        int dep = 1;
+        if (lane == 0) dep = wait_counter(p.ctrl, p.ctrl + kCtrlHqReady + d.slot, 1u) ? 1 : 0;
+        dep = __shfl_sync(0xffffffffu, dep, 0);
+        __syncwarp();  // order the other lanes' reads of h after lane 0's acquire
+        if (!dep) {
+          if (lane == 0) set_error(p.ctrl, kErrTimeout);
+          gabort = 1;
+          ok = false;
+        }
+      }
       const uint8_t* st = stages + (size_t)stage * kStageBytes;
 
       if (d.type == kRouter) {
@@ -396,17 +480,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
 #pragma unroll
         for (int r = 0; r < kMaxRR; ++r) {
           acc[r] = 0.f;
-          if (r < d.nrows) {
+          if (ok && r < d.nrows) {
             const float4* wr = reinterpret_cast<const float4*>(st + (size_t)r * p.H * 4);
 #pragma unroll
             for (int i = 0; i < kRouterChunks; ++i) {
-              const int c = tid + kCT * i;
-              if (c < rchunks) {
-                const float4 wv = wr[c];
-                acc[r] = fmaf(wv.x, xr[i].x, acc[r]);
-                acc[r] = fmaf(wv.y, xr[i].y, acc[r]);
-                acc[r] = fmaf(wv.z, xr[i].z, acc[r]);
-                acc[r] = fmaf(wv.w, xr[i].w, acc[r]);
+              const int cc = tg + kGT * i;
+              if (cc < rchunks) {
+                const float4 wv = wr[cc];
+                acc[r] = fmaf(wv.x, bf16_bits_to_f32(xr[i].x & 0xFFFFu), acc[r]);
+                acc[r] = fmaf(wv.y, bf16_bits_to_f32(xr[i].x >> 16), acc[r]);
+                acc[r] = fmaf(wv.z, bf16_bits_to_f32(xr[i].y & 0xFFFFu), acc[r]);
+                acc[r] = fmaf(wv.w, bf16_bits_to_f32(xr[i].y >> 16), acc[r]);
               }
             }
           }
@@ -417,23 +501,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         for (int r = 0; r < kMaxRR; ++r) {
           if (r < d.nrows) {
             const float v = warp_sum(acc[r]);
-            if (lane == 0) S.red[warp][r] = v;
+            if (lane == 0) S.red[grp][rbuf][gw][r] = v;
           }
         }
-        named_bar(1, kCT);
-        if (tid < d.nrows) {
-          float v = 0.f;
-          for (int w = 0; w < kCW; ++w) v += S.red[w][tid];
-          p.logits[d.row0 + tid] = v;
-          __threadfence();
+        named_bar(bar_id, kGT);
+        if (gabort) break;
+        if (gw == 0) {
+          if (lane < d.nrows) {
+            float v = 0.f;
+            for (int w = 0; w < kGW; ++w) v += S.red[grp][rbuf][w][lane];
+            p.logits[d.row0 + lane] = v;
+          }
+          __syncwarp();
+          uint32_t last = 0;
+          if (lane == 0) last = (atom_add_acq_rel(p.ctrl + kCtrlRouterDone, 1u) + 1 == (uint32_t)p.nR);
+          last = __shfl_sync(0xffffffffu, last, 0);
+          if (last) {
+            __syncwarp();
+            run_select(p, S);
+          }
         }
-        named_bar(1, kCT);
-        if (tid == 0) {
-          const uint32_t old = atom_add_acq_rel(p.ctrl + kCtrlRouterDone, 1u);
-          S.flag = (old + 1 == (uint32_t)p.nR) ? 1 : 0;
-        }
-        named_bar(1, kCT);
-        if (S.flag) run_select(p, S);
       } else if (d.type == kGateUp) {
         float v[NV_G];
         const size_t rb = (size_t)p.H / 2;
@@ -445,11 +532,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         for (int r = 0; r < NR_G; ++r) {
           const int lr = cg.phase * NR_G + r;
           float pg = 0.f, pu = 0.f;
-          if (lr < d.nrows) {
+          if (ok && lr < d.nrows) {
             const uint4 wg = *reinterpret_cast<const uint4*>(qg + lr * rb + cg.col * 16);
             const uint4 wu = *reinterpret_cast<const uint4*>(qu + lr * rb + cg.col * 16);
-            pg = f16_bits_to_f32(sg[lr * G + cg.col]) * dot_group(wg, xg);
-            pu = f16_bits_to_f32(su[lr * G + cg.col]) * dot_group(wu, xg);
+            pg = dot_scaled(wg, xq, f16_bits_to_f32(sg[lr * G + cg.col]));
+            pu = dot_scaled(wu, xq, f16_bits_to_f32(su[lr * G + cg.col]));
           }
           v[r] = pg;
           v[NR_G + r] = pu;
@@ -457,41 +544,48 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.empty[stage]);
         reduce_scatter<NV_G, SEG_G>(v);
-        S.red[warp][lane] = v[0];
-        named_bar(1, kCT);
-        if (tid < cg.P * NR_G) {
-          const int ph = tid / NR_G, i = tid % NR_G;
-          const int lr = ph * NR_G + i;
-          if (lr < d.nrows) {
-            int w0, lg, lu;
-            owner_of<NV_G, SEG_G>(ph, i, cg.wpr, w0, lg);
-            owner_of<NV_G, SEG_G>(ph, i + NR_G, cg.wpr, w0, lu);
-            float g = 0.f, u = 0.f;
-            for (int w = 0; w < cg.wpr; ++w) {
-              g += S.red[w0 + w][lg];
-              u += S.red[w0 + w][lu];
+        S.red[grp][rbuf][gw][lane] = v[0];
+        named_bar(bar_id, kGT);
+        if (gabort) break;
+        if (gw < fw_g) {
+          if (tg < cg.P * NR_G) {
+            const int ph = tg / NR_G, i = tg % NR_G;
+            const int lr = ph * NR_G + i;
+            if (lr < d.nrows) {
+              int w0, lg, lu;
+              owner_of<NV_G, SEG_G>(ph, i, cg.wpr, w0, lg);
+              owner_of<NV_G, SEG_G>(ph, i + NR_G, cg.wpr, w0, lu);
+              float g = 0.f, u = 0.f;
+              for (int w = 0; w < cg.wpr; ++w) {
+                g += S.red[grp][rbuf][w0 + w][lg];
+                u += S.red[grp][rbuf][w0 + w][lu];
+              }
+              p.hbuf[(size_t)d.slot * p.I + d.row0 + lr] = silu_mul(g, u);
             }
-            p.hbuf[(size_t)d.slot * p.I + d.row0 + lr] = silu_mul(g, u);
-            __threadfence();
+          }
+          __syncwarp();
+          uint32_t last = 0;
+          if (lane == 0)
+            last = (atom_add_acq_rel(p.ctrl + kCtrlGuDone + d.slot, 1u) + 1 ==
+                    (uint32_t)(p.nG * fw_g));
+          last = __shfl_sync(0xffffffffu, last, 0);
+          if (last) {
+            __syncwarp();
+            quantize_slot(p, d.slot);
           }
         }
-        named_bar(1, kCT);
-        if (tid == 0) atom_add_acq_rel(p.ctrl + kCtrlGuDone + d.slot, 1u);
       } else {  // kDown
-        XGroup hg;
+        XQ hq;
         {
-          float hf[32];
-          const float4* hp =
-              reinterpret_cast<const float4*>(p.hbuf + (size_t)d.slot * p.I + cd.col * 32);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float4 t4 = __ldcg(hp + i);
-            hf[4 * i] = t4.x;
-            hf[4 * i + 1] = t4.y;
-            hf[4 * i + 2] = t4.z;
-            hf[4 * i + 3] = t4.w;
-          }
-          xgroup_from_floats(hf, hg);
+          const size_t gi = (size_t)d.slot * GD + cd.col;
+          const uint4* src = reinterpret_cast<const uint4*>(p.hq + gi * 16);
+          const uint4 a0 = __ldcg(src), a1 = __ldcg(src + 1), a2 = __ldcg(src + 2),
+                      a3 = __ldcg(src + 3);
+          hq.ev[0] = a0.x; hq.ev[1] = a0.y; hq.ev[2] = a0.z; hq.ev[3] = a0.w;
+          hq.ev[4] = a1.x; hq.ev[5] = a1.y; hq.ev[6] = a1.z; hq.ev[7] = a1.w;
+          hq.od[0] = a2.x; hq.od[1] = a2.y; hq.od[2] = a2.z; hq.od[3] = a2.w;
+          hq.od[4] = a3.x; hq.od[5] = a3.y; hq.od[6] = a3.z; hq.od[7] = a3.w;
+          hq.f = __ldcg(p.hq_f + gi);
         }
         float v[NR_D];
         const size_t rb = (size_t)p.I / 2;
@@ -500,49 +594,50 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         for (int r = 0; r < NR_D; ++r) {
           const int lr = cd.phase * NR_D + r;
           v[r] = 0.f;
-          if (lr < d.nrows) {
+          if (ok && lr < d.nrows) {
             const uint4 wd = *reinterpret_cast<const uint4*>(st + lr * rb + cd.col * 16);
-            v[r] = f16_bits_to_f32(sd[lr * GD + cd.col]) * dot_group(wd, hg);
+            v[r] = dot_scaled(wd, hq, f16_bits_to_f32(sd[lr * GD + cd.col]));
           }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.empty[stage]);
         reduce_scatter<NR_D, SEG_D>(v);
-        S.red[warp][lane] = v[0];
-        named_bar(1, kCT);
-        if (tid < cd.P * NR_D) {
-          const int ph = tid / NR_D, i = tid % NR_D;
-          const int lr = ph * NR_D + i;
-          if (lr < d.nrows) {
-            int w0, l0;
-            owner_of<NR_D, SEG_D>(ph, i, cd.wpr, w0, l0);
-            float s = 0.f;
-            for (int w = 0; w < cd.wpr; ++w) s += S.red[w0 + w][l0];
-            p.ypart[(size_t)d.slot * p.H + d.row0 + lr] = s;
-            __threadfence();
+        S.red[grp][rbuf][gw][lane] = v[0];
+        named_bar(bar_id, kGT);
+        if (gabort) break;
+        if (gw < fw_d) {
+          if (tg < cd.P * NR_D) {
+            const int ph = tg / NR_D, i = tg % NR_D;
+            const int lr = ph * NR_D + i;
+            if (lr < d.nrows) {
+              int w0, l0;
+              owner_of<NR_D, SEG_D>(ph, i, cd.wpr, w0, l0);
+              float s = 0.f;
+              for (int w = 0; w < cd.wpr; ++w) s += S.red[grp][rbuf][w0 + w][l0];
+              p.ypart[(size_t)d.slot * p.H + d.row0 + lr] = s;
+            }
           }
-        }
-        named_bar(1, kCT);
-        if (tid == 0) {
+          __syncwarp();
           const int rblk = d.row0 / p.RD;
-          const uint32_t old = atom_add_acq_rel(p.ctrl + kCtrlRbDone + rblk, 1u);
-          S.flag = (old + 1 == (uint32_t)slots) ? 1 : 0;
-        }
-        named_bar(1, kCT);
-        if (S.flag) {
-          // last slot of this row block: fixed-order combine
-          for (int lr = tid; lr < d.nrows; lr += kCT) {
-            const int row = d.row0 + lr;
-            float acc = 0.f;
-            for (int j = 0; j < p.k; ++j)
-              acc = fmaf(__ldcg(p.w_ws + j), __ldcg(p.ypart + (size_t)j * p.H + row), acc);
-            if (p.has_shared) acc += __ldcg(p.ypart + (size_t)p.k * p.H + row);
-            p.y[row] = acc;
+          uint32_t last = 0;
+          if (lane == 0)
+            last = (atom_add_acq_rel(p.ctrl + kCtrlRbDone + rblk, 1u) + 1 ==
+                    (uint32_t)(slots * fw_d));
+          last = __shfl_sync(0xffffffffu, last, 0);
+          if (last) {
+            // last contribution to this row block: fixed-order combine
+            __syncwarp();
+            for (int lr = lane; lr < d.nrows; lr += 32) {
+              const int row = d.row0 + lr;
+              float acc = 0.f;
+              for (int j = 0; j < p.k; ++j)
+                acc = fmaf(__ldcg(p.w_ws + j), __ldcg(p.ypart + (size_t)j * p.H + row), acc);
+              if (p.has_shared) acc += __ldcg(p.ypart + (size_t)p.k * p.H + row);
+              p.y[row] = acc;
+            }
           }
         }
       }
-      cons_par ^= 1u << stage;
-      stage = (stage + 1 == kStages) ? 0 : stage + 1;
     }
   }
 
@@ -560,7 +655,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       c[kCtrlRouterDone] = 0;
       c[kCtrlSelReady] = 0;
       c[kCtrlAbort] = 0;
-      for (int j = 0; j < slots; ++j) c[kCtrlGuDone + j] = 0;
+      for (int j = 0; j < slots; ++j) {
+        c[kCtrlGuDone + j] = 0;
+        c[kCtrlHqReady + j] = 0;
+      }
       for (int b = 0; b < p.nD; ++b) c[kCtrlRbDone + b] = 0;
       c[kCtrlExit] = 0;
       __threadfence();
@@ -613,14 +711,14 @@ cudaError_t launch_g(const DecodeParams& p, int seg_d, cudaStream_t st) {
 
 int seg_of(int G) { return G >= 32 ? 32 : G; }
 
-// Rows per phase and concurrent phases of the column mapping with kCW warps.
+// Concurrent row phases of the column mapping over one group's warps.
 bool phases(int G, int& P) {
   if (G >= 32) {
     const int wpr = G / 32;
-    if (kCW % wpr) return false;
-    P = kCW / wpr;
+    if (kGW % wpr) return false;
+    P = kGW / wpr;
   } else {
-    P = kCW * (32 / G);
+    P = kGW * (32 / G);
   }
   return true;
 }
@@ -633,8 +731,8 @@ bool decode_plan(const moe_config& c, DecodeParams& p) {
   const int G = c.hidden / 32, GD = c.inter / 32;
   int PG, PD;
   if (!phases(G, PG) || !phases(GD, PD)) return false;
-  if (c.hidden / 4 > kRouterChunks * kCT) return false;
-  if (c.n_experts > 1024) return false;
+  if (c.hidden / 4 > kRouterChunks * kGT) return false;
+  if (c.n_experts > kMaxE) return false;
   const int sg = seg_of(G), sd = seg_of(GD);
   const int nrg = (sg / 2 < 8) ? sg / 2 : 8;
   const int nrd = (sd < 16) ? sd : 16;
@@ -658,7 +756,7 @@ bool decode_plan(const moe_config& c, DecodeParams& p) {
   p.nG = (p.I + p.RG - 1) / p.RG;
   p.nD = (p.H + p.RD - 1) / p.RD;
   if (kCtrlRbDone + p.nD > (int)(kCtrlBytes / 4)) return false;
-  if (p.k + p.has_shared > kCtrlRbDone - kCtrlGuDone) return false;
+  if (p.k + p.has_shared > kCtrlHqReady - kCtrlGuDone) return false;
   p.n_items = p.nR + (p.k + p.has_shared) * (p.nG + p.nD);
   return true;
 }

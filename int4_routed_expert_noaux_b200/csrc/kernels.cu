@@ -160,14 +160,14 @@ __global__ void __launch_bounds__(1024) select_kernel(
 // ---------------------------------------------------------------------------
 // Fused int4 gate/up + SiLU (one expert slot, a block of rows).  Column-
 // stationary: thread (col, phase) owns 16-byte chunk column `col` of every
-// row it visits, so its 32 inputs stay in registers as an XGroup.  Each
+// row it visits, so its 32 inputs stay in registers as an XQ.  Each
 // phase handles NR rows of gate and NR of up; one butterfly reduce-scatter
 // sums the 2*NR partial dots over the row's threads (with NV == SEG, lane l
 // of a segment ends with value index l % SEG: gate row r at r, up row r at
 // NR + r).  h = silu(g) * u is written to hbuf; g and u never leave the CTA.
 // grid.x = row blocks of `inter`, grid.y = token * slots + slot.
 
-__device__ __forceinline__ void load_x_group_bf16(const uint16_t* __restrict__ xp, XGroup& xg) {
+__device__ __forceinline__ void load_x_group_bf16(const uint16_t* __restrict__ xp, XQ& xg) {
   float xf[32];
   const uint4* p4 = reinterpret_cast<const uint4*>(xp);
 #pragma unroll
@@ -180,10 +180,10 @@ __device__ __forceinline__ void load_x_group_bf16(const uint16_t* __restrict__ x
       xf[8 * i + 2 * j + 1] = bf16_bits_to_f32(u[j] >> 16);
     }
   }
-  xgroup_from_floats(xf, xg);
+  xq_from_floats(xf, xg);
 }
 
-__device__ __forceinline__ void load_x_group_f32(const float* __restrict__ hp, XGroup& xg) {
+__device__ __forceinline__ void load_x_group_f32(const float* __restrict__ hp, XQ& xg) {
   float xf[32];
   const float4* p4 = reinterpret_cast<const float4*>(hp);
 #pragma unroll
@@ -194,7 +194,7 @@ __device__ __forceinline__ void load_x_group_f32(const float* __restrict__ hp, X
     xf[4 * i + 2] = v.z;
     xf[4 * i + 3] = v.w;
   }
-  xgroup_from_floats(xf, xg);
+  xq_from_floats(xf, xg);
 }
 
 template <int SEG>
@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(256) gate_up_kernel(
     return;
   }
   const ExpertPtrs ep = table[eid];
-  XGroup xg;
+  XQ xg;
   load_x_group_bf16(x + (size_t)t * H + cm.col * 32, xg);
 
   const size_t row_bytes = (size_t)H / 2, row_sc = (size_t)G;
@@ -238,8 +238,8 @@ __global__ void __launch_bounds__(256) gate_up_kernel(
       const uint4 qu = __ldg(reinterpret_cast<const uint4*>(ep.q_up + row * row_bytes) + cm.col);
       const float sg = f16_bits_to_f32(__ldg(ep.s_gate + row * row_sc + cm.col));
       const float su = f16_bits_to_f32(__ldg(ep.s_up + row * row_sc + cm.col));
-      pg = sg * dot_group(qg, xg);
-      pu = su * dot_group(qu, xg);
+      pg = dot_scaled(qg, xg, sg);
+      pu = dot_scaled(qu, xg, su);
     }
     v[r] = pg;
     v[NR + r] = pu;
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(256) down_combine_kernel(
       }
     }
     const ExpertPtrs ep = table[eid];
-    XGroup hg;
+    XQ hg;
     load_x_group_f32(hbuf + ((size_t)t * slots + slot) * I + cm.col * 32, hg);
 #pragma unroll
     for (int r = 0; r < NV; ++r) {
@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(256) down_combine_kernel(
       if (row < H) {
         const uint4 q = __ldg(reinterpret_cast<const uint4*>(ep.q_down + row * row_bytes) + cm.col);
         const float sc = f16_bits_to_f32(__ldg(ep.s_down + row * row_sc + cm.col));
-        acc[r] = fmaf(wj * sc, dot_group(q, hg), acc[r]);
+        acc[r] = fmaf(wj, dot_scaled(q, hg, sc), acc[r]);
       }
     }
   }
@@ -348,7 +348,7 @@ __global__ void __launch_bounds__(256) gemv_int4_kernel(
   const int G = cols >> 5;
   const ColMap cm = col_map(G);
   const int row0 = blockIdx.x * cm.P * NV;
-  XGroup xg;
+  XQ xg;
   load_x_group_f32(x + cm.col * 32, xg);
   float acc[NV];
 #pragma unroll
@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(256) gemv_int4_kernel(
     if (row < rows) {
       const uint4 w = __ldg(reinterpret_cast<const uint4*>(q + (size_t)row * (cols / 2)) + cm.col);
       const float sc = f16_bits_to_f32(__ldg(s + (size_t)row * G + cm.col));
-      acc[r] = sc * dot_group(w, xg);
+      acc[r] = dot_scaled(w, xg, sc);
     }
   }
   reduce_scatter<NV, SEG>(acc);
