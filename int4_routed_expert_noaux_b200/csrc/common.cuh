@@ -86,15 +86,16 @@ __device__ __forceinline__ uint32_t lop3_sel_xor(uint32_t a, uint32_t c1, uint32
 // integers.
 //
 // The group's 32 inputs x_k are held as int16 X_k = round(x_k * 2^e) with
-// one power-of-two exponent e per group, chosen so that max |X_k| <= 2^14
-// (exact for every input within 2^6 of the group's largest; otherwise the
-// representation error is below 2^-14 of the group's largest input).
+// one power-of-two exponent e per group, chosen so that the largest input
+// maps into [2^14, 2^15) (clamped to 32767): exact for every bf16 input
+// within 2^7 of the group's largest; otherwise the representation error is
+// at most 2^-15 of the group's largest input.
 // A packed word w holds codes q_{8i..8i+7} (nibble j = element 8i + j,
 // two's complement).  The bytes of (w & 0xF0F0F0F0), read as signed int8,
 // are exactly 16 * q of the odd elements; those of ((w << 4) & 0xF0F0F0F0)
 // are 16 * q of the even elements.  dp2a multiplies two int16 by two int8
 // and accumulates in int32, so four dp2a per word give 16 * sum q_k X_k with
-// no rounding (|sum| < 2^27 and a multiple of 16: the int32 -> fp32
+// no rounding (|sum| < 2^28 and a multiple of 16: the int32 -> fp32
 // conversion is exact too).  sum_k q_k x_k = that * 2^-e / 16.
 //
 // XQ holds the int16 pairs in dp2a order: for word i,
@@ -118,12 +119,12 @@ __device__ __forceinline__ void xq_from_floats(const float* x, XQ& g) {
   for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(x[i]));
   int ex = 0;
   if (m > 0.f) frexpf(m, &ex);  // m = fr * 2^ex, fr in [0.5, 1)
-  const int e = 14 - ex;        // m * 2^e < 2^14
+  const int e = 15 - ex;        // m * 2^e in [2^14, 2^15)
   const float sc = (m > 0.f) ? ldexpf(1.0f, e) : 0.f;
   g.f = (m > 0.f) ? ldexpf(1.0f, -e - 4) : 0.f;
   int X[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) X[i] = __float2int_rn(x[i] * sc);
+  for (int i = 0; i < 32; ++i) X[i] = max(-32767, min(32767, __float2int_rn(x[i] * sc)));
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     g.ev[2 * i] = pack_i16x2(X[8 * i + 0], X[8 * i + 2]);

@@ -62,6 +62,7 @@ struct ItemDesc {
 struct Smem {
   uint64_t full[kStages];
   uint64_t empty[kStages];
+  uint64_t gbar[kGroups];  // per-group item barrier (one arrival per warp)
   ItemDesc desc[kStages];
   float red[kGroups][2][kGW][32];
   int abort_flag[kGroups];
@@ -107,8 +108,16 @@ __device__ ItemDesc decode_ticket(const DecodeParams& p, int t) {
   return make_item(kDone, 0, 0, 0);
 }
 
-__device__ __forceinline__ void set_error(uint32_t* ctrl, uint32_t code) {
-  atomicCAS(ctrl + kCtrlErr, 0u, code);
+// Record an error: the first one also records where it happened (CTA,
+// warp, site, fill) in the control words kCtrlWhere..kCtrlWhere+3.
+__device__ __forceinline__ void set_error(uint32_t* ctrl, uint32_t code, uint32_t site = 0,
+                                          uint32_t fill = 0) {
+  if (atomicCAS(ctrl + kCtrlErr, 0u, code) == 0u) {
+    ctrl[kCtrlWhere + 0] = blockIdx.x;
+    ctrl[kCtrlWhere + 1] = threadIdx.x >> 5;
+    ctrl[kCtrlWhere + 2] = site;
+    ctrl[kCtrlWhere + 3] = fill;
+  }
   atomicExch(ctrl + kCtrlAbort, 1u);
 }
 
@@ -275,6 +284,24 @@ __device__ __forceinline__ void owner_of(int ph, int vi, int wpr, int& warp0, in
   }
 }
 
+// Bounded barrier of one consumer group: every warp arrives once, then waits
+// for phase `par`.  Returns false (in every lane of the warp) if the wait ran
+// out; the memory effects of the other warps before their arrival are
+// visible afterwards.
+__device__ __forceinline__ bool group_barrier(uint64_t* bar, uint32_t par) {
+  const int lane = threadIdx.x & 31;
+  __syncwarp();
+  int ok = 1;
+  if (lane == 0) {
+    mbar_arrive(bar);
+    ok = mbar_wait(bar, par, global_timer_ns() + kWaitNs) ? 1 : 0;
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) mbar_test(bar, par);
+  __syncwarp();
+  return ok != 0;
+}
+
 __device__ __forceinline__ ColMap group_col_map(int Gc, int gw, int lane) {
   ColMap m;
   if (Gc >= 32) {
@@ -312,6 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       mbar_init(&S.full[s], 1);
       mbar_init(&S.empty[s], kGW);
     }
+    for (int g = 0; g < kGroups; ++g) mbar_init(&S.gbar[g], kGW);
     S.abort_flag[0] = S.abort_flag[1] = 0;
     fence_mbar_init();
   }
@@ -335,14 +363,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
                 if (wait_counter(p.ctrl, p.ctrl + kCtrlSelReady, 1u)) {
                   sel_seen = true;
                 } else {
-                  set_error(p.ctrl, kErrTimeout);
+                  set_error(p.ctrl, kErrTimeout, 4, n);
                   d = make_item(kDone, 0, 0, 0);
                 }
               }
               if (d.type != kDone) {
                 d.eid = __ldcg(p.idx_ws + d.slot);
                 if (d.eid < 0 || d.eid >= p.E) {
-                  set_error(p.ctrl, kErrBadExpertId);
+                  set_error(p.ctrl, kErrBadExpertId, 5, n);
                   d = make_item(kDone, 0, 0, 0);
                 }
               }
@@ -355,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         if (n >= (uint32_t)kStages) {
           const uint64_t deadline = global_timer_ns() + kWaitNs;
           if (!mbar_wait(&S.empty[stage], ((n / kStages) - 1) & 1u, deadline)) {
-            set_error(p.ctrl, kErrTimeout);
+            set_error(p.ctrl, kErrTimeout, 6, n);
             // stop issuing; wait (bounded) for the fills already issued
             for (uint32_t m = n - kStages; m < n; ++m) {
               const uint64_t dl = global_timer_ns() + kWaitNs;
@@ -407,7 +435,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     const int grp = warp / kGW;
     const int gw = warp % kGW;                 // warp index inside the group
     const int tg = gw * 32 + lane;             // thread index inside the group
-    const int bar_id = 1 + grp;
     const int G = p.H >> 5, GD = p.I >> 5;
     const ColMap cg = group_col_map(G, gw, lane);
     const ColMap cd = group_col_map(GD, gw, lane);
@@ -445,6 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       const int stage = (int)(n % kStages);
       const uint32_t par = (n / kStages) & 1u;
       const int rbuf = c & 1;
+      const uint32_t gpar = c & 1u;  // one group barrier per iteration
       // Every path through this loop body passes the group barrier exactly
       // once, and wait results are uniform per warp, so a wait that runs out
       // in one warp can never leave a barrier or a shuffle half-joined.
@@ -454,12 +482,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       if (ok) {
         mbar_test(&S.full[stage], par);  // acquire the bulk-copied bytes in every lane
       } else {
-        if (lane == 0) set_error(p.ctrl, kErrTimeout);
+        if (lane == 0) set_error(p.ctrl, kErrTimeout, 1, n);
         gabort = 1;
       }
       const ItemDesc d = S.desc[stage];
       if (!ok || d.type == kDone) {
-        named_bar(bar_id, kGT);
+        group_barrier(&S.gbar[grp], gpar);
         break;
       }
       if (d.type == kDown) {
@@ -468,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         dep = __shfl_sync(0xffffffffu, dep, 0);
         __syncwarp();  // order the other lanes' reads of h after lane 0's acquire
         if (!dep) {
-          if (lane == 0) set_error(p.ctrl, kErrTimeout);
+          if (lane == 0) set_error(p.ctrl, kErrTimeout, 2, n);
           gabort = 1;
           ok = false;
         }
@@ -504,7 +532,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
             if (lane == 0) S.red[grp][rbuf][gw][r] = v;
           }
         }
-        named_bar(bar_id, kGT);
+        if (!group_barrier(&S.gbar[grp], gpar)) {
+          if (lane == 0) set_error(p.ctrl, kErrTimeout, 3, n);
+          gabort = 1;
+        }
         if (gabort) break;
         if (gw == 0) {
           if (lane < d.nrows) {
@@ -545,7 +576,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         if (lane == 0) mbar_arrive(&S.empty[stage]);
         reduce_scatter<NV_G, SEG_G>(v);
         S.red[grp][rbuf][gw][lane] = v[0];
-        named_bar(bar_id, kGT);
+        if (!group_barrier(&S.gbar[grp], gpar)) {
+          if (lane == 0) set_error(p.ctrl, kErrTimeout, 3, n);
+          gabort = 1;
+        }
         if (gabort) break;
         if (gw < fw_g) {
           if (tg < cg.P * NR_G) {
@@ -603,7 +637,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         if (lane == 0) mbar_arrive(&S.empty[stage]);
         reduce_scatter<NR_D, SEG_D>(v);
         S.red[grp][rbuf][gw][lane] = v[0];
-        named_bar(bar_id, kGT);
+        if (!group_barrier(&S.gbar[grp], gpar)) {
+          if (lane == 0) set_error(p.ctrl, kErrTimeout, 3, n);
+          gabort = 1;
+        }
         if (gabort) break;
         if (gw < fw_d) {
           if (tg < cd.P * NR_D) {

@@ -21,6 +21,7 @@ enum : int {
   kCtrlSelReady = 3,
   kCtrlExit = 4,
   kCtrlAbort = 5,
+  kCtrlWhere = 8,     // [4] where the first error happened (CTA, warp, site, fill)
   kCtrlGuDone = 16,   // [slots] finished gate/up finalizer warps
   kCtrlHqReady = 48,  // [slots] int16 h of the slot published
   kCtrlRbDone = 96,   // [row blocks of hidden] finished down finalizer warps
