@@ -15,18 +15,23 @@
 //    int16 fixed point with one exponent per group; the int4 group dot
 //    product is exact in integers (dp2a); one butterfly reduce-scatter plus
 //    a cross-warp sum finishes each row; one named barrier per item;
-//  * item order: router rows, shared-expert gate/up, shared-expert down,
-//    routed gate/up of slot 0, then (gate/up of slot j, down of slot j-1)
-//    for j = 1..k-1, then down of slot k-1.  Every dependency points to an
-//    earlier ticket, so in-order claiming always makes progress;
-//  * the warp that finishes the last router item runs the selection and
-//    publishes idx / w with a release flag; the producer acquires it before
-//    loading routed weights;
-//  * the warp that finishes the last gate/up item of a slot converts that
-//    slot's h to int16 groups once and flags it ready for the down items;
-//  * down items write per-slot partial rows; the warp that completes the
-//    last slot of a row block sums the partials in slot order
-//    (deterministic, no atomics on data) into y;
+//  * each CTA first computes its own block of router rows (a static
+//    split of the experts over the grid, the CTA's first fill); the CTA
+//    that finishes the last block runs the selection and publishes idx / w
+//    with a release flag; the producer acquires it before loading routed
+//    weights;
+//  * then work items come from a global ticket counter in the order:
+//    shared-expert gate/up, shared-expert down, routed gate/up of slots
+//    0..k-1, routed down of slots 0..k-1.  Every dependency points to an
+//    earlier ticket, so in-order claiming always makes progress, and each
+//    slot's down items come at least k-1 slots of work after its gate/up;
+//  * gate/up finalizer warps publish h rows and count themselves done with
+//    a release reduction; a down item waits for its slot's count, then each
+//    thread converts its own 32-row group of h to int16;
+//  * down items write per-slot partial rows; the warp whose release add
+//    completes a row block (checked one item later, off the critical path)
+//    sums the partials in slot order (deterministic, no atomics on data)
+//    into y;
 //  * every wait is bounded (1 s); a wait that runs out sets the workspace
 //    error word and the kernel winds down; the last CTA to exit resets the
 //    control counters so the next call starts clean.
@@ -82,8 +87,6 @@ __device__ __forceinline__ ItemDesc make_item(int type, int slot, int row0, int 
 }
 
 __device__ ItemDesc decode_ticket(const DecodeParams& p, int t) {
-  if (t < p.nR) return make_item(kRouter, 0, t * p.RR, min(p.RR, p.E - t * p.RR));
-  t -= p.nR;
   auto gu = [&](int slot, int b) {
     return make_item(kGateUp, slot, b * p.RG, min(p.RG, p.I - b * p.RG));
   };
@@ -96,16 +99,16 @@ __device__ ItemDesc decode_ticket(const DecodeParams& p, int t) {
     if (t < p.nD) return dn(p.k, t);
     t -= p.nD;
   }
-  if (t < p.nG) return gu(0, t);
-  t -= p.nG;
-  const int pair = p.nG + p.nD;
-  if (t < (p.k - 1) * pair) {
-    const int j = t / pair + 1, u = t % pair;
-    return u < p.nG ? gu(j, u) : dn(j - 1, u - p.nG);
-  }
-  t -= (p.k - 1) * pair;
-  if (t < p.nD) return dn(p.k - 1, t);
+  if (t < p.k * p.nG) return gu(t / p.nG, t % p.nG);
+  t -= p.k * p.nG;
+  if (t < p.k * p.nD) return dn(t / p.nD, t % p.nD);
   return make_item(kDone, 0, 0, 0);
+}
+
+// Router rows of CTA b: a static split of the E experts over the grid.
+__device__ __forceinline__ void router_rows(const DecodeParams& p, int b, int& r0, int& nr) {
+  r0 = (int)(((long long)b * p.E) / gridDim.x);
+  nr = (int)(((long long)(b + 1) * p.E) / gridDim.x) - r0;
 }
 
 // Record an error: the first one also records where it happened (CTA,
@@ -242,33 +245,20 @@ __device__ void run_select(const DecodeParams& p, Smem& S) {
   if (lane == 0) st_release(p.ctrl + kCtrlSelReady, 1u);
 }
 
-// Convert h of one slot (fp32 [I], complete) to int16 groups, by one warp.
-__device__ void quantize_slot(const DecodeParams& p, int slot) {
+// Fixed-order combine of one row block of y from the per-slot partials, by
+// one warp, once every slot's down item of the block has published.
+__device__ void combine_block(const DecodeParams& p, int row0, int nrows) {
   const int lane = threadIdx.x & 31;
-  const int ngroups = p.I >> 5;
-  const float* h = p.hbuf + (size_t)slot * p.I;
-  for (int gi = lane; gi < ngroups; gi += 32) {
-    float v[32];
-    const float4* hp = reinterpret_cast<const float4*>(h + gi * 32);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 t = __ldcg(hp + i);
-      v[4 * i] = t.x;
-      v[4 * i + 1] = t.y;
-      v[4 * i + 2] = t.z;
-      v[4 * i + 3] = t.w;
-    }
-    XQ q;
-    xq_from_floats(v, q);
-    uint4* dst = reinterpret_cast<uint4*>(p.hq + ((size_t)slot * ngroups + gi) * 16);
-    dst[0] = make_uint4(q.ev[0], q.ev[1], q.ev[2], q.ev[3]);
-    dst[1] = make_uint4(q.ev[4], q.ev[5], q.ev[6], q.ev[7]);
-    dst[2] = make_uint4(q.od[0], q.od[1], q.od[2], q.od[3]);
-    dst[3] = make_uint4(q.od[4], q.od[5], q.od[6], q.od[7]);
-    p.hq_f[(size_t)slot * ngroups + gi] = q.f;
-  }
+  if (lane == 0) fence_acq_rel();  // see the other warps' partials
   __syncwarp();
-  if (lane == 0) st_release(p.ctrl + kCtrlHqReady + slot, 1u);
+  for (int lr = lane; lr < nrows; lr += 32) {
+    const int row = row0 + lr;
+    float acc = 0.f;
+    for (int j = 0; j < p.k; ++j)
+      acc = fmaf(__ldcg(p.w_ws + j), __ldcg(p.ypart + (size_t)j * p.H + row), acc);
+    if (p.has_shared) acc += __ldcg(p.ypart + (size_t)p.k * p.H + row);
+    p.y[row] = acc;
+  }
 }
 
 // Lane holding reduce-scatter value `vi` of row phase `ph` (group-local warp).
@@ -351,11 +341,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       const uint64_t policy = l2_policy_evict_first();
       bool sel_seen = false;
       int dones = 0;
-      int t = (int)atomicAdd(p.ctrl + kCtrlTicket, 1u);
+      int rr0, rnr;
+      router_rows(p, blockIdx.x, rr0, rnr);
+      bool router_pending = rnr > 0;
+      int t = router_pending ? -1 : (int)atomicAdd(p.ctrl + kCtrlTicket, 1u);
       for (uint32_t n = 0;; ++n) {
         const int stage = (int)(n % kStages);
         ItemDesc d = make_item(kDone, 0, 0, 0);
-        if (dones == 0) {
+        if (router_pending) {
+          d = make_item(kRouter, 0, rr0, rnr);
+          router_pending = false;
+        } else if (dones == 0) {
           d = decode_ticket(p, t);
           if (d.type == kGateUp || d.type == kDown) {
             if (d.slot < p.k) {
@@ -467,6 +463,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     }
 
     int& gabort = S.abort_flag[grp];
+    int pend_row0 = -1, pend_nrows = 0;  // this warp's last down row block
+    uint32_t pend_old = 0;               // count before this warp's add (lane 0)
     for (uint32_t c = 0;; ++c) {
       const uint32_t n = 2 * c + grp;  // fill number consumed
       const int stage = (int)(n % kStages);
@@ -492,7 +490,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       }
       if (d.type == kDown) {
         int dep = 1;
-        if (lane == 0) dep = wait_counter(p.ctrl, p.ctrl + kCtrlHqReady + d.slot, 1u) ? 1 : 0;
+        if (lane == 0)
+          dep = wait_counter(p.ctrl, p.ctrl + kCtrlGuDone + d.slot, (uint32_t)(p.nG * fw_g)) ? 1 : 0;
         dep = __shfl_sync(0xffffffffu, dep, 0);
         __syncwarp();  // order the other lanes' reads of h after lane 0's acquire
         if (!dep) {
@@ -537,6 +536,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           gabort = 1;
         }
         if (gabort) break;
+        if (pend_row0 >= 0) {
+          const uint32_t last =
+              __shfl_sync(0xffffffffu, pend_old + 1 == (uint32_t)(slots * fw_d), 0);
+          if (last) combine_block(p, pend_row0, pend_nrows);
+          pend_row0 = -1;
+        }
         if (gw == 0) {
           if (lane < d.nrows) {
             float v = 0.f;
@@ -545,7 +550,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           }
           __syncwarp();
           uint32_t last = 0;
-          if (lane == 0) last = (atom_add_acq_rel(p.ctrl + kCtrlRouterDone, 1u) + 1 == (uint32_t)p.nR);
+          if (lane == 0) {
+            last = (atom_add_release(p.ctrl + kCtrlRouterDone, 1u) + 1 == (uint32_t)p.nR);
+            if (last) fence_acq_rel();  // see every block's logits
+          }
           last = __shfl_sync(0xffffffffu, last, 0);
           if (last) {
             __syncwarp();
@@ -581,6 +589,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           gabort = 1;
         }
         if (gabort) break;
+        if (pend_row0 >= 0) {
+          const uint32_t last =
+              __shfl_sync(0xffffffffu, pend_old + 1 == (uint32_t)(slots * fw_d), 0);
+          if (last) combine_block(p, pend_row0, pend_nrows);
+          pend_row0 = -1;
+        }
         if (gw < fw_g) {
           if (tg < cg.P * NR_G) {
             const int ph = tg / NR_G, i = tg % NR_G;
@@ -598,28 +612,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
             }
           }
           __syncwarp();
-          uint32_t last = 0;
-          if (lane == 0)
-            last = (atom_add_acq_rel(p.ctrl + kCtrlGuDone + d.slot, 1u) + 1 ==
-                    (uint32_t)(p.nG * fw_g));
-          last = __shfl_sync(0xffffffffu, last, 0);
-          if (last) {
-            __syncwarp();
-            quantize_slot(p, d.slot);
-          }
+          if (lane == 0) red_add_release(p.ctrl + kCtrlGuDone + d.slot, 1u);
         }
       } else {  // kDown
         XQ hq;
         {
-          const size_t gi = (size_t)d.slot * GD + cd.col;
-          const uint4* src = reinterpret_cast<const uint4*>(p.hq + gi * 16);
-          const uint4 a0 = __ldcg(src), a1 = __ldcg(src + 1), a2 = __ldcg(src + 2),
-                      a3 = __ldcg(src + 3);
-          hq.ev[0] = a0.x; hq.ev[1] = a0.y; hq.ev[2] = a0.z; hq.ev[3] = a0.w;
-          hq.ev[4] = a1.x; hq.ev[5] = a1.y; hq.ev[6] = a1.z; hq.ev[7] = a1.w;
-          hq.od[0] = a2.x; hq.od[1] = a2.y; hq.od[2] = a2.z; hq.od[3] = a2.w;
-          hq.od[4] = a3.x; hq.od[5] = a3.y; hq.od[6] = a3.z; hq.od[7] = a3.w;
-          hq.f = __ldcg(p.hq_f + gi);
+          float hf[32];
+          const float4* hp =
+              reinterpret_cast<const float4*>(p.hbuf + (size_t)d.slot * p.I + cd.col * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 t4 = __ldcg(hp + i);
+            hf[4 * i] = t4.x;
+            hf[4 * i + 1] = t4.y;
+            hf[4 * i + 2] = t4.z;
+            hf[4 * i + 3] = t4.w;
+          }
+          xq_from_floats(hf, hq);
         }
         float v[NR_D];
         const size_t rb = (size_t)p.I / 2;
@@ -642,6 +651,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           gabort = 1;
         }
         if (gabort) break;
+        if (pend_row0 >= 0) {
+          const uint32_t last =
+              __shfl_sync(0xffffffffu, pend_old + 1 == (uint32_t)(slots * fw_d), 0);
+          if (last) combine_block(p, pend_row0, pend_nrows);
+          pend_row0 = -1;
+        }
         if (gw < fw_d) {
           if (tg < cd.P * NR_D) {
             const int ph = tg / NR_D, i = tg % NR_D;
@@ -655,26 +670,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
             }
           }
           __syncwarp();
-          const int rblk = d.row0 / p.RD;
-          uint32_t last = 0;
+          // count this warp done; the result is looked at one item later
           if (lane == 0)
-            last = (atom_add_acq_rel(p.ctrl + kCtrlRbDone + rblk, 1u) + 1 ==
-                    (uint32_t)(slots * fw_d));
-          last = __shfl_sync(0xffffffffu, last, 0);
-          if (last) {
-            // last contribution to this row block: fixed-order combine
-            __syncwarp();
-            for (int lr = lane; lr < d.nrows; lr += 32) {
-              const int row = d.row0 + lr;
-              float acc = 0.f;
-              for (int j = 0; j < p.k; ++j)
-                acc = fmaf(__ldcg(p.w_ws + j), __ldcg(p.ypart + (size_t)j * p.H + row), acc);
-              if (p.has_shared) acc += __ldcg(p.ypart + (size_t)p.k * p.H + row);
-              p.y[row] = acc;
-            }
-          }
+            pend_old = atom_add_release(p.ctrl + kCtrlRbDone + d.row0 / p.RD, 1u);
+          pend_row0 = d.row0;
+          pend_nrows = d.nrows;
         }
       }
+    }
+    // a row block completed by this warp's last down item
+    if (!gabort && pend_row0 >= 0) {
+      const uint32_t last = __shfl_sync(0xffffffffu, pend_old + 1 == (uint32_t)(slots * fw_d), 0);
+      if (last) combine_block(p, pend_row0, pend_nrows);
     }
   }
 
@@ -692,10 +699,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       c[kCtrlRouterDone] = 0;
       c[kCtrlSelReady] = 0;
       c[kCtrlAbort] = 0;
-      for (int j = 0; j < slots; ++j) {
-        c[kCtrlGuDone + j] = 0;
-        c[kCtrlHqReady + j] = 0;
-      }
+      for (int j = 0; j < slots; ++j) c[kCtrlGuDone + j] = 0;
       for (int b = 0; b < p.nD; ++b) c[kCtrlRbDone + b] = 0;
       c[kCtrlExit] = 0;
       __threadfence();
@@ -789,11 +793,13 @@ bool decode_plan(const moe_config& c, DecodeParams& p) {
   if ((size_t)p.RG * (c.hidden / 2 + c.hidden / 16) * 2 > kStageBytes) return false;
   if ((size_t)p.RD * (c.inter / 2 + c.inter / 16) > kStageBytes) return false;
   if ((p.RG * (c.hidden / 16)) % 16 || (p.RD * (c.inter / 16)) % 16) return false;
-  p.nR = (p.E + p.RR - 1) / p.RR;
+  const int grid = num_sms();
+  if ((p.E + grid - 1) / grid > p.RR) return false;  // a CTA's router rows fill one stage
+  p.nR = p.E < grid ? p.E : grid;  // CTAs with at least one router row
   p.nG = (p.I + p.RG - 1) / p.RG;
   p.nD = (p.H + p.RD - 1) / p.RD;
   if (kCtrlRbDone + p.nD > (int)(kCtrlBytes / 4)) return false;
-  if (p.k + p.has_shared > kCtrlHqReady - kCtrlGuDone) return false;
+  if (p.k + p.has_shared > kCtrlRbDone - kCtrlGuDone) return false;
   p.n_items = p.nR + (p.k + p.has_shared) * (p.nG + p.nD);
   return true;
 }

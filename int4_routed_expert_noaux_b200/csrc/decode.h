@@ -23,8 +23,7 @@ enum : int {
   kCtrlAbort = 5,
   kCtrlWhere = 8,     // [4] where the first error happened (CTA, warp, site, fill)
   kCtrlGuDone = 16,   // [slots] finished gate/up finalizer warps
-  kCtrlHqReady = 48,  // [slots] int16 h of the slot published
-  kCtrlRbDone = 96,   // [row blocks of hidden] finished down finalizer warps
+  kCtrlRbDone = 64,   // [row blocks of hidden] finished down finalizer warps
 };
 
 struct DecodeParams {
@@ -41,11 +40,9 @@ struct DecodeParams {
   float* w_ws;        // [k]
   float* hbuf;        // [slots][I]
   float* ypart;       // [slots][H]
-  uint32_t* hq;       // [slots][I/32][16] int16 pairs of h, dot-product order
-  float* hq_f;        // [slots][I/32] group factors of hq
   int H, I, E, k, n_group, topk_group, has_shared;
   float rsf;
-  int RR, RG, RD;     // rows per router / gate-up / down item
+  int RR, RG, RD;     // rows per router block / gate-up / down item
   int nR, nG, nD, n_items;
 };
 
