@@ -109,6 +109,8 @@ WsLayout ws_layout(const moe_config* c, int T) {
   off = align_up(off + (size_t)T * slots * c->inter * 4, 256);
   L.ypart = off;
   off = align_up(off + (size_t)T * slots * c->hidden * 4, 256);
+  L.hq = off;
+  off = align_up(off + (size_t)T * slots * (c->inter / 32) * 68, 256);
   L.total = off;
   return L;
 }

@@ -50,13 +50,30 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// One probe that may suspend the thread in hardware for up to `hint_ns`
+// (it wakes earlier when the phase completes), so waiting warps do not take
+// issue slots from working ones.
+__device__ __forceinline__ bool mbar_test_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; "
+      "selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for phase `parity`, giving up at `deadline` (globaltimer ns).
 // Returns false on timeout.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t deadline) {
   if (mbar_test(bar, parity)) return true;
+  uint32_t sleep_ns = 32;  // deschedule between probes: waiting warps take no issue slots
   for (uint32_t it = 0;; ++it) {
+    __nanosleep(sleep_ns);
     if (mbar_test(bar, parity)) return true;
-    if ((it & 63) == 63 && global_timer_ns() > deadline) return false;
+    if (sleep_ns < 256) sleep_ns <<= 1;
+    if ((it & 7) == 7 && global_timer_ns() > deadline) return false;
   }
 }
 
@@ -76,6 +93,19 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
+}
+
+// L2 policy: evict-last (small tables read by many CTAs).
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// Order this thread's view of generic-proxy global writes (acquired from
+// other threads) before its subsequent async-proxy (bulk copy) reads.
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {

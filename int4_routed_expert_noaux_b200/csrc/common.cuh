@@ -122,9 +122,14 @@ __device__ __forceinline__ void xq_from_floats(const float* x, XQ& g) {
   const int e = 15 - ex;        // m * 2^e in [2^14, 2^15)
   const float sc = (m > 0.f) ? ldexpf(1.0f, e) : 0.f;
   g.f = (m > 0.f) ? ldexpf(1.0f, -e - 4) : 0.f;
+  // round to nearest even with the 1.5 * 2^23 bias: |x * sc| < 2^15, so the
+  // biased float holds the rounded integer in its low mantissa bits
   int X[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) X[i] = max(-32767, min(32767, __float2int_rn(x[i] * sc)));
+  for (int i = 0; i < 32; ++i) {
+    const float b = fmaf(x[i], sc, 12582912.0f);
+    X[i] = max(-32767, min(32767, (int)(__float_as_uint(b) - 0x4B400000u)));
+  }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     g.ev[2 * i] = pack_i16x2(X[8 * i + 0], X[8 * i + 2]);
@@ -146,20 +151,21 @@ __device__ __forceinline__ int dp2a_hi(uint32_t a, uint32_t b, int c) {
   return d;
 }
 
-// 16 * sum_k q_k X_k over the 32 codes of one 16-byte chunk.
+// 16 * sum_k q_k X_k over the 32 codes of one 16-byte chunk (four
+// independent dp2a chains of four).
 __device__ __forceinline__ int dotq_group(const uint4 w, const XQ& g) {
   const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-  int ae = 0, ao = 0;
+  int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint32_t odd = ws[i] & 0xF0F0F0F0u;
     const uint32_t even = (ws[i] << 4) & 0xF0F0F0F0u;
-    ae = dp2a_lo(g.ev[2 * i], even, ae);
-    ae = dp2a_hi(g.ev[2 * i + 1], even, ae);
-    ao = dp2a_lo(g.od[2 * i], odd, ao);
-    ao = dp2a_hi(g.od[2 * i + 1], odd, ao);
+    a0 = dp2a_lo(g.ev[2 * i], even, a0);
+    a1 = dp2a_hi(g.ev[2 * i + 1], even, a1);
+    a2 = dp2a_lo(g.od[2 * i], odd, a2);
+    a3 = dp2a_hi(g.od[2 * i + 1], odd, a3);
   }
-  return ae + ao;
+  return (a0 + a1) + (a2 + a3);
 }
 
 // sum_k (q_k * scale) x_k for one chunk: exact group sum, one rounding.

@@ -25,9 +25,12 @@
 //    0..k-1, routed down of slots 0..k-1.  Every dependency points to an
 //    earlier ticket, so in-order claiming always makes progress, and each
 //    slot's down items come at least k-1 slots of work after its gate/up;
-//  * gate/up finalizer warps publish h rows and count themselves done with
-//    a release reduction; a down item waits for its slot's count, then each
-//    thread converts its own 32-row group of h to int16;
+//  * gate/up finalizer warps publish h rows and count themselves done; the
+//    warp that completes a slot (it looks before its next wait, never after,
+//    so no fill can depend on it) converts the slot's h to int16 groups once
+//    (a 4.3 KB table for the GLM shape) and flags it; the producer acquires
+//    the flag and bulk-copies the table into the tail of each down item's
+//    stage, so down consumers read their inputs from shared memory;
 //  * down items write per-slot partial rows; the warp whose release add
 //    completes a row block (checked one item later, off the critical path)
 //    sums the partials in slot order (deterministic, no atomics on data)
@@ -56,6 +59,7 @@ constexpr uint32_t kStageBytes = 55296;
 constexpr int kRouterChunks = 8;         // 16-byte W chunks per thread per row
 constexpr int kMaxRR = 8;                // router rows per item
 constexpr int kMaxE = 256;
+constexpr int kMaxSlots = 33;
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 enum ItemType : int { kRouter = 0, kGateUp = 1, kDown = 2, kDone = 3 };
@@ -132,10 +136,12 @@ __device__ __forceinline__ bool aborted(const uint32_t* ctrl) {
 __device__ bool wait_counter(uint32_t* ctrl, const uint32_t* p, uint32_t target) {
   if (ld_acquire(p) >= target) return true;
   const uint64_t deadline = global_timer_ns() + kWaitNs;
+  uint32_t sleep_ns = 64;  // back off so that polling warps leave issue slots free
   for (uint32_t it = 0;; ++it) {
+    __nanosleep(sleep_ns);
     if (ld_acquire(p) >= target) return true;
-    __nanosleep(32);
-    if ((it & 15) == 15) {
+    if (sleep_ns < 512) sleep_ns <<= 1;
+    if ((it & 7) == 7) {
       if (aborted(ctrl) || global_timer_ns() > deadline) return false;
     }
   }
@@ -164,16 +170,29 @@ __device__ __forceinline__ ArgMaxF am_warp(ArgMaxF a) {
   return a;
 }
 
-// noaux_tc selection over the E logits, by one warp ("LightLX", "How it
-// works": the noaux_tc sigmoid router; colibri summary, "Principales
-// fonctionnalites implementees": routed_scaling_factor).
-__device__ void run_select(const DecodeParams& p, Smem& S) {
+// Selection for shapes whose groups do not align with lanes: scores staged
+// in shared memory, one lane per group, repeated warp arg-max.
+__device__ __noinline__ void run_select_generic(const DecodeParams& p, Smem& S) {
   const int lane = threadIdx.x & 31;
   const int per = p.E / p.n_group;
-  for (int e = lane; e < p.E; e += 32) {
-    const float s = 1.0f / (1.0f + expf(-__ldcg(p.logits + e)));
-    S.sc[e] = s;
-    S.sp[e] = s + __ldg(p.bias + e);
+  {
+    // issue every load of this lane before using any (one L2 round trip)
+    float lg[kMaxE / 32], bs[kMaxE / 32];
+#pragma unroll
+    for (int m = 0; m < kMaxE / 32; ++m) {
+      const int e = lane + 32 * m;
+      lg[m] = (e < p.E) ? __ldcg(p.logits + e) : 0.f;
+      bs[m] = (e < p.E) ? __ldg(p.bias + e) : 0.f;
+    }
+#pragma unroll
+    for (int m = 0; m < kMaxE / 32; ++m) {
+      const int e = lane + 32 * m;
+      if (e < p.E) {
+        const float s = 1.0f / (1.0f + expf(-lg[m]));
+        S.sc[e] = s;
+        S.sp[e] = s + bs[m];
+      }
+    }
   }
   __syncwarp();
   // group score: sum of the two largest bias-corrected scores (lane = group)
@@ -245,9 +264,43 @@ __device__ void run_select(const DecodeParams& p, Smem& S) {
   if (lane == 0) st_release(p.ctrl + kCtrlSelReady, 1u);
 }
 
+// Convert h of one slot (fp32 [I], complete) to int16 groups, by one warp:
+// the table holds, per 32-row group, the 16 words of XQ.ev/od and then, after
+// all groups, one factor per group.  Flags the slot ready for the producers.
+__device__ __noinline__ void quantize_slot(const DecodeParams& p, int slot) {
+  const int lane = threadIdx.x & 31;
+  const int ngroups = p.I >> 5;
+  if (lane == 0) fence_acq_rel();  // see every gate/up warp's h rows
+  __syncwarp();
+  const float* h = p.hbuf + (size_t)slot * p.I;
+  uint8_t* table = reinterpret_cast<uint8_t*>(p.hq) + (size_t)slot * ngroups * 68;
+  for (int gi = lane; gi < ngroups; gi += 32) {
+    float v[32];
+    const float4* hp = reinterpret_cast<const float4*>(h + gi * 32);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 t = __ldcg(hp + i);
+      v[4 * i] = t.x;
+      v[4 * i + 1] = t.y;
+      v[4 * i + 2] = t.z;
+      v[4 * i + 3] = t.w;
+    }
+    XQ q;
+    xq_from_floats(v, q);
+    uint4* dst = reinterpret_cast<uint4*>(table + gi * 64);
+    dst[0] = make_uint4(q.ev[0], q.ev[1], q.ev[2], q.ev[3]);
+    dst[1] = make_uint4(q.ev[4], q.ev[5], q.ev[6], q.ev[7]);
+    dst[2] = make_uint4(q.od[0], q.od[1], q.od[2], q.od[3]);
+    dst[3] = make_uint4(q.od[4], q.od[5], q.od[6], q.od[7]);
+    reinterpret_cast<float*>(table + ngroups * 64)[gi] = q.f;
+  }
+  __syncwarp();
+  if (lane == 0) st_release(p.ctrl + kCtrlHqReady + slot, 1u);
+}
+
 // Fixed-order combine of one row block of y from the per-slot partials, by
 // one warp, once every slot's down item of the block has published.
-__device__ void combine_block(const DecodeParams& p, int row0, int nrows) {
+__device__ __noinline__ void combine_block(const DecodeParams& p, int row0, int nrows) {
   const int lane = threadIdx.x & 31;
   if (lane == 0) fence_acq_rel();  // see the other warps' partials
   __syncwarp();
@@ -259,6 +312,141 @@ __device__ void combine_block(const DecodeParams& p, int row0, int nrows) {
     if (p.has_shared) acc += __ldcg(p.ypart + (size_t)p.k * p.H + row);
     p.y[row] = acc;
   }
+}
+
+// Order-preserving map of a float onto uint32 (larger float, larger key;
+// every key is > 0).
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// noaux_tc selection over the E logits, by one warp ("LightLX", "How it
+// works": the noaux_tc sigmoid router; colibri summary, "Principales
+// fonctionnalites implementees": routed_scaling_factor).  Lane l owns the
+// q = ceil(E / 32) consecutive experts l*q .. l*q+q-1 in registers; when a
+// group's experts are exactly L = per / q consecutive lanes (L a power of
+// two), group top-2 is a segmented butterfly and the top-k is k rounds of
+// two warp reductions (max of the score key, then min of the expert id
+// among the lanes holding it: ties go to the lower id).
+__device__ __noinline__ void run_select(const DecodeParams& p, Smem& S) {
+  const int lane = threadIdx.x & 31;
+  const int E = p.E, per = E / p.n_group, q = (E + 31) >> 5;
+  const int L = per / q;
+  if (per % q != 0 || L < 1 || (L & (L - 1)) != 0) {
+    run_select_generic(p, S);
+    return;
+  }
+  constexpr int kQ = kMaxE / 32;
+  float sc[kQ], sp[kQ];
+  {
+    float lg[kQ], bs[kQ];
+#pragma unroll
+    for (int j = 0; j < kQ; ++j) {
+      const int e = lane * q + j;
+      const bool valid = j < q && e < E;
+      lg[j] = valid ? __ldcg(p.logits + e) : 0.f;
+      bs[j] = valid ? __ldg(p.bias + e) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < kQ; ++j) {
+      sc[j] = 1.0f / (1.0f + expf(-lg[j]));
+      sp[j] = sc[j] + bs[j];
+    }
+  }
+  const int nmine = max(0, min(q, E - lane * q));  // experts this lane owns
+  // group score: the two largest sp of the group (lanes g*L .. g*L+L-1)
+  float t1 = -INFINITY, t2 = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < kQ; ++j) {
+    if (j < nmine) {
+      const float v = sp[j];
+      if (v > t1) {
+        t2 = t1;
+        t1 = v;
+      } else if (v > t2) {
+        t2 = v;
+      }
+    }
+  }
+  for (int o = 1; o < L; o <<= 1) {
+    const float p1 = __shfl_xor_sync(0xffffffffu, t1, o);
+    const float p2 = __shfl_xor_sync(0xffffffffu, t2, o);
+    const float n1 = fmaxf(t1, p1);
+    const float n2 = fmaxf(fminf(t1, p1), fmaxf(t2, p2));
+    t1 = n1;
+    t2 = n2;
+  }
+  const float gs_seg = (per >= 2) ? t1 + t2 : t1;
+  // keep topk_group groups: rank by (score desc, index asc); lane g holds group g
+  const int G = p.n_group;
+  const float gs = __shfl_sync(0xffffffffu, gs_seg, (lane < G ? lane : 0) * L);
+  int rank = 0;
+  for (int h = 0; h < G; ++h) {
+    const float o = __shfl_sync(0xffffffffu, gs, h);
+    if (o > gs || (o == gs && h < lane)) ++rank;
+  }
+  const unsigned kept_mask = __ballot_sync(0xffffffffu, lane < G && rank < p.topk_group);
+  const bool kept = (kept_mask >> (lane / L)) & 1u;
+  // top_k over the kept experts
+  uint32_t taken = 0;
+  uint32_t bk = 0;
+  int bj = 0;
+  auto local_best = [&]() {
+    bk = 0;
+    bj = 0;
+#pragma unroll
+    for (int j = 0; j < kQ; ++j) {
+      if (j < nmine && kept && !((taken >> j) & 1u)) {
+        const uint32_t key = order_key(sp[j]);
+        if (key > bk) {
+          bk = key;
+          bj = j;
+        }
+      }
+    }
+  };
+  local_best();
+  int my_sel = -1;
+  float my_s = 0.f;
+  for (int r = 0; r < p.k; ++r) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    const uint32_t cand = (bk == m && m != 0) ? (uint32_t)(lane * q + bj) : 0xFFFFFFFFu;
+    const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+    const int owner = (int)(win / (uint32_t)q);
+    float s_win = 0.f;
+#pragma unroll
+    for (int j = 0; j < kQ; ++j)
+      if (j == bj) s_win = sc[j];
+    s_win = __shfl_sync(0xffffffffu, s_win, owner);
+    if (lane == r) {
+      my_sel = (int)win;
+      my_s = s_win;
+    }
+    if (lane == owner) {
+      taken |= 1u << bj;
+      local_best();
+    }
+  }
+  // ascending ids; weights from the unbiased scores
+  int pos = 0;
+  for (int j = 0; j < p.k; ++j) {
+    const int other = __shfl_sync(0xffffffffu, my_sel, j);
+    if (lane < p.k && other < my_sel) ++pos;
+  }
+  float denom = (lane < p.k) ? my_s : 0.f;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, o);
+  denom += 1e-20f;
+  if (lane < p.k) {
+    const float wv = p.rsf * my_s / denom;
+    p.idx_ws[pos] = my_sel;
+    p.w_ws[pos] = wv;
+    if (p.idx_out) p.idx_out[pos] = my_sel;
+    if (p.w_out) p.w_out[pos] = wv;
+  }
+  __syncwarp();
+  if (lane == 0) st_release(p.ctrl + kCtrlSelReady, 1u);
 }
 
 // Lane holding reduce-scatter value `vi` of row phase `ph` (group-local warp).
@@ -340,6 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     if (lane == 0) {
       const uint64_t policy = l2_policy_evict_first();
       bool sel_seen = false;
+      uint64_t hq_seen = 0;  // bit j: slot j's int16 h table acquired
       int dones = 0;
       int rr0, rnr;
       router_rows(p, blockIdx.x, rr0, rnr);
@@ -353,6 +542,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           router_pending = false;
         } else if (dones == 0) {
           d = decode_ticket(p, t);
+          if (d.type == kDown) {
+            // the slot's int16 h table must be published before it is copied
+            if (!((hq_seen >> d.slot) & 1ull)) {
+              if (wait_counter(p.ctrl, p.ctrl + kCtrlHqReady + d.slot, 1u)) {
+                hq_seen |= 1ull << d.slot;
+                fence_proxy_async();  // order the table's stores before the bulk read
+              } else {
+                set_error(p.ctrl, kErrTimeout, 7, n);
+                d = make_item(kDone, 0, 0, 0);
+              }
+            }
+          }
           if (d.type == kGateUp || d.type == kDown) {
             if (d.slot < p.k) {
               if (!sel_seen) {
@@ -407,10 +608,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         } else if (d.type == kDown) {
           const ExpertPtrs ep = p.table[d.eid];
           const uint32_t qb = (uint32_t)d.nrows * (p.I / 2), sb = (uint32_t)d.nrows * (p.I / 16);
-          mbar_arrive_expect_tx(&S.full[stage], qb + sb);
+          const uint32_t hb = (uint32_t)(p.I / 32) * 68;
+          mbar_arrive_expect_tx(&S.full[stage], qb + sb + hb);
           bulk_g2s(dst, ep.q_down + (size_t)d.row0 * (p.I / 2), qb, &S.full[stage], policy);
           bulk_g2s(dst + p.RD * (p.I / 2), ep.s_down + (size_t)d.row0 * (p.I / 32), sb,
                    &S.full[stage], policy);
+          bulk_g2s(dst + p.RD * (p.I / 2) + p.RD * (p.I / 16),
+                   reinterpret_cast<const uint8_t*>(p.hq) + (size_t)d.slot * hb, hb,
+                   &S.full[stage], l2_policy_evict_last());
         } else {
           mbar_arrive(&S.full[stage]);  // a DONE fill: one per consumer group
           if (++dones == kGroups) {
@@ -454,55 +659,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       }
       xq_from_floats(xf, xq);
     }
-    uint2 xr[kRouterChunks];
-    const int rchunks = p.H >> 2;
-#pragma unroll
-    for (int i = 0; i < kRouterChunks; ++i) {
-      const int c = tg + kGT * i;
-      xr[i] = (c < rchunks) ? __ldg(reinterpret_cast<const uint2*>(p.x) + c) : make_uint2(0, 0);
-    }
-
     int& gabort = S.abort_flag[grp];
     int pend_row0 = -1, pend_nrows = 0;  // this warp's last down row block
+    int pend_gu = -1;                    // slot of this warp's last gate/up item
+    uint32_t pend_gu_old = 0;            // gate/up count before this warp's add
     uint32_t pend_old = 0;               // count before this warp's add (lane 0)
-    for (uint32_t c = 0;; ++c) {
-      const uint32_t n = 2 * c + grp;  // fill number consumed
-      const int stage = (int)(n % kStages);
-      const uint32_t par = (n / kStages) & 1u;
-      const int rbuf = c & 1;
-      const uint32_t gpar = c & 1u;  // one group barrier per iteration
-      // Every path through this loop body passes the group barrier exactly
-      // once, and wait results are uniform per warp, so a wait that runs out
-      // in one warp can never leave a barrier or a shuffle half-joined.
-      int okw = 0;
-      if (lane == 0) okw = mbar_wait(&S.full[stage], par, global_timer_ns() + kWaitNs) ? 1 : 0;
-      bool ok = __shfl_sync(0xffffffffu, okw, 0) != 0;
-      if (ok) {
-        mbar_test(&S.full[stage], par);  // acquire the bulk-copied bytes in every lane
-      } else {
-        if (lane == 0) set_error(p.ctrl, kErrTimeout, 1, n);
-        gabort = 1;
-      }
-      const ItemDesc d = S.desc[stage];
-      if (!ok || d.type == kDone) {
-        group_barrier(&S.gbar[grp], gpar);
-        break;
-      }
-      if (d.type == kDown) {
-        int dep = 1;
-        if (lane == 0)
-          dep = wait_counter(p.ctrl, p.ctrl + kCtrlGuDone + d.slot, (uint32_t)(p.nG * fw_g)) ? 1 : 0;
-        dep = __shfl_sync(0xffffffffu, dep, 0);
-        __syncwarp();  // order the other lanes' reads of h after lane 0's acquire
-        if (!dep) {
-          if (lane == 0) set_error(p.ctrl, kErrTimeout, 2, n);
-          gabort = 1;
-          ok = false;
+    // Group 0 of a CTA with router rows: fill 0 is the router block.  It is
+    // handled before the main loop so its bf16 inputs are dead afterwards.
+    uint32_t c_first = 0;
+    {
+      int rr0, rnr;
+      router_rows(p, blockIdx.x, rr0, rnr);
+      if (grp == 0 && rnr > 0) {
+        c_first = 1;
+        uint2 xr[kRouterChunks];
+        const int rchunks = p.H >> 2;
+#pragma unroll
+        for (int i = 0; i < kRouterChunks; ++i) {
+          const int cc = tg + kGT * i;
+          xr[i] = (cc < rchunks) ? __ldg(reinterpret_cast<const uint2*>(p.x) + cc) : make_uint2(0, 0);
         }
-      }
-      const uint8_t* st = stages + (size_t)stage * kStageBytes;
-
-      if (d.type == kRouter) {
+        const int stage = 0, rbuf = 0;
+        const uint32_t gpar = 0u;
+        int okw = 0;
+        if (lane == 0) okw = mbar_wait(&S.full[0], 0u, global_timer_ns() + kWaitNs) ? 1 : 0;
+        const bool ok = __shfl_sync(0xffffffffu, okw, 0) != 0;
+        if (ok) {
+          mbar_test(&S.full[0], 0u);
+        } else {
+          if (lane == 0) set_error(p.ctrl, kErrTimeout, 1, 0);
+          gabort = 1;
+        }
+        const ItemDesc d = S.desc[0];
+        const uint8_t* st = stages;
         float acc[kMaxRR];
 #pragma unroll
         for (int r = 0; r < kMaxRR; ++r) {
@@ -532,17 +721,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           }
         }
         if (!group_barrier(&S.gbar[grp], gpar)) {
-          if (lane == 0) set_error(p.ctrl, kErrTimeout, 3, n);
+          if (lane == 0) set_error(p.ctrl, kErrTimeout, 3, 0);
           gabort = 1;
         }
-        if (gabort) break;
-        if (pend_row0 >= 0) {
-          const uint32_t last =
-              __shfl_sync(0xffffffffu, pend_old + 1 == (uint32_t)(slots * fw_d), 0);
-          if (last) combine_block(p, pend_row0, pend_nrows);
-          pend_row0 = -1;
-        }
-        if (gw == 0) {
+        if (!gabort && gw == 0) {
           if (lane < d.nrows) {
             float v = 0.f;
             for (int w = 0; w < kGW; ++w) v += S.red[grp][rbuf][w][lane];
@@ -560,25 +742,59 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
             run_select(p, S);
           }
         }
-      } else if (d.type == kGateUp) {
+      }
+    }
+    for (uint32_t c = c_first;; ++c) {
+      if (gabort) break;
+      // A slot completed by this warp's previous gate/up item is converted
+      // before waiting for the next fill: the producer may hold that fill
+      // back until the conversion is published.
+      if (pend_gu >= 0) {
+        const uint32_t last =
+            __shfl_sync(0xffffffffu, pend_gu_old + 1 == (uint32_t)(p.nG * fw_g), 0);
+        if (last) quantize_slot(p, pend_gu);
+        pend_gu = -1;
+      }
+      const uint32_t n = 2 * c + grp;  // fill number consumed
+      const int stage = (int)(n % kStages);
+      const uint32_t par = (n / kStages) & 1u;
+      const int rbuf = c & 1;
+      const uint32_t gpar = c & 1u;  // one group barrier per iteration
+      // Every path through this loop body passes the group barrier exactly
+      // once, and wait results are uniform per warp, so a wait that runs out
+      // in one warp can never leave a barrier or a shuffle half-joined.
+      int okw = 0;
+      if (lane == 0) okw = mbar_wait(&S.full[stage], par, global_timer_ns() + kWaitNs) ? 1 : 0;
+      bool ok = __shfl_sync(0xffffffffu, okw, 0) != 0;
+      if (ok) {
+        mbar_test(&S.full[stage], par);  // acquire the bulk-copied bytes in every lane
+      } else {
+        if (lane == 0) set_error(p.ctrl, kErrTimeout, 1, n);
+        gabort = 1;
+      }
+      const ItemDesc d = S.desc[stage];
+      if (!ok || d.type == kDone) {
+        group_barrier(&S.gbar[grp], gpar);
+        break;
+      }
+      const uint8_t* st = stages + (size_t)stage * kStageBytes;
+
+      if (d.type == kGateUp) {
         float v[NV_G];
         const size_t rb = (size_t)p.H / 2;
         const uint8_t* qg = st;
         const uint8_t* qu = st + (size_t)p.RG * rb;
         const uint16_t* sg = reinterpret_cast<const uint16_t*>(st + 2 * (size_t)p.RG * rb);
         const uint16_t* su = sg + (size_t)p.RG * G;
+        // Rows past nrows (a partial last item) are computed from whatever
+        // the stage holds and dropped at the finalize: no branch in the loop.
 #pragma unroll
         for (int r = 0; r < NR_G; ++r) {
           const int lr = cg.phase * NR_G + r;
-          float pg = 0.f, pu = 0.f;
-          if (ok && lr < d.nrows) {
-            const uint4 wg = *reinterpret_cast<const uint4*>(qg + lr * rb + cg.col * 16);
-            const uint4 wu = *reinterpret_cast<const uint4*>(qu + lr * rb + cg.col * 16);
-            pg = dot_scaled(wg, xq, f16_bits_to_f32(sg[lr * G + cg.col]));
-            pu = dot_scaled(wu, xq, f16_bits_to_f32(su[lr * G + cg.col]));
-          }
-          v[r] = pg;
-          v[NR_G + r] = pu;
+          const uint4 wg = *reinterpret_cast<const uint4*>(qg + lr * rb + cg.col * 16);
+          const uint4 wu = *reinterpret_cast<const uint4*>(qu + lr * rb + cg.col * 16);
+          v[r] = dot_scaled(wg, xq, f16_bits_to_f32(sg[lr * G + cg.col]));
+          v[NR_G + r] = dot_scaled(wu, xq, f16_bits_to_f32(su[lr * G + cg.col]));
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.empty[stage]);
@@ -595,6 +811,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           if (last) combine_block(p, pend_row0, pend_nrows);
           pend_row0 = -1;
         }
+
         if (gw < fw_g) {
           if (tg < cg.P * NR_G) {
             const int ph = tg / NR_G, i = tg % NR_G;
@@ -612,23 +829,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
             }
           }
           __syncwarp();
-          if (lane == 0) red_add_release(p.ctrl + kCtrlGuDone + d.slot, 1u);
+          // count this warp done; the result is looked at before the next wait
+          if (lane == 0) pend_gu_old = atom_add_release(p.ctrl + kCtrlGuDone + d.slot, 1u);
+          pend_gu = d.slot;
         }
       } else {  // kDown
         XQ hq;
         {
-          float hf[32];
-          const float4* hp =
-              reinterpret_cast<const float4*>(p.hbuf + (size_t)d.slot * p.I + cd.col * 32);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float4 t4 = __ldcg(hp + i);
-            hf[4 * i] = t4.x;
-            hf[4 * i + 1] = t4.y;
-            hf[4 * i + 2] = t4.z;
-            hf[4 * i + 3] = t4.w;
-          }
-          xq_from_floats(hf, hq);
+          const uint8_t* tab = st + (size_t)p.RD * (p.I / 2) + (size_t)p.RD * (p.I / 16);
+          const uint4* src = reinterpret_cast<const uint4*>(tab + cd.col * 64);
+          const uint4 a0 = src[0], a1 = src[1], a2 = src[2], a3 = src[3];
+          hq.ev[0] = a0.x; hq.ev[1] = a0.y; hq.ev[2] = a0.z; hq.ev[3] = a0.w;
+          hq.ev[4] = a1.x; hq.ev[5] = a1.y; hq.ev[6] = a1.z; hq.ev[7] = a1.w;
+          hq.od[0] = a2.x; hq.od[1] = a2.y; hq.od[2] = a2.z; hq.od[3] = a2.w;
+          hq.od[4] = a3.x; hq.od[5] = a3.y; hq.od[6] = a3.z; hq.od[7] = a3.w;
+          hq.f = reinterpret_cast<const float*>(tab + GD * 64)[cd.col];
         }
         float v[NR_D];
         const size_t rb = (size_t)p.I / 2;
@@ -636,11 +851,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
 #pragma unroll
         for (int r = 0; r < NR_D; ++r) {
           const int lr = cd.phase * NR_D + r;
-          v[r] = 0.f;
-          if (ok && lr < d.nrows) {
-            const uint4 wd = *reinterpret_cast<const uint4*>(st + lr * rb + cd.col * 16);
-            v[r] = dot_scaled(wd, hq, f16_bits_to_f32(sd[lr * GD + cd.col]));
-          }
+          const uint4 wd = *reinterpret_cast<const uint4*>(st + lr * rb + cd.col * 16);
+          v[r] = dot_scaled(wd, hq, f16_bits_to_f32(sd[lr * GD + cd.col]));
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.empty[stage]);
@@ -657,6 +869,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           if (last) combine_block(p, pend_row0, pend_nrows);
           pend_row0 = -1;
         }
+
         if (gw < fw_d) {
           if (tg < cd.P * NR_D) {
             const int ph = tg / NR_D, i = tg % NR_D;
@@ -678,7 +891,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         }
       }
     }
-    // a row block completed by this warp's last down item
+    // a slot or row block completed by this warp's last items
+    if (!gabort && pend_gu >= 0) {
+      const uint32_t last =
+          __shfl_sync(0xffffffffu, pend_gu_old + 1 == (uint32_t)(p.nG * fw_g), 0);
+      if (last) quantize_slot(p, pend_gu);
+    }
     if (!gabort && pend_row0 >= 0) {
       const uint32_t last = __shfl_sync(0xffffffffu, pend_old + 1 == (uint32_t)(slots * fw_d), 0);
       if (last) combine_block(p, pend_row0, pend_nrows);
@@ -699,7 +917,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       c[kCtrlRouterDone] = 0;
       c[kCtrlSelReady] = 0;
       c[kCtrlAbort] = 0;
-      for (int j = 0; j < slots; ++j) c[kCtrlGuDone + j] = 0;
+      for (int j = 0; j < slots; ++j) {
+        c[kCtrlGuDone + j] = 0;
+        c[kCtrlHqReady + j] = 0;
+      }
       for (int b = 0; b < p.nD; ++b) c[kCtrlRbDone + b] = 0;
       c[kCtrlExit] = 0;
       __threadfence();
@@ -787,11 +1008,18 @@ bool decode_plan(const moe_config& c, DecodeParams& p) {
   p.rsf = c.routed_scaling_factor;
   p.RG = PG * nrg;
   p.RD = PD * nrd;
+  {
+    // a down item also carries the slot's int16 h table (68 bytes per group)
+    const size_t hb = (size_t)GD * 68, rowb = (size_t)c.inter / 2 + c.inter / 16;
+    const int fit = (int)((kStageBytes - hb) / rowb);
+    if (fit < p.RD) p.RD = fit & ~3;
+    if (p.RD < 4 || hb % 16) return false;
+  }
   p.RR = (int)(kStageBytes / ((uint32_t)c.hidden * 4));
   if (p.RR > kMaxRR) p.RR = kMaxRR;
   if (p.RR < 1) return false;
   if ((size_t)p.RG * (c.hidden / 2 + c.hidden / 16) * 2 > kStageBytes) return false;
-  if ((size_t)p.RD * (c.inter / 2 + c.inter / 16) > kStageBytes) return false;
+  if ((size_t)p.RD * (c.inter / 2 + c.inter / 16) + (size_t)GD * 68 > kStageBytes) return false;
   if ((p.RG * (c.hidden / 16)) % 16 || (p.RD * (c.inter / 16)) % 16) return false;
   const int grid = num_sms();
   if ((p.E + grid - 1) / grid > p.RR) return false;  // a CTA's router rows fill one stage
@@ -799,7 +1027,8 @@ bool decode_plan(const moe_config& c, DecodeParams& p) {
   p.nG = (p.I + p.RG - 1) / p.RG;
   p.nD = (p.H + p.RD - 1) / p.RD;
   if (kCtrlRbDone + p.nD > (int)(kCtrlBytes / 4)) return false;
-  if (p.k + p.has_shared > kCtrlRbDone - kCtrlGuDone) return false;
+  if (p.k + p.has_shared > kMaxSlots || p.k + p.has_shared > kCtrlHqReady - kCtrlGuDone)
+    return false;
   p.n_items = p.nR + (p.k + p.has_shared) * (p.nG + p.nD);
   return true;
 }

@@ -23,7 +23,8 @@ enum : int {
   kCtrlAbort = 5,
   kCtrlWhere = 8,     // [4] where the first error happened (CTA, warp, site, fill)
   kCtrlGuDone = 16,   // [slots] finished gate/up finalizer warps
-  kCtrlRbDone = 64,   // [row blocks of hidden] finished down finalizer warps
+  kCtrlHqReady = 56,  // [slots] the slot's int16 h table is published
+  kCtrlRbDone = 96,   // [row blocks of hidden] finished down finalizer warps
 };
 
 struct DecodeParams {
@@ -40,6 +41,7 @@ struct DecodeParams {
   float* w_ws;        // [k]
   float* hbuf;        // [slots][I]
   float* ypart;       // [slots][H]
+  uint32_t* hq;       // [slots][I/32 * 68 bytes]: int16 h groups, then factors
   int H, I, E, k, n_group, topk_group, has_shared;
   float rsf;
   int RR, RG, RD;     // rows per router block / gate-up / down item

@@ -49,6 +49,7 @@ moe_status forward_impl(const moe_layer* l, const uint16_t* x, int T, float* y, 
     p.w_ws = reinterpret_cast<float*>(ws + L.w);
     p.hbuf = reinterpret_cast<float*>(ws + L.hbuf);
     p.ypart = reinterpret_cast<float*>(ws + L.ypart);
+    p.hq = reinterpret_cast<uint32_t*>(ws + L.hq);
     cudaError_t e = launch_decode(p, st);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "decode launch");
   }
