@@ -153,6 +153,85 @@ moe_status moe_layer_forward(const moe_layer* layer, const void* x_dev, int T,
                              float* w_out_dev, void* ws_dev, size_t ws_bytes,
                              void* stream);
 
+/* ---- stacked layers (pre-norm residual stream) --------------------------- */
+
+/* One decoder MoE step on an fp32 residual stream (the reading of a stack of
+ * layers: RMSNorm with unit gain before each MoE block, as in the upstream
+ * model -- "LightLX", "How it works": RMSNorm):
+ *   x_next = x + MoE(bf16(x / sqrt(mean(x^2) + norm_eps)))
+ * x_dev, x_next_dev fp32 [hidden], distinct.  xn_out_dev (nullable) receives
+ * the bf16 normalised input the experts saw.  One token (T = 1); the shape
+ * must be one the fused decode kernel covers (MOE_ERR_UNSUPPORTED otherwise).
+ * The workspace is that of moe_workspace_bytes(cfg, 1). */
+moe_status moe_layer_forward_residual(const moe_layer* layer, const float* x_dev,
+                                      float* x_next_dev, uint16_t* xn_out_dev,
+                                      int32_t* idx_out_dev, float* w_out_dev,
+                                      float norm_eps, void* ws_dev,
+                                      size_t ws_bytes, void* stream);
+
+/* n_layers residual steps in order, one token: layers[l] maps x_l to
+ * x_{l+1}; x_in_dev = x_0, x_out_dev = x_{n_layers}; x_tmp_dev is a third
+ * fp32 [hidden] buffer (unused for one layer).  idx_out_dev (nullable)
+ * int32 [n_layers][top_k].  All launches are enqueued on stream (capturable
+ * into a CUDA graph). */
+moe_status moe_stack_forward(const moe_layer* const* layers, int n_layers,
+                             const float* x_in_dev, float* x_out_dev,
+                             float* x_tmp_dev, int32_t* idx_out_dev,
+                             float norm_eps, void* ws_dev, size_t ws_bytes,
+                             void* stream);
+
+/* ---- host-streamed experts: per-layer LRU cache in HBM ------------------ */
+/* colibri summary ("Show HN: run GLM 5.2 on a slow computer"), section
+ * "Execution d'un MoE basee sur le streaming disque": a per-layer LRU cache
+ * of routed experts in front of a larger store; "Principales fonctionnalites
+ * implementees": the next expert block is read while another is multiplied.
+ * Here the store is pinned host memory and the cache is HBM. */
+typedef struct moe_cache moe_cache;
+
+/* host_experts: host array [n_layers][n_experts] of moe_expert whose six
+ * pointers are pinned host memory (cudaHostAlloc / registered), caller-owned,
+ * alive until moe_cache_destroy.  Allocates n_layers * slots_per_layer expert
+ * slots in HBM (MOE_ERR_OOM if they do not fit) and a copy stream.
+ * top_k <= slots_per_layer <= n_experts. */
+moe_status moe_cache_create(const moe_config* cfg, int n_layers,
+                            int slots_per_layer,
+                            const moe_expert* host_experts, moe_cache** out);
+void moe_cache_destroy(moe_cache* cache);
+
+/* The layer view of `layer` (created on first call, owned by the cache):
+ * router weight / bias and the shared expert are resident device tensors as
+ * in moe_layer_create; routed entries point into the cache's slots and are
+ * valid for the ids of the latest moe_cache_acquire of that layer. */
+moe_status moe_cache_layer(moe_cache* cache, int layer,
+                           const float* w_router_dev, const float* bias_dev,
+                           const moe_expert* shared_host, moe_layer** view);
+
+/* Make experts ids_host[0..n) (ascending, distinct) of `layer` resident:
+ * LRU bookkeeping on the host; every miss is copied host -> slot with
+ * cudaMemcpyAsync on the cache's copy stream (after the layer's last
+ * release event, so no slot still in use is overwritten); compute_stream
+ * then waits for the copies and the layer view's pointer table is updated
+ * on it.  Replacement: hits are touched in ascending id order, then each
+ * miss in ascending id order takes the lowest empty slot, else the least
+ * recently used slot not holding one of ids.  n <= slots_per_layer, n <= 32. */
+moe_status moe_cache_acquire(moe_cache* cache, int layer,
+                             const int32_t* ids_host, int n,
+                             void* compute_stream);
+/* Mark the end of the compute that reads `layer`'s slots on compute_stream. */
+moe_status moe_cache_release(moe_cache* cache, int layer, void* compute_stream);
+/* Cumulative counters of a layer (any pointer nullable). */
+moe_status moe_cache_stats(const moe_cache* cache, int layer, uint64_t* hits,
+                           uint64_t* misses, uint64_t* bytes_h2d);
+/* Wait for the cache's copy stream. */
+moe_status moe_cache_sync(moe_cache* cache);
+
+/* The cache's replacement rule run on the host over a trace [T][n_layers][k]
+ * of ascending ids (no GPU needed): per-layer hits and misses after T calls
+ * with `capacity` slots, all empty at the start. */
+moe_status moe_lru_replay(int n_layers, int n_experts, int capacity, int k,
+                          int T, const int32_t* trace, uint64_t* hits,
+                          uint64_t* misses);
+
 /* ---- diagnostics ------------------------------------------------------- */
 
 /* One dequantising int4 GEMV with the layer kernels' group dot product:

@@ -78,6 +78,26 @@ def lib():
         L.moe_expert_ffn.argtypes = [p, p, i, p, p, p, p, sz, p]
         L.moe_layer_forward.restype = st
         L.moe_layer_forward.argtypes = [p, p, i, p, p, p, p, sz, p]
+        L.moe_layer_forward_residual.restype = st
+        L.moe_layer_forward_residual.argtypes = [p, p, p, p, p, p, ctypes.c_float, p, sz, p]
+        L.moe_stack_forward.restype = st
+        L.moe_stack_forward.argtypes = [p, i, p, p, p, p, ctypes.c_float, p, sz, p]
+        L.moe_cache_create.restype = st
+        L.moe_cache_create.argtypes = [p, i, i, p, ctypes.POINTER(p)]
+        L.moe_cache_destroy.restype = None
+        L.moe_cache_destroy.argtypes = [p]
+        L.moe_cache_layer.restype = st
+        L.moe_cache_layer.argtypes = [p, i, p, p, p, ctypes.POINTER(p)]
+        L.moe_cache_acquire.restype = st
+        L.moe_cache_acquire.argtypes = [p, i, p, i, p]
+        L.moe_cache_release.restype = st
+        L.moe_cache_release.argtypes = [p, i, p]
+        L.moe_cache_stats.restype = st
+        L.moe_cache_stats.argtypes = [p, i, p, p, p]
+        L.moe_cache_sync.restype = st
+        L.moe_cache_sync.argtypes = [p]
+        L.moe_lru_replay.restype = st
+        L.moe_lru_replay.argtypes = [i, i, i, i, i, p, p, p]
         L.moe_debug_gemv_int4.restype = st
         L.moe_debug_gemv_int4.argtypes = [p, p, i, i, p, p, p]
         _lib = L
@@ -165,6 +185,108 @@ class Layer:
         check(lib().moe_layer_forward(self.handle, _ptr(x), T, _ptr(y), _ptr(idx), _ptr(w),
                                       _ptr(ws), ws.numel(), _stream(stream)),
               "moe_layer_forward")
+
+
+NORM_EPS = 1e-6
+
+
+def forward_residual(layer, x, x_next, ws, xn=None, idx=None, w=None, eps=NORM_EPS, stream=None):
+    """x_next = x + MoE(bf16(RMSNorm(x))) for one token (fp32 [hidden] tensors)."""
+    check(lib().moe_layer_forward_residual(layer.handle, _ptr(x), _ptr(x_next), _ptr(xn),
+                                           _ptr(idx), _ptr(w), float(eps), _ptr(ws), ws.numel(),
+                                           _stream(stream)), "moe_layer_forward_residual")
+
+
+def stack_forward(layers, x_in, x_out, x_tmp, ws, idx=None, eps=NORM_EPS, stream=None):
+    """Residual steps through layers[0..L-1] for one token."""
+    arr = (ctypes.c_void_p * len(layers))(*[l.handle.value for l in layers])
+    check(lib().moe_stack_forward(arr, len(layers), _ptr(x_in), _ptr(x_out), _ptr(x_tmp), _ptr(idx),
+                                  float(eps), _ptr(ws), ws.numel(), _stream(stream)),
+          "moe_stack_forward")
+
+
+def lru_replay(trace, n_experts, capacity):
+    """The cache's LRU rule on a host trace [T][L][k] -> (hits[L], misses[L])."""
+    import numpy as np
+    tr = np.ascontiguousarray(trace, dtype=np.int32)
+    T, Lyr, k = tr.shape
+    hits = np.zeros(Lyr, dtype=np.uint64)
+    misses = np.zeros(Lyr, dtype=np.uint64)
+    check(lib().moe_lru_replay(Lyr, n_experts, capacity, k, T, tr.ctypes.data, hits.ctypes.data,
+                               misses.ctypes.data), "moe_lru_replay")
+    return hits, misses
+
+
+class _LayerView:
+    """A moe_layer owned by something else (a cache view)."""
+
+    def __init__(self, handle, cfg):
+        self.handle = handle
+        self.cfg = cfg
+
+    route = Layer.route
+    expert_ffn = Layer.expert_ffn
+    forward = Layer.forward
+
+
+class Cache:
+    """Per-layer LRU cache of routed experts in HBM over a pinned host store.
+
+    host_experts: list over layers of lists over experts of dicts name ->
+    pinned host address (int) or pinned tensor."""
+
+    def __init__(self, cfg, host_experts, slots_per_layer):
+        self.cfg = cfg
+        n_layers = len(host_experts)
+        arr = (Expert * (n_layers * cfg.n_experts))()
+        for l, layer in enumerate(host_experts):
+            for e, d in enumerate(layer):
+                arr[l * cfg.n_experts + e] = Expert.from_ptrs({k: _addr(v) for k, v in d.items()})
+        out = ctypes.c_void_p()
+        check(lib().moe_cache_create(ctypes.byref(cfg), n_layers, int(slots_per_layer), arr,
+                                     ctypes.byref(out)), "moe_cache_create")
+        self.handle = out
+        self._keep = host_experts
+        self._views = {}
+
+    def layer(self, l, w_router, bias, shared):
+        if l not in self._views:
+            sh = Expert.from_ptrs({k: _addr(v) for k, v in shared.items()}) if shared else None
+            out = ctypes.c_void_p()
+            check(lib().moe_cache_layer(self.handle, int(l), _addr(w_router), _addr(bias),
+                                        ctypes.byref(sh) if sh is not None else None,
+                                        ctypes.byref(out)), "moe_cache_layer")
+            self._views[l] = (_LayerView(out, self.cfg), (w_router, bias, shared))
+        return self._views[l][0]
+
+    def acquire(self, l, ids, stream=None):
+        import numpy as np
+        a = np.ascontiguousarray(ids, dtype=np.int32)
+        check(lib().moe_cache_acquire(self.handle, int(l), a.ctypes.data, a.size, _stream(stream)),
+              "moe_cache_acquire")
+
+    def release(self, l, stream=None):
+        check(lib().moe_cache_release(self.handle, int(l), _stream(stream)), "moe_cache_release")
+
+    def stats(self, l):
+        h, m, b = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_uint64()
+        check(lib().moe_cache_stats(self.handle, int(l), ctypes.byref(h), ctypes.byref(m),
+                                    ctypes.byref(b)), "moe_cache_stats")
+        return h.value, m.value, b.value
+
+    def sync(self):
+        check(lib().moe_cache_sync(self.handle), "moe_cache_sync")
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib().moe_cache_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def gemv_int4(q, s, rows, cols, x, y, stream=None):

@@ -280,6 +280,55 @@ moe_status moe_layer_forward(const moe_layer* l, const void* x, int T, float* y,
                       (cudaStream_t)stream);
 }
 
+moe_status moe_layer_forward_residual(const moe_layer* l, const float* x_dev, float* x_next_dev,
+                                      uint16_t* xn_out_dev, int32_t* idx_out_dev,
+                                      float* w_out_dev, float norm_eps, void* ws, size_t ws_bytes,
+                                      void* stream) {
+  g_last_error[0] = 0;
+  if (!l) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+  moe_status s;
+  if ((s = check_device_ptr(x_dev, 16, "x")) != MOE_OK) return s;
+  if ((s = check_device_ptr(x_next_dev, 16, "x_next")) != MOE_OK) return s;
+  if (x_dev == x_next_dev) return fail(MOE_ERR_INVALID_ARG, "x and x_next must not alias");
+  if (xn_out_dev && (s = check_device_ptr(xn_out_dev, 4, "xn_out")) != MOE_OK) return s;
+  if (idx_out_dev && (s = check_device_ptr(idx_out_dev, 4, "idx_out")) != MOE_OK) return s;
+  if (w_out_dev && (s = check_device_ptr(w_out_dev, 4, "w_out")) != MOE_OK) return s;
+  if (!(norm_eps >= 0.f)) return fail(MOE_ERR_INVALID_ARG, "norm_eps must be >= 0");
+  WsLayout L;
+  if ((s = check_ws(l, 1, ws, ws_bytes, &L)) != MOE_OK) return s;
+  return residual_impl(l, x_dev, norm_eps, x_next_dev, xn_out_dev, idx_out_dev, w_out_dev,
+                       (uint8_t*)ws, L, (cudaStream_t)stream);
+}
+
+moe_status moe_stack_forward(const moe_layer* const* layers, int n_layers, const float* x_in_dev,
+                             float* x_out_dev, float* x_tmp_dev, int32_t* idx_out_dev,
+                             float norm_eps, void* ws, size_t ws_bytes, void* stream) {
+  g_last_error[0] = 0;
+  if (!layers || n_layers < 1) return fail(MOE_ERR_INVALID_ARG, "need at least one layer");
+  if (n_layers > 1 && !x_tmp_dev) return fail(MOE_ERR_INVALID_ARG, "x_tmp is needed for more than one layer");
+  const moe_config& c0 = layers[0]->cfg;
+  for (int l = 1; l < n_layers; ++l) {
+    if (!layers[l]) return fail(MOE_ERR_INVALID_ARG, "layers[%d] is NULL", l);
+    if (layers[l]->cfg.hidden != c0.hidden || layers[l]->cfg.top_k != c0.top_k)
+      return fail(MOE_ERR_INVALID_ARG, "layers differ in shape");
+  }
+  if (x_tmp_dev && (x_tmp_dev == x_out_dev || x_tmp_dev == x_in_dev))
+    return fail(MOE_ERR_INVALID_ARG, "x_tmp must be a separate buffer");
+  // ping-pong so that the last layer writes x_out
+  const float* cur = x_in_dev;
+  for (int l = 0; l < n_layers; ++l) {
+    const bool last = (l == n_layers - 1);
+    float* nxt = ((n_layers - 1 - l) % 2 == 0) ? x_out_dev : x_tmp_dev;
+    if (last) nxt = x_out_dev;
+    int32_t* idx = idx_out_dev ? idx_out_dev + (size_t)l * c0.top_k : nullptr;
+    moe_status s = moe_layer_forward_residual(layers[l], cur, nxt, nullptr, idx, nullptr, norm_eps,
+                                              ws, ws_bytes, stream);
+    if (s != MOE_OK) return s;
+    cur = nxt;
+  }
+  return MOE_OK;
+}
+
 moe_status moe_debug_gemv_int4(const uint8_t* q, const uint16_t* s, int rows, int cols,
                                const float* x, float* y, void* stream) {
   g_last_error[0] = 0;

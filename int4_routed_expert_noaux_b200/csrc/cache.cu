@@ -1,0 +1,342 @@
+// cache.cu -- per-layer LRU cache of routed experts in HBM, fed from a
+// pinned host store by cudaMemcpyAsync on a side stream (colibri summary,
+// "Execution d'un MoE basee sur le streaming disque": a per-layer LRU cache
+// of routed experts; "Principales fonctionnalites implementees": expert
+// readahead while another expert block is multiplied).
+//
+// Replacement rule, per layer and per call: ids already cached are hits and
+// are touched in ascending id order; then every missing id, in ascending
+// order, takes an empty slot (the lowest) or else the least recently used
+// slot whose expert is not among the call's ids.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <new>
+#include <vector>
+
+#include "layer.h"
+#include "moe.h"
+
+namespace moe {
+
+// The replacement rule on its own (host only).
+class LruPolicy {
+ public:
+  LruPolicy(int n_experts, int slots)
+      : slot_expert_(slots, -1), stamp_(slots, 0), expert_slot_(n_experts, -1) {}
+
+  struct Load {
+    int expert, slot, evicted;
+  };
+
+  // ids ascending, distinct.  Fills loads (misses) and returns the hit count.
+  int access(const int32_t* ids, int n, std::vector<Load>& loads) {
+    loads.clear();
+    int hits = 0;
+    for (int j = 0; j < n; ++j) {
+      const int s = expert_slot_[ids[j]];
+      if (s >= 0) {
+        stamp_[s] = ++clock_;
+        ++hits;
+      }
+    }
+    for (int j = 0; j < n; ++j) {
+      const int e = ids[j];
+      if (expert_slot_[e] >= 0) continue;
+      int victim = -1;
+      for (int s = 0; s < (int)slot_expert_.size() && victim < 0; ++s)
+        if (slot_expert_[s] < 0) victim = s;
+      if (victim < 0) {
+        for (int s = 0; s < (int)slot_expert_.size(); ++s) {
+          bool current = false;
+          for (int jj = 0; jj < n; ++jj)
+            if (slot_expert_[s] == ids[jj]) current = true;
+          if (current) continue;
+          if (victim < 0 || stamp_[s] < stamp_[victim]) victim = s;
+        }
+      }
+      const int old = slot_expert_[victim];
+      if (old >= 0) expert_slot_[old] = -1;
+      slot_expert_[victim] = e;
+      expert_slot_[e] = victim;
+      stamp_[victim] = ++clock_;
+      loads.push_back(Load{e, victim, old});
+    }
+    return hits;
+  }
+
+ private:
+  std::vector<int> slot_expert_;
+  std::vector<uint64_t> stamp_;
+  std::vector<int> expert_slot_;
+  uint64_t clock_ = 0;
+};
+
+namespace {
+
+constexpr int kMaxTableUpdates = 32;
+
+struct TableUpdate {
+  int n;
+  int ids[kMaxTableUpdates];
+  ExpertPtrs ptrs[kMaxTableUpdates];
+};
+
+// Writes new pointer-table entries; the entries travel as kernel arguments,
+// so the update is ordered on the compute stream with no host staging.
+__global__ void table_update_kernel(ExpertPtrs* table, TableUpdate u) {
+  const int i = threadIdx.x;
+  if (i < u.n) table[u.ids[i]] = u.ptrs[i];
+}
+
+}  // namespace
+
+}  // namespace moe
+
+using namespace moe;
+
+struct moe_cache {
+  moe_config cfg;
+  int n_layers = 0, slots = 0;
+  size_t expert_bytes = 0;
+  size_t off[6] = {0, 0, 0, 0, 0, 0};  // tensor offsets inside a slot
+  std::vector<moe_expert> host;        // [L][E] pinned host experts (caller-owned)
+  uint8_t* dev_slots = nullptr;        // [L][slots][expert_bytes]
+  cudaStream_t copy_stream = nullptr;
+  std::vector<cudaEvent_t> copied;     // per layer: loads of the last acquire done
+  std::vector<cudaEvent_t> used;       // per layer: compute of the last release done
+  std::vector<bool> used_valid;
+  std::vector<LruPolicy> lru;
+  std::vector<moe_layer*> views;       // per layer, created by moe_cache_layer
+  std::vector<uint64_t> hits, misses, bytes;
+  std::vector<LruPolicy::Load> loads;  // scratch
+};
+
+namespace {
+
+size_t expert_bytes_of(const moe_config& c, size_t off[6]) {
+  const size_t H = c.hidden, I = c.inter;
+  const size_t qgu = I * H / 2, sgu = I * (H / 32) * 2, qd = H * I / 2, sd = H * (I / 32) * 2;
+  off[0] = 0;                 // q_gate
+  off[1] = off[0] + qgu;      // q_up
+  off[2] = off[1] + qgu;      // s_gate
+  off[3] = off[2] + sgu;      // s_up
+  off[4] = off[3] + sgu;      // q_down
+  off[5] = off[4] + qd;       // s_down
+  return off[5] + sd;
+}
+
+moe_status check_host_ptr(const void* p, const char* name) {
+  if (!p) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", name);
+  cudaPointerAttributes a;
+  cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MOE_ERR_INVALID_ARG, "%s: not a registered host pointer", name);
+  }
+  if (a.type != cudaMemoryTypeHost)
+    return fail(MOE_ERR_INVALID_ARG, "%s is not pinned host memory", name);
+  return MOE_OK;
+}
+
+ExpertPtrs slot_ptrs(const moe_cache* c, int layer, int slot) {
+  const uint8_t* b = c->dev_slots + ((size_t)layer * c->slots + slot) * c->expert_bytes;
+  return ExpertPtrs{b + c->off[0], b + c->off[1], reinterpret_cast<const uint16_t*>(b + c->off[2]),
+                    reinterpret_cast<const uint16_t*>(b + c->off[3]), b + c->off[4],
+                    reinterpret_cast<const uint16_t*>(b + c->off[5])};
+}
+
+}  // namespace
+
+extern "C" {
+#pragma GCC visibility push(default)
+
+moe_status moe_lru_replay(int n_layers, int n_experts, int capacity, int k, int T,
+                          const int32_t* trace, uint64_t* hits, uint64_t* misses) {
+  if (n_layers < 1 || n_experts < 1 || k < 1 || capacity < k || T < 0 || !trace || !hits ||
+      !misses)
+    return fail(MOE_ERR_INVALID_ARG, "bad LRU replay arguments");
+  std::vector<LruPolicy::Load> loads;
+  for (int l = 0; l < n_layers; ++l) {
+    LruPolicy lru(n_experts, capacity);
+    uint64_t h = 0, m = 0;
+    for (int t = 0; t < T; ++t) {
+      const int32_t* ids = trace + ((size_t)t * n_layers + l) * k;
+      for (int j = 0; j < k; ++j)
+        if (ids[j] < 0 || ids[j] >= n_experts || (j && ids[j] <= ids[j - 1]))
+          return fail(MOE_ERR_INVALID_ARG, "trace ids must be ascending and in range");
+      h += lru.access(ids, k, loads);
+      m += loads.size();
+    }
+    hits[l] = h;
+    misses[l] = m;
+  }
+  return MOE_OK;
+}
+
+moe_status moe_cache_create(const moe_config* cfg, int n_layers, int slots_per_layer,
+                            const moe_expert* host_experts, moe_cache** out) {
+  if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  moe_status s = check_config(cfg);
+  if (s != MOE_OK) return s;
+  if (n_layers < 1) return fail(MOE_ERR_INVALID_ARG, "n_layers must be >= 1");
+  if (slots_per_layer < cfg->top_k || slots_per_layer > cfg->n_experts)
+    return fail(MOE_ERR_INVALID_ARG, "slots_per_layer must be in [top_k, n_experts]");
+  if (!host_experts) return fail(MOE_ERR_INVALID_ARG, "host_experts is NULL");
+  const size_t n = (size_t)n_layers * cfg->n_experts;
+  for (size_t i = 0; i < n; ++i) {
+    const moe_expert& e = host_experts[i];
+    const void* ptrs[6] = {e.q_gate, e.q_up, e.s_gate, e.s_up, e.q_down, e.s_down};
+    for (int t = 0; t < 6; ++t)
+      if ((s = check_host_ptr(ptrs[t], "host expert tensor")) != MOE_OK) return s;
+  }
+  moe_cache* c = new (std::nothrow) moe_cache();
+  if (!c) return fail(MOE_ERR_OOM, "host allocation failed");
+  c->cfg = *cfg;
+  c->n_layers = n_layers;
+  c->slots = slots_per_layer;
+  c->expert_bytes = expert_bytes_of(*cfg, c->off);
+  c->host.assign(host_experts, host_experts + n);
+  const size_t dev_bytes = (size_t)n_layers * slots_per_layer * c->expert_bytes;
+  size_t free_b = 0, total_b = 0;
+  cudaError_t ce = cudaMemGetInfo(&free_b, &total_b);
+  if (ce == cudaSuccess && dev_bytes + (256u << 20) > free_b) {
+    delete c;
+    return fail(MOE_ERR_OOM, "cache needs %zu bytes of HBM, %zu free", dev_bytes, free_b);
+  }
+  ce = cudaMalloc(&c->dev_slots, dev_bytes);
+  if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&c->copy_stream, cudaStreamNonBlocking);
+  c->copied.assign(n_layers, nullptr);
+  c->used.assign(n_layers, nullptr);
+  c->used_valid.assign(n_layers, false);
+  for (int l = 0; l < n_layers && ce == cudaSuccess; ++l) {
+    ce = cudaEventCreateWithFlags(&c->copied[l], cudaEventDisableTiming);
+    if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->used[l], cudaEventDisableTiming);
+  }
+  if (ce != cudaSuccess) {
+    s = cuda_fail(ce, "moe_cache_create");
+    moe_cache_destroy(c);
+    return s;
+  }
+  for (int l = 0; l < n_layers; ++l) c->lru.emplace_back(cfg->n_experts, slots_per_layer);
+  c->views.assign(n_layers, nullptr);
+  c->hits.assign(n_layers, 0);
+  c->misses.assign(n_layers, 0);
+  c->bytes.assign(n_layers, 0);
+  *out = c;
+  return MOE_OK;
+}
+
+void moe_cache_destroy(moe_cache* c) {
+  if (!c) return;
+  if (c->copy_stream) cudaStreamSynchronize(c->copy_stream);
+  for (moe_layer* v : c->views) moe_layer_destroy(v);
+  for (cudaEvent_t e : c->copied)
+    if (e) cudaEventDestroy(e);
+  for (cudaEvent_t e : c->used)
+    if (e) cudaEventDestroy(e);
+  if (c->copy_stream) cudaStreamDestroy(c->copy_stream);
+  if (c->dev_slots) cudaFree(c->dev_slots);
+  delete c;
+}
+
+moe_status moe_cache_layer(moe_cache* c, int layer, const float* w_router_dev,
+                           const float* bias_dev, const moe_expert* shared_host,
+                           moe_layer** view) {
+  if (!c || !view) return fail(MOE_ERR_INVALID_ARG, "cache or view is NULL");
+  if (layer < 0 || layer >= c->n_layers) return fail(MOE_ERR_INVALID_ARG, "layer out of range");
+  *view = nullptr;
+  if (c->views[layer]) {
+    *view = c->views[layer];
+    return MOE_OK;
+  }
+  // every routed entry starts at slot 0 of the layer; the kernels only read
+  // the entries of selected experts, which acquire sets first
+  std::vector<moe_expert> tab(c->cfg.n_experts);
+  const ExpertPtrs s0 = slot_ptrs(c, layer, 0);
+  for (int e = 0; e < c->cfg.n_experts; ++e)
+    tab[e] = moe_expert{s0.q_gate, s0.q_up, s0.s_gate, s0.s_up, s0.q_down, s0.s_down};
+  moe_layer* l = nullptr;
+  moe_status s = moe_layer_create(&c->cfg, w_router_dev, bias_dev, tab.data(), shared_host, &l);
+  if (s != MOE_OK) return s;
+  c->views[layer] = l;
+  *view = l;
+  return MOE_OK;
+}
+
+moe_status moe_cache_acquire(moe_cache* c, int layer, const int32_t* ids_host, int n,
+                             void* compute_stream) {
+  if (!c || !ids_host) return fail(MOE_ERR_INVALID_ARG, "cache or ids is NULL");
+  if (layer < 0 || layer >= c->n_layers) return fail(MOE_ERR_INVALID_ARG, "layer out of range");
+  if (!c->views[layer]) return fail(MOE_ERR_INVALID_ARG, "create the layer view first (moe_cache_layer)");
+  if (n < 1 || n > c->slots || n > kMaxTableUpdates)
+    return fail(MOE_ERR_INVALID_ARG, "n = %d outside 1..min(slots, %d)", n, kMaxTableUpdates);
+  for (int j = 0; j < n; ++j)
+    if (ids_host[j] < 0 || ids_host[j] >= c->cfg.n_experts || (j && ids_host[j] <= ids_host[j - 1]))
+      return fail(MOE_ERR_INVALID_ARG, "ids must be ascending, distinct and in range");
+  cudaStream_t cs = (cudaStream_t)compute_stream;
+  const int hits = c->lru[layer].access(ids_host, n, c->loads);
+  c->hits[layer] += hits;
+  if (c->loads.empty()) return MOE_OK;
+  cudaError_t ce = cudaSuccess;
+  // a victim slot may still be read by this layer's previously released compute
+  if (c->used_valid[layer]) ce = cudaStreamWaitEvent(c->copy_stream, c->used[layer], 0);
+  TableUpdate u;
+  u.n = 0;
+  moe_layer* view = c->views[layer];
+  for (const LruPolicy::Load& ld : c->loads) {
+    const moe_expert& he = c->host[(size_t)layer * c->cfg.n_experts + ld.expert];
+    const ExpertPtrs d = slot_ptrs(c, layer, ld.slot);
+    const void* src[6] = {he.q_gate, he.q_up, he.s_gate, he.s_up, he.q_down, he.s_down};
+    void* dst[6] = {(void*)d.q_gate, (void*)d.q_up, (void*)d.s_gate,
+                    (void*)d.s_up, (void*)d.q_down, (void*)d.s_down};
+    const size_t sz[6] = {c->off[1] - c->off[0], c->off[2] - c->off[1], c->off[3] - c->off[2],
+                          c->off[4] - c->off[3], c->off[5] - c->off[4],
+                          c->expert_bytes - c->off[5]};
+    for (int t = 0; t < 6 && ce == cudaSuccess; ++t)
+      ce = cudaMemcpyAsync(dst[t], src[t], sz[t], cudaMemcpyHostToDevice, c->copy_stream);
+    u.ids[u.n] = ld.expert;
+    u.ptrs[u.n] = d;
+    view->host_table[ld.expert] = d;
+    ++u.n;
+    c->misses[layer] += 1;
+    c->bytes[layer] += c->expert_bytes;
+  }
+  if (ce == cudaSuccess) ce = cudaEventRecord(c->copied[layer], c->copy_stream);
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(cs, c->copied[layer], 0);
+  if (ce == cudaSuccess) {
+    table_update_kernel<<<1, kMaxTableUpdates, 0, cs>>>(view->table, u);
+    ce = cudaGetLastError();
+  }
+  return ce == cudaSuccess ? MOE_OK : cuda_fail(ce, "moe_cache_acquire");
+}
+
+moe_status moe_cache_release(moe_cache* c, int layer, void* compute_stream) {
+  if (!c) return fail(MOE_ERR_INVALID_ARG, "cache is NULL");
+  if (layer < 0 || layer >= c->n_layers) return fail(MOE_ERR_INVALID_ARG, "layer out of range");
+  cudaError_t ce = cudaEventRecord(c->used[layer], (cudaStream_t)compute_stream);
+  if (ce != cudaSuccess) return cuda_fail(ce, "moe_cache_release");
+  c->used_valid[layer] = true;
+  return MOE_OK;
+}
+
+moe_status moe_cache_stats(const moe_cache* c, int layer, uint64_t* hits, uint64_t* misses,
+                           uint64_t* bytes_h2d) {
+  if (!c) return fail(MOE_ERR_INVALID_ARG, "cache is NULL");
+  if (layer < 0 || layer >= c->n_layers) return fail(MOE_ERR_INVALID_ARG, "layer out of range");
+  if (hits) *hits = c->hits[layer];
+  if (misses) *misses = c->misses[layer];
+  if (bytes_h2d) *bytes_h2d = c->bytes[layer];
+  return MOE_OK;
+}
+
+moe_status moe_cache_sync(moe_cache* c) {
+  if (!c) return fail(MOE_ERR_INVALID_ARG, "cache is NULL");
+  cudaError_t ce = cudaStreamSynchronize(c->copy_stream);
+  return ce == cudaSuccess ? MOE_OK : cuda_fail(ce, "moe_cache_sync");
+}
+
+#pragma GCC visibility pop
+}  // extern "C"

@@ -75,6 +75,8 @@ struct Smem {
   ItemDesc desc[kStages];
   float red[kGroups][2][kGW][32];
   int abort_flag[kGroups];
+  float norm_part[kThreads / 32];
+  float inv_rms;
   float sc[kMaxE];
   float sp[kMaxE];
 };
@@ -298,6 +300,13 @@ __device__ __noinline__ void quantize_slot(const DecodeParams& p, int slot) {
   if (lane == 0) st_release(p.ctrl + kCtrlHqReady + slot, 1u);
 }
 
+// bf16 bit pattern of layer input element i: x[i] itself, or, for a
+// residual (pre-norm) step, bf16(x_resid[i] * inv_rms).
+__device__ __forceinline__ uint32_t input_bf16(const DecodeParams& p, int i, float inv_rms) {
+  if (p.x_resid) return f32_to_bf16_rne(p.x_resid[i] * inv_rms);
+  return p.x[i];
+}
+
 // Fixed-order combine of one row block of y from the per-slot partials, by
 // one warp, once every slot's down item of the block has published.
 __device__ __noinline__ void combine_block(const DecodeParams& p, int row0, int nrows) {
@@ -310,6 +319,7 @@ __device__ __noinline__ void combine_block(const DecodeParams& p, int row0, int 
     for (int j = 0; j < p.k; ++j)
       acc = fmaf(__ldcg(p.w_ws + j), __ldcg(p.ypart + (size_t)j * p.H + row), acc);
     if (p.has_shared) acc += __ldcg(p.ypart + (size_t)p.k * p.H + row);
+    if (p.x_resid) acc = p.x_resid[row] + acc;  // residual stream: x + MoE(norm(x))
     p.y[row] = acc;
   }
 }
@@ -521,7 +531,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     S.abort_flag[0] = S.abort_flag[1] = 0;
     fence_mbar_init();
   }
+  if (p.x_resid) {
+    // RMSNorm with unit gain ("LightLX", "How it works": RMSNorm of the
+    // upstream model): every CTA forms the same fixed-order sum of squares.
+    float part = 0.f;
+    for (int i = threadIdx.x; i < p.H; i += kThreads) part = fmaf(p.x_resid[i], p.x_resid[i], part);
+    part = warp_sum(part);
+    if (lane == 0) S.norm_part[warp] = part;
+  }
   __syncthreads();
+  if (p.x_resid && threadIdx.x == 0) {
+    float ss = 0.f;
+    for (int w = 0; w < kThreads / 32; ++w) ss += S.norm_part[w];
+    S.inv_rms = 1.0f / sqrtf(ss / (float)p.H + p.norm_eps);
+  }
+  __syncthreads();
+  const float inv_rms = p.x_resid ? S.inv_rms : 1.0f;
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
@@ -646,15 +671,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     XQ xq;
     {
       float xf[32];
-      const uint4* xp = reinterpret_cast<const uint4*>(p.x + cg.col * 32);
+      if (p.x_resid) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 v = __ldg(xp + i);
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+        for (int i = 0; i < 32; ++i) {
+          const uint32_t b = input_bf16(p, cg.col * 32 + i, inv_rms);
+          xf[i] = bf16_bits_to_f32(b);
+          if (blockIdx.x == 0 && grp == 0 && cg.phase == 0 && p.xn_out)
+            p.xn_out[cg.col * 32 + i] = (uint16_t)b;
+        }
+      } else {
+        const uint4* xp = reinterpret_cast<const uint4*>(p.x + cg.col * 32);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          xf[8 * i + 2 * j] = bf16_bits_to_f32(u[j] & 0xFFFFu);
-          xf[8 * i + 2 * j + 1] = bf16_bits_to_f32(u[j] >> 16);
+        for (int i = 0; i < 4; ++i) {
+          const uint4 v = __ldg(xp + i);
+          const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            xf[8 * i + 2 * j] = bf16_bits_to_f32(u[j] & 0xFFFFu);
+            xf[8 * i + 2 * j + 1] = bf16_bits_to_f32(u[j] >> 16);
+          }
         }
       }
       xq_from_floats(xf, xq);
@@ -677,7 +712,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
 #pragma unroll
         for (int i = 0; i < kRouterChunks; ++i) {
           const int cc = tg + kGT * i;
-          xr[i] = (cc < rchunks) ? __ldg(reinterpret_cast<const uint2*>(p.x) + cc) : make_uint2(0, 0);
+          if (cc >= rchunks) {
+            xr[i] = make_uint2(0, 0);
+          } else if (p.x_resid) {
+            xr[i].x = input_bf16(p, 4 * cc, inv_rms) | (input_bf16(p, 4 * cc + 1, inv_rms) << 16);
+            xr[i].y = input_bf16(p, 4 * cc + 2, inv_rms) | (input_bf16(p, 4 * cc + 3, inv_rms) << 16);
+          } else {
+            xr[i] = __ldg(reinterpret_cast<const uint2*>(p.x) + cc);
+          }
         }
         const int stage = 0, rbuf = 0;
         const uint32_t gpar = 0u;

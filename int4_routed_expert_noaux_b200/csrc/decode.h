@@ -31,8 +31,11 @@ struct DecodeParams {
   const ExpertPtrs* table;
   const float* w_router;
   const float* bias;
-  const uint16_t* x;  // bf16 [H]
-  float* y;           // fp32 [H]
+  const uint16_t* x;  // bf16 [H] (plain step), or
+  const float* x_resid;  // fp32 [H] residual stream (pre-norm step), nullable
+  float norm_eps;     // RMSNorm epsilon of the pre-norm step
+  uint16_t* xn_out;   // bf16 [H] normalised input of the pre-norm step, nullable
+  float* y;           // fp32 [H]: MoE(x), or x_resid + MoE(bf16(RMSNorm(x_resid)))
   int32_t* idx_out;   // nullable
   float* w_out;       // nullable
   uint32_t* ctrl;

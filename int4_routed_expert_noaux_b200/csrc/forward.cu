@@ -32,32 +32,58 @@ moe_status ffn_impl(const moe_layer* l, const uint16_t* x, int T, const int32_t*
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "expert launch");
 }
 
+static moe_status launch_fused(const moe_layer* l, const uint16_t* x, const float* x_resid,
+                               float norm_eps, uint16_t* xn_out, float* y, int32_t* idx_out,
+                               float* w_out, uint8_t* ws, const WsLayout& L, cudaStream_t st,
+                               bool* used) {
+  DecodeParams p;
+  *used = false;
+  if (!decode_plan(l->cfg, p)) return MOE_OK;
+  *used = true;
+  p.table = l->table;
+  p.w_router = l->w_router;
+  p.bias = l->bias;
+  p.x = x;
+  p.x_resid = x_resid;
+  p.norm_eps = norm_eps;
+  p.xn_out = xn_out;
+  p.y = y;
+  p.idx_out = idx_out;
+  p.w_out = w_out;
+  p.ctrl = reinterpret_cast<uint32_t*>(ws + L.ctrl);
+  p.logits = reinterpret_cast<float*>(ws + L.logits);
+  p.idx_ws = reinterpret_cast<int32_t*>(ws + L.idx);
+  p.w_ws = reinterpret_cast<float*>(ws + L.w);
+  p.hbuf = reinterpret_cast<float*>(ws + L.hbuf);
+  p.ypart = reinterpret_cast<float*>(ws + L.ypart);
+  p.hq = reinterpret_cast<uint32_t*>(ws + L.hq);
+  cudaError_t e = launch_decode(p, st);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "decode launch");
+}
+
 moe_status forward_impl(const moe_layer* l, const uint16_t* x, int T, float* y, int32_t* idx_out,
                         float* w_out, uint8_t* ws, const WsLayout& L, cudaStream_t st) {
-  DecodeParams p;
-  if (T == 1 && decode_plan(l->cfg, p)) {
-    p.table = l->table;
-    p.w_router = l->w_router;
-    p.bias = l->bias;
-    p.x = x;
-    p.y = y;
-    p.idx_out = idx_out;
-    p.w_out = w_out;
-    p.ctrl = reinterpret_cast<uint32_t*>(ws + L.ctrl);
-    p.logits = reinterpret_cast<float*>(ws + L.logits);
-    p.idx_ws = reinterpret_cast<int32_t*>(ws + L.idx);
-    p.w_ws = reinterpret_cast<float*>(ws + L.w);
-    p.hbuf = reinterpret_cast<float*>(ws + L.hbuf);
-    p.ypart = reinterpret_cast<float*>(ws + L.ypart);
-    p.hq = reinterpret_cast<uint32_t*>(ws + L.hq);
-    cudaError_t e = launch_decode(p, st);
-    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "decode launch");
+  if (T == 1) {
+    bool used = false;
+    moe_status s = launch_fused(l, x, nullptr, 0.f, nullptr, y, idx_out, w_out, ws, L, st, &used);
+    if (used || s != MOE_OK) return s;
   }
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
   float* w = w_out ? w_out : reinterpret_cast<float*>(ws + L.w);
   moe_status s = route_impl(l, x, T, idx, w, nullptr, ws, L, st);
   if (s != MOE_OK) return s;
   return ffn_impl(l, x, T, idx, w, y, ws, L, st);
+}
+
+moe_status residual_impl(const moe_layer* l, const float* x_resid, float norm_eps, float* x_next,
+                         uint16_t* xn_out, int32_t* idx_out, float* w_out, uint8_t* ws,
+                         const WsLayout& L, cudaStream_t st) {
+  bool used = false;
+  moe_status s = launch_fused(l, nullptr, x_resid, norm_eps, xn_out, x_next, idx_out, w_out, ws,
+                              L, st, &used);
+  if (s != MOE_OK) return s;
+  if (!used) return fail(MOE_ERR_UNSUPPORTED, "the pre-norm step needs the fused decode kernel's shapes");
+  return MOE_OK;
 }
 
 }  // namespace moe

@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 import int4_routed_expert_noaux_b200 as moe
@@ -58,3 +59,25 @@ def test_create_rejects_null_pointers():
     assert rc == 1
     assert b"NULL" in moe.lib().moe_last_error()
     assert not out.value
+
+
+def test_library_lru_matches_oracle_lru():
+    # the cache's replacement rule (C++ in the library) against the oracle's
+    # independent simulation, on Zipf traces at several capacities
+    import oracle
+    for seed, (L, E, k, T) in enumerate([(3, 256, 8, 300), (2, 16, 2, 200), (1, 64, 6, 500)]):
+        tr = synth.zipf_trace(seed, L, E, k, T)
+        for cap in sorted({k, k + 1, 2 * k, 4 * k, E // 2, E}):
+            if cap < k or cap > E:
+                continue
+            h1, m1 = moe.lru_replay(tr, E, cap)
+            h2, m2 = oracle.lru_sim(tr, E, cap)
+            assert np.array_equal(h1, h2) and np.array_equal(m1, m2), (seed, cap)
+
+
+def test_lru_replay_rejects_bad_traces():
+    tr = np.array([[[3, 1]]], dtype=np.int32)  # not ascending
+    with pytest.raises(moe.MoeError):
+        moe.lru_replay(tr, 8, 2)
+    with pytest.raises(moe.MoeError):
+        moe.lru_replay(np.array([[[0, 1]]], dtype=np.int32), 8, 1)  # capacity < k
