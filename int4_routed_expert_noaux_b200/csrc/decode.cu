@@ -21,10 +21,11 @@
 //    with a release flag; the producer acquires it before loading routed
 //    weights;
 //  * then work items come from a global ticket counter in the order:
-//    shared-expert gate/up, shared-expert down, routed gate/up of slots
-//    0..k-1, routed down of slots 0..k-1.  Every dependency points to an
-//    earlier ticket, so in-order claiming always makes progress, and each
-//    slot's down items come at least k-1 slots of work after its gate/up;
+//    shared-expert gate/up, routed gate/up of slots 0..k-1, routed down of
+//    slots 0..k-2, shared-expert down, routed down of slot k-1.  Every
+//    dependency points to an earlier ticket, so in-order claiming always
+//    makes progress, and every slot's down items come well after its
+//    gate/up items;
 //  * gate/up finalizer warps publish h rows and count themselves done; the
 //    warp that completes a slot (it looks before its next wait, never after,
 //    so no fill can depend on it) converts the slot's h to int16 groups once
@@ -93,6 +94,9 @@ __device__ __forceinline__ ItemDesc make_item(int type, int slot, int row0, int 
 }
 
 __device__ ItemDesc decode_ticket(const DecodeParams& p, int t) {
+  // shared gate/up, routed gate/up 0..k-1, routed down 0..k-2, shared down,
+  // routed down k-1: the shared expert's down items (ready early) sit between
+  // the last routed slot's gate/up and its down items.
   auto gu = [&](int slot, int b) {
     return make_item(kGateUp, slot, b * p.RG, min(p.RG, p.I - b * p.RG));
   };
@@ -102,12 +106,16 @@ __device__ ItemDesc decode_ticket(const DecodeParams& p, int t) {
   if (p.has_shared) {
     if (t < p.nG) return gu(p.k, t);
     t -= p.nG;
-    if (t < p.nD) return dn(p.k, t);
-    t -= p.nD;
   }
   if (t < p.k * p.nG) return gu(t / p.nG, t % p.nG);
   t -= p.k * p.nG;
-  if (t < p.k * p.nD) return dn(t / p.nD, t % p.nD);
+  if (t < (p.k - 1) * p.nD) return dn(t / p.nD, t % p.nD);
+  t -= (p.k - 1) * p.nD;
+  if (p.has_shared) {
+    if (t < p.nD) return dn(p.k, t);
+    t -= p.nD;
+  }
+  if (t < p.nD) return dn(p.k - 1, t);
   return make_item(kDone, 0, 0, 0);
 }
 
@@ -276,16 +284,27 @@ __device__ __noinline__ void quantize_slot(const DecodeParams& p, int slot) {
   __syncwarp();
   const float* h = p.hbuf + (size_t)slot * p.I;
   uint8_t* table = reinterpret_cast<uint8_t*>(p.hq) + (size_t)slot * ngroups * 68;
-  for (int gi = lane; gi < ngroups; gi += 32) {
+  for (int gi0 = lane; gi0 < ngroups; gi0 += 64) {
+    // two groups per pass, all loads issued before any is used
+    float4 raw[2][8];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int gi = gi0 + 32 * u;
+      const float4* hp = reinterpret_cast<const float4*>(h + (size_t)min(gi, ngroups - 1) * 32);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) raw[u][i] = __ldcg(hp + i);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+    const int gi = gi0 + 32 * u;
+    if (gi >= ngroups) break;
     float v[32];
-    const float4* hp = reinterpret_cast<const float4*>(h + gi * 32);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float4 t = __ldcg(hp + i);
-      v[4 * i] = t.x;
-      v[4 * i + 1] = t.y;
-      v[4 * i + 2] = t.z;
-      v[4 * i + 3] = t.w;
+      v[4 * i] = raw[u][i].x;
+      v[4 * i + 1] = raw[u][i].y;
+      v[4 * i + 2] = raw[u][i].z;
+      v[4 * i + 3] = raw[u][i].w;
     }
     XQ q;
     xq_from_floats(v, q);
@@ -295,6 +314,7 @@ __device__ __noinline__ void quantize_slot(const DecodeParams& p, int slot) {
     dst[2] = make_uint4(q.od[0], q.od[1], q.od[2], q.od[3]);
     dst[3] = make_uint4(q.od[4], q.od[5], q.od[6], q.od[7]);
     reinterpret_cast<float*>(table + ngroups * 64)[gi] = q.f;
+    }
   }
   __syncwarp();
   if (lane == 0) st_release(p.ctrl + kCtrlHqReady + slot, 1u);
@@ -398,44 +418,52 @@ __device__ __noinline__ void run_select(const DecodeParams& p, Smem& S) {
   }
   const unsigned kept_mask = __ballot_sync(0xffffffffu, lane < G && rank < p.topk_group);
   const bool kept = (kept_mask >> (lane / L)) & 1u;
-  // top_k over the kept experts
-  uint32_t taken = 0;
-  uint32_t bk = 0;
-  int bj = 0;
-  auto local_best = [&]() {
-    bk = 0;
-    bj = 0;
+  // top_k over the kept experts: each lane sorts its candidates once
+  // (descending key; equal keys keep the lower id first), then every round
+  // is two warp reductions and a pop from the winning lane's list
+  uint32_t key[kQ];
+  int jid[kQ];
 #pragma unroll
-    for (int j = 0; j < kQ; ++j) {
-      if (j < nmine && kept && !((taken >> j) & 1u)) {
-        const uint32_t key = order_key(sp[j]);
-        if (key > bk) {
-          bk = key;
-          bj = j;
-        }
-      }
+  for (int j = 0; j < kQ; ++j) {
+    key[j] = (j < nmine && kept) ? order_key(sp[j]) : 0u;
+    jid[j] = j;
+  }
+#pragma unroll
+  for (int a = 1; a < kQ; ++a) {  // insertion sort, fully unrolled
+#pragma unroll
+    for (int b = a; b > 0; --b) {
+      const bool sw = key[b] > key[b - 1];
+      const uint32_t k0 = key[b - 1], k1 = key[b];
+      const int j0 = jid[b - 1], j1 = jid[b];
+      key[b - 1] = sw ? k1 : k0;
+      key[b] = sw ? k0 : k1;
+      jid[b - 1] = sw ? j1 : j0;
+      jid[b] = sw ? j0 : j1;
     }
-  };
-  local_best();
+  }
   int my_sel = -1;
   float my_s = 0.f;
   for (int r = 0; r < p.k; ++r) {
-    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
-    const uint32_t cand = (bk == m && m != 0) ? (uint32_t)(lane * q + bj) : 0xFFFFFFFFu;
+    const uint32_t m = __reduce_max_sync(0xffffffffu, key[0]);
+    const uint32_t cand = (key[0] == m && m != 0) ? (uint32_t)(lane * q + jid[0]) : 0xFFFFFFFFu;
     const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
     const int owner = (int)(win / (uint32_t)q);
-    float s_win = 0.f;
+    float s_head = 0.f;
 #pragma unroll
     for (int j = 0; j < kQ; ++j)
-      if (j == bj) s_win = sc[j];
-    s_win = __shfl_sync(0xffffffffu, s_win, owner);
+      if (j == jid[0]) s_head = sc[j];
+    const float s_win = __shfl_sync(0xffffffffu, s_head, owner);
     if (lane == r) {
       my_sel = (int)win;
       my_s = s_win;
     }
-    if (lane == owner) {
-      taken |= 1u << bj;
-      local_best();
+    if (lane == owner) {  // pop the head
+#pragma unroll
+      for (int j = 0; j + 1 < kQ; ++j) {
+        key[j] = key[j + 1];
+        jid[j] = jid[j + 1];
+      }
+      key[kQ - 1] = 0u;
     }
   }
   // ascending ids; weights from the unbiased scores
