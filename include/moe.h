@@ -153,6 +153,34 @@ moe_status moe_layer_forward(const moe_layer* layer, const void* x_dev, int T,
                              float* w_out_dev, void* ws_dev, size_t ws_bytes,
                              void* stream);
 
+/* moe_layer_forward for one token (T = 1) without a caller workspace, so
+ * that the call allocates no device memory: its scratch is a fixed
+ * 512 KiB array in the library's device image (one per device), and the
+ * call makes no cudaMalloc, cudaFree or other allocating call.  The pages
+ * have no counterpart to this entry point; it exists for callers that may
+ * not allocate (for example while another component owns the allocator).
+ *   x_dev bf16 [hidden]; y_dev fp32 [hidden]; idx_out_dev int32 [top_k] and
+ *   w_out_dev fp32 [top_k] nullable, as in moe_layer_forward.
+ *   status_out_dev (nullable) uint32: after the kernel, the device error word
+ *   of this call (0 = none; 1 = expert id out of range, 2 = a device-side
+ *   wait ran out), written on `stream`.
+ * Results are bitwise those of moe_layer_forward(layer, x_dev, 1, ...).
+ * Shapes whose one-token workspace, moe_workspace_bytes(cfg, 1), exceeds
+ * 512 KiB are refused with MOE_ERR_UNSUPPORTED.  The current device must be
+ * the layer's.  Each call first clears the array's control words on
+ * `stream`, then runs the same kernels as moe_layer_forward.
+ * The first call on each device resolves the array's address
+ * (cudaGetSymbolAddress, which may load the module) and sets the decode
+ * kernel's shared-memory attribute: make it before any stream capture.
+ * All calls on one device share the one array: calls that can overlap on
+ * the device (different streams, or host threads without ordering between
+ * them) race on it and give undefined results; calls on one stream are
+ * ordered and safe. */
+moe_status moe_layer_forward_noalloc(const moe_layer* layer, const void* x_dev,
+                                     float* y_dev, int32_t* idx_out_dev,
+                                     float* w_out_dev, uint32_t* status_out_dev,
+                                     void* stream);
+
 /* ---- stacked layers (pre-norm residual stream) --------------------------- */
 
 /* One decoder MoE step on an fp32 residual stream (the reading of a stack of

@@ -78,6 +78,8 @@ def lib():
         L.moe_expert_ffn.argtypes = [p, p, i, p, p, p, p, sz, p]
         L.moe_layer_forward.restype = st
         L.moe_layer_forward.argtypes = [p, p, i, p, p, p, p, sz, p]
+        L.moe_layer_forward_noalloc.restype = st
+        L.moe_layer_forward_noalloc.argtypes = [p, p, p, p, p, p, p]
         L.moe_layer_forward_residual.restype = st
         L.moe_layer_forward_residual.argtypes = [p, p, p, p, p, p, ctypes.c_float, p, sz, p]
         L.moe_stack_forward.restype = st
@@ -185,6 +187,15 @@ class Layer:
         check(lib().moe_layer_forward(self.handle, _ptr(x), T, _ptr(y), _ptr(idx), _ptr(w),
                                       _ptr(ws), ws.numel(), _stream(stream)),
               "moe_layer_forward")
+
+
+def forward_noalloc(layer, x, y, idx=None, w=None, status=None, stream=None):
+    """Layer.forward for one token with the library's fixed scratch array
+    (no workspace argument, no device allocation).  status: optional int32
+    device tensor of one element that receives the device error word."""
+    check(lib().moe_layer_forward_noalloc(layer.handle, _ptr(x), _ptr(y), _ptr(idx), _ptr(w),
+                                          _ptr(status), _stream(stream)),
+          "moe_layer_forward_noalloc")
 
 
 NORM_EPS = 1e-6

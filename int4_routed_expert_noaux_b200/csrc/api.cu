@@ -24,6 +24,8 @@ moe_status fail(moe_status s, const char* fmt, ...) {
   return s;
 }
 
+void clear_last_error() { g_last_error[0] = 0; }
+
 moe_status cuda_fail(cudaError_t e, const char* what) {
   return fail(e == cudaErrorMemoryAllocation ? MOE_ERR_OOM : MOE_ERR_CUDA, "%s: %s", what,
               cudaGetErrorString(e));
@@ -60,7 +62,7 @@ moe_status check_config(const moe_config* c) {
   return MOE_OK;
 }
 
-static moe_status check_device_ptr(const void* p, size_t align, const char* name) {
+moe_status check_device_ptr(const void* p, size_t align, const char* name) {
   if (!p) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", name);
   if (reinterpret_cast<uintptr_t>(p) % align)
     return fail(MOE_ERR_INVALID_ARG, "%s is not %zu-byte aligned", name, align);

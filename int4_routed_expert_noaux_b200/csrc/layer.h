@@ -31,8 +31,10 @@ struct WsLayout {
 WsLayout ws_layout(const moe_config* c, int T);
 moe_status fail(moe_status s, const char* fmt, ...);
 moe_status cuda_fail(cudaError_t e, const char* what);
+void clear_last_error();
 moe_status check_config(const moe_config* c);
 moe_status check_expert(const moe_expert* e, const char* what);
+moe_status check_device_ptr(const void* p, size_t align, const char* name);
 ExpertPtrs to_ptrs(const moe_expert& e);
 
 moe_status route_impl(const moe_layer* l, const uint16_t* x, int T, int32_t* idx, float* w,
