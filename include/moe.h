@@ -115,9 +115,11 @@ moe_status moe_layer_set_expert(moe_layer* layer, int e,
 /* ---- workspace --------------------------------------------------------- */
 
 /* Bytes of device workspace a call with T tokens needs.  The workspace must
- * be 256-byte aligned and zero-filled before its first use; every call that
- * returns MOE_OK leaves its control words zero again.  One workspace must not
- * be used by two calls that can run at the same time. */
+ * be 256-byte aligned and zero-filled before its first use, and the caller
+ * must not write it between calls (moe_ws_check aside): the fused kernel
+ * leaves its counters zero after every call but keeps a call count and the
+ * router score records, tagged with that count, from call to call.  One
+ * workspace must not be used by two calls that can run at the same time. */
 size_t moe_workspace_bytes(const moe_config* cfg, int T);
 
 /* Synchronise the stream, then read the device error word of a workspace.
@@ -167,11 +169,12 @@ moe_status moe_layer_forward(const moe_layer* layer, const void* x_dev, int T,
  * Results are bitwise those of moe_layer_forward(layer, x_dev, 1, ...).
  * Shapes whose one-token workspace, moe_workspace_bytes(cfg, 1), exceeds
  * 512 KiB are refused with MOE_ERR_UNSUPPORTED.  The current device must be
- * the layer's.  Each call first clears the array's control words on
- * `stream`, then runs the same kernels as moe_layer_forward.
+ * the layer's.  Each call first clears the array's error word on `stream`,
+ * then runs the same kernels as moe_layer_forward.
  * The first call on each device resolves the array's address
- * (cudaGetSymbolAddress, which may load the module) and sets the decode
- * kernel's shared-memory attribute: make it before any stream capture.
+ * (cudaGetSymbolAddress, which may load the module), zero-fills the array's
+ * control words on `stream` and sets the decode kernel's shared-memory
+ * attribute: make it before any stream capture.
  * All calls on one device share the one array: calls that can overlap on
  * the device (different streams, or host threads without ordering between
  * them) race on it and give undefined results; calls on one stream are

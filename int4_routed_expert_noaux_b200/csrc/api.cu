@@ -102,7 +102,8 @@ WsLayout ws_layout(const moe_config* c, int T) {
   L.ctrl = off;
   off += kCtrlBytes;
   L.logits = off;
-  off = align_up(off + (size_t)T * c->n_experts * 4, 256);
+  // router logits of the step kernels, or the fused kernel's score records
+  off = align_up(off + (size_t)T * c->n_experts * 8, 256);
   L.idx = off;
   off = align_up(off + (size_t)T * k * 4, 256);
   L.w = off;
@@ -112,7 +113,6 @@ WsLayout ws_layout(const moe_config* c, int T) {
   L.ypart = off;
   off = align_up(off + (size_t)T * slots * c->hidden * 4, 256);
   L.hq = off;
-  off = align_up(off + (size_t)T * slots * (c->inter / 32) * 68, 256);
   L.total = off;
   return L;
 }

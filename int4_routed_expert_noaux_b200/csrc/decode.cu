@@ -3,7 +3,8 @@
 // int4 expert FFNs, weighted combine) in ONE launch.
 //
 // Design (sm_100a):
-//  * one CTA per SM: a producer warp and two consumer groups of 6 warps;
+//  * one CTA per SM: a producer warp, a selection warp and two consumer
+//    groups of 6 warps;
 //  * the producer claims work items from a global ticket counter, in a fixed
 //    order, and moves each item's weights HBM -> shared memory with 1-D bulk
 //    async copies (the TMA engine) into a 4-stage ring of 54 KB stages,
@@ -14,24 +15,26 @@
 //    column of the rows it visits and keeps its 32 inputs in registers as
 //    int16 fixed point with one exponent per group; the int4 group dot
 //    product is exact in integers (dp2a); one butterfly reduce-scatter plus
-//    a cross-warp sum finishes each row; one named barrier per item;
-//  * each CTA first computes its own block of router rows (a static
-//    split of the experts over the grid, the CTA's first fill); the CTA
-//    that finishes the last block runs the selection and publishes idx / w
-//    with a release flag; the producer acquires it before loading routed
-//    weights;
-//  * then work items come from a global ticket counter in the order:
-//    shared-expert gate/up, routed gate/up of slots 0..k-1, routed down of
-//    slots 0..k-2, shared-expert down, routed down of slot k-1.  Every
-//    dependency points to an earlier ticket, so in-order claiming always
-//    makes progress, and every slot's down items come well after its
-//    gate/up items;
-//  * gate/up finalizer warps publish h rows and count themselves done; the
-//    warp that completes a slot (it looks before its next wait, never after,
-//    so no fill can depend on it) converts the slot's h to int16 groups once
-//    (a 4.3 KB table for the GLM shape) and flags it; the producer acquires
-//    the flag and bulk-copies the table into the tail of each down item's
-//    stage, so down consumers read their inputs from shared memory;
+//    a cross-warp sum finishes each row; one group barrier per item;
+//  * each CTA first computes its own block of router rows (a static split
+//    of the experts over the first CTAs, the CTA's first fill) and
+//    publishes each row's sigmoid score as a 64-bit record tagged with the
+//    call's epoch (one single-copy-atomic store: no flag, no fence);
+//  * a selection warp in every CTA polls the E records until all carry this
+//    call's epoch and runs the noaux_tc selection itself (every CTA reads the
+//    same scores with the same code, so all reach the same bits); it hands
+//    the expert ids and weights to its producer and consumers through
+//    shared memory;
+//  * work items come from a global ticket counter in the order:
+//    shared-expert gate/up, shared-expert down, routed gate/up of slots
+//    0..k-1, routed down of slots 0..k-1.  Every dependency points to an
+//    earlier ticket, so in-order claiming always makes progress; the shared
+//    expert's items keep HBM busy while the routed experts are selected;
+//  * gate/up finalizer warps publish h rows (fp32) and count themselves done
+//    with a release add (nothing waits on its result); the producer waits
+//    until a slot's count is complete and bulk-copies the slot's h (8 KB for
+//    the GLM shape, from L2) into the tail of each down item's stage; down
+//    consumers convert their own 32-row group of h to int16 fixed point;
 //  * down items write per-slot partial rows; the warp whose release add
 //    completes a row block (checked one item later, off the critical path)
 //    sums the partials in slot order (deterministic, no atomics on data)
@@ -53,8 +56,9 @@ namespace {
 constexpr int kGW = 6;                   // warps per consumer group
 constexpr int kGT = kGW * 32;            // threads per consumer group
 constexpr int kGroups = 2;
-constexpr int kThreads = kGroups * kGT + 32;
+constexpr int kThreads = kGroups * kGT + 64;
 constexpr int kProducerWarp = kGroups * kGW;
+constexpr int kSelectWarp = kProducerWarp + 1;
 constexpr int kStages = 4;
 constexpr uint32_t kStageBytes = 55296;
 constexpr int kRouterChunks = 8;         // 16-byte W chunks per thread per row
@@ -73,7 +77,11 @@ struct Smem {
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t gbar[kGroups];  // per-group item barrier (one arrival per warp)
+  uint64_t selbar;         // the selection warp has published sel_*
   ItemDesc desc[kStages];
+  int sel_idx[kMaxSlots];  // selected expert ids, ascending
+  float sel_w[kMaxSlots];  // their combine weights
+  int sel_ok;
   float red[kGroups][2][kGW][32];
   int abort_flag[kGroups];
   float norm_part[kThreads / 32];
@@ -94,9 +102,7 @@ __device__ __forceinline__ ItemDesc make_item(int type, int slot, int row0, int 
 }
 
 __device__ ItemDesc decode_ticket(const DecodeParams& p, int t) {
-  // shared gate/up, routed gate/up 0..k-1, routed down 0..k-2, shared down,
-  // routed down k-1: the shared expert's down items (ready early) sit between
-  // the last routed slot's gate/up and its down items.
+  // shared gate/up, shared down, routed gate/up 0..k-1, routed down 0..k-1
   auto gu = [&](int slot, int b) {
     return make_item(kGateUp, slot, b * p.RG, min(p.RG, p.I - b * p.RG));
   };
@@ -106,23 +112,25 @@ __device__ ItemDesc decode_ticket(const DecodeParams& p, int t) {
   if (p.has_shared) {
     if (t < p.nG) return gu(p.k, t);
     t -= p.nG;
-  }
-  if (t < p.k * p.nG) return gu(t / p.nG, t % p.nG);
-  t -= p.k * p.nG;
-  if (t < (p.k - 1) * p.nD) return dn(t / p.nD, t % p.nD);
-  t -= (p.k - 1) * p.nD;
-  if (p.has_shared) {
     if (t < p.nD) return dn(p.k, t);
     t -= p.nD;
   }
-  if (t < p.nD) return dn(p.k - 1, t);
+  if (t < p.k * p.nG) return gu(t / p.nG, t % p.nG);
+  t -= p.k * p.nG;
+  if (t < p.k * p.nD) return dn(t / p.nD, t % p.nD);
   return make_item(kDone, 0, 0, 0);
 }
 
-// Router rows of CTA b: a static split of the E experts over the grid.
+// Router rows of CTA b: a static split of the E experts over the first nR
+// CTAs (every one of them gets at least one row).
 __device__ __forceinline__ void router_rows(const DecodeParams& p, int b, int& r0, int& nr) {
-  r0 = (int)(((long long)b * p.E) / gridDim.x);
-  nr = (int)(((long long)(b + 1) * p.E) / gridDim.x) - r0;
+  if (b >= p.nR) {
+    r0 = p.E;
+    nr = 0;
+    return;
+  }
+  r0 = (int)(((long long)b * p.E) / p.nR);
+  nr = (int)(((long long)(b + 1) * p.E) / p.nR) - r0;
 }
 
 // Record an error: the first one also records where it happened (CTA,
@@ -180,31 +188,12 @@ __device__ __forceinline__ ArgMaxF am_warp(ArgMaxF a) {
   return a;
 }
 
-// Selection for shapes whose groups do not align with lanes: scores staged
-// in shared memory, one lane per group, repeated warp arg-max.
+// Selection for shapes whose groups do not align with lanes: one lane per
+// group, repeated warp arg-max over S.sp / S.sc.  Results go to
+// S.sel_idx / S.sel_w (and, from CTA 0, to the caller's idx_out / w_out).
 __device__ __noinline__ void run_select_generic(const DecodeParams& p, Smem& S) {
   const int lane = threadIdx.x & 31;
   const int per = p.E / p.n_group;
-  {
-    // issue every load of this lane before using any (one L2 round trip)
-    float lg[kMaxE / 32], bs[kMaxE / 32];
-#pragma unroll
-    for (int m = 0; m < kMaxE / 32; ++m) {
-      const int e = lane + 32 * m;
-      lg[m] = (e < p.E) ? __ldcg(p.logits + e) : 0.f;
-      bs[m] = (e < p.E) ? __ldg(p.bias + e) : 0.f;
-    }
-#pragma unroll
-    for (int m = 0; m < kMaxE / 32; ++m) {
-      const int e = lane + 32 * m;
-      if (e < p.E) {
-        const float s = 1.0f / (1.0f + expf(-lg[m]));
-        S.sc[e] = s;
-        S.sp[e] = s + bs[m];
-      }
-    }
-  }
-  __syncwarp();
   // group score: sum of the two largest bias-corrected scores (lane = group)
   float gs = 0.f;
   if (lane < p.n_group) {
@@ -265,59 +254,13 @@ __device__ __noinline__ void run_select_generic(const DecodeParams& p, Smem& S) 
   denom += 1e-20f;
   if (lane < p.k) {
     const float wv = p.rsf * s_mine / denom;
-    p.idx_ws[pos] = my_sel;
-    p.w_ws[pos] = wv;
-    if (p.idx_out) p.idx_out[pos] = my_sel;
-    if (p.w_out) p.w_out[pos] = wv;
-  }
-  __syncwarp();
-  if (lane == 0) st_release(p.ctrl + kCtrlSelReady, 1u);
-}
-
-// Convert h of one slot (fp32 [I], complete) to int16 groups, by one warp:
-// the table holds, per 32-row group, the 16 words of XQ.ev/od and then, after
-// all groups, one factor per group.  Flags the slot ready for the producers.
-__device__ __noinline__ void quantize_slot(const DecodeParams& p, int slot) {
-  const int lane = threadIdx.x & 31;
-  const int ngroups = p.I >> 5;
-  if (lane == 0) fence_acq_rel();  // see every gate/up warp's h rows
-  __syncwarp();
-  const float* h = p.hbuf + (size_t)slot * p.I;
-  uint8_t* table = reinterpret_cast<uint8_t*>(p.hq) + (size_t)slot * ngroups * 68;
-  for (int gi0 = lane; gi0 < ngroups; gi0 += 64) {
-    // two groups per pass, all loads issued before any is used
-    float4 raw[2][8];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int gi = gi0 + 32 * u;
-      const float4* hp = reinterpret_cast<const float4*>(h + (size_t)min(gi, ngroups - 1) * 32);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) raw[u][i] = __ldcg(hp + i);
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-    const int gi = gi0 + 32 * u;
-    if (gi >= ngroups) break;
-    float v[32];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[4 * i] = raw[u][i].x;
-      v[4 * i + 1] = raw[u][i].y;
-      v[4 * i + 2] = raw[u][i].z;
-      v[4 * i + 3] = raw[u][i].w;
-    }
-    XQ q;
-    xq_from_floats(v, q);
-    uint4* dst = reinterpret_cast<uint4*>(table + gi * 64);
-    dst[0] = make_uint4(q.ev[0], q.ev[1], q.ev[2], q.ev[3]);
-    dst[1] = make_uint4(q.ev[4], q.ev[5], q.ev[6], q.ev[7]);
-    dst[2] = make_uint4(q.od[0], q.od[1], q.od[2], q.od[3]);
-    dst[3] = make_uint4(q.od[4], q.od[5], q.od[6], q.od[7]);
-    reinterpret_cast<float*>(table + ngroups * 64)[gi] = q.f;
+    S.sel_idx[pos] = my_sel;
+    S.sel_w[pos] = wv;
+    if (blockIdx.x == 0) {
+      if (p.idx_out) p.idx_out[pos] = my_sel;
+      if (p.w_out) p.w_out[pos] = wv;
     }
   }
-  __syncwarp();
-  if (lane == 0) st_release(p.ctrl + kCtrlHqReady + slot, 1u);
 }
 
 // bf16 bit pattern of layer input element i: x[i] itself, or, for a
@@ -329,7 +272,8 @@ __device__ __forceinline__ uint32_t input_bf16(const DecodeParams& p, int i, flo
 
 // Fixed-order combine of one row block of y from the per-slot partials, by
 // one warp, once every slot's down item of the block has published.
-__device__ __noinline__ void combine_block(const DecodeParams& p, int row0, int nrows) {
+__device__ __noinline__ void combine_block(const DecodeParams& p, const float* wsel, int row0,
+                                          int nrows) {
   const int lane = threadIdx.x & 31;
   if (lane == 0) fence_acq_rel();  // see the other warps' partials
   __syncwarp();
@@ -337,7 +281,7 @@ __device__ __noinline__ void combine_block(const DecodeParams& p, int row0, int 
     const int row = row0 + lr;
     float acc = 0.f;
     for (int j = 0; j < p.k; ++j)
-      acc = fmaf(__ldcg(p.w_ws + j), __ldcg(p.ypart + (size_t)j * p.H + row), acc);
+      acc = fmaf(wsel[j], __ldcg(p.ypart + (size_t)j * p.H + row), acc);
     if (p.has_shared) acc += __ldcg(p.ypart + (size_t)p.k * p.H + row);
     if (p.x_resid) acc = p.x_resid[row] + acc;  // residual stream: x + MoE(norm(x))
     p.y[row] = acc;
@@ -351,40 +295,48 @@ __device__ __forceinline__ uint32_t order_key(float v) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// noaux_tc selection over the E logits, by one warp ("LightLX", "How it
-// works": the noaux_tc sigmoid router; colibri summary, "Principales
-// fonctionnalites implementees": routed_scaling_factor).  Lane l owns the
-// q = ceil(E / 32) consecutive experts l*q .. l*q+q-1 in registers; when a
-// group's experts are exactly L = per / q consecutive lanes (L a power of
-// two), group top-2 is a segmented butterfly and the top-k is k rounds of
-// two warp reductions (max of the score key, then min of the expert id
-// among the lanes holding it: ties go to the lower id).
+// Compare-exchange of the per-lane candidate lists: position a before b in
+// the order (key descending, expert index ascending).
+__device__ __forceinline__ void cx(uint32_t (&key)[kMaxE / 32], int (&jid)[kMaxE / 32],
+                                   float (&sl)[kMaxE / 32], int a, int b) {
+  const bool sw = key[b] > key[a] || (key[b] == key[a] && jid[b] < jid[a]);
+  const uint32_t ka = key[a], kb = key[b];
+  const int ja = jid[a], jb = jid[b];
+  const float sa = sl[a], sb = sl[b];
+  key[a] = sw ? kb : ka;
+  key[b] = sw ? ka : kb;
+  jid[a] = sw ? jb : ja;
+  jid[b] = sw ? ja : jb;
+  sl[a] = sw ? sb : sa;
+  sl[b] = sw ? sa : sb;
+}
+
+// noaux_tc selection over S.sp (sigmoid + bias) and S.sc (sigmoid), by one
+// warp ("LightLX", "How it works": the noaux_tc sigmoid router; colibri
+// summary, "Principales fonctionnalites implementees": routed_scaling_factor).
+// Lane l owns the q = ceil(E / 32) consecutive experts l*q .. l*q+q-1 in
+// registers; when a group's experts are exactly L = per / q consecutive
+// lanes (L a power of two), group top-2 is a segmented butterfly, each lane
+// sorts its kept candidates with a sorting network, and the top-k is k
+// rounds of two warp reductions (max of the score key, then min of the
+// expert id among the lanes holding it: ties go to the lower id).  Results
+// go to S.sel_idx / S.sel_w (and, from CTA 0, to idx_out / w_out).
 __device__ __noinline__ void run_select(const DecodeParams& p, Smem& S) {
   const int lane = threadIdx.x & 31;
   const int E = p.E, per = E / p.n_group, q = (E + 31) >> 5;
   const int L = per / q;
-  if (per % q != 0 || L < 1 || (L & (L - 1)) != 0) {
+  constexpr int kQ = kMaxE / 32;
+  if (per % q != 0 || L < 1 || (L & (L - 1)) != 0 || q > kQ) {
     run_select_generic(p, S);
     return;
   }
-  constexpr int kQ = kMaxE / 32;
-  float sc[kQ], sp[kQ];
-  {
-    float lg[kQ], bs[kQ];
-#pragma unroll
-    for (int j = 0; j < kQ; ++j) {
-      const int e = lane * q + j;
-      const bool valid = j < q && e < E;
-      lg[j] = valid ? __ldcg(p.logits + e) : 0.f;
-      bs[j] = valid ? __ldg(p.bias + e) : 0.f;
-    }
-#pragma unroll
-    for (int j = 0; j < kQ; ++j) {
-      sc[j] = 1.0f / (1.0f + expf(-lg[j]));
-      sp[j] = sc[j] + bs[j];
-    }
-  }
   const int nmine = max(0, min(q, E - lane * q));  // experts this lane owns
+  float sc[kQ], sp[kQ];
+#pragma unroll
+  for (int j = 0; j < kQ; ++j) {
+    sp[j] = (j < nmine) ? S.sp[lane * q + j] : 0.f;
+    sc[j] = (j < nmine) ? S.sc[lane * q + j] : 0.f;
+  }
   // group score: the two largest sp of the group (lanes g*L .. g*L+L-1)
   float t1 = -INFINITY, t2 = -INFINITY;
 #pragma unroll
@@ -408,51 +360,46 @@ __device__ __noinline__ void run_select(const DecodeParams& p, Smem& S) {
     t2 = n2;
   }
   const float gs_seg = (per >= 2) ? t1 + t2 : t1;
-  // keep topk_group groups: rank by (score desc, index asc); lane g holds group g
+  // keep topk_group groups: rank by (score desc, index asc); lane g holds
+  // group g (n_group <= E / q <= 32); the shuffles are independent
   const int G = p.n_group;
   const float gs = __shfl_sync(0xffffffffu, gs_seg, (lane < G ? lane : 0) * L);
   int rank = 0;
-  for (int h = 0; h < G; ++h) {
-    const float o = __shfl_sync(0xffffffffu, gs, h);
-    if (o > gs || (o == gs && h < lane)) ++rank;
+#pragma unroll
+  for (int h = 0; h < 32; ++h) {
+    if (h < G) {
+      const float o = __shfl_sync(0xffffffffu, gs, h);
+      if (o > gs || (o == gs && h < lane)) ++rank;
+    }
   }
   const unsigned kept_mask = __ballot_sync(0xffffffffu, lane < G && rank < p.topk_group);
   const bool kept = (kept_mask >> (lane / L)) & 1u;
-  // top_k over the kept experts: each lane sorts its candidates once
-  // (descending key; equal keys keep the lower id first), then every round
-  // is two warp reductions and a pop from the winning lane's list
+  // each lane sorts its kept candidates once (a sorting network)
   uint32_t key[kQ];
   int jid[kQ];
+  float sl[kQ];
 #pragma unroll
   for (int j = 0; j < kQ; ++j) {
     key[j] = (j < nmine && kept) ? order_key(sp[j]) : 0u;
     jid[j] = j;
+    sl[j] = sc[j];
   }
-#pragma unroll
-  for (int a = 1; a < kQ; ++a) {  // insertion sort, fully unrolled
-#pragma unroll
-    for (int b = a; b > 0; --b) {
-      const bool sw = key[b] > key[b - 1];
-      const uint32_t k0 = key[b - 1], k1 = key[b];
-      const int j0 = jid[b - 1], j1 = jid[b];
-      key[b - 1] = sw ? k1 : k0;
-      key[b] = sw ? k0 : k1;
-      jid[b - 1] = sw ? j1 : j0;
-      jid[b] = sw ? j0 : j1;
-    }
-  }
+  static_assert(kQ == 8, "the network below sorts 8 candidates");
+  cx(key, jid, sl, 0, 1); cx(key, jid, sl, 2, 3); cx(key, jid, sl, 4, 5); cx(key, jid, sl, 6, 7);
+  cx(key, jid, sl, 0, 2); cx(key, jid, sl, 1, 3); cx(key, jid, sl, 4, 6); cx(key, jid, sl, 5, 7);
+  cx(key, jid, sl, 1, 2); cx(key, jid, sl, 5, 6);
+  cx(key, jid, sl, 0, 4); cx(key, jid, sl, 1, 5); cx(key, jid, sl, 2, 6); cx(key, jid, sl, 3, 7);
+  cx(key, jid, sl, 2, 4); cx(key, jid, sl, 3, 5);
+  cx(key, jid, sl, 1, 2); cx(key, jid, sl, 3, 4); cx(key, jid, sl, 5, 6);
+  // top_k: the best head, lowest expert id among equal heads, is popped
   int my_sel = -1;
   float my_s = 0.f;
   for (int r = 0; r < p.k; ++r) {
     const uint32_t m = __reduce_max_sync(0xffffffffu, key[0]);
-    const uint32_t cand = (key[0] == m && m != 0) ? (uint32_t)(lane * q + jid[0]) : 0xFFFFFFFFu;
+    const uint32_t cand = (key[0] == m && m != 0u) ? (uint32_t)(lane * q + jid[0]) : 0xFFFFFFFFu;
     const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
-    const int owner = (int)(win / (uint32_t)q);
-    float s_head = 0.f;
-#pragma unroll
-    for (int j = 0; j < kQ; ++j)
-      if (j == jid[0]) s_head = sc[j];
-    const float s_win = __shfl_sync(0xffffffffu, s_head, owner);
+    const int owner = __ffs(__ballot_sync(0xffffffffu, cand == win)) - 1;
+    const float s_win = __shfl_sync(0xffffffffu, sl[0], owner);
     if (lane == r) {
       my_sel = (int)win;
       my_s = s_win;
@@ -462,15 +409,19 @@ __device__ __noinline__ void run_select(const DecodeParams& p, Smem& S) {
       for (int j = 0; j + 1 < kQ; ++j) {
         key[j] = key[j + 1];
         jid[j] = jid[j + 1];
+        sl[j] = sl[j + 1];
       }
       key[kQ - 1] = 0u;
     }
   }
   // ascending ids; weights from the unbiased scores
   int pos = 0;
-  for (int j = 0; j < p.k; ++j) {
-    const int other = __shfl_sync(0xffffffffu, my_sel, j);
-    if (lane < p.k && other < my_sel) ++pos;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    if (j < p.k) {
+      const int other = __shfl_sync(0xffffffffu, my_sel, j);
+      if (lane < p.k && other < my_sel) ++pos;
+    }
   }
   float denom = (lane < p.k) ? my_s : 0.f;
 #pragma unroll
@@ -478,13 +429,13 @@ __device__ __noinline__ void run_select(const DecodeParams& p, Smem& S) {
   denom += 1e-20f;
   if (lane < p.k) {
     const float wv = p.rsf * my_s / denom;
-    p.idx_ws[pos] = my_sel;
-    p.w_ws[pos] = wv;
-    if (p.idx_out) p.idx_out[pos] = my_sel;
-    if (p.w_out) p.w_out[pos] = wv;
+    S.sel_idx[pos] = my_sel;
+    S.sel_w[pos] = wv;
+    if (blockIdx.x == 0) {
+      if (p.idx_out) p.idx_out[pos] = my_sel;
+      if (p.w_out) p.w_out[pos] = wv;
+    }
   }
-  __syncwarp();
-  if (lane == 0) st_release(p.ctrl + kCtrlSelReady, 1u);
 }
 
 // Lane holding reduce-scatter value `vi` of row phase `ph` (group-local warp).
@@ -556,6 +507,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       mbar_init(&S.empty[s], kGW);
     }
     for (int g = 0; g < kGroups; ++g) mbar_init(&S.gbar[g], kGW);
+    mbar_init(&S.selbar, 1);
+    S.sel_ok = 0;
     S.abort_flag[0] = S.abort_flag[1] = 0;
     fence_mbar_init();
   }
@@ -575,13 +528,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   }
   __syncthreads();
   const float inv_rms = p.x_resid ? S.inv_rms : 1.0f;
+  // this call's epoch: one more than the last finished call's
+  const uint32_t epoch = *reinterpret_cast<volatile const uint32_t*>(p.ctrl + kCtrlEpoch) + 1u;
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t policy = l2_policy_evict_first();
       bool sel_seen = false;
-      uint64_t hq_seen = 0;  // bit j: slot j's int16 h table acquired
+      uint64_t h_seen = 0;  // bit j: slot j's h acquired
       int dones = 0;
       int rr0, rnr;
       router_rows(p, blockIdx.x, rr0, rnr);
@@ -596,11 +551,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         } else if (dones == 0) {
           d = decode_ticket(p, t);
           if (d.type == kDown) {
-            // the slot's int16 h table must be published before it is copied
-            if (!((hq_seen >> d.slot) & 1ull)) {
-              if (wait_counter(p.ctrl, p.ctrl + kCtrlHqReady + d.slot, 1u)) {
-                hq_seen |= 1ull << d.slot;
-                fence_proxy_async();  // order the table's stores before the bulk read
+            // every gate/up item of the slot must have published its h rows
+            // before the slot's h is copied
+            if (!((h_seen >> d.slot) & 1ull)) {
+              if (wait_counter(p.ctrl, p.ctrl + kCtrlGuDone + d.slot, (uint32_t)p.gu_count)) {
+                h_seen |= 1ull << d.slot;
+                fence_proxy_async();  // order the h stores before the bulk read
               } else {
                 set_error(p.ctrl, kErrTimeout, 7, n);
                 d = make_item(kDone, 0, 0, 0);
@@ -610,7 +566,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           if (d.type == kGateUp || d.type == kDown) {
             if (d.slot < p.k) {
               if (!sel_seen) {
-                if (wait_counter(p.ctrl, p.ctrl + kCtrlSelReady, 1u)) {
+                // the selection warp's result (mbarrier: release / acquire)
+                if (mbar_wait(&S.selbar, 0u, global_timer_ns() + kWaitNs) && S.sel_ok) {
                   sel_seen = true;
                 } else {
                   set_error(p.ctrl, kErrTimeout, 4, n);
@@ -618,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
                 }
               }
               if (d.type != kDone) {
-                d.eid = __ldcg(p.idx_ws + d.slot);
+                d.eid = S.sel_idx[d.slot];
                 if (d.eid < 0 || d.eid >= p.E) {
                   set_error(p.ctrl, kErrBadExpertId, 5, n);
                   d = make_item(kDone, 0, 0, 0);
@@ -661,14 +618,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         } else if (d.type == kDown) {
           const ExpertPtrs ep = p.table[d.eid];
           const uint32_t qb = (uint32_t)d.nrows * (p.I / 2), sb = (uint32_t)d.nrows * (p.I / 16);
-          const uint32_t hb = (uint32_t)(p.I / 32) * 68;
+          const uint32_t hb = (uint32_t)p.I * 4;
           mbar_arrive_expect_tx(&S.full[stage], qb + sb + hb);
           bulk_g2s(dst, ep.q_down + (size_t)d.row0 * (p.I / 2), qb, &S.full[stage], policy);
           bulk_g2s(dst + p.RD * (p.I / 2), ep.s_down + (size_t)d.row0 * (p.I / 32), sb,
                    &S.full[stage], policy);
           bulk_g2s(dst + p.RD * (p.I / 2) + p.RD * (p.I / 16),
-                   reinterpret_cast<const uint8_t*>(p.hq) + (size_t)d.slot * hb, hb,
-                   &S.full[stage], l2_policy_evict_last());
+                   p.hbuf + (size_t)d.slot * p.I, hb, &S.full[stage], l2_policy_evict_last());
         } else {
           mbar_arrive(&S.full[stage]);  // a DONE fill: one per consumer group
           if (++dones == kGroups) {
@@ -683,6 +639,63 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         }
         t = (int)atomicAdd(p.ctrl + kCtrlTicket, 1u);
       }
+    }
+  } else if (warp == kSelectWarp) {
+    // ------------------------------------------------------------ selection
+    // the bias of this lane's experts (e = lane + 32 m), fetched while the
+    // router runs; then poll the score records until every one carries this
+    // call's epoch (bounded)
+    float bs[kMaxE / 32];
+#pragma unroll
+    for (int m = 0; m < kMaxE / 32; ++m) {
+      const int e = lane + 32 * m;
+      bs[m] = e < p.E ? __ldg(p.bias + e) : 0.f;
+    }
+    uint64_t rec[kMaxE / 32];
+    bool ok = true;
+    {
+      const uint64_t deadline = global_timer_ns() + kWaitNs;
+      uint32_t sleep_ns = 32;
+      for (uint32_t it = 0;; ++it) {
+#pragma unroll
+        for (int m = 0; m < kMaxE / 32; ++m) {
+          const int e = lane + 32 * m;
+          rec[m] = e < p.E ? ld_relaxed_u64(p.scores + e) : (uint64_t)epoch << 32;
+        }
+        bool mine = true;
+#pragma unroll
+        for (int m = 0; m < kMaxE / 32; ++m) mine = mine && (uint32_t)(rec[m] >> 32) == epoch;
+        if (__all_sync(0xffffffffu, mine)) break;
+        if ((it & 7) == 7) {
+          const int stop = lane == 0 && (aborted(p.ctrl) || global_timer_ns() > deadline);
+          if (__shfl_sync(0xffffffffu, stop, 0)) {
+            ok = false;
+            break;
+          }
+        }
+        __nanosleep(sleep_ns);
+        if (sleep_ns < 256) sleep_ns <<= 1;
+      }
+    }
+    if (ok) {
+#pragma unroll
+      for (int m = 0; m < kMaxE / 32; ++m) {
+        const int e = lane + 32 * m;
+        if (e < p.E) {
+          const float s = __uint_as_float((uint32_t)rec[m]);
+          S.sc[e] = s;
+          S.sp[e] = s + bs[m];
+        }
+      }
+      __syncwarp();
+      run_select(p, S);
+    } else if (lane == 0) {
+      set_error(p.ctrl, kErrTimeout, 8, 0);
+    }
+    __syncwarp();
+    if (lane == 0) {
+      S.sel_ok = ok ? 1 : 0;
+      mbar_arrive(&S.selbar);
     }
   } else {
     // ------------------------------------------------------------ consumers
@@ -724,8 +737,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     }
     int& gabort = S.abort_flag[grp];
     int pend_row0 = -1, pend_nrows = 0;  // this warp's last down row block
-    int pend_gu = -1;                    // slot of this warp's last gate/up item
-    uint32_t pend_gu_old = 0;            // gate/up count before this warp's add
     uint32_t pend_old = 0;               // count before this warp's add (lane 0)
     // Group 0 of a CTA with router rows: fill 0 is the router block.  It is
     // handled before the main loop so its bf16 inputs are dead afterwards.
@@ -795,36 +806,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           gabort = 1;
         }
         if (!gabort && gw == 0) {
+          // the sigmoid score of each row, tagged with this call's epoch
           if (lane < d.nrows) {
             float v = 0.f;
             for (int w = 0; w < kGW; ++w) v += S.red[grp][rbuf][w][lane];
-            p.logits[d.row0 + lane] = v;
-          }
-          __syncwarp();
-          uint32_t last = 0;
-          if (lane == 0) {
-            last = (atom_add_release(p.ctrl + kCtrlRouterDone, 1u) + 1 == (uint32_t)p.nR);
-            if (last) fence_acq_rel();  // see every block's logits
-          }
-          last = __shfl_sync(0xffffffffu, last, 0);
-          if (last) {
-            __syncwarp();
-            run_select(p, S);
+            const float sg = 1.0f / (1.0f + expf(-v));
+            st_relaxed_u64(p.scores + d.row0 + lane,
+                           ((uint64_t)epoch << 32) | __float_as_uint(sg));
           }
         }
       }
     }
     for (uint32_t c = c_first;; ++c) {
       if (gabort) break;
-      // A slot completed by this warp's previous gate/up item is converted
-      // before waiting for the next fill: the producer may hold that fill
-      // back until the conversion is published.
-      if (pend_gu >= 0) {
-        const uint32_t last =
-            __shfl_sync(0xffffffffu, pend_gu_old + 1 == (uint32_t)(p.nG * fw_g), 0);
-        if (last) quantize_slot(p, pend_gu);
-        pend_gu = -1;
-      }
       const uint32_t n = 2 * c + grp;  // fill number consumed
       const int stage = (int)(n % kStages);
       const uint32_t par = (n / kStages) & 1u;
@@ -878,42 +872,43 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         if (pend_row0 >= 0) {
           const uint32_t last =
               __shfl_sync(0xffffffffu, pend_old + 1 == (uint32_t)(slots * fw_d), 0);
-          if (last) combine_block(p, pend_row0, pend_nrows);
+          if (last) combine_block(p, S.sel_w, pend_row0, pend_nrows);
           pend_row0 = -1;
         }
 
         if (gw < fw_g) {
-          if (tg < cg.P * NR_G) {
+          // item row tg (= phase * NR_G + i) of this finalizer thread
+          if (tg < cg.P * NR_G && tg < d.nrows) {
             const int ph = tg / NR_G, i = tg % NR_G;
-            const int lr = ph * NR_G + i;
-            if (lr < d.nrows) {
-              int w0, lg, lu;
-              owner_of<NV_G, SEG_G>(ph, i, cg.wpr, w0, lg);
-              owner_of<NV_G, SEG_G>(ph, i + NR_G, cg.wpr, w0, lu);
-              float g = 0.f, u = 0.f;
-              for (int w = 0; w < cg.wpr; ++w) {
-                g += S.red[grp][rbuf][w0 + w][lg];
-                u += S.red[grp][rbuf][w0 + w][lu];
-              }
-              p.hbuf[(size_t)d.slot * p.I + d.row0 + lr] = silu_mul(g, u);
+            int w0, lg, lu;
+            owner_of<NV_G, SEG_G>(ph, i, cg.wpr, w0, lg);
+            owner_of<NV_G, SEG_G>(ph, i + NR_G, cg.wpr, w0, lu);
+            float g = 0.f, u = 0.f;
+            for (int w = 0; w < cg.wpr; ++w) {
+              g += S.red[grp][rbuf][w0 + w][lg];
+              u += S.red[grp][rbuf][w0 + w][lu];
             }
+            p.hbuf[(size_t)d.slot * p.I + d.row0 + tg] = silu_mul(g, u);
           }
           __syncwarp();
-          // count this warp done; the result is looked at before the next wait
-          if (lane == 0) pend_gu_old = atom_add_release(p.ctrl + kCtrlGuDone + d.slot, 1u);
-          pend_gu = d.slot;
+          // count this warp done (nothing waits for the result)
+          if (lane == 0) red_add_release(p.ctrl + kCtrlGuDone + d.slot, 1u);
         }
       } else {  // kDown
-        XQ hq;
+        XQ hq;  // this thread's 32-row group of h, as int16 fixed point
         {
-          const uint8_t* tab = st + (size_t)p.RD * (p.I / 2) + (size_t)p.RD * (p.I / 16);
-          const uint4* src = reinterpret_cast<const uint4*>(tab + cd.col * 64);
-          const uint4 a0 = src[0], a1 = src[1], a2 = src[2], a3 = src[3];
-          hq.ev[0] = a0.x; hq.ev[1] = a0.y; hq.ev[2] = a0.z; hq.ev[3] = a0.w;
-          hq.ev[4] = a1.x; hq.ev[5] = a1.y; hq.ev[6] = a1.z; hq.ev[7] = a1.w;
-          hq.od[0] = a2.x; hq.od[1] = a2.y; hq.od[2] = a2.z; hq.od[3] = a2.w;
-          hq.od[4] = a3.x; hq.od[5] = a3.y; hq.od[6] = a3.z; hq.od[7] = a3.w;
-          hq.f = reinterpret_cast<const float*>(tab + GD * 64)[cd.col];
+          const float4* hs = reinterpret_cast<const float4*>(
+              st + (size_t)p.RD * (p.I / 2) + (size_t)p.RD * (p.I / 16)) + cd.col * 8;
+          float hv[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 t = hs[i];
+            hv[4 * i] = t.x;
+            hv[4 * i + 1] = t.y;
+            hv[4 * i + 2] = t.z;
+            hv[4 * i + 3] = t.w;
+          }
+          xq_from_floats(hv, hq);
         }
         float v[NR_D];
         const size_t rb = (size_t)p.I / 2;
@@ -936,7 +931,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         if (pend_row0 >= 0) {
           const uint32_t last =
               __shfl_sync(0xffffffffu, pend_old + 1 == (uint32_t)(slots * fw_d), 0);
-          if (last) combine_block(p, pend_row0, pend_nrows);
+          if (last) combine_block(p, S.sel_w, pend_row0, pend_nrows);
           pend_row0 = -1;
         }
 
@@ -961,15 +956,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         }
       }
     }
-    // a slot or row block completed by this warp's last items
-    if (!gabort && pend_gu >= 0) {
-      const uint32_t last =
-          __shfl_sync(0xffffffffu, pend_gu_old + 1 == (uint32_t)(p.nG * fw_g), 0);
-      if (last) quantize_slot(p, pend_gu);
-    }
+    // a row block completed by this warp's last down item
     if (!gabort && pend_row0 >= 0) {
       const uint32_t last = __shfl_sync(0xffffffffu, pend_old + 1 == (uint32_t)(slots * fw_d), 0);
-      if (last) combine_block(p, pend_row0, pend_nrows);
+      if (last) combine_block(p, S.sel_w, pend_row0, pend_nrows);
     }
   }
 
@@ -980,18 +970,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     const uint32_t old = atomicAdd(p.ctrl + kCtrlExit, 1u);
     if (old + 1 == gridDim.x) {
       // last CTA out: reset the counters for the next call (the error word
-      // is left for the host to read)
+      // is left for the host to read) and advance the epoch
       __threadfence();
       volatile uint32_t* c = p.ctrl;
       c[kCtrlTicket] = 0;
-      c[kCtrlRouterDone] = 0;
-      c[kCtrlSelReady] = 0;
       c[kCtrlAbort] = 0;
-      for (int j = 0; j < slots; ++j) {
-        c[kCtrlGuDone + j] = 0;
-        c[kCtrlHqReady + j] = 0;
-      }
+      for (int j = 0; j < slots; ++j) c[kCtrlGuDone + j] = 0;
       for (int b = 0; b < p.nD; ++b) c[kCtrlRbDone + b] = 0;
+      c[kCtrlEpoch] = epoch;
       c[kCtrlExit] = 0;
       __threadfence();
     }
@@ -1079,8 +1065,8 @@ bool decode_plan(const moe_config& c, DecodeParams& p) {
   p.RG = PG * nrg;
   p.RD = PD * nrd;
   {
-    // a down item also carries the slot's int16 h table (68 bytes per group)
-    const size_t hb = (size_t)GD * 68, rowb = (size_t)c.inter / 2 + c.inter / 16;
+    // a down item also carries the slot's fp32 h
+    const size_t hb = (size_t)c.inter * 4, rowb = (size_t)c.inter / 2 + c.inter / 16;
     const int fit = (int)((kStageBytes - hb) / rowb);
     if (fit < p.RD) p.RD = fit & ~3;
     if (p.RD < 4 || hb % 16) return false;
@@ -1089,16 +1075,18 @@ bool decode_plan(const moe_config& c, DecodeParams& p) {
   if (p.RR > kMaxRR) p.RR = kMaxRR;
   if (p.RR < 1) return false;
   if ((size_t)p.RG * (c.hidden / 2 + c.hidden / 16) * 2 > kStageBytes) return false;
-  if ((size_t)p.RD * (c.inter / 2 + c.inter / 16) + (size_t)GD * 68 > kStageBytes) return false;
+  if ((size_t)p.RD * (c.inter / 2 + c.inter / 16) + (size_t)c.inter * 4 > kStageBytes) return false;
   if ((p.RG * (c.hidden / 16)) % 16 || (p.RD * (c.inter / 16)) % 16) return false;
   const int grid = num_sms();
   if ((p.E + grid - 1) / grid > p.RR) return false;  // a CTA's router rows fill one stage
   p.nR = p.E < grid ? p.E : grid;  // CTAs with at least one router row
   p.nG = (p.I + p.RG - 1) / p.RG;
   p.nD = (p.H + p.RD - 1) / p.RD;
-  if (kCtrlRbDone + p.nD > (int)(kCtrlBytes / 4)) return false;
-  if (p.k + p.has_shared > kMaxSlots || p.k + p.has_shared > kCtrlHqReady - kCtrlGuDone)
-    return false;
+  p.gu_count = p.nG * ((p.RG + 31) / 32);  // finalizer warps per item: ceil(RG / 32)
+  const int slots = p.k + p.has_shared;
+  // the control words' ranges
+  if (slots > kMaxSlots || slots > kCtrlRbDone - kCtrlGuDone) return false;
+  if (p.nD > kCtrlWords - kCtrlRbDone) return false;
   p.n_items = p.nR + (p.k + p.has_shared) * (p.nG + p.nD);
   return true;
 }

@@ -11,20 +11,20 @@
 namespace moe {
 
 // Control words at the start of a workspace (uint32 indices).  Word 0 is the
-// error word the host reads; the rest are counters of the fused kernel,
-// zero between calls.
+// error word the host reads.  The counters of the fused kernel are zero
+// between calls; the epoch word counts the kernel's calls on this workspace
+// (router score records carry the epoch of the call that wrote them).
 constexpr size_t kCtrlBytes = 4096;
 enum : int {
   kCtrlErr = 0,
   kCtrlTicket = 1,
-  kCtrlRouterDone = 2,
-  kCtrlSelReady = 3,
+  kCtrlEpoch = 2,
   kCtrlExit = 4,
   kCtrlAbort = 5,
-  kCtrlWhere = 8,     // [4] where the first error happened (CTA, warp, site, fill)
-  kCtrlGuDone = 16,   // [slots] finished gate/up finalizer warps
-  kCtrlHqReady = 56,  // [slots] the slot's int16 h table is published
-  kCtrlRbDone = 96,   // [row blocks of hidden] finished down finalizer warps
+  kCtrlWhere = 8,    // [4] where the first error happened (CTA, warp, site, fill)
+  kCtrlGuDone = 16,  // [slots] finished gate/up finalizer warps of the slot
+  kCtrlRbDone = 64,  // [row blocks of hidden] finished down finalizer warps
+  kCtrlWords = (int)(kCtrlBytes / 4),
 };
 
 struct DecodeParams {
@@ -39,15 +39,13 @@ struct DecodeParams {
   int32_t* idx_out;   // nullable
   float* w_out;       // nullable
   uint32_t* ctrl;
-  float* logits;      // [E]
-  int32_t* idx_ws;    // [k]
-  float* w_ws;        // [k]
+  uint64_t* scores;   // [E]: (epoch << 32) | bits of sigmoid(logit), per expert
   float* hbuf;        // [slots][I]
   float* ypart;       // [slots][H]
-  uint32_t* hq;       // [slots][I/32 * 68 bytes]: int16 h groups, then factors
   int H, I, E, k, n_group, topk_group, has_shared;
   float rsf;
-  int RR, RG, RD;     // rows per router block / gate-up / down item
+  int RR, RG, RD;     // rows per router block / gate-up item / down item
+  int gu_count;       // finalizer-warp arrivals that complete one slot's h
   int nR, nG, nD, n_items;
 };
 

@@ -51,12 +51,9 @@ static moe_status launch_fused(const moe_layer* l, const uint16_t* x, const floa
   p.idx_out = idx_out;
   p.w_out = w_out;
   p.ctrl = reinterpret_cast<uint32_t*>(ws + L.ctrl);
-  p.logits = reinterpret_cast<float*>(ws + L.logits);
-  p.idx_ws = reinterpret_cast<int32_t*>(ws + L.idx);
-  p.w_ws = reinterpret_cast<float*>(ws + L.w);
+  p.scores = reinterpret_cast<uint64_t*>(ws + L.logits);
   p.hbuf = reinterpret_cast<float*>(ws + L.hbuf);
   p.ypart = reinterpret_cast<float*>(ws + L.ypart);
-  p.hq = reinterpret_cast<uint32_t*>(ws + L.hq);
   cudaError_t e = launch_decode(p, st);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "decode launch");
 }

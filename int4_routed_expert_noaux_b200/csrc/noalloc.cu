@@ -12,17 +12,21 @@ namespace moe {
 
 // Largest scratch the call takes: the one-token workspace of the shape,
 // ws_layout(cfg, 1).total.  A 6144 x 2048 layer with top-8 of 256 experts
-// and one shared expert needs 339,712 bytes.
+// and one shared expert needs 301,568 bytes.
 constexpr size_t kStaticScratchBytes = 512u << 10;
 constexpr int kStaticMaxDevices = 64;
+// control words plus the largest router score area (256 experts x 8 bytes)
+constexpr size_t kStaticClearBytes = kCtrlBytes + 256 * 8;
 
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
 static std::atomic<uint8_t*> g_scratch_addr[kStaticMaxDevices];
 static std::mutex g_scratch_mu;
 
-// Address of g_static_scratch on `dev` (the current device), resolved once.
-static moe_status scratch_address(int dev, uint8_t** out) {
+// Address of g_static_scratch on `dev` (the current device), resolved once;
+// the first resolution also zero-fills the control words and the router
+// score records on `st` (the array starts zeroed at module load as well).
+static moe_status scratch_address(int dev, cudaStream_t st, uint8_t** out) {
   uint8_t* a = g_scratch_addr[dev].load(std::memory_order_acquire);
   if (!a) {
     std::lock_guard<std::mutex> lock(g_scratch_mu);
@@ -32,6 +36,8 @@ static moe_status scratch_address(int dev, uint8_t** out) {
       cudaError_t e = cudaGetSymbolAddress(&sym, g_static_scratch);
       if (e != cudaSuccess) return cuda_fail(e, "scratch symbol address");
       a = static_cast<uint8_t*>(sym);
+      e = cudaMemsetAsync(a, 0, kStaticClearBytes, st);
+      if (e != cudaSuccess) return cuda_fail(e, "scratch clear");
       g_scratch_addr[dev].store(a, std::memory_order_release);
     }
   }
@@ -69,14 +75,14 @@ moe_status moe_layer_forward_noalloc(const moe_layer* l, const void* x, float* y
                 l->device);
   if (dev < 0 || dev >= kStaticMaxDevices)
     return fail(MOE_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kStaticMaxDevices);
-  uint8_t* ws = nullptr;
-  if ((s = scratch_address(dev, &ws)) != MOE_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
-  // The control words (error word, tickets, dependency counts) must start at
-  // zero; clearing them on every call also recovers from a call whose kernel
-  // stopped early and left counts behind.
-  ce = cudaMemsetAsync(ws + L.ctrl, 0, kCtrlBytes, st);
-  if (ce != cudaSuccess) return cuda_fail(ce, "scratch clear");
+  uint8_t* ws = nullptr;
+  if ((s = scratch_address(dev, st, &ws)) != MOE_OK) return s;
+  // The kernels return their counters to zero on every exit, stopped early
+  // or not, and the epoch word must keep counting; only the error word of an
+  // earlier call is cleared, so that status_out reports this call alone.
+  ce = cudaMemsetAsync(ws + L.ctrl, 0, sizeof(uint32_t), st);
+  if (ce != cudaSuccess) return cuda_fail(ce, "error word clear");
   if ((s = forward_impl(l, (const uint16_t*)x, 1, y, idx_out, w_out, ws, L, st)) != MOE_OK)
     return s;
   if (status_out) {

@@ -225,7 +225,14 @@ def test_many_decode_calls_one_workspace(shape, n):
     for t in range(n):
         L.forward(x[t:t + 1], ys[t:t + 1], ws, idx=idx[t:t + 1], w=w[t:t + 1])
     moe.ws_check(ws)
-    assert int(ws[4:4096].count_nonzero().item()) == 0  # counters reset
+    # the counters are back to zero; the epoch word counts the calls and every
+    # router score record (after the 4 KB of control words) carries the last
+    # call's epoch
+    words = ws[:4096].view(torch.int32).cpu().numpy()
+    assert words[2] == n
+    assert np.count_nonzero(np.delete(words[1:], 1)) == 0
+    recs = ws[4096:4096 + 8 * shape.n_experts].view(torch.int64).cpu().numpy()
+    assert np.all((recs >> 32) == n)
     check_forward(shape, dl, x_bits, ys.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy())
 
 

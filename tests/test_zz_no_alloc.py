@@ -66,8 +66,8 @@ def test_noalloc_matches_workspace_forward(shape):
 
 def test_noalloc_refuses_shapes_beyond_the_scratch():
     needs_gpu()
-    # one token of a 8192 x 4096 layer needs more than the fixed array holds
-    shape = synth.Shape(hidden=8192, inter=4096, n_experts=16, n_shared=1, top_k=8,
+    # one token of a 8192 x 8192 layer needs more than the fixed array holds
+    shape = synth.Shape(hidden=8192, inter=8192, n_experts=16, n_shared=1, top_k=8,
                         n_group=1, topk_group=1)
     cfg = moe.Config.from_shape(shape)
     assert moe.workspace_bytes(cfg, 1) > SCRATCH_BYTES
