@@ -90,6 +90,38 @@ struct Smem {
   float sp[kMaxE];
 };
 
+// The out-of-line helpers take their arguments by value: a reference to the
+// kernel's parameters would make the compiler copy them into local memory,
+// whose loads miss L1 and wait on L2 while the weights stream.
+struct SelArgs {
+  int E, k, n_group, topk_group, sel_q, sel_lgL, sel_fast;
+  float rsf;
+  int32_t* idx_out;  // written by CTA 0 only (nullable)
+  float* w_out;
+};
+
+__device__ __forceinline__ SelArgs sel_args(const DecodeParams& p) {
+  SelArgs a;
+  a.E = p.E;
+  a.k = p.k;
+  a.n_group = p.n_group;
+  a.topk_group = p.topk_group;
+  a.sel_q = p.sel_q;
+  a.sel_lgL = p.sel_lgL;
+  a.sel_fast = p.sel_fast;
+  a.rsf = p.rsf;
+  a.idx_out = p.idx_out;
+  a.w_out = p.w_out;
+  return a;
+}
+
+struct CombineArgs {
+  int k, H, has_shared;
+  const float* ypart;
+  const float* x_resid;
+  float* y;
+};
+
 __device__ __forceinline__ ItemDesc make_item(int type, int slot, int row0, int nrows) {
   ItemDesc d;
   d.type = type;
@@ -101,7 +133,7 @@ __device__ __forceinline__ ItemDesc make_item(int type, int slot, int row0, int 
   return d;
 }
 
-__device__ ItemDesc decode_ticket(const DecodeParams& p, int t) {
+__device__ __forceinline__ ItemDesc decode_ticket(const DecodeParams& p, int t) {
   // shared gate/up, shared down, routed gate/up 0..k-1, routed down 0..k-1
   auto gu = [&](int slot, int b) {
     return make_item(kGateUp, slot, b * p.RG, min(p.RG, p.I - b * p.RG));
@@ -191,7 +223,7 @@ __device__ __forceinline__ ArgMaxF am_warp(ArgMaxF a) {
 // Selection for shapes whose groups do not align with lanes: one lane per
 // group, repeated warp arg-max over S.sp / S.sc.  Results go to
 // S.sel_idx / S.sel_w (and, from CTA 0, to the caller's idx_out / w_out).
-__device__ __noinline__ void run_select_generic(const DecodeParams& p, Smem& S) {
+__device__ __noinline__ void run_select_generic(const SelArgs p, Smem& S) {
   const int lane = threadIdx.x & 31;
   const int per = p.E / p.n_group;
   // group score: sum of the two largest bias-corrected scores (lane = group)
@@ -272,7 +304,7 @@ __device__ __forceinline__ uint32_t input_bf16(const DecodeParams& p, int i, flo
 
 // Fixed-order combine of one row block of y from the per-slot partials, by
 // one warp, once every slot's down item of the block has published.
-__device__ __noinline__ void combine_block(const DecodeParams& p, const float* wsel, int row0,
+__device__ __noinline__ void combine_block(const CombineArgs p, const float* wsel, int row0,
                                           int nrows) {
   const int lane = threadIdx.x & 31;
   if (lane == 0) fence_acq_rel();  // see the other warps' partials
@@ -321,59 +353,55 @@ __device__ __forceinline__ void cx(uint32_t (&key)[kMaxE / 32], int (&jid)[kMaxE
 // rounds of two warp reductions (max of the score key, then min of the
 // expert id among the lanes holding it: ties go to the lower id).  Results
 // go to S.sel_idx / S.sel_w (and, from CTA 0, to idx_out / w_out).
-__device__ __noinline__ void run_select(const DecodeParams& p, Smem& S) {
-  const int lane = threadIdx.x & 31;
-  const int E = p.E, per = E / p.n_group, q = (E + 31) >> 5;
-  const int L = per / q;
-  constexpr int kQ = kMaxE / 32;
-  if (per % q != 0 || L < 1 || (L & (L - 1)) != 0 || q > kQ) {
+__device__ __noinline__ void run_select(const SelArgs p, Smem& S) {
+  if (!p.sel_fast) {
     run_select_generic(p, S);
     return;
   }
-  const int nmine = max(0, min(q, E - lane * q));  // experts this lane owns
+  // Branch-free: every shuffle and reduction runs in all lanes with no
+  // data-dependent guard around it (guarded warp collectives cost tens of
+  // cycles each in convergence handling).
+  const int lane = threadIdx.x & 31;
+  const int q = p.sel_q, lgL = p.sel_lgL, L = 1 << lgL;
+  constexpr int kQ = kMaxE / 32;
+  const int nmine = max(0, min(q, p.E - lane * q));  // experts this lane owns
   float sc[kQ], sp[kQ];
 #pragma unroll
   for (int j = 0; j < kQ; ++j) {
-    sp[j] = (j < nmine) ? S.sp[lane * q + j] : 0.f;
+    sp[j] = (j < nmine) ? S.sp[lane * q + j] : -INFINITY;
     sc[j] = (j < nmine) ? S.sc[lane * q + j] : 0.f;
   }
   // group score: the two largest sp of the group (lanes g*L .. g*L+L-1)
   float t1 = -INFINITY, t2 = -INFINITY;
 #pragma unroll
   for (int j = 0; j < kQ; ++j) {
-    if (j < nmine) {
-      const float v = sp[j];
-      if (v > t1) {
-        t2 = t1;
-        t1 = v;
-      } else if (v > t2) {
-        t2 = v;
-      }
-    }
+    t2 = fmaxf(t2, fminf(t1, sp[j]));
+    t1 = fmaxf(t1, sp[j]);
   }
-  for (int o = 1; o < L; o <<= 1) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
     const float p1 = __shfl_xor_sync(0xffffffffu, t1, o);
     const float p2 = __shfl_xor_sync(0xffffffffu, t2, o);
-    const float n1 = fmaxf(t1, p1);
     const float n2 = fmaxf(fminf(t1, p1), fmaxf(t2, p2));
-    t1 = n1;
-    t2 = n2;
+    const float n1 = fmaxf(t1, p1);
+    t1 = (o < L) ? n1 : t1;
+    t2 = (o < L) ? n2 : t2;
   }
+  const int per = q << lgL;
   const float gs_seg = (per >= 2) ? t1 + t2 : t1;
   // keep topk_group groups: rank by (score desc, index asc); lane g holds
-  // group g (n_group <= E / q <= 32); the shuffles are independent
+  // group g (n_group <= 32), lanes past the groups hold -inf
   const int G = p.n_group;
-  const float gs = __shfl_sync(0xffffffffu, gs_seg, (lane < G ? lane : 0) * L);
+  float gs = __shfl_sync(0xffffffffu, gs_seg, (lane < G ? lane : 0) << lgL);
+  gs = (lane < G) ? gs : -INFINITY;
   int rank = 0;
 #pragma unroll
   for (int h = 0; h < 32; ++h) {
-    if (h < G) {
-      const float o = __shfl_sync(0xffffffffu, gs, h);
-      if (o > gs || (o == gs && h < lane)) ++rank;
-    }
+    const float o = __shfl_sync(0xffffffffu, gs, h);
+    rank += (o > gs || (o == gs && h < lane)) ? 1 : 0;
   }
   const unsigned kept_mask = __ballot_sync(0xffffffffu, lane < G && rank < p.topk_group);
-  const bool kept = (kept_mask >> (lane / L)) & 1u;
+  const bool kept = (kept_mask >> (lane >> lgL)) & 1u;
   // each lane sorts its kept candidates once (a sorting network)
   uint32_t key[kQ];
   int jid[kQ];
@@ -391,37 +419,33 @@ __device__ __noinline__ void run_select(const DecodeParams& p, Smem& S) {
   cx(key, jid, sl, 0, 4); cx(key, jid, sl, 1, 5); cx(key, jid, sl, 2, 6); cx(key, jid, sl, 3, 7);
   cx(key, jid, sl, 2, 4); cx(key, jid, sl, 3, 5);
   cx(key, jid, sl, 1, 2); cx(key, jid, sl, 3, 4); cx(key, jid, sl, 5, 6);
-  // top_k: the best head, lowest expert id among equal heads, is popped
-  int my_sel = -1;
+  // top_k: the best head, lowest expert id among equal heads, is popped;
+  // lane r keeps the r-th pick (lanes past k keep INT_MAX for the ordering)
+  int my_sel = 0x7FFFFFFF;
   float my_s = 0.f;
   for (int r = 0; r < p.k; ++r) {
     const uint32_t m = __reduce_max_sync(0xffffffffu, key[0]);
     const uint32_t cand = (key[0] == m && m != 0u) ? (uint32_t)(lane * q + jid[0]) : 0xFFFFFFFFu;
     const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
-    const int owner = __ffs(__ballot_sync(0xffffffffu, cand == win)) - 1;
-    const float s_win = __shfl_sync(0xffffffffu, sl[0], owner);
-    if (lane == r) {
-      my_sel = (int)win;
-      my_s = s_win;
-    }
-    if (lane == owner) {  // pop the head
+    const bool own = cand == win && m != 0u;
+    const int owner = __ffs(__ballot_sync(0xffffffffu, own)) - 1;
+    const float s_win = __shfl_sync(0xffffffffu, sl[0], owner & 31);
+    my_sel = (lane == r) ? (int)win : my_sel;  // no candidate left: -1
+    my_s = (lane == r) ? s_win : my_s;
 #pragma unroll
-      for (int j = 0; j + 1 < kQ; ++j) {
-        key[j] = key[j + 1];
-        jid[j] = jid[j + 1];
-        sl[j] = sl[j + 1];
-      }
-      key[kQ - 1] = 0u;
+    for (int j = 0; j + 1 < kQ; ++j) {  // pop the owner's head
+      key[j] = own ? key[j + 1] : key[j];
+      jid[j] = own ? jid[j + 1] : jid[j];
+      sl[j] = own ? sl[j + 1] : sl[j];
     }
+    key[kQ - 1] = own ? 0u : key[kQ - 1];
   }
   // ascending ids; weights from the unbiased scores
   int pos = 0;
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
-    if (j < p.k) {
-      const int other = __shfl_sync(0xffffffffu, my_sel, j);
-      if (lane < p.k && other < my_sel) ++pos;
-    }
+    const int other = __shfl_sync(0xffffffffu, my_sel, j);
+    pos += (other < my_sel) ? 1 : 0;
   }
   float denom = (lane < p.k) ? my_s : 0.f;
 #pragma unroll
@@ -688,7 +712,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         }
       }
       __syncwarp();
-      run_select(p, S);
+      run_select(sel_args(p), S);
     } else if (lane == 0) {
       set_error(p.ctrl, kErrTimeout, 8, 0);
     }
@@ -736,6 +760,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       xq_from_floats(xf, xq);
     }
     int& gabort = S.abort_flag[grp];
+    CombineArgs comb;
+    comb.k = p.k;
+    comb.H = p.H;
+    comb.has_shared = p.has_shared;
+    comb.ypart = p.ypart;
+    comb.x_resid = p.x_resid;
+    comb.y = p.y;
     int pend_row0 = -1, pend_nrows = 0;  // this warp's last down row block
     uint32_t pend_old = 0;               // count before this warp's add (lane 0)
     // Group 0 of a CTA with router rows: fill 0 is the router block.  It is
@@ -817,26 +848,41 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         }
       }
     }
-    for (uint32_t c = c_first;; ++c) {
+    // Group 1 starts with two placeholder items (a gate/up, then a down
+    // item) that run the real loop body on whatever the stage holds and
+    // publish nothing: the instructions of both paths are fetched while the
+    // first weights are still on their way, not when they have arrived.
+    int warm = (grp == 1 && p.warm) ? 2 : 0;
+    uint32_t c = c_first;
+    for (uint32_t it = c_first;; ++it) {  // it: group barrier phases used
       if (gabort) break;
+      const bool fake = warm > 0;
       const uint32_t n = 2 * c + grp;  // fill number consumed
       const int stage = (int)(n % kStages);
       const uint32_t par = (n / kStages) & 1u;
-      const int rbuf = c & 1;
-      const uint32_t gpar = c & 1u;  // one group barrier per iteration
+      const int rbuf = it & 1;
+      const uint32_t gpar = it & 1u;  // one group barrier per iteration
       // Every path through this loop body passes the group barrier exactly
       // once, and wait results are uniform per warp, so a wait that runs out
       // in one warp can never leave a barrier or a shuffle half-joined.
-      int okw = 0;
-      if (lane == 0) okw = mbar_wait(&S.full[stage], par, global_timer_ns() + kWaitNs) ? 1 : 0;
-      bool ok = __shfl_sync(0xffffffffu, okw, 0) != 0;
-      if (ok) {
-        mbar_test(&S.full[stage], par);  // acquire the bulk-copied bytes in every lane
-      } else {
-        if (lane == 0) set_error(p.ctrl, kErrTimeout, 1, n);
-        gabort = 1;
+      bool ok = true;
+      if (!fake) {
+        int okw = 0;
+        if (lane == 0) okw = mbar_wait(&S.full[stage], par, global_timer_ns() + kWaitNs) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, okw, 0) != 0;
+        if (ok) {
+          mbar_test(&S.full[stage], par);  // acquire the bulk-copied bytes in every lane
+        } else {
+          if (lane == 0) set_error(p.ctrl, kErrTimeout, 1, n);
+          gabort = 1;
+        }
       }
-      const ItemDesc d = S.desc[stage];
+      const ItemDesc d = fake ? make_item(warm == 2 ? kGateUp : kDown, 0, 0, 0) : S.desc[stage];
+      if (fake) {
+        --warm;
+      } else {
+        ++c;
+      }
       if (!ok || d.type == kDone) {
         group_barrier(&S.gbar[grp], gpar);
         break;
@@ -861,7 +907,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           v[NR_G + r] = dot_scaled(wu, xq, f16_bits_to_f32(su[lr * G + cg.col]));
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.empty[stage]);
+        if (lane == 0 && !fake) mbar_arrive(&S.empty[stage]);
         reduce_scatter<NV_G, SEG_G>(v);
         S.red[grp][rbuf][gw][lane] = v[0];
         if (!group_barrier(&S.gbar[grp], gpar)) {
@@ -872,7 +918,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         if (pend_row0 >= 0) {
           const uint32_t last =
               __shfl_sync(0xffffffffu, pend_old + 1 == (uint32_t)(slots * fw_d), 0);
-          if (last) combine_block(p, S.sel_w, pend_row0, pend_nrows);
+          if (last) combine_block(comb, S.sel_w, pend_row0, pend_nrows);
           pend_row0 = -1;
         }
 
@@ -892,7 +938,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           }
           __syncwarp();
           // count this warp done (nothing waits for the result)
-          if (lane == 0) red_add_release(p.ctrl + kCtrlGuDone + d.slot, 1u);
+          if (lane == 0 && !fake) red_add_release(p.ctrl + kCtrlGuDone + d.slot, 1u);
         }
       } else {  // kDown
         XQ hq;  // this thread's 32-row group of h, as int16 fixed point
@@ -920,7 +966,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           v[r] = dot_scaled(wd, hq, f16_bits_to_f32(sd[lr * GD + cd.col]));
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.empty[stage]);
+        if (lane == 0 && !fake) mbar_arrive(&S.empty[stage]);
         reduce_scatter<NR_D, SEG_D>(v);
         S.red[grp][rbuf][gw][lane] = v[0];
         if (!group_barrier(&S.gbar[grp], gpar)) {
@@ -931,11 +977,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         if (pend_row0 >= 0) {
           const uint32_t last =
               __shfl_sync(0xffffffffu, pend_old + 1 == (uint32_t)(slots * fw_d), 0);
-          if (last) combine_block(p, S.sel_w, pend_row0, pend_nrows);
+          if (last) combine_block(comb, S.sel_w, pend_row0, pend_nrows);
           pend_row0 = -1;
         }
 
-        if (gw < fw_d) {
+        if (gw < fw_d && !fake) {
           if (tg < cd.P * NR_D) {
             const int ph = tg / NR_D, i = tg % NR_D;
             const int lr = ph * NR_D + i;
@@ -959,7 +1005,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     // a row block completed by this warp's last down item
     if (!gabort && pend_row0 >= 0) {
       const uint32_t last = __shfl_sync(0xffffffffu, pend_old + 1 == (uint32_t)(slots * fw_d), 0);
-      if (last) combine_block(p, S.sel_w, pend_row0, pend_nrows);
+      if (last) combine_block(comb, S.sel_w, pend_row0, pend_nrows);
     }
   }
 
@@ -1062,6 +1108,14 @@ bool decode_plan(const moe_config& c, DecodeParams& p) {
   p.topk_group = c.topk_group;
   p.has_shared = c.n_shared;
   p.rsf = c.routed_scaling_factor;
+  {
+    const int per = c.n_experts / c.n_group, q = (c.n_experts + 31) / 32;
+    const int L = per / q;
+    p.sel_q = q;
+    p.sel_lgL = 0;
+    while ((1 << p.sel_lgL) < L) ++p.sel_lgL;
+    p.sel_fast = per % q == 0 && L >= 1 && (1 << p.sel_lgL) == L && q <= kMaxE / 32;
+  }
   p.RG = PG * nrg;
   p.RD = PD * nrd;
   {
