@@ -848,26 +848,41 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         }
       }
     }
-    for (uint32_t c = c_first;; ++c) {
+    // Group 1 starts with two placeholder items (a gate/up, then a down
+    // item) that run the real loop body on whatever the stage holds and
+    // publish nothing: the instructions of both paths are fetched while the
+    // first weights are still on their way, not when they have arrived.
+    int warm = (grp == 1 && p.warm) ? 2 : 0;
+    uint32_t c = c_first;
+    for (uint32_t it = c_first;; ++it) {  // it: group barrier phases used
       if (gabort) break;
+      const bool fake = warm > 0;
       const uint32_t n = 2 * c + grp;  // fill number consumed
       const int stage = (int)(n % kStages);
       const uint32_t par = (n / kStages) & 1u;
-      const int rbuf = c & 1;
-      const uint32_t gpar = c & 1u;  // one group barrier per iteration
+      const int rbuf = it & 1;
+      const uint32_t gpar = it & 1u;  // one group barrier per iteration
       // Every path through this loop body passes the group barrier exactly
       // once, and wait results are uniform per warp, so a wait that runs out
       // in one warp can never leave a barrier or a shuffle half-joined.
-      int okw = 0;
-      if (lane == 0) okw = mbar_wait(&S.full[stage], par, global_timer_ns() + kWaitNs) ? 1 : 0;
-      const bool ok = __shfl_sync(0xffffffffu, okw, 0) != 0;
-      if (ok) {
-        mbar_test(&S.full[stage], par);  // acquire the bulk-copied bytes in every lane
-      } else {
-        if (lane == 0) set_error(p.ctrl, kErrTimeout, 1, n);
-        gabort = 1;
+      bool ok = true;
+      if (!fake) {
+        int okw = 0;
+        if (lane == 0) okw = mbar_wait(&S.full[stage], par, global_timer_ns() + kWaitNs) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, okw, 0) != 0;
+        if (ok) {
+          mbar_test(&S.full[stage], par);  // acquire the bulk-copied bytes in every lane
+        } else {
+          if (lane == 0) set_error(p.ctrl, kErrTimeout, 1, n);
+          gabort = 1;
+        }
       }
-      const ItemDesc d = S.desc[stage];
+      const ItemDesc d = fake ? make_item(warm == 2 ? kGateUp : kDown, 0, 0, 0) : S.desc[stage];
+      if (fake) {
+        --warm;
+      } else {
+        ++c;
+      }
       if (!ok || d.type == kDone) {
         group_barrier(&S.gbar[grp], gpar);
         break;
@@ -892,7 +907,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           v[NR_G + r] = dot_scaled(wu, xq, f16_bits_to_f32(su[lr * G + cg.col]));
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.empty[stage]);
+        if (lane == 0 && !fake) mbar_arrive(&S.empty[stage]);
         reduce_scatter<NV_G, SEG_G>(v);
         S.red[grp][rbuf][gw][lane] = v[0];
         if (!group_barrier(&S.gbar[grp], gpar)) {
@@ -923,7 +938,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           }
           __syncwarp();
           // count this warp done (nothing waits for the result)
-          if (lane == 0) red_add_release(p.ctrl + kCtrlGuDone + d.slot, 1u);
+          if (lane == 0 && !fake) red_add_release(p.ctrl + kCtrlGuDone + d.slot, 1u);
         }
       } else {  // kDown
         XQ hq;  // this thread's 32-row group of h, as int16 fixed point
@@ -951,7 +966,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           v[r] = dot_scaled(wd, hq, f16_bits_to_f32(sd[lr * GD + cd.col]));
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.empty[stage]);
+        if (lane == 0 && !fake) mbar_arrive(&S.empty[stage]);
         reduce_scatter<NR_D, SEG_D>(v);
         S.red[grp][rbuf][gw][lane] = v[0];
         if (!group_barrier(&S.gbar[grp], gpar)) {
@@ -966,7 +981,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           pend_row0 = -1;
         }
 
-        if (gw < fw_d) {
+        if (gw < fw_d && !fake) {
           if (tg < cd.P * NR_D) {
             const int ph = tg / NR_D, i = tg % NR_D;
             const int lr = ph * NR_D + i;

@@ -47,6 +47,7 @@ struct DecodeParams {
   // selection layout: lane l owns experts l*sel_q .. l*sel_q+sel_q-1 and a
   // group is 2^sel_lgL consecutive lanes (sel_fast), else the generic path
   int sel_fast, sel_q, sel_lgL;
+  int warm;           // consumer group 1 first runs one placeholder item of each kind
   int RR, RG, RD;     // rows per router block / gate-up item / down item
   int gu_count;       // finalizer-warp arrivals that complete one slot's h
   int nR, nG, nD, n_items;

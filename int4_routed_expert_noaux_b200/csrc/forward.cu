@@ -53,6 +53,7 @@ static moe_status launch_fused(const moe_layer* l, const uint16_t* x, const floa
   p.ctrl = reinterpret_cast<uint32_t*>(ws + L.ctrl);
   p.scores = reinterpret_cast<uint64_t*>(ws + L.logits);
   p.hbuf = reinterpret_cast<float*>(ws + L.hbuf);
+  p.warm = 1;
   p.ypart = reinterpret_cast<float*>(ws + L.ypart);
   cudaError_t e = launch_decode(p, st);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "decode launch");
