@@ -26,10 +26,14 @@
 //    the expert ids and weights to its producer and consumers through
 //    shared memory;
 //  * work items come from a global ticket counter in the order:
-//    shared-expert gate/up, shared-expert down, routed gate/up of slots
-//    0..k-1, routed down of slots 0..k-1.  Every dependency points to an
+//    shared-expert gate/up, routed gate/up of slots 0..k-1, shared-expert
+//    down, routed down of slots 0..k-1.  Every dependency points to an
 //    earlier ticket, so in-order claiming always makes progress; the shared
-//    expert's items keep HBM busy while the routed experts are selected;
+//    expert's gate/up items keep HBM busy while the routed experts are
+//    selected, and no producer waits on a down item's inputs early on;
+//  * consumer group 1 first runs one placeholder gate/up and one placeholder
+//    down item through the loop body (nothing published), so that both code
+//    paths are fetched while the first weights are in flight;
 //  * gate/up finalizer warps publish h rows (fp32) and count themselves done
 //    with a release add (nothing waits on its result); the producer waits
 //    until a slot's count is complete and bulk-copies the slot's h (8 KB for
@@ -134,7 +138,7 @@ __device__ __forceinline__ ItemDesc make_item(int type, int slot, int row0, int 
 }
 
 __device__ __forceinline__ ItemDesc decode_ticket(const DecodeParams& p, int t) {
-  // shared gate/up, shared down, routed gate/up 0..k-1, routed down 0..k-1
+  // shared gate/up, routed gate/up 0..k-1, shared down, routed down 0..k-1
   auto gu = [&](int slot, int b) {
     return make_item(kGateUp, slot, b * p.RG, min(p.RG, p.I - b * p.RG));
   };
@@ -144,11 +148,13 @@ __device__ __forceinline__ ItemDesc decode_ticket(const DecodeParams& p, int t) 
   if (p.has_shared) {
     if (t < p.nG) return gu(p.k, t);
     t -= p.nG;
-    if (t < p.nD) return dn(p.k, t);
-    t -= p.nD;
   }
   if (t < p.k * p.nG) return gu(t / p.nG, t % p.nG);
   t -= p.k * p.nG;
+  if (p.has_shared) {
+    if (t < p.nD) return dn(p.k, t);
+    t -= p.nD;
+  }
   if (t < p.k * p.nD) return dn(t / p.nD, t % p.nD);
   return make_item(kDone, 0, 0, 0);
 }
