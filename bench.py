@@ -50,6 +50,18 @@ def parse():
     p.add_argument("--small", action="store_true", help="tiny layer (smoke/profiling only)")
     p.add_argument("--experts", type=int, default=0,
                    help="routed experts per layer (profiling only; default: the shape's 256)")
+    p.add_argument("--mode", default="layer", choices=["layer", "verify", "stack", "stream"],
+                   help="layer: batch-1 decode of one layer (the headline); verify: T-token "
+                        "calls; stack: one token through 24 layers; stream: host-streamed "
+                        "experts through the LRU cache")
+    p.add_argument("--verify-T", default="2,3,4,8,32", help="tokens per verify call")
+    p.add_argument("--correlated", action="store_true",
+                   help="verify: draft tokens x0 + 0.05 eps (heavily shared experts)")
+    p.add_argument("--stack-layers", type=int, default=24)
+    p.add_argument("--stream-layers", type=int, default=8,
+                   help="stream: layers in pinned host memory (capped by free host RAM)")
+    p.add_argument("--stream-caps", default="8,16,32,64,128", help="stream: cache slots per layer")
+    p.add_argument("--stream-tokens", type=int, default=512)
     return p.parse_args()
 
 
@@ -210,6 +222,9 @@ def main():
     if args.impl == "reference":
         run_reference(args, shape)
         return
+    if args.mode != "layer":
+        run_mode(args, shape)
+        return
 
     import torch
     import int4_routed_expert_noaux_b200 as moe
@@ -368,6 +383,202 @@ def main():
 
 def launches_per_forward():
     return 1
+
+
+# ---------------------------------------------------------------------------
+# other modes: one JSON line per configuration, same keys where they apply
+
+def _timed(stream, fn, steps, warmup):
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, warmup)):
+            fn()
+    stream.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(steps):
+            fn()
+        ev1.record(stream)
+    stream.synchronize()
+    return ev0.elapsed_time(ev1)
+
+
+def _graph(stream, fn):
+    import torch
+    with torch.cuda.stream(stream):
+        fn()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    stream.synchronize()
+    return g
+
+
+def _line(args, shape, extra):
+    base = {"metric": METRIC, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+            "warmup": max(3, args.warmup), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int4xf32", "data": "synthetic", "mode": args.mode}
+    base.update(extra)
+    print(json.dumps(base), flush=True)
+
+
+def run_mode(args, shape):
+    import torch
+    import int4_routed_expert_noaux_b200 as moe
+    import synth
+    from synth.layers import DeviceLayer
+    torch.cuda.set_device(0)
+    cfg = moe.Config.from_shape(shape)
+    peak, peak_kind = peaks()
+    stream = torch.cuda.Stream()
+    E, H = shape.n_experts, shape.hidden
+    fixed = E * H * 4 + E * 4
+
+    if args.mode == "verify":
+        copies = max(1, args.copies)
+        dls = [DeviceLayer(shape, 0, c) for c in range(copies)]
+        views = [moe.Layer(cfg, d.w_router, d.bias, d.routed, d.shared) for d in dls]
+        for T in [int(v) for v in args.verify_T.split(",")]:
+            calls = max(copies, args.tokens // T)
+            if args.correlated:
+                xb = np.concatenate([synth.correlated_tokens(shape, 7 + c, T) for c in range(calls)])
+            else:
+                xb = synth.tokens(shape, 0, 0, calls * T)
+            x = torch.from_numpy(xb.view(np.int16)).cuda()
+            y = torch.empty((calls * T, H), dtype=torch.float32, device="cuda")
+            idx = torch.empty((calls * T, shape.top_k), dtype=torch.int32, device="cuda")
+            ws = moe.alloc_workspace(cfg, T)
+
+            def step():
+                for c in range(calls):
+                    sl = slice(c * T, (c + 1) * T)
+                    views[c % copies].forward(x[sl], y[sl], ws, idx=idx[sl], stream=stream)
+            g = _graph(stream, step)
+            ms = _timed(stream, g.replay, args.steps, args.warmup)
+            moe.ws_check(ws, stream)
+            ids = idx.cpu().numpy().reshape(calls, T, shape.top_k)
+            uniq = [len(np.unique(ids[c])) for c in range(calls)]
+            byts = sum(fixed + (u + shape.n_shared) * shape.expert_bytes + T * (H * 2 + H * 4)
+                       for u in uniq)
+            call_us = ms * 1000.0 / (args.steps * calls)
+            achieved = byts / calls / (call_us * 1e-6) / 1e9
+            _line(args, shape, {
+                "value": calls * T * args.steps / (ms / 1000.0), "ms_per_step": ms / args.steps,
+                "config": {"workload": "GLM-5.2-shaped MoE layer, batched verify calls",
+                           "T": T, "calls_per_step": calls, "correlated": args.correlated,
+                           "layer_copies": copies, "mean_distinct_routed_experts": float(np.mean(uniq))},
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                             "frac": achieved / peak, "traffic": None, "peak_source": peak_kind,
+                             "kernel": "moe_layer_forward (T tokens)",
+                             "algorithmic_bytes_per_launch": byts / calls, "launch_us": call_us},
+                "gpu_launches": calls * args.steps * 8})
+        return
+
+    if args.mode == "stack":
+        L = args.stack_layers
+        dls = [DeviceLayer(shape, 0, l) for l in range(L)]
+        views = [moe.Layer(cfg, d.w_router, d.bias, d.routed, d.shared) for d in dls]
+        n = max(1, min(args.tokens, 200))
+        xb = synth.tokens(shape, 0, 0, n)
+        x0 = torch.from_numpy(synth.bf16_to_f32(xb)).cuda()
+        xo = torch.empty_like(x0)
+        tmp = torch.empty((H,), dtype=torch.float32, device="cuda")
+        ws = moe.alloc_workspace(cfg, 1)
+
+        def step():
+            for t in range(n):
+                moe.stack_forward(views, x0[t], xo[t], tmp, ws, stream=stream)
+        g = _graph(stream, step)
+        ms = _timed(stream, g.replay, args.steps, args.warmup)
+        moe.ws_check(ws, stream)
+        if not torch.isfinite(xo).all():
+            raise RuntimeError("non-finite stack outputs")
+        byts = L * algorithmic_bytes_per_token(shape)
+        tok_us = ms * 1000.0 / (args.steps * n)
+        achieved = byts / (tok_us * 1e-6) / 1e9
+        _line(args, shape, {
+            "value": n * args.steps / (ms / 1000.0), "ms_per_step": ms / args.steps,
+            "config": {"workload": f"{L} GLM-5.2-shaped MoE layers, one token through all "
+                                   "(pre-norm residual stream), all experts resident",
+                       "layers": L, "tokens_per_step": n,
+                       "hbm_weight_bytes": L * ((E + shape.n_shared) * shape.expert_bytes + fixed)},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "peak_source": peak_kind,
+                         "kernel": "moe_stack_forward (per token)",
+                         "algorithmic_bytes_per_launch": byts, "launch_us": tok_us},
+            "gpu_launches": n * args.steps * L})
+        return
+
+    if args.mode == "stream":
+        import psutil
+        stride = synth.expert_stride(shape)
+        layer_bytes = E * stride
+        avail = psutil.virtual_memory().available
+        L = max(1, min(args.stream_layers, int(avail * 0.25) // layer_bytes))
+        host, keep = [], []
+        for l in range(L):
+            buf = torch.empty(layer_bytes, dtype=torch.uint8).pin_memory()
+            keep.append(buf)
+            base = buf.data_ptr()
+            experts = []
+            for e in range(E):
+                offs = synth.expert_into(shape, 0, l, e, base + e * stride)
+                experts.append({k: base + e * stride + o for k, o in offs.items()})
+            host.append(experts)
+        dls = [DeviceLayer(shape, 0, l, routed=False) for l in range(L)]
+        # measured host->device bandwidth of pinned memory (>= 1 GB copies)
+        probe = torch.empty(min(layer_bytes, 2 << 30), dtype=torch.uint8, device="cuda")
+        hb_ms = _timed(stream, lambda: probe.copy_(keep[0][:probe.numel()], non_blocking=True), 3, 1)
+        h2d_gbs = 3 * probe.numel() / (hb_ms / 1000.0) / 1e9
+        del probe
+        trace = synth.zipf_trace(5, L, E, shape.top_k, args.stream_tokens)
+        xb = synth.tokens(shape, 0, 0, args.stream_tokens)
+        x = torch.from_numpy(xb.view(np.int16)).cuda()
+        ids_dev = torch.from_numpy(trace.astype(np.int32)).cuda()
+        w = torch.full((1, shape.top_k), shape.rsf / shape.top_k, dtype=torch.float32, device="cuda")
+        y = torch.empty((1, H), dtype=torch.float32, device="cuda")
+        ws = moe.alloc_workspace(cfg, 1)
+        for cap in [int(v) for v in args.stream_caps.split(",")]:
+            cache = moe.Cache(cfg, host, cap)
+            views = [cache.layer(l, dls[l].w_router, dls[l].bias, dls[l].shared) for l in range(L)]
+            torch.cuda.synchronize()
+            ev0 = torch.cuda.Event(enable_timing=True)
+            ev1 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                ev0.record(stream)
+                for t in range(args.stream_tokens):
+                    for l in range(L):
+                        cache.acquire(l, trace[t, l], stream=stream)
+                        views[l].expert_ffn(x[t:t + 1], ids_dev[t, l:l + 1], w, y, ws, stream=stream)
+                        cache.release(l, stream=stream)
+                ev1.record(stream)
+            stream.synchronize()
+            cache.sync()
+            ms = ev0.elapsed_time(ev1)
+            moe.ws_check(ws, stream)
+            hits = misses = moved = 0
+            for l in range(L):
+                h, m, b = cache.stats(l)
+                hits, misses, moved = hits + h, misses + m, moved + b
+            link = moved / (ms / 1000.0) / 1e9
+            _line(args, shape, {
+                "value": args.stream_tokens / (ms / 1000.0), "ms_per_step": ms,
+                "config": {"workload": f"{L} GLM-5.2-shaped MoE layers in pinned host memory, "
+                                       "per-layer LRU cache in HBM, Zipf(1.1) trace",
+                           "layers": L, "cache_slots_per_layer": cap,
+                           "tokens": args.stream_tokens, "routing": "trace; weights rsf/k",
+                           "hit_rate": hits / max(1, hits + misses),
+                           "host_bytes_per_layer": layer_bytes},
+                "roofline": {"bound": "h2d", "achieved": link, "peak": h2d_gbs, "unit": "GB/s",
+                             "frac": link / h2d_gbs, "traffic": moved, "peak_source":
+                             "measured pinned cudaMemcpyAsync, same run",
+                             "kernel": "expert loads (cudaMemcpyAsync, side stream)"},
+                "gpu_launches": args.stream_tokens * L * 7})
+            cache.close()
+        return
 
 
 if __name__ == "__main__":

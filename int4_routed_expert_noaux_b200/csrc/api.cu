@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "kernels.h"
 #include "layer.h"
 #include "moe.h"
 
@@ -112,7 +113,17 @@ WsLayout ws_layout(const moe_config* c, int T) {
   off = align_up(off + (size_t)T * slots * c->inter * 4, 256);
   L.ypart = off;
   off = align_up(off + (size_t)T * slots * c->hidden * 4, 256);
+  // batched path: int16 groups of x and of h, per-expert token lists
+  L.xq = off;
+  off = align_up(off + (size_t)T * (c->hidden / 32) * 64, 256);
+  L.xqf = off;
+  off = align_up(off + (size_t)T * (c->hidden / 32) * 4, 256);
   L.hq = off;
+  off = align_up(off + (size_t)T * slots * (c->inter / 32) * 64, 256);
+  L.hqf = off;
+  off = align_up(off + (size_t)T * slots * (c->inter / 32) * 4, 256);
+  L.lists = off;
+  off = align_up(off + union_lists_ints(T, k, c->n_experts, c->n_shared) * 4, 256);
   L.total = off;
   return L;
 }

@@ -21,14 +21,11 @@ moe_status route_impl(const moe_layer* l, const uint16_t* x, int T, int32_t* idx
 moe_status ffn_impl(const moe_layer* l, const uint16_t* x, int T, const int32_t* idx,
                     const float* w, float* y, uint8_t* ws, const WsLayout& L, cudaStream_t st) {
   const moe_config& c = l->cfg;
-  const int slots = c.top_k + c.n_shared;
-  float* hbuf = reinterpret_cast<float*>(ws + L.hbuf);
-  uint32_t* err = reinterpret_cast<uint32_t*>(ws + L.ctrl);
-  cudaError_t e = launch_gate_up(l->table, idx, c.n_experts, c.top_k, slots, x, T, c.hidden,
-                                 c.inter, hbuf, err, st);
-  if (e == cudaSuccess)
-    e = launch_down_combine(l->table, idx, w, c.n_experts, c.top_k, slots, hbuf, T, c.hidden,
-                            c.inter, y, err, st);
+  cudaError_t e = launch_union_ffn(
+      l->table, idx, w, x, T, c.hidden, c.inter, c.n_experts, c.top_k, c.n_shared, ws + L.xq,
+      reinterpret_cast<float*>(ws + L.xqf), ws + L.hq, reinterpret_cast<float*>(ws + L.hqf),
+      reinterpret_cast<int*>(ws + L.lists), reinterpret_cast<float*>(ws + L.hbuf),
+      reinterpret_cast<float*>(ws + L.ypart), y, reinterpret_cast<uint32_t*>(ws + L.ctrl), st);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "expert launch");
 }
 

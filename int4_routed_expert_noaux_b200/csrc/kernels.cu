@@ -1,7 +1,7 @@
-// kernels.cu -- step kernels of the routed-MoE layer: router GEMV, noaux_tc
-// selection, fused int4 gate/up + SiLU, int4 down projection with the
-// weighted combine.  Used by moe_route / moe_expert_ffn and by the batched
-// path; the T = 1 decode path uses the fused persistent kernel instead.
+// kernels.cu -- step kernels of the routed-MoE layer: router GEMV and
+// noaux_tc selection for T tokens (moe_route and the batched path), and a
+// plain dequantising int4 GEMV for one-hot checks.  The experts of T > 1
+// calls run in union.cu; a T = 1 call runs the fused persistent kernel.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -158,30 +158,9 @@ __global__ void __launch_bounds__(1024) select_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Fused int4 gate/up + SiLU (one expert slot, a block of rows).  Column-
-// stationary: thread (col, phase) owns 16-byte chunk column `col` of every
-// row it visits, so its 32 inputs stay in registers as an XQ.  Each
-// phase handles NR rows of gate and NR of up; one butterfly reduce-scatter
-// sums the 2*NR partial dots over the row's threads (with NV == SEG, lane l
-// of a segment ends with value index l % SEG: gate row r at r, up row r at
-// NR + r).  h = silu(g) * u is written to hbuf; g and u never leave the CTA.
-// grid.x = row blocks of `inter`, grid.y = token * slots + slot.
-
-__device__ __forceinline__ void load_x_group_bf16(const uint16_t* __restrict__ xp, XQ& xg) {
-  float xf[32];
-  const uint4* p4 = reinterpret_cast<const uint4*>(xp);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint4 v = __ldg(p4 + i);
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      xf[8 * i + 2 * j] = bf16_bits_to_f32(u[j] & 0xFFFFu);
-      xf[8 * i + 2 * j + 1] = bf16_bits_to_f32(u[j] >> 16);
-    }
-  }
-  xq_from_floats(xf, xg);
-}
+// Plain dequantising int4 GEMV, y[r] = sum_c q[r][c] * scale[r][c/32] * x[c]
+// (fp32 x and y), built from the same group dot product as the layer
+// kernels.  Exposed for one-hot checks of the packing and scale indexing.
 
 __device__ __forceinline__ void load_x_group_f32(const float* __restrict__ hp, XQ& xg) {
   float xf[32];
@@ -196,149 +175,6 @@ __device__ __forceinline__ void load_x_group_f32(const float* __restrict__ hp, X
   }
   xq_from_floats(xf, xg);
 }
-
-template <int SEG>
-__global__ void __launch_bounds__(256) gate_up_kernel(
-    const ExpertPtrs* __restrict__ table, const int32_t* __restrict__ idx,
-    int n_experts, int top_k, int slots, const uint16_t* __restrict__ x,
-    int H, int I, float* __restrict__ hbuf, uint32_t* __restrict__ err) {
-  constexpr int NV = SEG;        // values reduced per phase (gate + up)
-  constexpr int NR = NV / 2;     // rows per phase
-  __shared__ float red[32][33];  // cross-warp partials [warp][lane]
-  const int G = H >> 5;
-  const ColMap cm = col_map(G);
-  const int t = blockIdx.y / slots, slot = blockIdx.y % slots;
-  int eid = n_experts;  // slot == top_k: the shared expert
-  if (slot < top_k) {
-    eid = idx[(size_t)t * top_k + slot];
-    if (eid < 0 || eid >= n_experts) {
-      if (threadIdx.x == 0) atomicCAS(err, 0u, (uint32_t)kErrBadExpertId);
-      eid = -1;
-    }
-  }
-  float* hrow = hbuf + ((size_t)t * slots + slot) * I;
-  const int row0 = blockIdx.x * cm.P * NR;
-  if (eid < 0) {  // skipped term: h = 0
-    for (int r = threadIdx.x; r < cm.P * NR; r += blockDim.x)
-      if (row0 + r < I) hrow[row0 + r] = 0.f;
-    return;
-  }
-  const ExpertPtrs ep = table[eid];
-  XQ xg;
-  load_x_group_bf16(x + (size_t)t * H + cm.col * 32, xg);
-
-  const size_t row_bytes = (size_t)H / 2, row_sc = (size_t)G;
-  float v[NV];
-#pragma unroll
-  for (int r = 0; r < NR; ++r) {
-    const int row = row0 + cm.phase * NR + r;
-    float pg = 0.f, pu = 0.f;
-    if (row < I) {
-      const uint4 qg = __ldg(reinterpret_cast<const uint4*>(ep.q_gate + row * row_bytes) + cm.col);
-      const uint4 qu = __ldg(reinterpret_cast<const uint4*>(ep.q_up + row * row_bytes) + cm.col);
-      const float sg = f16_bits_to_f32(__ldg(ep.s_gate + row * row_sc + cm.col));
-      const float su = f16_bits_to_f32(__ldg(ep.s_up + row * row_sc + cm.col));
-      pg = dot_scaled(qg, xg, sg);
-      pu = dot_scaled(qu, xg, su);
-    }
-    v[r] = pg;
-    v[NR + r] = pu;
-  }
-  reduce_scatter<NV, SEG>(v);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int vi = lane % SEG;
-  if (cm.wpr == 1) {
-    const float u = __shfl_down_sync(0xffffffffu, v[0], NR, SEG);
-    const int row = row0 + cm.phase * NR + vi;
-    if (vi < NR && row < I) hrow[row] = silu_mul(v[0], u);
-  } else {
-    red[warp][lane] = v[0];
-    __syncthreads();
-    if (cm.wir == 0 && lane < NR) {
-      float g = 0.f, u = 0.f;
-      for (int w = 0; w < cm.wpr; ++w) {
-        g += red[warp + w][lane];
-        u += red[warp + w][lane + NR];
-      }
-      const int row = row0 + cm.phase * NR + lane;
-      if (row < I) hrow[row] = silu_mul(g, u);
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// int4 down projection with the weighted combine (one token, a block of
-// output rows).  For each row the thread of chunk column `col` accumulates,
-// in slot order, w_j * scale * dot(q_down row chunk, h_j group) over the
-// routed slots and the shared expert (weight 1); one reduce-scatter and a
-// fixed-order cross-warp sum give y[row] directly.  The K = inter dimension
-// is split over the row's threads and reduced without atomics, and no
-// per-expert partial goes to memory.
-// grid.x = row blocks of `hidden`, grid.y = token.
-
-template <int SEG, int NV>
-__global__ void __launch_bounds__(256) down_combine_kernel(
-    const ExpertPtrs* __restrict__ table, const int32_t* __restrict__ idx,
-    const float* __restrict__ wts, int n_experts, int top_k, int slots,
-    const float* __restrict__ hbuf, int H, int I, float* __restrict__ y,
-    uint32_t* __restrict__ err) {
-  __shared__ float red[32][33];
-  const int G = I >> 5;
-  const ColMap cm = col_map(G);
-  const int t = blockIdx.y;
-  const int row0 = blockIdx.x * cm.P * NV;
-  const size_t row_bytes = (size_t)I / 2, row_sc = (size_t)G;
-  float acc[NV];
-#pragma unroll
-  for (int r = 0; r < NV; ++r) acc[r] = 0.f;
-
-  for (int slot = 0; slot < slots; ++slot) {
-    int eid = n_experts;
-    float wj = 1.0f;
-    if (slot < top_k) {
-      eid = idx[(size_t)t * top_k + slot];
-      wj = wts[(size_t)t * top_k + slot];
-      if (eid < 0 || eid >= n_experts) {
-        if (threadIdx.x == 0) atomicCAS(err, 0u, (uint32_t)kErrBadExpertId);
-        continue;
-      }
-    }
-    const ExpertPtrs ep = table[eid];
-    XQ hg;
-    load_x_group_f32(hbuf + ((size_t)t * slots + slot) * I + cm.col * 32, hg);
-#pragma unroll
-    for (int r = 0; r < NV; ++r) {
-      const int row = row0 + cm.phase * NV + r;
-      if (row < H) {
-        const uint4 q = __ldg(reinterpret_cast<const uint4*>(ep.q_down + row * row_bytes) + cm.col);
-        const float sc = f16_bits_to_f32(__ldg(ep.s_down + row * row_sc + cm.col));
-        acc[r] = fmaf(wj, dot_scaled(q, hg, sc), acc[r]);
-      }
-    }
-  }
-  reduce_scatter<NV, SEG>(acc);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int vi = reduce_index<NV, SEG>(lane);
-  const bool owner = (lane % (SEG / NV)) == 0;
-  if (cm.wpr == 1) {
-    const int row = row0 + cm.phase * NV + vi;
-    if (owner && row < H) y[(size_t)t * H + row] = acc[0];
-  } else {
-    red[warp][lane] = acc[0];
-    __syncthreads();
-    if (cm.wir == 0 && owner) {
-      float s = 0.f;
-      for (int w = 0; w < cm.wpr; ++w) s += red[warp + w][lane];
-      const int row = row0 + cm.phase * NV + vi;
-      if (row < H) y[(size_t)t * H + row] = s;
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Plain dequantising int4 GEMV, y[r] = sum_c q[r][c] * scale[r][c/32] * x[c]
-// (fp32 x and y), built from the same group dot product as the layer
-// kernels.  Exposed for one-hot checks of the packing and scale indexing.
 
 template <int SEG, int NV>
 __global__ void __launch_bounds__(256) gemv_int4_kernel(
@@ -403,61 +239,6 @@ cudaError_t launch_select(const float* logits, const float* bias, int T, int E, 
   select_kernel<<<T, 32 * n_group, 0, st>>>(logits, bias, E, n_group, topk_group, top_k, rsf,
                                             idx, w, scores);
   return cudaGetLastError();
-}
-
-template <int SEG>
-static cudaError_t gate_up_seg(const ExpertPtrs* table, const int32_t* idx, int E, int top_k,
-                               int slots, const uint16_t* x, int T, int H, int I, float* hbuf,
-                               uint32_t* err, cudaStream_t st) {
-  const int G = H / 32;
-  const int nw = warps_for(G);
-  const int P = (G >= 32) ? nw / (G / 32) : nw * (32 / G);
-  const int rows = P * (SEG / 2);
-  dim3 grid((I + rows - 1) / rows, T * slots);
-  gate_up_kernel<SEG><<<grid, nw * 32, 0, st>>>(table, idx, E, top_k, slots, x, H, I, hbuf, err);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_gate_up(const ExpertPtrs* table, const int32_t* idx, int E, int top_k,
-                           int slots, const uint16_t* x, int T, int H, int I, float* hbuf,
-                           uint32_t* err, cudaStream_t st) {
-  const int G = H / 32;
-  switch (G >= 32 ? 32 : G) {
-    case 32: return gate_up_seg<32>(table, idx, E, top_k, slots, x, T, H, I, hbuf, err, st);
-    case 16: return gate_up_seg<16>(table, idx, E, top_k, slots, x, T, H, I, hbuf, err, st);
-    case 8: return gate_up_seg<8>(table, idx, E, top_k, slots, x, T, H, I, hbuf, err, st);
-    case 4: return gate_up_seg<4>(table, idx, E, top_k, slots, x, T, H, I, hbuf, err, st);
-    case 2: return gate_up_seg<2>(table, idx, E, top_k, slots, x, T, H, I, hbuf, err, st);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
-template <int SEG, int NV>
-static cudaError_t down_seg(const ExpertPtrs* table, const int32_t* idx, const float* w, int E,
-                            int top_k, int slots, const float* hbuf, int T, int H, int I,
-                            float* y, uint32_t* err, cudaStream_t st) {
-  const int G = I / 32;
-  const int nw = warps_for(G);
-  const int P = (G >= 32) ? nw / (G / 32) : nw * (32 / G);
-  const int rows = P * NV;
-  dim3 grid((H + rows - 1) / rows, T);
-  down_combine_kernel<SEG, NV><<<grid, nw * 32, 0, st>>>(table, idx, w, E, top_k, slots, hbuf,
-                                                         H, I, y, err);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_down_combine(const ExpertPtrs* table, const int32_t* idx, const float* w,
-                                int E, int top_k, int slots, const float* hbuf, int T, int H,
-                                int I, float* y, uint32_t* err, cudaStream_t st) {
-  const int G = I / 32;
-  switch (G >= 32 ? 32 : G) {
-    case 32: return down_seg<32, 4>(table, idx, w, E, top_k, slots, hbuf, T, H, I, y, err, st);
-    case 16: return down_seg<16, 4>(table, idx, w, E, top_k, slots, hbuf, T, H, I, y, err, st);
-    case 8: return down_seg<8, 4>(table, idx, w, E, top_k, slots, hbuf, T, H, I, y, err, st);
-    case 4: return down_seg<4, 4>(table, idx, w, E, top_k, slots, hbuf, T, H, I, y, err, st);
-    case 2: return down_seg<2, 2>(table, idx, w, E, top_k, slots, hbuf, T, H, I, y, err, st);
-    default: return cudaErrorInvalidValue;
-  }
 }
 
 template <int SEG, int NV>

@@ -1,5 +1,5 @@
-// kernels.h -- launchers of the step kernels (kernels.cu) and of the fused
-// decode kernel (decode.cu).
+// kernels.h -- launchers of the step kernels (kernels.cu: router, selection,
+// test GEMV) and of the batched expert path (union.cu).
 #pragma once
 
 #include <cuda_runtime.h>
@@ -14,12 +14,15 @@ cudaError_t launch_router_logits(const float* w, const uint16_t* x, int T, int H
 cudaError_t launch_select(const float* logits, const float* bias, int T, int E, int n_group,
                           int topk_group, int top_k, float rsf, int32_t* idx, float* w,
                           float* scores, cudaStream_t st);
-cudaError_t launch_gate_up(const ExpertPtrs* table, const int32_t* idx, int E, int top_k,
-                           int slots, const uint16_t* x, int T, int H, int I, float* hbuf,
-                           uint32_t* err, cudaStream_t st);
-cudaError_t launch_down_combine(const ExpertPtrs* table, const int32_t* idx, const float* w,
-                                int E, int top_k, int slots, const float* hbuf, int T, int H,
-                                int I, float* y, uint32_t* err, cudaStream_t st);
+// The batched expert path (union.cu): distinct experts read once for all
+// their tokens.  Scratch: xq (T * H/32 groups), hq (T * slots * I/32 groups),
+// lists (union_lists_ints ints), hbuf (T * slots * I), ypart (T * slots * H).
+size_t union_lists_ints(int T, int k, int E, int has_shared);
+cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const float* w,
+                             const uint16_t* x, int T, int H, int I, int E, int k, int has_shared,
+                             uint8_t* xq_words, float* xq_fac, uint8_t* hq_words, float* hq_fac,
+                             int* lists, float* hbuf, float* ypart, float* y, uint32_t* err,
+                             cudaStream_t st);
 
 cudaError_t launch_gemv_int4(const uint8_t* q, const uint16_t* s, int rows, int cols,
                              const float* x, float* y, cudaStream_t st);

@@ -1,0 +1,327 @@
+// union.cu -- the batched (T tokens per call) expert path: every distinct
+// selected expert is read from HBM once for all the tokens routed to it
+// ("colibri", "Notes": batch-union of the experts of the draft tokens; the
+// MTP verify step of "LightLX").
+//
+//   xq_table        x (bf16) or h (fp32) rows -> int16 groups (XQ words and
+//                   factors), once per row, shared by every expert that reads
+//                   the row
+//   build_lists     per-expert token lists from idx [T][k] (one CTA):
+//                   distinct experts in ascending id, the shared expert last
+//                   with all T tokens, entries of each expert in token order
+//   union_gemm<2>   gate/up of one distinct expert for a block of rows and all
+//                   its tokens: h = silu(g) * u, written per (token, slot)
+//   union_gemm<1>   down of one distinct expert: partial y per (token, slot)
+//   combine         y[t] = sum_j w[t][j] ypart[t][j] + ypart[t][shared],
+//                   fixed order, no atomics
+//
+// The group dot product is the exact integer one of the decode kernel
+// (dp2a over int16 inputs); only the order of the fp32 sums differs.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kUnionThreads = 256;
+constexpr int kTokChunk = 16;  // tokens of one expert per pass (fp32 accumulators)
+constexpr int kGroupBlock = 32;  // 32-input groups staged per k step
+constexpr int kListMaxE = 257;   // routed experts + shared
+
+// ---------------------------------------------------------------------------
+template <bool kBf16>
+__global__ void __launch_bounds__(256) xq_table_kernel(const void* __restrict__ in, int rows,
+                                                       int K, uint8_t* __restrict__ words,
+                                                       float* __restrict__ fac) {
+  const int G = K >> 5;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= rows * G) return;
+  const int row = i / G, g = i % G;
+  float xf[32];
+  if (kBf16) {
+    const uint4* p4 =
+        reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(in) + (size_t)row * K + g * 32);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 v = __ldg(p4 + j);
+      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        xf[8 * j + 2 * h] = bf16_bits_to_f32(u[h] & 0xFFFFu);
+        xf[8 * j + 2 * h + 1] = bf16_bits_to_f32(u[h] >> 16);
+      }
+    }
+  } else {
+    const float4* p4 =
+        reinterpret_cast<const float4*>(static_cast<const float*>(in) + (size_t)row * K + g * 32);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 v = p4[j];
+      xf[4 * j] = v.x;
+      xf[4 * j + 1] = v.y;
+      xf[4 * j + 2] = v.z;
+      xf[4 * j + 3] = v.w;
+    }
+  }
+  XQ q;
+  xq_from_floats(xf, q);
+  uint4* dst = reinterpret_cast<uint4*>(words + (size_t)i * 64);
+  dst[0] = make_uint4(q.ev[0], q.ev[1], q.ev[2], q.ev[3]);
+  dst[1] = make_uint4(q.ev[4], q.ev[5], q.ev[6], q.ev[7]);
+  dst[2] = make_uint4(q.od[0], q.od[1], q.od[2], q.od[3]);
+  dst[3] = make_uint4(q.od[4], q.od[5], q.od[6], q.od[7]);
+  fac[i] = q.f;
+}
+
+// ---------------------------------------------------------------------------
+// lists: [0] U; u_expert [E + 1]; u_off [E + 2]; list_tok [T slots];
+// list_pos [T slots] (pos = t * slots + j: the (token, slot) row of hbuf,
+// ypart).  Out-of-range ids set the error word and are left out.
+__global__ void __launch_bounds__(256) build_lists_kernel(const int32_t* __restrict__ idx, int T,
+                                                          int k, int E, int has_shared,
+                                                          int* __restrict__ lists,
+                                                          uint32_t* __restrict__ err) {
+  __shared__ int cnt[kListMaxE];
+  __shared__ int base[kListMaxE];
+  const int slots = k + has_shared;
+  const int n_list = T * slots;
+  int* u_expert = lists + 1;
+  int* u_off = u_expert + (E + 1);
+  int* list_tok = u_off + (E + 2);
+  int* list_pos = list_tok + n_list;
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
+    const int e = idx[i];
+    if (e >= 0 && e < E) {
+      atomicAdd(&cnt[e], 1);
+    } else {
+      atomicCAS(err, 0u, (uint32_t)kErrBadExpertId);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (has_shared) cnt[E] = T;
+    int U = 0, off = 0;
+    for (int e = 0; e <= E; ++e) {
+      if (cnt[e] > 0) {
+        u_expert[U] = e;
+        u_off[U] = off;
+        base[e] = off;
+        off += cnt[e];
+        ++U;
+      }
+    }
+    u_off[U] = off;
+    lists[0] = U;
+  }
+  __syncthreads();
+  // each expert appends its entries in (token, slot) order
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    if (cnt[e] == 0) continue;
+    int pos = base[e];
+    for (int i = 0; i < T * k; ++i) {
+      if (idx[i] == e) {
+        const int t = i / k, j = i % k;
+        list_tok[pos] = t;
+        list_pos[pos] = t * slots + j;
+        ++pos;
+      }
+    }
+  }
+  if (has_shared) {
+    for (int t = threadIdx.x; t < T; t += blockDim.x) {
+      list_tok[base[E] + t] = t;
+      list_pos[base[E] + t] = t * slots + k;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// One distinct expert (blockIdx.y) times a block of rows (blockIdx.x) for all
+// its tokens.  Thread (m, q) = (tid / 4, tid % 4) owns matrix row m of the
+// block (MATS == 2: rows 0..31 gate, 32..63 up; MATS == 1: 64 down rows) and
+// every fourth group of each k step (groups 4i + q); the k step's int16 inputs of up to
+// 16 tokens are staged in shared memory, each weight chunk is loaded once
+// and used for every token.
+struct UnionArgs {
+  const ExpertPtrs* table;
+  const int* lists;
+  int E, n_list;
+  const uint8_t* xq_words;  // [input rows][G] 64-byte XQ words
+  const float* xq_fac;      // [input rows][G]
+  int G;                    // 32-input groups of a matrix row
+  int R;                    // rows of one matrix
+  int in_is_pos;            // input row of an entry: list_pos (1) or list_tok (0)
+  float* out;               // [T slots][R]
+};
+
+template <int MATS>
+__global__ void __launch_bounds__(kUnionThreads) union_gemm_kernel(const UnionArgs a) {
+  constexpr int RBM = 64 / MATS;  // rows of one matrix per CTA
+  // one 16-byte pad per group: the four column quarters of a warp read four
+  // consecutive groups from four different bank quads
+  __shared__ __align__(16) uint4 sX[kTokChunk][kGroupBlock][5];
+  __shared__ float sF[kTokChunk][kGroupBlock];
+  __shared__ float sO[MATS][RBM][kTokChunk + 1];
+  const int U = a.lists[0];
+  const int u = blockIdx.y;
+  if (u >= U) return;  // uniform per CTA, before any barrier
+  const int* u_expert = a.lists + 1;
+  const int* u_off = u_expert + (a.E + 1);
+  const int* list_tok = u_off + (a.E + 2);
+  const int* list_pos = list_tok + a.n_list;
+  const int* in_idx = a.in_is_pos ? list_pos : list_tok;
+  const int e = u_expert[u];
+  const int base = u_off[u], n = u_off[u + 1] - base;
+  const int row0 = blockIdx.x * RBM;
+  const int tid = threadIdx.x, m = tid >> 2, q = tid & 3;
+  const int mat = m / RBM, r = m % RBM, row = row0 + r;
+  const bool active = row < a.R;
+  const ExpertPtrs ep = a.table[e];
+  const uint8_t* codes = (MATS == 2) ? (mat == 0 ? ep.q_gate : ep.q_up) : ep.q_down;
+  const uint16_t* scales = (MATS == 2) ? (mat == 0 ? ep.s_gate : ep.s_up) : ep.s_down;
+  const uint4* wrow = reinterpret_cast<const uint4*>(codes + (size_t)(active ? row : 0) * a.G * 16);
+  const uint16_t* srow = scales + (size_t)(active ? row : 0) * a.G;
+
+  for (int tc = 0; tc < n; tc += kTokChunk) {
+    const int nt = min(kTokChunk, n - tc);
+    float acc[kTokChunk];
+#pragma unroll
+    for (int ti = 0; ti < kTokChunk; ++ti) acc[ti] = 0.f;
+    for (int kb = 0; kb < a.G; kb += kGroupBlock) {
+      const int kbn = min(kGroupBlock, a.G - kb);
+      // this thread's weight chunks of the k step, loaded before the barrier
+      uint4 w[8];
+      float sc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int g = 4 * i + q;
+        const bool ok = active && g < kbn;
+        w[i] = ok ? __ldg(wrow + kb + g) : make_uint4(0, 0, 0, 0);
+        sc[i] = ok ? f16_bits_to_f32(__ldg(srow + kb + g)) : 0.f;
+      }
+      __syncthreads();  // the previous step's inputs are no longer read
+      for (int i = tid; i < nt * kbn * 4; i += kUnionThreads) {
+        const int ti = i / (kbn * 4), rem = i % (kbn * 4);
+        const int rin = in_idx[base + tc + ti];
+        sX[ti][rem >> 2][rem & 3] = *reinterpret_cast<const uint4*>(
+            a.xq_words + ((size_t)rin * a.G + kb + (rem >> 2)) * 64 + (rem & 3) * 16);
+      }
+      for (int i = tid; i < nt * kbn; i += kUnionThreads) {
+        const int ti = i / kbn, gi = i % kbn;
+        sF[ti][gi] = a.xq_fac[(size_t)in_idx[base + tc + ti] * a.G + kb + gi];
+      }
+      __syncthreads();
+#pragma unroll
+      for (int ti = 0; ti < kTokChunk; ++ti) {
+        if (ti < nt) {
+          float s = 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int g = 4 * i + q;
+            if (g < kbn) {
+              XQ xg;
+              const uint4 a0 = sX[ti][g][0], a1 = sX[ti][g][1], a2 = sX[ti][g][2], a3 = sX[ti][g][3];
+              xg.ev[0] = a0.x; xg.ev[1] = a0.y; xg.ev[2] = a0.z; xg.ev[3] = a0.w;
+              xg.ev[4] = a1.x; xg.ev[5] = a1.y; xg.ev[6] = a1.z; xg.ev[7] = a1.w;
+              xg.od[0] = a2.x; xg.od[1] = a2.y; xg.od[2] = a2.z; xg.od[3] = a2.w;
+              xg.od[4] = a3.x; xg.od[5] = a3.y; xg.od[6] = a3.z; xg.od[7] = a3.w;
+              xg.f = sF[ti][g];
+              s += dot_scaled(w[i], xg, sc[i]);
+            }
+          }
+          acc[ti] += s;
+        }
+      }
+    }
+    // the four column quarters of a row are lanes 4m .. 4m+3
+#pragma unroll
+    for (int ti = 0; ti < kTokChunk; ++ti) {
+      acc[ti] += __shfl_xor_sync(0xffffffffu, acc[ti], 1);
+      acc[ti] += __shfl_xor_sync(0xffffffffu, acc[ti], 2);
+    }
+    if (q == 0) {
+#pragma unroll
+      for (int ti = 0; ti < kTokChunk; ++ti) sO[mat][r][ti] = acc[ti];
+    }
+    __syncthreads();
+    for (int i = tid; i < RBM * nt; i += kUnionThreads) {
+      const int rr = i % RBM, ti = i / RBM;
+      if (row0 + rr < a.R) {
+        const float v = (MATS == 2) ? silu_mul(sO[0][rr][ti], sO[1][rr][ti]) : sO[0][rr][ti];
+        a.out[(size_t)list_pos[base + tc + ti] * a.R + row0 + rr] = v;
+      }
+    }
+    __syncthreads();  // sO is rewritten by the next token chunk
+  }
+}
+
+// y[t][row] = sum_j w[t][j] * ypart[t][j][row] (+ the shared expert's row),
+// in slot order; terms of out-of-range ids are left out.
+__global__ void __launch_bounds__(256) union_combine_kernel(
+    const int32_t* __restrict__ idx, const float* __restrict__ w, const float* __restrict__ ypart,
+    int T, int H, int k, int E, int has_shared, float* __restrict__ y) {
+  const int t = blockIdx.y;
+  const int row = blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= H) return;
+  const int slots = k + has_shared;
+  float acc = 0.f;
+  for (int j = 0; j < k; ++j) {
+    const int e = idx[t * k + j];
+    if (e >= 0 && e < E)
+      acc = fmaf(w[t * k + j], ypart[((size_t)t * slots + j) * H + row], acc);
+  }
+  if (has_shared) acc += ypart[((size_t)t * slots + k) * H + row];
+  y[(size_t)t * H + row] = acc;
+}
+
+}  // namespace
+
+size_t union_lists_ints(int T, int k, int E, int has_shared) {
+  return 1 + (size_t)(E + 1) + (E + 2) + 2 * (size_t)T * (k + has_shared);
+}
+
+cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const float* w,
+                             const uint16_t* x, int T, int H, int I, int E, int k, int has_shared,
+                             uint8_t* xq_words, float* xq_fac, uint8_t* hq_words, float* hq_fac,
+                             int* lists, float* hbuf, float* ypart, float* y, uint32_t* err,
+                             cudaStream_t st) {
+  if (E + 1 > kListMaxE) return cudaErrorInvalidValue;
+  const int slots = k + has_shared;
+  const int G = H / 32, GD = I / 32;
+  const int n_list = T * slots;
+  const int umax = (E < T * k ? E : T * k) + has_shared;
+  xq_table_kernel<true><<<(T * G + 255) / 256, 256, 0, st>>>(x, T, H, xq_words, xq_fac);
+  build_lists_kernel<<<1, 256, 0, st>>>(idx, T, k, E, has_shared, lists, err);
+  UnionArgs a;
+  a.table = table;
+  a.lists = lists;
+  a.E = E;
+  a.n_list = n_list;
+  a.xq_words = xq_words;
+  a.xq_fac = xq_fac;
+  a.G = G;
+  a.R = I;
+  a.in_is_pos = 0;
+  a.out = hbuf;
+  union_gemm_kernel<2><<<dim3((I + 31) / 32, umax), kUnionThreads, 0, st>>>(a);
+  xq_table_kernel<false><<<(n_list * GD + 255) / 256, 256, 0, st>>>(hbuf, n_list, I, hq_words,
+                                                                    hq_fac);
+  a.xq_words = hq_words;
+  a.xq_fac = hq_fac;
+  a.G = GD;
+  a.R = H;
+  a.in_is_pos = 1;
+  a.out = ypart;
+  union_gemm_kernel<1><<<dim3((H + 63) / 64, umax), kUnionThreads, 0, st>>>(a);
+  union_combine_kernel<<<dim3((H + 255) / 256, T), 256, 0, st>>>(idx, w, ypart, T, H, k, E,
+                                                                 has_shared, y);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

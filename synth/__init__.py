@@ -151,6 +151,30 @@ def expert(shape, seed, layer, expert_id):
     return out
 
 
+def expert_into(shape, seed, layer, expert_id, base_ptr):
+    """Generate one expert (same values as expert()) into caller memory at
+    base_ptr, laid out as expert_layout(shape) in order, each tensor 256-byte
+    aligned; returns {name: byte offset}."""
+    lib = _load_host()
+    offs, off = {}, 0
+    for name, dt, shp, tag in expert_layout(shape):
+        n = int(np.prod(shp))
+        k = key(seed, layer, expert_id, tag)
+        if dt == np.uint8:
+            lib.synth_fill_bytes(k, ctypes.c_void_p(base_ptr + off), n)
+        else:
+            lib.synth_fill_scales_f16(k, ctypes.c_void_p(base_ptr + off), n, SCALE_LO, SCALE_HI)
+        offs[name] = off
+        off += (n * np.dtype(dt).itemsize + 255) // 256 * 256
+    return offs
+
+
+def expert_stride(shape):
+    """Bytes one expert takes in expert_into's layout."""
+    return sum((int(np.prod(shp)) * np.dtype(dt).itemsize + 255) // 256 * 256
+               for _, dt, shp, _ in expert_layout(shape))
+
+
 def router(shape, seed, layer):
     """Router weight fp32 [E][H] ~ N(0, 0.02) and bias fp32 [E] ~ U(-0.1, 0.1)."""
     lib = _load_host()

@@ -20,19 +20,23 @@ def expert_offsets(shape):
 class DeviceLayer:
     """Synthetic layer `layer` of `seed` on the current CUDA device."""
 
-    def __init__(self, shape, seed, layer, device="cuda", stream=None):
+    def __init__(self, shape, seed, layer, device="cuda", stream=None, routed=True):
+        """routed=False: router, bias and shared expert only (the routed
+        experts live elsewhere, e.g. in a pinned host store)."""
         import torch
         self.shape, self.seed, self.layer = shape, seed, layer
         n = shape.n_experts + shape.n_shared
-        self.slab = torch.empty(n * shape.expert_bytes, dtype=torch.uint8, device=device)
+        ids = list(range(n)) if routed else list(range(shape.n_experts, n))
+        self.slab = torch.empty(max(1, len(ids)) * shape.expert_bytes, dtype=torch.uint8,
+                                device=device)
         base = self.slab.data_ptr()
         offs = expert_offsets(shape)
         st = (stream or torch.cuda.current_stream()).cuda_stream
-        self.experts = []
-        for e in range(n):
-            ptrs = {k: base + e * shape.expert_bytes + o for k, o in offs.items()}
+        self.experts = [None] * n
+        for i, e in enumerate(ids):
+            ptrs = {k: base + i * shape.expert_bytes + o for k, o in offs.items()}
             synth.fill_expert_device(shape, seed, layer, e, ptrs, st)
-            self.experts.append(ptrs)
+            self.experts[e] = ptrs
         w, b = synth.router(shape, seed, layer)
         self.w_router = torch.from_numpy(w).to(device)
         self.bias = torch.from_numpy(b).to(device)

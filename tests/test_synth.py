@@ -87,3 +87,12 @@ def test_device_generator_matches_host():
     for name, dt, shp, tag in synth.expert_layout(sh):
         dev = bufs[name].cpu().numpy().view(dt).reshape(shp)
         assert np.array_equal(dev, host[name]), name
+
+
+def test_expert_into_matches_expert():
+    # the in-place generator (pinned host stores) gives the same tensors
+    buf = np.zeros(synth.expert_stride(synth.TINY), dtype=np.uint8)
+    offs = synth.expert_into(synth.TINY, 0, 2, 5, buf.ctypes.data)
+    for name, a in synth.expert(synth.TINY, 0, 2, 5).items():
+        got = buf[offs[name]:offs[name] + a.nbytes].view(a.dtype).reshape(a.shape)
+        assert np.array_equal(got, a), name
