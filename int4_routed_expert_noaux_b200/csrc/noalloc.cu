@@ -12,7 +12,7 @@ namespace moe {
 
 // Largest scratch the call takes: the one-token workspace of the shape,
 // ws_layout(cfg, 1).total.  A 6144 x 2048 layer with top-8 of 256 experts
-// and one shared expert needs 301,568 bytes.
+// and one shared expert needs 356,096 bytes.
 constexpr size_t kStaticScratchBytes = 512u << 10;
 constexpr int kStaticMaxDevices = 64;
 // control words plus the largest router score area (256 experts x 8 bytes)
