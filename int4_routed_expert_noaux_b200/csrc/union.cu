@@ -20,6 +20,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "async.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -28,8 +29,6 @@ namespace moe {
 namespace {
 
 constexpr int kUnionThreads = 256;
-constexpr int kTokChunk = 16;  // tokens of one expert per pass (fp32 accumulators)
-constexpr int kGroupBlock = 32;  // 32-input groups staged per k step
 constexpr int kListMaxE = 257;   // routed experts + shared
 
 // ---------------------------------------------------------------------------
@@ -143,11 +142,13 @@ __global__ void __launch_bounds__(256) build_lists_kernel(const int32_t* __restr
 
 // ---------------------------------------------------------------------------
 // One distinct expert (blockIdx.y) times a block of rows (blockIdx.x) for all
-// its tokens.  Thread (m, q) = (tid / 4, tid % 4) owns matrix row m of the
-// block (MATS == 2: rows 0..31 gate, 32..63 up; MATS == 1: 64 down rows) and
-// every fourth group of each k step (groups 4i + q); the k step's int16 inputs of up to
-// 16 tokens are staged in shared memory, each weight chunk is loaded once
-// and used for every token.
+// its tokens, up to kTok tokens per pass.  Thread (m, q) = (warp * 8 +
+// lane % 8, lane / 8) owns matrix row m of the block (MATS == 2: rows 0..31
+// gate, 32..63 up; MATS == 1: 64 down rows) and groups 4i + q of each k step.
+// A k step (kKB groups) of weights, scales and the tokens' int16 inputs is
+// brought into shared memory by cp.async, kNS - 1 steps ahead of the step
+// being computed, so DRAM latency overlaps the dot products; every weight
+// chunk is read from HBM once per pass and used for every token of the pass.
 struct UnionArgs {
   const ExpertPtrs* table;
   const int* lists;
@@ -160,14 +161,49 @@ struct UnionArgs {
   float* out;               // [T slots][R]
 };
 
+constexpr int kTok = 8;     // tokens per pass
+constexpr int kKB = 16;     // groups per k step
+constexpr int kNS = 3;      // pipeline stages
+constexpr int kRowPad = kKB + 1;  // chunks per staged row: 8 consecutive rows hit 8 bank quads
+
+struct UStage {
+  uint4 w[64][kRowPad];     // weight chunks of the block's 64 matrix rows
+  uint16_t s[64][kKB];      // their fp16 scales
+  uint4 x[kTok][kKB][4];    // XQ words of the pass's tokens
+  float f[kTok][kKB];       // XQ factors
+};
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async4(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_addr(dst)), "l"(src),
+               "r"(valid ? 4 : 0)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+size_t union_smem_bytes(int mats) {
+  return (size_t)kNS * sizeof(UStage) + (size_t)mats * (64 / mats) * (kTok + 1) * sizeof(float);
+}
+
 template <int MATS>
 __global__ void __launch_bounds__(kUnionThreads) union_gemm_kernel(const UnionArgs a) {
   constexpr int RBM = 64 / MATS;  // rows of one matrix per CTA
-  // one 16-byte pad per group: the four column quarters of a warp read four
-  // consecutive groups from four different bank quads
-  __shared__ __align__(16) uint4 sX[kTokChunk][kGroupBlock][5];
-  __shared__ float sF[kTokChunk][kGroupBlock];
-  __shared__ float sO[MATS][RBM][kTokChunk + 1];
+  extern __shared__ __align__(16) uint8_t usmem[];
+  UStage* st = reinterpret_cast<UStage*>(usmem);
+  float(*sO)[RBM][kTok + 1] = reinterpret_cast<float(*)[RBM][kTok + 1]>(usmem + kNS * sizeof(UStage));
   const int U = a.lists[0];
   const int u = blockIdx.y;
   if (u >= U) return;  // uniform per CTA, before any barrier
@@ -179,75 +215,95 @@ __global__ void __launch_bounds__(kUnionThreads) union_gemm_kernel(const UnionAr
   const int e = u_expert[u];
   const int base = u_off[u], n = u_off[u + 1] - base;
   const int row0 = blockIdx.x * RBM;
-  const int tid = threadIdx.x, m = tid >> 2, q = tid & 3;
-  const int mat = m / RBM, r = m % RBM, row = row0 + r;
-  const bool active = row < a.R;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int m = (tid >> 5) * 8 + (lane & 7), q = lane >> 3;
+  const int mat = m / RBM, r = m % RBM;
   const ExpertPtrs ep = a.table[e];
-  const uint8_t* codes = (MATS == 2) ? (mat == 0 ? ep.q_gate : ep.q_up) : ep.q_down;
-  const uint16_t* scales = (MATS == 2) ? (mat == 0 ? ep.s_gate : ep.s_up) : ep.s_down;
-  const uint4* wrow = reinterpret_cast<const uint4*>(codes + (size_t)(active ? row : 0) * a.G * 16);
-  const uint16_t* srow = scales + (size_t)(active ? row : 0) * a.G;
+  const int nk = (a.G + kKB - 1) / kKB;
 
-  for (int tc = 0; tc < n; tc += kTokChunk) {
-    const int nt = min(kTokChunk, n - tc);
-    float acc[kTokChunk];
+  // issue the copies of k step ks of the pass starting at token tc into stage sb
+  auto issue = [&](int sb, int ks, int tc, int nt) {
+    UStage& S = st[sb];
+    const int kb = ks * kKB, kbn = min(kKB, a.G - kb);
+    for (int c = tid; c < 64 * kKB; c += kUnionThreads) {  // weight chunks
+      const int mm = c / kKB, g = c % kKB;
+      const int rr = row0 + mm % RBM;
+      const uint8_t* codes = (MATS == 2) ? ((mm / RBM) == 0 ? ep.q_gate : ep.q_up) : ep.q_down;
+      const bool ok = rr < a.R && g < kbn;
+      cp_async16(&S.w[mm][g], codes + ((size_t)(ok ? rr : row0) * a.G + kb + (ok ? g : 0)) * 16, ok);
+    }
+    for (int c = tid; c < 64 * (kKB / 2); c += kUnionThreads) {  // scale pairs
+      const int mm = c / (kKB / 2), g = 2 * (c % (kKB / 2));
+      const int rr = row0 + mm % RBM;
+      const uint16_t* sc = (MATS == 2) ? ((mm / RBM) == 0 ? ep.s_gate : ep.s_up) : ep.s_down;
+      const bool ok = rr < a.R && g < kbn;
+      cp_async4(&S.s[mm][g], sc + (size_t)(ok ? rr : row0) * a.G + kb + (ok ? g : 0), ok);
+    }
+    for (int c = tid; c < kTok * kKB * 4; c += kUnionThreads) {  // token inputs
+      const int ti = c / (kKB * 4), g = (c / 4) % kKB, wv = c % 4;
+      const bool ok = ti < nt && g < kbn;
+      const int rin = in_idx[base + tc + (ok ? ti : 0)];
+      cp_async16(&S.x[ti][g][wv],
+                 a.xq_words + ((size_t)rin * a.G + kb + (ok ? g : 0)) * 64 + wv * 16, ok);
+    }
+    for (int c = tid; c < kTok * kKB; c += kUnionThreads) {
+      const int ti = c / kKB, g = c % kKB;
+      const bool ok = ti < nt && g < kbn;
+      const int rin = in_idx[base + tc + (ok ? ti : 0)];
+      cp_async4(&S.f[ti][g], a.xq_fac + (size_t)rin * a.G + kb + (ok ? g : 0), ok);
+    }
+  };
+
+  for (int tc = 0; tc < n; tc += kTok) {
+    const int nt = min(kTok, n - tc);
+    float acc[kTok];
 #pragma unroll
-    for (int ti = 0; ti < kTokChunk; ++ti) acc[ti] = 0.f;
-    for (int kb = 0; kb < a.G; kb += kGroupBlock) {
-      const int kbn = min(kGroupBlock, a.G - kb);
-      // this thread's weight chunks of the k step, loaded before the barrier
-      uint4 w[8];
-      float sc[8];
+    for (int ti = 0; ti < kTok; ++ti) acc[ti] = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+    for (int s0 = 0; s0 < kNS - 1; ++s0) {
+      if (s0 < nk) issue(s0, s0, tc, nt);
+      cp_async_commit();
+    }
+    for (int ks = 0; ks < nk; ++ks) {
+      cp_async_wait<kNS - 2>();  // step ks has landed (this thread's copies)
+      __syncthreads();           // ... everyone's; step ks - 1 is no longer read
+      if (ks + kNS - 1 < nk) issue((ks + kNS - 1) % kNS, ks + kNS - 1, tc, nt);
+      cp_async_commit();
+      const UStage& S = st[ks % kNS];
+      const int kbn = min(kKB, a.G - ks * kKB);
+#pragma unroll
+      for (int i = 0; i < kKB / 4; ++i) {
         const int g = 4 * i + q;
-        const bool ok = active && g < kbn;
-        w[i] = ok ? __ldg(wrow + kb + g) : make_uint4(0, 0, 0, 0);
-        sc[i] = ok ? f16_bits_to_f32(__ldg(srow + kb + g)) : 0.f;
-      }
-      __syncthreads();  // the previous step's inputs are no longer read
-      for (int i = tid; i < nt * kbn * 4; i += kUnionThreads) {
-        const int ti = i / (kbn * 4), rem = i % (kbn * 4);
-        const int rin = in_idx[base + tc + ti];
-        sX[ti][rem >> 2][rem & 3] = *reinterpret_cast<const uint4*>(
-            a.xq_words + ((size_t)rin * a.G + kb + (rem >> 2)) * 64 + (rem & 3) * 16);
-      }
-      for (int i = tid; i < nt * kbn; i += kUnionThreads) {
-        const int ti = i / kbn, gi = i % kbn;
-        sF[ti][gi] = a.xq_fac[(size_t)in_idx[base + tc + ti] * a.G + kb + gi];
-      }
-      __syncthreads();
+        if (g < kbn) {
+          const uint4 w = S.w[m][g];
+          const float sc = f16_bits_to_f32(S.s[m][g]);
 #pragma unroll
-      for (int ti = 0; ti < kTokChunk; ++ti) {
-        if (ti < nt) {
-          float s = 0.f;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int g = 4 * i + q;
-            if (g < kbn) {
+          for (int ti = 0; ti < kTok; ++ti) {
+            if (ti < nt) {
               XQ xg;
-              const uint4 a0 = sX[ti][g][0], a1 = sX[ti][g][1], a2 = sX[ti][g][2], a3 = sX[ti][g][3];
+              const uint4 a0 = S.x[ti][g][0], a1 = S.x[ti][g][1], a2 = S.x[ti][g][2],
+                          a3 = S.x[ti][g][3];
               xg.ev[0] = a0.x; xg.ev[1] = a0.y; xg.ev[2] = a0.z; xg.ev[3] = a0.w;
               xg.ev[4] = a1.x; xg.ev[5] = a1.y; xg.ev[6] = a1.z; xg.ev[7] = a1.w;
               xg.od[0] = a2.x; xg.od[1] = a2.y; xg.od[2] = a2.z; xg.od[3] = a2.w;
               xg.od[4] = a3.x; xg.od[5] = a3.y; xg.od[6] = a3.z; xg.od[7] = a3.w;
-              xg.f = sF[ti][g];
-              s += dot_scaled(w[i], xg, sc[i]);
+              xg.f = S.f[ti][g];
+              acc[ti] += dot_scaled(w, xg, sc);
             }
           }
-          acc[ti] += s;
         }
       }
     }
-    // the four column quarters of a row are lanes 4m .. 4m+3
+    cp_async_wait<0>();
+    // the four column quarters of a row are lanes l, l + 8, l + 16, l + 24
 #pragma unroll
-    for (int ti = 0; ti < kTokChunk; ++ti) {
-      acc[ti] += __shfl_xor_sync(0xffffffffu, acc[ti], 1);
-      acc[ti] += __shfl_xor_sync(0xffffffffu, acc[ti], 2);
+    for (int ti = 0; ti < kTok; ++ti) {
+      acc[ti] += __shfl_xor_sync(0xffffffffu, acc[ti], 8);
+      acc[ti] += __shfl_xor_sync(0xffffffffu, acc[ti], 16);
     }
     if (q == 0) {
 #pragma unroll
-      for (int ti = 0; ti < kTokChunk; ++ti) sO[mat][r][ti] = acc[ti];
+      for (int ti = 0; ti < kTok; ++ti) sO[mat][r][ti] = acc[ti];
     }
     __syncthreads();
     for (int i = tid; i < RBM * nt; i += kUnionThreads) {
@@ -257,7 +313,7 @@ __global__ void __launch_bounds__(kUnionThreads) union_gemm_kernel(const UnionAr
         a.out[(size_t)list_pos[base + tc + ti] * a.R + row0 + rr] = v;
       }
     }
-    __syncthreads();  // sO is rewritten by the next token chunk
+    __syncthreads();  // sO and the stages are rewritten by the next pass
   }
 }
 
@@ -309,7 +365,20 @@ cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const 
   a.R = I;
   a.in_is_pos = 0;
   a.out = hbuf;
-  union_gemm_kernel<2><<<dim3((I + 31) / 32, umax), kUnionThreads, 0, st>>>(a);
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    cudaError_t ce = cudaFuncSetAttribute(union_gemm_kernel<2>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)union_smem_bytes(2));
+    if (ce == cudaSuccess)
+      ce = cudaFuncSetAttribute(union_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)union_smem_bytes(1));
+    if (ce != cudaSuccess) return ce;
+    configured[dev] = true;
+  }
+  union_gemm_kernel<2><<<dim3((I + 31) / 32, umax), kUnionThreads, union_smem_bytes(2), st>>>(a);
   xq_table_kernel<false><<<(n_list * GD + 255) / 256, 256, 0, st>>>(hbuf, n_list, I, hq_words,
                                                                     hq_fac);
   a.xq_words = hq_words;
@@ -318,7 +387,7 @@ cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const 
   a.R = H;
   a.in_is_pos = 1;
   a.out = ypart;
-  union_gemm_kernel<1><<<dim3((H + 63) / 64, umax), kUnionThreads, 0, st>>>(a);
+  union_gemm_kernel<1><<<dim3((H + 63) / 64, umax), kUnionThreads, union_smem_bytes(1), st>>>(a);
   union_combine_kernel<<<dim3((H + 255) / 256, T), 256, 0, st>>>(idx, w, ypart, T, H, k, E,
                                                                  has_shared, y);
   return cudaGetLastError();
