@@ -301,13 +301,10 @@ def main():
     ms = ev0.elapsed_time(ev1)
     moe.ws_check(ws, stream)
     if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dist)
         dist.barrier()
     ms_step = ms / args.steps
-    tokens_total = n * args.steps * world
-    value = tokens_total / (ms / 1000.0)
+    value = job_rate(n * args.steps, world, ms)
 
     # e2e: host buffers, per-token pinned H2D of x and D2H of y in the timed region
     x_host = torch.from_numpy(x_bits.view(np.int16)).pin_memory()
@@ -337,10 +334,8 @@ def main():
     stream.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     if dist:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = n * e2e_steps * world / (e2e_ms / 1000.0)
+        e2e_ms = max_over_ranks(e2e_ms, dist)
+    e2e_value = job_rate(n * e2e_steps, world, e2e_ms)
     if not np.all(np.isfinite(y_host.numpy())):
         raise RuntimeError("non-finite outputs")
 
@@ -383,6 +378,22 @@ def main():
 
 def launches_per_forward():
     return 1
+
+
+def max_over_ranks(value, dist=None, device="cuda"):
+    """The largest value over all ranks (every rank gets it): a multi-GPU
+    time is the slowest rank's."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank, world, ms):
+    """Whole-job throughput: units of all ranks over the slowest rank's time."""
+    return units_per_rank * world / (ms / 1000.0)
 
 
 # ---------------------------------------------------------------------------
