@@ -79,10 +79,15 @@ def algorithmic_bytes_per_token(shape):
     return ((shape.top_k + shape.n_shared) * shape.expert_bytes + E * H * 4 + E * 4 + H * 2 + H * 4)
 
 
+DECODE_SOURCES = ("decode.cu", "decode.h", "common.cuh", "async.cuh", "forward.cu")
+
+
 def kernel_source_hash():
+    """Hash of the sources of the one-token decode kernel (the kernel the
+    roofline's traffic figure belongs to)."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "int4_routed_expert_noaux_b200", "csrc")
-    for fn in sorted(os.listdir(d)):
+    for fn in DECODE_SOURCES:
         h.update(open(os.path.join(d, fn), "rb").read())
     return h.hexdigest()[:16]
 

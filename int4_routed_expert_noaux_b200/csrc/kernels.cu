@@ -12,24 +12,24 @@ namespace moe {
 
 // ---------------------------------------------------------------------------
 // Router GEMV ("LightLX", "How it works": one router logit per routed
-// expert).  One warp per expert row of W (fp32 [E][H]); lanes stride the row
-// in 16-byte chunks (4 weights); all T tokens are accumulated per chunk.
-// logits [T][E].
+// expert).  One CTA per expert row of W (fp32 [E][H]): each thread holds its
+// 16-byte chunks of the row and accumulates them against TT tokens at a
+// time; a block reduction gives the TT logits.  logits [T][E].
 
 template <int TT>
 __global__ void __launch_bounds__(256) router_logits_kernel(
     const float* __restrict__ w, const uint16_t* __restrict__ x, int T, int H,
     int E, float* __restrict__ logits) {
+  __shared__ float red[TT][8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (e >= E) return;
+  const int e = blockIdx.x;
   const float4* wr = reinterpret_cast<const float4*>(w + (size_t)e * H);
   const int nchunk = H >> 2;
   for (int t0 = 0; t0 < T; t0 += TT) {
     float acc[TT];
 #pragma unroll
     for (int t = 0; t < TT; ++t) acc[t] = 0.f;
-    for (int c = lane; c < nchunk; c += 32) {
+    for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
       const float4 wv = __ldg(wr + c);
 #pragma unroll
       for (int t = 0; t < TT; ++t) {
@@ -45,8 +45,15 @@ __global__ void __launch_bounds__(256) router_logits_kernel(
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
       const float s = warp_sum(acc[t]);
-      if (lane == 0 && t0 + t < T) logits[(size_t)(t0 + t) * E + e] = s;
+      if (lane == 0) red[t][warp] = s;
     }
+    __syncthreads();
+    if (threadIdx.x < TT && t0 + threadIdx.x < T) {
+      float s = 0.f;
+      for (int w8 = 0; w8 < (int)(blockDim.x >> 5); ++w8) s += red[threadIdx.x][w8];
+      logits[(size_t)(t0 + threadIdx.x) * E + e] = s;
+    }
+    __syncthreads();
   }
 }
 
@@ -228,8 +235,7 @@ static int warps_for(int G) {
 
 cudaError_t launch_router_logits(const float* w, const uint16_t* x, int T, int H, int E,
                                  float* logits, cudaStream_t st) {
-  const int wpb = 8;
-  router_logits_kernel<8><<<(E + wpb - 1) / wpb, wpb * 32, 0, st>>>(w, x, T, H, E, logits);
+  router_logits_kernel<8><<<E, 256, 0, st>>>(w, x, T, H, E, logits);
   return cudaGetLastError();
 }
 

@@ -103,20 +103,53 @@ __global__ void __launch_bounds__(256) build_lists_kernel(const int32_t* __restr
     }
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    if (has_shared) cnt[E] = T;
-    int U = 0, off = 0;
-    for (int e = 0; e <= E; ++e) {
-      if (cnt[e] > 0) {
-        u_expert[U] = e;
-        u_off[U] = off;
-        base[e] = off;
-        off += cnt[e];
-        ++U;
+  if (threadIdx.x == 0 && has_shared) cnt[E] = T;
+  __syncthreads();
+  // exclusive scans of (expert used, entries) over experts 0..E, ascending:
+  // thread i owns experts 2i and 2i + 1 (E + 1 <= 512)
+  {
+    __shared__ int wu[8], ws[8];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int e0 = 2 * threadIdx.x, e1 = e0 + 1;
+    const int c0 = e0 <= E ? cnt[e0] : 0, c1 = e1 <= E ? cnt[e1] : 0;
+    const int nu = (c0 > 0) + (c1 > 0), ns = c0 + c1;
+    int iu = nu, is = ns;  // inclusive warp scans
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, iu, o), b = __shfl_up_sync(0xffffffffu, is, o);
+      if (lane >= o) {
+        iu += a;
+        is += b;
       }
     }
-    u_off[U] = off;
-    lists[0] = U;
+    if (lane == 31) {
+      wu[warp] = iu;
+      ws[warp] = is;
+    }
+    __syncthreads();
+    int bu = 0, bs = 0;
+    for (int w = 0; w < warp; ++w) {
+      bu += wu[w];
+      bs += ws[w];
+    }
+    int uu = bu + iu - nu, off = bs + is - ns;  // exclusive prefixes
+    if (c0 > 0) {
+      u_expert[uu] = e0;
+      u_off[uu] = off;
+      base[e0] = off;
+      ++uu;
+      off += c0;
+    }
+    if (c1 > 0) {
+      u_expert[uu] = e1;
+      u_off[uu] = off;
+      base[e1] = off;
+    }
+    if (threadIdx.x == blockDim.x - 1) {
+      const int U = bu + iu, total = bs + is;
+      u_off[U] = total;
+      lists[0] = U;
+    }
   }
   __syncthreads();
   // each expert appends its entries in (token, slot) order
