@@ -254,53 +254,90 @@ __global__ void __launch_bounds__(kUnionThreads) union_gemm_kernel(const UnionAr
   const ExpertPtrs ep = a.table[e];
   const int nk = (a.G + kKB - 1) / kKB;
 
-  // issue the copies of k step ks of the pass starting at token tc into stage sb
-  auto issue = [&](int sb, int ks, int tc, int nt) {
+  static_assert(64 * kKB == 4 * kUnionThreads && 64 * kKB / 2 == 2 * kUnionThreads &&
+                    kTok * kKB * 4 == 2 * kUnionThreads && kTok * kKB <= kUnionThreads,
+                "the copy assignment below");
+  // This thread's copies of every k step, as source pointers advanced by the
+  // step: weight chunks (4), scale pairs (2), token input chunks (2) and one
+  // token factor.  Row sources are fixed for the CTA, token sources per pass.
+  const int gw_ = tid & (kKB - 1), gs_ = 2 * (tid & (kKB / 2 - 1));
+  const uint8_t* wsrc[4];
+  bool wok[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int mm = (tid >> 4) + 16 * j, rr = row0 + mm % RBM;
+    const uint8_t* codes = (MATS == 2) ? ((mm / RBM) == 0 ? ep.q_gate : ep.q_up) : ep.q_down;
+    wok[j] = rr < a.R;
+    wsrc[j] = codes + ((size_t)(wok[j] ? rr : row0) * a.G + min(gw_, a.G - 1)) * 16;
+  }
+  const uint16_t* ssrc[2];
+  bool sok[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int mm = (tid >> 3) + 32 * j, rr = row0 + mm % RBM;
+    const uint16_t* sc = (MATS == 2) ? ((mm / RBM) == 0 ? ep.s_gate : ep.s_up) : ep.s_down;
+    sok[j] = rr < a.R;
+    ssrc[j] = sc + (size_t)(sok[j] ? rr : row0) * a.G + min(gs_, a.G - 2);
+  }
+  const int xg_ = (tid >> 2) & (kKB - 1), xw_ = tid & 3;
+  const uint8_t* xsrc[2];
+  bool xok[2];
+  const float* fsrc = a.xq_fac;
+  bool fok = false;
+
+  // a copy that is not needed (row or token past the end, group past the
+  // step) reads nothing (source size 0) from its in-range base pointer
+  auto issue = [&](int sb, int ks) {
     UStage& S = st[sb];
     const int kb = ks * kKB, kbn = min(kKB, a.G - kb);
-    for (int c = tid; c < 64 * kKB; c += kUnionThreads) {  // weight chunks
-      const int mm = c / kKB, g = c % kKB;
-      const int rr = row0 + mm % RBM;
-      const uint8_t* codes = (MATS == 2) ? ((mm / RBM) == 0 ? ep.q_gate : ep.q_up) : ep.q_down;
-      const bool ok = rr < a.R && g < kbn;
-      cp_async16(&S.w[mm][g], codes + ((size_t)(ok ? rr : row0) * a.G + kb + (ok ? g : 0)) * 16, ok);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const bool ok = wok[j] && gw_ < kbn;
+      cp_async16(&S.w[(tid >> 4) + 16 * j][gw_], ok ? wsrc[j] + (size_t)kb * 16 : wsrc[j], ok);
     }
-    for (int c = tid; c < 64 * (kKB / 2); c += kUnionThreads) {  // scale pairs
-      const int mm = c / (kKB / 2), g = 2 * (c % (kKB / 2));
-      const int rr = row0 + mm % RBM;
-      const uint16_t* sc = (MATS == 2) ? ((mm / RBM) == 0 ? ep.s_gate : ep.s_up) : ep.s_down;
-      const bool ok = rr < a.R && g < kbn;
-      cp_async4(&S.s[mm][g], sc + (size_t)(ok ? rr : row0) * a.G + kb + (ok ? g : 0), ok);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const bool ok = sok[j] && gs_ < kbn;
+      cp_async4(&S.s[(tid >> 3) + 32 * j][gs_], ok ? ssrc[j] + kb : ssrc[j], ok);
     }
-    for (int c = tid; c < kTok * kKB * 4; c += kUnionThreads) {  // token inputs
-      const int ti = c / (kKB * 4), g = (c / 4) % kKB, wv = c % 4;
-      const bool ok = ti < nt && g < kbn;
-      const int rin = in_idx[base + tc + (ok ? ti : 0)];
-      cp_async16(&S.x[ti][g][wv],
-                 a.xq_words + ((size_t)rin * a.G + kb + (ok ? g : 0)) * 64 + wv * 16, ok);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const bool ok = xok[j] && xg_ < kbn;
+      cp_async16(&S.x[(tid >> 6) + 4 * j][xg_][xw_], ok ? xsrc[j] + (size_t)kb * 64 : xsrc[j], ok);
     }
-    for (int c = tid; c < kTok * kKB; c += kUnionThreads) {
-      const int ti = c / kKB, g = c % kKB;
-      const bool ok = ti < nt && g < kbn;
-      const int rin = in_idx[base + tc + (ok ? ti : 0)];
-      cp_async4(&S.f[ti][g], a.xq_fac + (size_t)rin * a.G + kb + (ok ? g : 0), ok);
+    if (tid < kTok * kKB) {
+      const bool ok = fok && (tid % kKB) < kbn;
+      cp_async4(&S.f[tid / kKB][tid % kKB], ok ? fsrc + kb : fsrc, ok);
     }
   };
 
   for (int tc = 0; tc < n; tc += kTok) {
     const int nt = min(kTok, n - tc);
+    // this pass's token sources
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int ti = (tid >> 6) + 4 * j;
+      xok[j] = ti < nt;
+      const int rin = in_idx[base + tc + (xok[j] ? ti : 0)];
+      xsrc[j] = a.xq_words + ((size_t)rin * a.G + min(xg_, a.G - 1)) * 64 + xw_ * 16;
+    }
+    if (tid < kTok * kKB) {
+      const int ti = tid / kKB;
+      fok = ti < nt;
+      fsrc = a.xq_fac + (size_t)in_idx[base + tc + (fok ? ti : 0)] * a.G + min(tid % kKB, a.G - 1);
+    }
     float acc[kTok];
 #pragma unroll
     for (int ti = 0; ti < kTok; ++ti) acc[ti] = 0.f;
 #pragma unroll
     for (int s0 = 0; s0 < kNS - 1; ++s0) {
-      if (s0 < nk) issue(s0, s0, tc, nt);
+      if (s0 < nk) issue(s0, s0);
       cp_async_commit();
     }
     for (int ks = 0; ks < nk; ++ks) {
       cp_async_wait<kNS - 2>();  // step ks has landed (this thread's copies)
       __syncthreads();           // ... everyone's; step ks - 1 is no longer read
-      if (ks + kNS - 1 < nk) issue((ks + kNS - 1) % kNS, ks + kNS - 1, tc, nt);
+      if (ks + kNS - 1 < nk) issue((ks + kNS - 1) % kNS, ks + kNS - 1);
       cp_async_commit();
       const UStage& S = st[ks % kNS];
       const int kbn = min(kKB, a.G - ks * kKB);
