@@ -168,6 +168,30 @@ __device__ __forceinline__ int dotq_group(const uint4 w, const XQ& g) {
   return (a0 + a1) + (a2 + a3);
 }
 
+// dotq_group with the chunk's words already split into even-element and
+// odd-element bytes (16 * q), for a chunk used against several inputs.
+__device__ __forceinline__ void split_chunk(const uint4 w, uint32_t (&even)[4], uint32_t (&odd)[4]) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    odd[i] = ws[i] & 0xF0F0F0F0u;
+    even[i] = (ws[i] << 4) & 0xF0F0F0F0u;
+  }
+}
+
+__device__ __forceinline__ int dotq_group_split(const uint32_t (&even)[4], const uint32_t (&odd)[4],
+                                                const XQ& g) {
+  int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    a0 = dp2a_lo(g.ev[2 * i], even[i], a0);
+    a1 = dp2a_hi(g.ev[2 * i + 1], even[i], a1);
+    a2 = dp2a_lo(g.od[2 * i], odd[i], a2);
+    a3 = dp2a_hi(g.od[2 * i + 1], odd[i], a3);
+  }
+  return (a0 + a1) + (a2 + a3);
+}
+
 // sum_k (q_k * scale) x_k for one chunk: exact group sum, one rounding.
 __device__ __forceinline__ float dot_scaled(const uint4 w, const XQ& g, float scale) {
   return (float)dotq_group(w, g) * (scale * g.f);

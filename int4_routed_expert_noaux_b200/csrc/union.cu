@@ -345,7 +345,8 @@ __global__ void __launch_bounds__(kUnionThreads) union_gemm_kernel(const UnionAr
       for (int i = 0; i < kKB / 4; ++i) {
         const int g = 4 * i + q;
         if (g < kbn) {
-          const uint4 w = S.w[m][g];
+          uint32_t even[4], odd[4];
+          split_chunk(S.w[m][g], even, odd);  // once, for every token
           const float sc = f16_bits_to_f32(S.s[m][g]);
 #pragma unroll
           for (int ti = 0; ti < kTok; ++ti) {
@@ -358,7 +359,7 @@ __global__ void __launch_bounds__(kUnionThreads) union_gemm_kernel(const UnionAr
               xg.od[0] = a2.x; xg.od[1] = a2.y; xg.od[2] = a2.z; xg.od[3] = a2.w;
               xg.od[4] = a3.x; xg.od[5] = a3.y; xg.od[6] = a3.z; xg.od[7] = a3.w;
               xg.f = S.f[ti][g];
-              acc[ti] += dot_scaled(w, xg, sc);
+              acc[ti] += (float)dotq_group_split(even, odd, xg) * (sc * xg.f);
             }
           }
         }
