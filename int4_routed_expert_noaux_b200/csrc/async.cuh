@@ -50,20 +50,6 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// One probe that may suspend the thread in hardware for up to `hint_ns`
-// (it wakes earlier when the phase completes), so waiting warps do not take
-// issue slots from working ones.
-__device__ __forceinline__ bool mbar_test_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; "
-      "selp.u32 %0, 1, 0, p; }"
-      : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
-
 // Wait for phase `parity`, giving up at `deadline` (globaltimer ns).
 // Returns false on timeout.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t deadline) {
@@ -114,14 +100,6 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   return v;
 }
 
-// Relaxed (not ordering) load at gpu scope, for polling; pair it with a fence
-// once the value is seen.
-__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
 // 64-bit relaxed load / store at gpu scope: single-copy atomic, so a record
 // that carries its own validity tag needs no fence.
 __device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
@@ -132,17 +110,6 @@ __device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
 
 __device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-__device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
-               : "memory");
-  return old;
 }
 
 __device__ __forceinline__ void red_add_release(uint32_t* p, uint32_t v) {
@@ -159,11 +126,6 @@ __device__ __forceinline__ uint32_t atom_add_release(uint32_t* p, uint32_t v) {
 
 __device__ __forceinline__ void fence_acq_rel() {
   asm volatile("fence.acq_rel.gpu;" ::: "memory");
-}
-
-// Named barrier over `count` threads (a multiple of 32).
-__device__ __forceinline__ void named_bar(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 }  // namespace moe

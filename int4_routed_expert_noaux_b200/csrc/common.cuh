@@ -46,42 +46,6 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
 }
 
 // ---------------------------------------------------------------------------
-// packed fp32x2 arithmetic (sm_100 FFMA2)
-
-__device__ __forceinline__ unsigned long long pack_f2(float lo, float hi) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-
-__device__ __forceinline__ void unpack_f2(unsigned long long v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-
-__device__ __forceinline__ unsigned long long pack_u2(uint32_t lo, uint32_t hi) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
-  return r;
-}
-
-// d = a * b + c, element-wise on two packed floats, round to nearest.
-__device__ __forceinline__ unsigned long long ffma2(unsigned long long a,
-                                                    unsigned long long b,
-                                                    unsigned long long c) {
-  unsigned long long d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-
-// r = c1 ? (a ^ c2) : c2, bitwise (one LOP3: a = 0xF0, c1 = 0xCC, c2 = 0xAA
-// gives the truth table 0x6A).
-__device__ __forceinline__ uint32_t lop3_sel_xor(uint32_t a, uint32_t c1, uint32_t c2) {
-  uint32_t r;
-  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(r) : "r"(a), "r"(c1), "r"(c2));
-  return r;
-}
-
-// ---------------------------------------------------------------------------
 // int4 dot product of one 32-input scale group (16 packed bytes), exact in
 // integers.
 //
