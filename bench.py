@@ -15,7 +15,7 @@ With --gpus N (torchrun) each rank runs its own replica of the workload
 (independent tokens, no data-path collective): weak scaling.
 
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
-workload on the host cores (the reference arm of this build).
+workload on the host cores: there is no other implementation to run.
 """
 import argparse
 import hashlib
