@@ -301,11 +301,14 @@ __device__ __noinline__ void run_select_generic(const SelArgs p, Smem& S) {
   }
 }
 
-// bf16 bit pattern of layer input element i: x[i] itself, or, for a
-// residual (pre-norm) step, bf16(x_resid[i] * inv_rms).
-__device__ __forceinline__ uint32_t input_bf16(const DecodeParams& p, int i, float inv_rms) {
-  if (p.x_resid) return f32_to_bf16_rne(p.x_resid[i] * inv_rms);
-  return p.x[i];
+// Four consecutive inputs of a residual (pre-norm) step, i0 % 4 == 0, as
+// bf16(x_resid * inv_rms) pairs in two words (one 16-byte load).
+__device__ __forceinline__ uint2 norm_bf16x4(const float* x_resid, int i0, float inv_rms) {
+  const float4 v = __ldg(reinterpret_cast<const float4*>(x_resid + i0));
+  uint2 r;
+  r.x = (uint32_t)f32_to_bf16_rne(v.x * inv_rms) | ((uint32_t)f32_to_bf16_rne(v.y * inv_rms) << 16);
+  r.y = (uint32_t)f32_to_bf16_rne(v.z * inv_rms) | ((uint32_t)f32_to_bf16_rne(v.w * inv_rms) << 16);
+  return r;
 }
 
 // Fixed-order combine of one row block of y from the per-slot partials, by
@@ -743,12 +746,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     {
       float xf[32];
       if (p.x_resid) {
+        const bool write_xn = blockIdx.x == 0 && grp == 0 && cg.phase == 0 && p.xn_out;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const uint32_t b = input_bf16(p, cg.col * 32 + i, inv_rms);
-          xf[i] = bf16_bits_to_f32(b);
-          if (blockIdx.x == 0 && grp == 0 && cg.phase == 0 && p.xn_out)
-            p.xn_out[cg.col * 32 + i] = (uint16_t)b;
+        for (int i = 0; i < 8; ++i) {
+          const uint2 b = norm_bf16x4(p.x_resid, cg.col * 32 + 4 * i, inv_rms);
+          xf[4 * i] = bf16_bits_to_f32(b.x & 0xFFFFu);
+          xf[4 * i + 1] = bf16_bits_to_f32(b.x >> 16);
+          xf[4 * i + 2] = bf16_bits_to_f32(b.y & 0xFFFFu);
+          xf[4 * i + 3] = bf16_bits_to_f32(b.y >> 16);
+          if (write_xn) {  // xn_out is 4-byte aligned
+            uint32_t* xo = reinterpret_cast<uint32_t*>(p.xn_out + cg.col * 32 + 4 * i);
+            xo[0] = b.x;
+            xo[1] = b.y;
+          }
         }
       } else {
         const uint4* xp = reinterpret_cast<const uint4*>(p.x + cg.col * 32);
@@ -791,8 +801,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           if (cc >= rchunks) {
             xr[i] = make_uint2(0, 0);
           } else if (p.x_resid) {
-            xr[i].x = input_bf16(p, 4 * cc, inv_rms) | (input_bf16(p, 4 * cc + 1, inv_rms) << 16);
-            xr[i].y = input_bf16(p, 4 * cc + 2, inv_rms) | (input_bf16(p, 4 * cc + 3, inv_rms) << 16);
+            xr[i] = norm_bf16x4(p.x_resid, 4 * cc, inv_rms);
           } else {
             xr[i] = __ldg(reinterpret_cast<const uint2*>(p.x) + cc);
           }
