@@ -129,6 +129,13 @@ moe_status moe_ws_check(void* ws_dev, size_t ws_bytes, void* stream);
 
 /* ---- the hot path ------------------------------------------------------ */
 
+/* Pointer rules for moe_route, moe_expert_ffn, moe_layer_forward,
+ * moe_layer_forward_noalloc, moe_layer_forward_residual and moe_stack_forward:
+ * all buffers are device memory of the current device; x / y / x_next buffers start on a 16-byte boundary; idx,
+ * w, scores, xn_out and status buffers on a 4-byte boundary.  A NULL (where
+ * not nullable), host or misaligned pointer returns MOE_ERR_INVALID_ARG
+ * before anything is launched. */
+
 /* Steps 1-2 for T tokens.  x_dev bf16 [T][hidden]; idx_dev int32 [T][top_k]
  * (ascending expert ids); w_dev fp32 [T][top_k]; scores_dev fp32
  * [T][n_experts] = sigmoid scores s (nullable, for inspection).
@@ -190,7 +197,8 @@ moe_status moe_layer_forward_noalloc(const moe_layer* layer, const void* x_dev,
  * layers: RMSNorm with unit gain before each MoE block, as in the upstream
  * model -- "LightLX", "How it works": RMSNorm):
  *   x_next = x + MoE(bf16(x / sqrt(mean(x^2) + norm_eps)))
- * x_dev, x_next_dev fp32 [hidden], distinct.  xn_out_dev (nullable) receives
+ * x_dev, x_next_dev fp32 [hidden], distinct, 16-byte aligned.  xn_out_dev
+ * (nullable, 4-byte aligned) receives
  * the bf16 normalised input the experts saw.  One token (T = 1); the shape
  * must be one the fused decode kernel covers (MOE_ERR_UNSUPPORTED otherwise).
  * The workspace is that of moe_workspace_bytes(cfg, 1). */

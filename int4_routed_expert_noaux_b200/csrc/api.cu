@@ -319,6 +319,7 @@ moe_status moe_stack_forward(const moe_layer* const* layers, int n_layers, const
   g_last_error[0] = 0;
   if (!layers || n_layers < 1) return fail(MOE_ERR_INVALID_ARG, "need at least one layer");
   if (n_layers > 1 && !x_tmp_dev) return fail(MOE_ERR_INVALID_ARG, "x_tmp is needed for more than one layer");
+  if (!layers[0]) return fail(MOE_ERR_INVALID_ARG, "layers[0] is NULL");
   const moe_config& c0 = layers[0]->cfg;
   for (int l = 1; l < n_layers; ++l) {
     if (!layers[l]) return fail(MOE_ERR_INVALID_ARG, "layers[%d] is NULL", l);

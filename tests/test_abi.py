@@ -61,6 +61,17 @@ def test_create_rejects_null_pointers():
     assert not out.value
 
 
+
+def test_stack_rejects_bad_layer_lists():
+    """moe_stack_forward checks its layer list before it touches any pointer."""
+    L = moe.lib()
+    arr = (ctypes.c_void_p * 2)(None, None)
+    assert L.moe_stack_forward(arr, 0, None, None, None, None, 1e-6, None, 0, None) == 1
+    assert L.moe_stack_forward(arr, 2, None, None, None, None, 1e-6, None, 0, None) == 1
+    assert b"x_tmp" in L.moe_last_error()
+    assert L.moe_stack_forward(arr, 1, None, None, None, None, 1e-6, None, 0, None) == 1
+    assert b"layers[0] is NULL" in L.moe_last_error()
+
 def test_library_lru_matches_oracle_lru():
     # the cache's replacement rule (C++ in the library) against the oracle's
     # independent simulation, on Zipf traces at several capacities
