@@ -141,6 +141,34 @@ def test_expert_ffn_closed_form():
     assert np.allclose(y, y_exp, rtol=1e-15, atol=1e-300)
 
 
+
+def test_expert_ffn_silu_special_values():
+    # SiLU values that follow from the definition without evaluating it:
+    # silu(0) = 0; sigmoid(ln 3) = 3/4, so silu(ln 3) = 0.75 ln 3; silu(42) is
+    # 42 and silu(-42) is 0 to well below fp64 resolution (e^-42 < 1e-18).
+    # Catches a sign flip inside the sigmoid, SiLU applied to up, or a
+    # different activation (ReLU, GELU) in its place.
+    H, I, gs = 32, 4, 32
+    sh = Shape(hidden=H, inter=I, n_experts=1, top_k=1, n_group=1, topk_group=1,
+               group_size=gs, rsf=1.0)
+    x = np.zeros(H)
+    x[0:4] = [0.0, math.log(3.0), 42.0, -42.0]   # gate inputs
+    x[8:12] = [5.0, 2.0, 1.0, 3.0]               # up inputs
+    gate_codes = np.zeros((I, H), dtype=np.int64)
+    up_codes = np.zeros((I, H), dtype=np.int64)
+    for i in range(I):
+        gate_codes[i, i] = 1
+        up_codes[i, 8 + i] = 1
+    ones = lambda n, m: f16_bits(np.ones((n, m // gs)))
+    e = dict(q_gate=pack_int4(gate_codes), s_gate=ones(I, H),
+             q_up=pack_int4(up_codes), s_up=ones(I, H),
+             q_down=pack_int4(np.zeros((H, I), dtype=np.int64)), s_down=ones(H, I))
+    _, h = oracle.expert_ffn(sh, e, x, return_h=True)
+    assert h[0] == 0.0
+    assert abs(h[1] - 0.75 * math.log(3.0) * 2.0) <= 4e-16 * abs(h[1])
+    assert h[2] == 42.0
+    assert abs(h[3]) < 1e-15
+
 # ---------------------------------------------------------------------------
 # router logits
 
@@ -292,6 +320,23 @@ def test_route_bias_only_steers_selection():
     s0, s7 = 1 / (1 + math.exp(-2.0)), 1 / (1 + math.exp(5.0))
     assert np.allclose(w[0], [2.0 * s0 / (s0 + s7), 2.0 * s7 / (s0 + s7)], rtol=1e-14)
 
+
+
+def test_route_sigmoid_scores_closed_form():
+    # The score is the logistic sigmoid of the logit: at 0, +-ln 3, ln 7,
+    # ln 15 and -ln 7 it takes the values 1/2, 3/4, 1/4, 7/8, 15/16, 1/8; at
+    # +-40 it is 1 and e^-40 to fp64 resolution.  Weights of the two winners
+    # (scores 1 and 15/16, rsf 2) are 32/31 and 30/31.  Catches softmax in
+    # place of the sigmoid, a sign flip, or weights from the biased scores.
+    sh = Shape(hidden=32, inter=32, n_experts=8, top_k=2, n_group=1, topk_group=1,
+               group_size=32, rsf=2.0)
+    ln = math.log
+    logits = np.array([[0.0, ln(3.0), -ln(3.0), ln(7.0), 40.0, -40.0, -ln(7.0), ln(15.0)]])
+    idx, w, _, s = oracle.route(sh, logits, np.zeros(8, dtype=np.float32))
+    want = [0.5, 0.75, 0.25, 0.875, 1.0, math.exp(-40.0), 0.125, 0.9375]
+    assert np.allclose(s[0], want, rtol=1e-15, atol=0)
+    assert idx.tolist() == [[4, 7]]
+    assert np.allclose(w[0], [32 / 31, 30 / 31], rtol=1e-15, atol=0)
 
 # ---------------------------------------------------------------------------
 # combine: linearity and the single-expert case (P9)
