@@ -118,7 +118,9 @@ moe_status moe_layer_set_expert(moe_layer* layer, int e,
  * be 256-byte aligned and zero-filled before its first use, and the caller
  * must not write it between calls (moe_ws_check aside): the fused kernel
  * leaves its counters zero after every call but keeps a call count and the
- * router score records, tagged with that count, from call to call.  One
+ * router score records, tagged with that count, from call to call, in a
+ * region that no other call writes.  A workspace sized for T tokens serves
+ * every call with T or fewer tokens, one-token and batched calls mixed.  One
  * workspace must not be used by two calls that can run at the same time. */
 size_t moe_workspace_bytes(const moe_config* cfg, int T);
 

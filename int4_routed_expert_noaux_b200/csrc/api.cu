@@ -102,9 +102,13 @@ WsLayout ws_layout(const moe_config* c, int T) {
   size_t off = 0;
   L.ctrl = off;
   off += kCtrlBytes;
+  // the fused one-token kernel's epoch-tagged router score records, kept
+  // from call to call: a region that no other call writes
+  L.records = off;
+  off = align_up(off + (size_t)c->n_experts * 8, 256);
+  // fp32 router logits of the step kernels
   L.logits = off;
-  // router logits of the step kernels, or the fused kernel's score records
-  off = align_up(off + (size_t)T * c->n_experts * 8, 256);
+  off = align_up(off + (size_t)T * c->n_experts * 4, 256);
   L.idx = off;
   off = align_up(off + (size_t)T * k * 4, 256);
   L.w = off;

@@ -48,7 +48,7 @@ static moe_status launch_fused(const moe_layer* l, const uint16_t* x, const floa
   p.idx_out = idx_out;
   p.w_out = w_out;
   p.ctrl = reinterpret_cast<uint32_t*>(ws + L.ctrl);
-  p.scores = reinterpret_cast<uint64_t*>(ws + L.logits);
+  p.scores = reinterpret_cast<uint64_t*>(ws + L.records);
   p.hbuf = reinterpret_cast<float*>(ws + L.hbuf);
   p.warm = 1;
   p.ypart = reinterpret_cast<float*>(ws + L.ypart);

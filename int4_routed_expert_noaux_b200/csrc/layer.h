@@ -25,7 +25,7 @@ constexpr int kMaxTokens = 64;
 
 // Byte offsets inside a workspace.
 struct WsLayout {
-  size_t ctrl, logits, idx, w, hbuf, ypart, xq, xqf, hq, hqf, lists, total;
+  size_t ctrl, records, logits, idx, w, hbuf, ypart, xq, xqf, hq, hqf, lists, total;
 };
 
 WsLayout ws_layout(const moe_config* c, int T);

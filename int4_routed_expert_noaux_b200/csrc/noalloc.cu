@@ -12,10 +12,11 @@ namespace moe {
 
 // Largest scratch the call takes: the one-token workspace of the shape,
 // ws_layout(cfg, 1).total.  A 6144 x 2048 layer with top-8 of 256 experts
-// and one shared expert needs 356,096 bytes.
+// and one shared expert needs 357,120 bytes.
 constexpr size_t kStaticScratchBytes = 512u << 10;
 constexpr int kStaticMaxDevices = 64;
-// control words plus the largest router score area (256 experts x 8 bytes)
+// control words plus the router score records that follow them (8 bytes per
+// expert; the fused kernel, their only user, takes at most 256 experts)
 constexpr size_t kStaticClearBytes = kCtrlBytes + 256 * 8;
 
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];

@@ -43,6 +43,10 @@ def test_status_strings_and_config_checks():
     assert glm > 0 and glm % 256 == 0
     assert moe.workspace_bytes(cfg, 0) == 0
     assert moe.workspace_bytes(cfg, 65) == 0
+    # a workspace sized for T tokens serves every smaller call
+    sizes = [moe.workspace_bytes(cfg, T) for T in range(1, 65)]
+    assert all(a < b for a, b in zip(sizes, sizes[1:]))
+    assert all(v % 256 == 0 for v in sizes)
     assert moe.workspace_bytes(moe.Config.from_shape(synth.TINY), 4) > 0
     bad = moe.Config.from_shape(synth.GLM)
     bad.hidden = 6000

@@ -236,6 +236,39 @@ def test_many_decode_calls_one_workspace(shape, n):
     check_forward(shape, dl, x_bits, ys.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy())
 
 
+
+@pytest.mark.parametrize("shape", [synth.TINY, synth.GLM], ids=["tiny", "glm"])
+def test_one_token_and_batched_calls_share_a_workspace(shape):
+    # A workspace sized for 4 tokens serves one-token and batched calls in
+    # any order.  The batched call leaves the one-token kernel's epoch-tagged
+    # score records untouched (they would otherwise hold logit bits that a
+    # later epoch could match), and the one-token result stays bitwise that
+    # of a fresh workspace.
+    dl, L = get_layer(shape)
+    cfg = moe.Config.from_shape(shape)
+    x_bits = synth.tokens(shape, 0, 500, 5)
+    x = to_dev_bf16(x_bits)
+    dev = dict(dtype=torch.float32, device="cuda")
+    y_ref = torch.empty((1, shape.hidden), **dev)
+    ws_fresh = moe.alloc_workspace(cfg, 1)
+    L.forward(x[0:1], y_ref, ws_fresh)
+    moe.ws_check(ws_fresh)
+    ws = moe.alloc_workspace(cfg, 4)
+    y1, y2 = torch.empty_like(y_ref), torch.empty_like(y_ref)
+    y4 = torch.empty((4, shape.hidden), **dev)
+    idx4 = torch.empty((4, shape.top_k), dtype=torch.int32, device="cuda")
+    w4 = torch.empty((4, shape.top_k), **dev)
+    records = lambda: ws[4096:4096 + 8 * shape.n_experts].view(torch.int64).cpu().numpy()
+    L.forward(x[0:1], y1, ws)
+    L.forward(x[1:5], y4, ws, idx=idx4, w=w4)
+    moe.ws_check(ws)
+    assert np.all((records() >> 32) == 1)
+    L.forward(x[0:1], y2, ws)
+    moe.ws_check(ws)
+    assert np.all((records() >> 32) == 2)
+    assert torch.equal(y1, y_ref) and torch.equal(y2, y_ref)
+    check_forward(shape, dl, x_bits[1:5], y4.cpu().numpy(), idx4.cpu().numpy(), w4.cpu().numpy())
+
 def test_fused_decode_matches_step_kernels():
     shape = synth.GLM
     dl, L = get_layer(shape)
