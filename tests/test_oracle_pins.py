@@ -220,6 +220,35 @@ def test_select_hand_worked_group_rule():
     assert m2[0] == 0.0
 
 
+def test_select_group_sum_in_fp32():
+    # The kernel-precision variant (round_group_f32) forms each group score
+    # as the fp32 sum of the two addends, each rounded to fp32 first: the
+    # float32 arithmetic a one-warp selection does.  Two hand cases, four
+    # experts in two groups of two, keep one group, top-1:
+    sh = Shape(hidden=32, inter=32, n_experts=4, top_k=1, n_group=2, topk_group=1,
+               group_size=32, rsf=1.0)
+    f32 = lambda v: float(np.float32(v))
+    # (a) the SUM is rounded: 1 + 1.5*2^-24 and 1 + 1.75*2^-24 (exact fp32
+    # addends) both round to 1 + 2^-23, a tie kept by the lower group.
+    # Without rounding the sum (or in fp64) group 1 wins.
+    sp_a = np.array([[1.0, 1.5 * 2.0**-24, 1.0, 1.75 * 2.0**-24]])
+    assert f32(1.0 + 1.5 * 2.0**-24) == f32(1.0 + 1.75 * 2.0**-24) == 1.0 + 2.0**-23
+    assert oracle.select_scores(sh, sp_a, sp_a, round_group_f32=True)[0].tolist() == [[0]]
+    assert oracle.select_scores(sh, sp_a, sp_a)[0].tolist() == [[2]]
+    # (b) each ADDEND is rounded first: 2^-24 + 2^-50 rounds to 2^-24, and
+    # 1 + 2^-24 is a tie between fp32 neighbours that goes to even (1.0),
+    # below group 1's exact 1 + 2^-23.  Rounding only the exact sum would
+    # give 1 + 2^-23 for group 0 too, a tie won by group 0.
+    sp_b = np.array([[1.0, 2.0**-24 + 2.0**-50, 1.0, 2.0**-23]])
+    assert f32(2.0**-24 + 2.0**-50) == 2.0**-24
+    assert f32(1.0 + 2.0**-24) == 1.0
+    assert f32(1.0 + 2.0**-24 + 2.0**-50) == 1.0 + 2.0**-23
+    assert oracle.select_scores(sh, sp_b, sp_b, round_group_f32=True)[0].tolist() == [[2]]
+    assert oracle.select_scores(sh, sp_b, sp_b)[0].tolist() == [[2]]
+    # So a variant that skips the sum's rounding (or rounds nothing) fails
+    # (a), and one that rounds only the exact sum fails (b).
+
+
 def test_select_ties_lower_index():
     sh = Shape(hidden=32, inter=32, n_experts=8, top_k=3, n_group=1, topk_group=1,
                group_size=32, rsf=1.0)
