@@ -49,6 +49,8 @@ def lib():
         L.orc_select_scores.argtypes = [p, p, p, i, i, p, p, p]
         L.orc_route.restype = i
         L.orc_route.argtypes = [p, p, p, i, p, p, p, p]
+        L.orc_topp.restype = i
+        L.orc_topp.argtypes = [p, p, i, d, p, p, p, p]
         L.orc_gemv_int4.argtypes = [p, p, i, i, i, p, p]
         L.orc_expert_ffn.argtypes = [p, p, p, p, p]
         L.orc_experts_combine.argtypes = [p, p, p, p, i, p, p, p]
@@ -137,6 +139,23 @@ def route(shape, logits, bias):
     if rc != 0:
         raise ValueError("oracle routing rejected the configuration")
     return idx, w, margin, s
+
+
+def topp(shape, s, idx, w, p):
+    """Adaptive expert top-p (reading R16) on routes from route() /
+    select_scores(): returns (idx, w, n_keep, margin); dropped slots are -1
+    with weight 0, after the kept ids (ascending)."""
+    s = _c(np.atleast_2d(s), np.float64)
+    idx = np.array(np.atleast_2d(idx), dtype=np.int32, copy=True, order="C")
+    w = np.array(np.atleast_2d(w), dtype=np.float64, copy=True, order="C")
+    T = idx.shape[0]
+    n_keep = np.empty((T,), dtype=np.int32)
+    margin = np.empty((T,), dtype=np.float64)
+    rc = lib().orc_topp(ctypes.byref(cfg(shape)), _p(s), T, float(p), _p(idx), _p(w),
+                        _p(n_keep), _p(margin))
+    if rc != 0:
+        raise ValueError("oracle top-p rejected the arguments")
+    return idx, w, n_keep, margin
 
 
 def gemv_int4(q, s, cols, group_size, x):

@@ -216,6 +216,90 @@ int orc_route(const orc_cfg* c, const double* logits, const float* bias,
   return rc;
 }
 
+/* Adaptive expert top-p (colibri summary, "Telechargement et execution du
+ * modele": the --topp 0.7 option, adaptive expert top-p, and "Benchmarks
+ * communautaires"; the pages give no formula, reading R16): of the k
+ * selected experts, keep the fewest, taken in descending weight (ties: the
+ * lower id first), whose weights add up to at least p * rsf; the kept
+ * weights are normalised again over the kept experts (R4 on the kept set).
+ * Kept ids ascending first, then -1 with weight 0 for the dropped slots.
+ * p >= 1 keeps all k. */
+int orc_topp(const orc_cfg* c, const double* s, int T, double p, int32_t* idx,
+             double* w, int32_t* n_keep, double* margin) {
+  if (!cfg_ok(c) || T < 0 || !(p > 0.0)) return -1;
+  const int E = c->n_experts, k = c->top_k;
+  int32_t* ord = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+  int32_t* kept = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+  if (!ord || !kept) {
+    free(ord); free(kept);
+    return -1;
+  }
+  for (int t = 0; t < T; ++t) {
+    int32_t* it = idx + (size_t)t * k;
+    double* wt = w + (size_t)t * k;
+    const double* st = s + (size_t)t * E;
+    /* positions of the k selected experts in descending weight, ties to
+     * the lower id (selection sort: k is small) */
+    char* used = (char*)calloc((size_t)k, 1);
+    for (int r = 0; r < k; ++r) {
+      int best = -1;
+      for (int j = 0; j < k; ++j) {
+        if (used[j]) continue;
+        if (best < 0 || wt[j] > wt[best] || (wt[j] == wt[best] && it[j] < it[best])) best = j;
+      }
+      used[best] = 1;
+      ord[r] = best;
+    }
+    free(used);
+    /* the shortest prefix whose share of rsf reaches p */
+    int m = k;
+    double cum = 0.0, before = 0.0;
+    if (p < 1.0) {
+      for (int r = 0; r < k; ++r) {
+        before = cum;
+        cum += wt[ord[r]] / c->rsf;
+        if (cum >= p) {
+          m = r + 1;
+          break;
+        }
+      }
+    }
+    double mg = INFINITY;
+    if (p < 1.0 && m <= k) {
+      const double a = cum - p, b = p - before;
+      mg = a < b ? a : b;
+      if (m < k) {
+        const double gap = (wt[ord[m - 1]] - wt[ord[m]]) / c->rsf;
+        if (gap < mg) mg = gap;
+      }
+    }
+    /* kept ids ascending; weights from the unbiased scores over the kept */
+    for (int r = 0; r < m; ++r) kept[r] = it[ord[r]];
+    for (int a = 1; a < m; ++a)
+      for (int b = a; b > 0 && kept[b - 1] > kept[b]; --b) {
+        const int32_t tmp = kept[b];
+        kept[b] = kept[b - 1];
+        kept[b - 1] = tmp;
+      }
+    double denom = 0.0;
+    for (int r = 0; r < m; ++r) denom += st[kept[r]];
+    denom += 1e-20;
+    for (int r = 0; r < k; ++r) {
+      if (r < m) {
+        it[r] = kept[r];
+        wt[r] = c->rsf * st[kept[r]] / denom;
+      } else {
+        it[r] = -1;
+        wt[r] = 0.0;
+      }
+    }
+    if (n_keep) n_keep[t] = m;
+    if (margin) margin[t] = mg;
+  }
+  free(ord); free(kept);
+  return 0;
+}
+
 /* ---- experts ------------------------------------------------------------ */
 
 /* Dequantise-on-use GEMV of a packed int4 matrix (colibri summary: int4
@@ -263,6 +347,7 @@ void orc_experts_combine(const orc_cfg* c, const orc_expert* experts,
     double* yt = y + (size_t)t * H;
     for (int h = 0; h < H; ++h) yt[h] = 0.0;
     for (int j = 0; j < k; ++j) {
+      if (idx[(size_t)t * k + j] < 0) continue;   /* dropped by top-p (R16) */
       orc_expert_ffn(c, &experts[idx[(size_t)t * k + j]], xt, ye, NULL);
       for (int h = 0; h < H; ++h) yt[h] += w[(size_t)t * k + j] * ye[h];
     }

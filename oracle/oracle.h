@@ -96,6 +96,18 @@ int orc_route(const orc_cfg* c, const double* logits, const float* bias,
               int T, int32_t* idx, double* w, double* margin,
               double* scores_out);
 
+/* Adaptive expert top-p (reading R16) applied in place to routes from
+ * orc_select_scores / orc_route: idx [T][k] (ascending), w [T][k], s the
+ * unbiased scores [T][E].  Keeps the fewest experts, in descending weight
+ * (ties: lower id), whose weights reach p * rsf; kept weights are
+ * renormalised over the kept experts; dropped slots become id -1, weight 0,
+ * after the kept ids.  n_keep[t] (nullable) = experts kept; margin[t]
+ * (nullable) = the smaller of |cumulative share - p| at the boundary and the
+ * share gap between the last kept and first dropped expert (infinite for
+ * p >= 1).  p > 0; p >= 1 keeps all. */
+int orc_topp(const orc_cfg* c, const double* s, int T, double p, int32_t* idx,
+             double* w, int32_t* n_keep, double* margin);
+
 /* y[r] = sum_col (q[r][col] * fp16(s[r][col / gs])) * x[col], for r < rows.
  * q packed per R5 with cols / 2 bytes per row; s has cols / gs per row. */
 void orc_gemv_int4(const uint8_t* q, const uint16_t* s, int rows, int cols,
@@ -114,7 +126,8 @@ int orc_layer_forward(const orc_cfg* c, const float* w_router,
                       const orc_expert* shared, const uint16_t* x_bf16, int T,
                       double* y, int32_t* idx, double* w, double* margin);
 
-/* Expert part only, for given routes: y[t] = sum_j w[t][j] * FFN_{idx[t][j]}
+/* Expert part only, for given routes (an id of -1 is skipped: a slot
+ * dropped by top-p): y[t] = sum_j w[t][j] * FFN_{idx[t][j]}
  * (x_t) + FFN_shared(x_t).  x as doubles [T][H]. */
 void orc_experts_combine(const orc_cfg* c, const orc_expert* experts,
                          const orc_expert* shared, const double* x, int T,

@@ -249,6 +249,87 @@ def test_select_group_sum_in_fp32():
     # (a), and one that rounds only the exact sum fails (b).
 
 
+def test_topp_hand_cases():
+    # R16: keep the fewest selected experts, taken in descending weight
+    # (ties: the lower id first), whose weights reach p * rsf; the kept
+    # weights are normalised again over the kept experts.
+    sh = Shape(hidden=32, inter=32, n_experts=16, top_k=4, n_group=1, topk_group=1,
+               group_size=32, rsf=2.0)
+    s = np.zeros(16)
+    s[[3, 7, 9, 12]] = [0.8, 0.4, 0.2, 0.2]          # shares .5 .25 .125 .125
+    idx, w, _ = oracle.select_scores(sh, s[None], s[None])
+    # p = 0.7: .5 < .7 <= .75, so the two heaviest, weights 2 * (.8, .4) / 1.2
+    i2, w2, n2, m2 = oracle.topp(sh, s[None], idx, w, 0.7)
+    assert i2.tolist() == [[3, 7, -1, -1]] and n2.tolist() == [2]
+    assert np.allclose(w2, [[4 / 3, 2 / 3, 0.0, 0.0]], rtol=1e-15, atol=0)
+    assert m2[0] == pytest.approx(0.05, abs=1e-15)
+    # p reached exactly (.75): two kept, boundary margin 0 (flagged)
+    _, _, n3, m3 = oracle.topp(sh, s[None], idx, w, 0.75)
+    assert n3.tolist() == [2] and m3[0] == 0.0
+    # p = 1 keeps every selected expert with its weight
+    i4, w4, n4, m4 = oracle.topp(sh, s[None], idx, w, 1.0)
+    assert i4.tolist() == idx.tolist() and np.array_equal(w4, w) and n4[0] == 4
+    assert m4[0] == np.inf
+    # a tiny p keeps only the heaviest, at weight rsf
+    i5, w5, n5, _ = oracle.topp(sh, s[None], idx, w, 1e-9)
+    assert i5.tolist() == [[3, -1, -1, -1]] and w5[0, 0] == pytest.approx(2.0, rel=1e-15)
+    # equal weights across the boundary: the lower ids are kept, margin 0
+    s2 = np.zeros(16)
+    s2[[2, 5, 8, 11]] = 0.5
+    idx2, wq, _ = oracle.select_scores(sh, s2[None], s2[None])
+    i6, w6, n6, m6 = oracle.topp(sh, s2[None], idx2, wq, 0.6)
+    assert i6.tolist() == [[2, 5, 8, -1]] and n6[0] == 3 and m6[0] == 0.0
+    assert np.allclose(w6[0, :3], 2 / 3, rtol=1e-15, atol=0)
+
+
+def test_topp_brute_force():
+    # Independently of the prefix scan: the kept set is the smallest subset
+    # of the selected experts whose weights reach p * rsf, and of the subsets
+    # of that size the heaviest.  Trials whose decision is within 1e-9 of a
+    # tie are skipped (the two formulations may then differ in rounding).
+    sh = Shape(hidden=32, inter=32, n_experts=16, top_k=4, n_group=4, topk_group=2,
+               group_size=32, rsf=2.5)
+    rng = np.random.default_rng(21)
+    checked = 0
+    for _ in range(400):
+        s = 1 / (1 + np.exp(-rng.normal(0, 1.5, size=16)))
+        sp = s + rng.uniform(-0.1, 0.1, size=16)
+        p = float(rng.uniform(0.05, 0.999))
+        idx, w, _ = oracle.select_scores(sh, s[None], sp[None])
+        i2, w2, n, m = oracle.topp(sh, s[None], idx, w, p)
+        if m[0] < 1e-9:
+            continue
+        sel = idx[0].tolist()
+        share = {e: s[e] / sum(s[x] for x in sel) for e in sel}
+        best = None
+        for r in range(1, 5):
+            cands = [c for c in itertools.combinations(sel, r) if sum(share[e] for e in c) >= p]
+            if cands:
+                best = max(cands, key=lambda c: sum(share[e] for e in c))
+                break
+        assert sorted(best) == [e for e in i2[0].tolist() if e >= 0]
+        assert n[0] == len(best)
+        kept = sorted(best)
+        assert np.allclose(w2[0, :len(kept)], [2.5 * s[e] / sum(s[x] for x in kept) for e in kept],
+                           rtol=1e-14)
+        assert np.all(i2[0, len(kept):] == -1) and np.all(w2[0, len(kept):] == 0)
+        checked += 1
+    assert checked > 300
+
+
+def test_combine_skips_dropped_slots():
+    # an id of -1 (a slot dropped by top-p) contributes nothing
+    sh = synth.TINY
+    rng = np.random.default_rng(8)
+    ex = {e: synth.expert(sh, 0, 0, e) for e in (3, 9)}
+    x = rng.normal(size=(1, sh.hidden))
+    y_one = oracle.experts_combine(sh, ex, None, x, np.array([[3, -1]], dtype=np.int32),
+                                   np.array([[1.5, 0.0]]))
+    y_ref = oracle.experts_combine(sh, ex, None, x, np.array([[3, 9]], dtype=np.int32),
+                                   np.array([[1.5, 0.0]]))
+    assert np.array_equal(y_one, y_ref)
+
+
 def test_select_ties_lower_index():
     sh = Shape(hidden=32, inter=32, n_experts=8, top_k=3, n_group=1, topk_group=1,
                group_size=32, rsf=1.0)
