@@ -112,6 +112,20 @@ void moe_layer_destroy(moe_layer* layer);
 moe_status moe_layer_set_expert(moe_layer* layer, int e,
                                 const moe_expert* expert_host, void* stream);
 
+/* Adaptive expert top-p of a layer (colibri summary, "Telechargement et
+ * execution du modele": the --topp option, adaptive expert top-p, fewer
+ * expert bytes read; the pages give no formula, so the rule here is this
+ * library's reading): of the top_k experts the router selects, keep the
+ * fewest, taken in descending weight (ties: the lower id first), whose
+ * weights add up to at least p * routed_scaling_factor, and normalise the
+ * kept weights again over the kept experts.  Routes then carry the kept ids
+ * ascending followed by -1 (weight 0) for each dropped slot; -1 entries are
+ * skipped by moe_expert_ffn.  p >= 1 turns it off (the default); p must be
+ * > 0.  With top-p on, one-token calls take the batched path, and
+ * moe_layer_forward_residual / moe_stack_forward return
+ * MOE_ERR_UNSUPPORTED.  Not thread-safe against calls on the same layer. */
+moe_status moe_layer_set_top_p(moe_layer* layer, float p);
+
 /* ---- workspace --------------------------------------------------------- */
 
 /* Bytes of device workspace a call with T tokens needs.  The workspace must
@@ -148,8 +162,8 @@ moe_status moe_route(const moe_layer* layer, const void* x_dev, int T,
 
 /* Steps 3-5 for T tokens with given routes: y_dev fp32 [T][hidden] =
  * sum_j w[t][j] * FFN_{idx[t][j]}(x_t) + FFN_shared(x_t).  Expert ids must be
- * in [0, n_experts); an out-of-range id sets the workspace error word and its
- * term is skipped.  1 <= T <= 64. */
+ * in [0, n_experts), or -1 for a slot dropped by top-p (skipped); any other
+ * id sets the workspace error word and its term is skipped.  1 <= T <= 64. */
 moe_status moe_expert_ffn(const moe_layer* layer, const void* x_dev, int T,
                           const int32_t* idx_dev, const float* w_dev,
                           float* y_dev, void* ws_dev, size_t ws_bytes,
@@ -250,11 +264,18 @@ moe_status moe_cache_layer(moe_cache* cache, int layer,
 /* Make experts ids_host[0..n) (ascending, distinct) of `layer` resident:
  * LRU bookkeeping on the host; every miss is copied host -> slot with
  * cudaMemcpyAsync on the cache's copy stream (after the layer's last
- * release event, so no slot still in use is overwritten); compute_stream
- * then waits for the copies and the layer view's pointer table is updated
- * on it.  Replacement: hits are touched in ascending id order, then each
- * miss in ascending id order takes the lowest empty slot, else the least
- * recently used slot not holding one of ids.  n <= slots_per_layer, n <= 32. */
+ * release event, so no slot still in use is overwritten; if the layer was
+ * acquired again with no release in between, after everything enqueued on
+ * compute_stream so far); compute_stream then waits for the copies and the
+ * layer view's pointer table is updated on it.  Replacement: hits are
+ * touched in ascending id order, then each miss in ascending id order takes
+ * the lowest empty slot, else the least recently used slot not holding one
+ * of ids.  n <= slots_per_layer, n <= 32.
+ * Transactional: the replacement state, the counters and the pointer table
+ * change only when every copy was enqueued.  On a failed enqueue the call
+ * returns MOE_ERR_CUDA and the layer keeps its previous state, except that
+ * the slots its copies may have reached are marked empty (so a later
+ * acquire reloads rather than trusts them). */
 moe_status moe_cache_acquire(moe_cache* cache, int layer,
                              const int32_t* ids_host, int n,
                              void* compute_stream);
@@ -265,6 +286,11 @@ moe_status moe_cache_stats(const moe_cache* cache, int layer, uint64_t* hits,
                            uint64_t* misses, uint64_t* bytes_h2d);
 /* Wait for the cache's copy stream. */
 moe_status moe_cache_sync(moe_cache* cache);
+/* Wait at most timeout_ms for the cache's copy stream, polling it from the
+ * host (cudaStreamQuery): MOE_OK when every enqueued copy has finished,
+ * MOE_ERR_TIMEOUT when the deadline passes first (the copies go on; a later
+ * wait can succeed), MOE_ERR_CUDA if the stream reports an error. */
+moe_status moe_cache_wait(moe_cache* cache, int timeout_ms);
 
 /* The cache's replacement rule run on the host over a trace [T][n_layers][k]
  * of ascending ids (no GPU needed): per-layer hits and misses after T calls
@@ -285,6 +311,25 @@ moe_status moe_lru_replay(int n_layers, int n_experts, int capacity, int k,
 moe_status moe_debug_gemv_int4(const uint8_t* q_dev, const uint16_t* s_dev,
                                int rows, int cols, const float* x_dev,
                                float* y_dev, void* stream);
+
+/* Host-side fault injection for tests of the error paths (nothing is
+ * injected unless armed; one armed fault at a time, process-wide):
+ *   MOE_FAULT_CACHE_ALLOC  the n-th later device allocation of
+ *                          moe_cache_create fails (as cudaErrorMemoryAllocation)
+ *   MOE_FAULT_CACHE_COPY   the n-th later host -> device copy enqueue of
+ *                          moe_cache_acquire fails (as cudaErrorInvalidValue)
+ *   MOE_FAULT_CACHE_STALL  the next moe_cache_acquire that copies holds its
+ *                          copy stream for n ms first (a host function)
+ *   MOE_FAULT_NONE         disarm
+ * No GPU work is faulted: the failures are return codes the library makes
+ * up on the host. */
+typedef enum {
+  MOE_FAULT_NONE = 0,
+  MOE_FAULT_CACHE_ALLOC = 1,
+  MOE_FAULT_CACHE_COPY = 2,
+  MOE_FAULT_CACHE_STALL = 3
+} moe_fault;
+moe_status moe_debug_inject_fault(int kind, int n);
 
 const char* moe_status_string(moe_status s);
 /* Text of the last failure on the calling thread ("" if none). */

@@ -66,6 +66,8 @@ def lib():
         L.moe_layer_create.argtypes = [p, p, p, p, p, ctypes.POINTER(p)]
         L.moe_layer_destroy.restype = None
         L.moe_layer_destroy.argtypes = [p]
+        L.moe_layer_set_top_p.restype = st
+        L.moe_layer_set_top_p.argtypes = [p, ctypes.c_float]
         L.moe_layer_set_expert.restype = st
         L.moe_layer_set_expert.argtypes = [p, i, p, p]
         L.moe_workspace_bytes.restype = sz
@@ -98,6 +100,10 @@ def lib():
         L.moe_cache_stats.argtypes = [p, i, p, p, p]
         L.moe_cache_sync.restype = st
         L.moe_cache_sync.argtypes = [p]
+        L.moe_cache_wait.restype = st
+        L.moe_cache_wait.argtypes = [p, i]
+        L.moe_debug_inject_fault.restype = st
+        L.moe_debug_inject_fault.argtypes = [i, i]
         L.moe_lru_replay.restype = st
         L.moe_lru_replay.argtypes = [i, i, i, i, i, p, p, p]
         L.moe_debug_gemv_int4.restype = st
@@ -172,6 +178,10 @@ class Layer:
         check(lib().moe_layer_set_expert(self.handle, int(e), ctypes.byref(ex), _stream(stream)),
               "moe_layer_set_expert")
 
+    def set_top_p(self, p):
+        """Adaptive expert top-p (moe_layer_set_top_p); p >= 1 turns it off."""
+        check(lib().moe_layer_set_top_p(self.handle, float(p)), "moe_layer_set_top_p")
+
     def route(self, x, idx, w, ws, scores=None, stream=None):
         T = x.shape[0]
         check(lib().moe_route(self.handle, _ptr(x), T, _ptr(idx), _ptr(w), _ptr(scores),
@@ -238,6 +248,7 @@ class _LayerView:
     route = Layer.route
     expert_ffn = Layer.expert_ffn
     forward = Layer.forward
+    set_top_p = Layer.set_top_p
 
 
 class Cache:
@@ -288,6 +299,11 @@ class Cache:
     def sync(self):
         check(lib().moe_cache_sync(self.handle), "moe_cache_sync")
 
+    def wait(self, timeout_ms):
+        """Wait at most timeout_ms for the copies (MoeError MOE_ERR_TIMEOUT
+        if they are still running then)."""
+        check(lib().moe_cache_wait(self.handle, int(timeout_ms)), "moe_cache_wait")
+
     def close(self):
         if getattr(self, "handle", None):
             lib().moe_cache_destroy(self.handle)
@@ -298,6 +314,15 @@ class Cache:
             self.close()
         except Exception:
             pass
+
+
+FAULT_NONE, FAULT_CACHE_ALLOC, FAULT_CACHE_COPY, FAULT_CACHE_STALL = 0, 1, 2, 3
+
+
+def inject_fault(kind, n=0):
+    """Arm a host-side fault of the library's error paths (moe.h,
+    moe_debug_inject_fault); kind FAULT_NONE disarms."""
+    check(lib().moe_debug_inject_fault(int(kind), int(n)), "moe_debug_inject_fault")
 
 
 def gemv_int4(q, s, rows, cols, x, y, stream=None):

@@ -235,6 +235,13 @@ moe_status moe_layer_set_expert(moe_layer* l, int e, const moe_expert* ex, void*
   return ce == cudaSuccess ? MOE_OK : cuda_fail(ce, "moe_layer_set_expert");
 }
 
+moe_status moe_layer_set_top_p(moe_layer* l, float p) {
+  if (!l) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+  if (!(p > 0.f)) return fail(MOE_ERR_INVALID_ARG, "top_p must be > 0 (>= 1 turns it off)");
+  l->top_p = p >= 1.f ? 1.f : p;
+  return MOE_OK;
+}
+
 size_t moe_workspace_bytes(const moe_config* cfg, int T) {
   if (check_config(cfg) != MOE_OK || T < 1 || T > kMaxTokens) return 0;
   return ws_layout(cfg, T).total;

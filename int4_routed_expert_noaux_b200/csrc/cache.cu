@@ -12,7 +12,10 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+#include <chrono>
 #include <new>
+#include <thread>
 #include <vector>
 
 #include "layer.h"
@@ -29,6 +32,14 @@ class LruPolicy {
   struct Load {
     int expert, slot, evicted;
   };
+
+  // Forget whatever slot `slot` holds (it becomes empty).
+  void invalidate(int slot) {
+    const int old = slot_expert_[slot];
+    if (old >= 0) expert_slot_[old] = -1;
+    slot_expert_[slot] = -1;
+    stamp_[slot] = 0;
+  }
 
   // ids ascending, distinct.  Fills loads (misses) and returns the hit count.
   int access(const int32_t* ids, int n, std::vector<Load>& loads) {
@@ -73,7 +84,25 @@ class LruPolicy {
   uint64_t clock_ = 0;
 };
 
+// Host-side fault injection for tests (off unless armed through
+// moe_debug_inject_fault): the n-th later event of a kind fails.
+std::atomic<int> g_inject_kind{0};
+std::atomic<int> g_inject_after{0};
+
+bool inject(int kind) {
+  if (g_inject_kind.load(std::memory_order_acquire) != kind) return false;
+  if (g_inject_after.fetch_sub(1, std::memory_order_acq_rel) != 0) return false;
+  g_inject_kind.store(0, std::memory_order_release);
+  return true;
+}
+
 namespace {
+
+// Host function run in stream order: holds the stream for `ms` milliseconds
+// (an injected stall; host memory and time only, no GPU work).
+void CUDART_CB hold_stream(void* ms) {
+  std::this_thread::sleep_for(std::chrono::milliseconds((intptr_t)ms));
+}
 
 constexpr int kMaxTableUpdates = 32;
 
@@ -107,6 +136,7 @@ struct moe_cache {
   std::vector<cudaEvent_t> copied;     // per layer: loads of the last acquire done
   std::vector<cudaEvent_t> used;       // per layer: compute of the last release done
   std::vector<bool> used_valid;
+  std::vector<bool> acquired;          // per layer: acquired, not yet released
   std::vector<LruPolicy> lru;
   std::vector<moe_layer*> views;       // per layer, created by moe_cache_layer
   std::vector<uint64_t> hits, misses, bytes;
@@ -206,11 +236,13 @@ moe_status moe_cache_create(const moe_config* cfg, int n_layers, int slots_per_l
     delete c;
     return fail(MOE_ERR_OOM, "cache needs %zu bytes of HBM, %zu free", dev_bytes, free_b);
   }
-  ce = cudaMalloc(&c->dev_slots, dev_bytes);
+  ce = inject(MOE_FAULT_CACHE_ALLOC) ? cudaErrorMemoryAllocation
+                                      : cudaMalloc(&c->dev_slots, dev_bytes);
   if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&c->copy_stream, cudaStreamNonBlocking);
   c->copied.assign(n_layers, nullptr);
   c->used.assign(n_layers, nullptr);
   c->used_valid.assign(n_layers, false);
+  c->acquired.assign(n_layers, false);
   for (int l = 0; l < n_layers && ce == cudaSuccess; ++l) {
     ce = cudaEventCreateWithFlags(&c->copied[l], cudaEventDisableTiming);
     if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->used[l], cudaEventDisableTiming);
@@ -277,16 +309,37 @@ moe_status moe_cache_acquire(moe_cache* c, int layer, const int32_t* ids_host, i
     if (ids_host[j] < 0 || ids_host[j] >= c->cfg.n_experts || (j && ids_host[j] <= ids_host[j - 1]))
       return fail(MOE_ERR_INVALID_ARG, "ids must be ascending, distinct and in range");
   cudaStream_t cs = (cudaStream_t)compute_stream;
-  const int hits = c->lru[layer].access(ids_host, n, c->loads);
-  c->hits[layer] += hits;
-  if (c->loads.empty()) return MOE_OK;
+  // The replacement is planned on a copy of the layer's state and committed
+  // (with the counters and the pointer table) only once every copy of every
+  // miss is enqueued.
+  LruPolicy plan = c->lru[layer];
+  const int hits = plan.access(ids_host, n, c->loads);
+  if (c->loads.empty()) {
+    c->lru[layer] = plan;
+    c->hits[layer] += hits;
+    c->acquired[layer] = true;
+    return MOE_OK;
+  }
   cudaError_t ce = cudaSuccess;
-  // a victim slot may still be read by this layer's previously released compute
-  if (c->used_valid[layer]) ce = cudaStreamWaitEvent(c->copy_stream, c->used[layer], 0);
+  // A victim slot may still be read by compute enqueued earlier for this
+  // layer: that of the last release, or -- acquired again with no release
+  // in between -- everything enqueued on the compute stream so far.
+  if (c->acquired[layer]) {
+    ce = cudaEventRecord(c->used[layer], cs);
+    if (ce == cudaSuccess) c->used_valid[layer] = true;
+  }
+  if (ce == cudaSuccess && c->used_valid[layer])
+    ce = cudaStreamWaitEvent(c->copy_stream, c->used[layer], 0);
+  if (ce == cudaSuccess && g_inject_kind.load(std::memory_order_acquire) == MOE_FAULT_CACHE_STALL) {
+    const int ms = g_inject_after.exchange(0);
+    g_inject_kind.store(0, std::memory_order_release);
+    ce = cudaLaunchHostFunc(c->copy_stream, hold_stream, reinterpret_cast<void*>((intptr_t)ms));
+  }
   TableUpdate u;
   u.n = 0;
-  moe_layer* view = c->views[layer];
+  int reached = 0;  // loads whose slot a copy may have written
   for (const LruPolicy::Load& ld : c->loads) {
+    if (ce != cudaSuccess) break;
     const moe_expert& he = c->host[(size_t)layer * c->cfg.n_experts + ld.expert];
     const ExpertPtrs d = slot_ptrs(c, layer, ld.slot);
     const void* src[6] = {he.q_gate, he.q_up, he.s_gate, he.s_up, he.q_down, he.s_down};
@@ -295,22 +348,35 @@ moe_status moe_cache_acquire(moe_cache* c, int layer, const int32_t* ids_host, i
     const size_t sz[6] = {c->off[1] - c->off[0], c->off[2] - c->off[1], c->off[3] - c->off[2],
                           c->off[4] - c->off[3], c->off[5] - c->off[4],
                           c->expert_bytes - c->off[5]};
+    ++reached;
     for (int t = 0; t < 6 && ce == cudaSuccess; ++t)
-      ce = cudaMemcpyAsync(dst[t], src[t], sz[t], cudaMemcpyHostToDevice, c->copy_stream);
+      ce = inject(MOE_FAULT_CACHE_COPY)
+               ? cudaErrorInvalidValue
+               : cudaMemcpyAsync(dst[t], src[t], sz[t], cudaMemcpyHostToDevice, c->copy_stream);
     u.ids[u.n] = ld.expert;
     u.ptrs[u.n] = d;
-    view->host_table[ld.expert] = d;
     ++u.n;
-    c->misses[layer] += 1;
-    c->bytes[layer] += c->expert_bytes;
   }
   if (ce == cudaSuccess) ce = cudaEventRecord(c->copied[layer], c->copy_stream);
   if (ce == cudaSuccess) ce = cudaStreamWaitEvent(cs, c->copied[layer], 0);
   if (ce == cudaSuccess) {
-    table_update_kernel<<<1, kMaxTableUpdates, 0, cs>>>(view->table, u);
+    table_update_kernel<<<1, kMaxTableUpdates, 0, cs>>>(c->views[layer]->table, u);
     ce = cudaGetLastError();
   }
-  return ce == cudaSuccess ? MOE_OK : cuda_fail(ce, "moe_cache_acquire");
+  if (ce != cudaSuccess) {
+    // Roll back: the layer keeps its committed state, except that a slot a
+    // copy may have reached no longer counts as holding anything.
+    for (int i = 0; i < reached; ++i) c->lru[layer].invalidate(c->loads[i].slot);
+    return cuda_fail(ce, "moe_cache_acquire");
+  }
+  c->lru[layer] = plan;
+  moe_layer* view = c->views[layer];
+  for (int i = 0; i < u.n; ++i) view->host_table[u.ids[i]] = u.ptrs[i];
+  c->hits[layer] += hits;
+  c->misses[layer] += u.n;
+  c->bytes[layer] += (uint64_t)u.n * c->expert_bytes;
+  c->acquired[layer] = true;
+  return MOE_OK;
 }
 
 moe_status moe_cache_release(moe_cache* c, int layer, void* compute_stream) {
@@ -319,6 +385,7 @@ moe_status moe_cache_release(moe_cache* c, int layer, void* compute_stream) {
   cudaError_t ce = cudaEventRecord(c->used[layer], (cudaStream_t)compute_stream);
   if (ce != cudaSuccess) return cuda_fail(ce, "moe_cache_release");
   c->used_valid[layer] = true;
+  c->acquired[layer] = false;
   return MOE_OK;
 }
 
@@ -336,6 +403,29 @@ moe_status moe_cache_sync(moe_cache* c) {
   if (!c) return fail(MOE_ERR_INVALID_ARG, "cache is NULL");
   cudaError_t ce = cudaStreamSynchronize(c->copy_stream);
   return ce == cudaSuccess ? MOE_OK : cuda_fail(ce, "moe_cache_sync");
+}
+
+moe_status moe_cache_wait(moe_cache* c, int timeout_ms) {
+  if (!c) return fail(MOE_ERR_INVALID_ARG, "cache is NULL");
+  if (timeout_ms < 0) return fail(MOE_ERR_INVALID_ARG, "timeout_ms must be >= 0");
+  const auto deadline = std::chrono::steady_clock::now() + std::chrono::milliseconds(timeout_ms);
+  for (;;) {
+    const cudaError_t ce = cudaStreamQuery(c->copy_stream);
+    if (ce == cudaSuccess) return MOE_OK;
+    if (ce != cudaErrorNotReady) return cuda_fail(ce, "moe_cache_wait");
+    if (std::chrono::steady_clock::now() >= deadline)
+      return fail(MOE_ERR_TIMEOUT, "expert copies still running after %d ms", timeout_ms);
+    std::this_thread::sleep_for(std::chrono::microseconds(50));
+  }
+}
+
+moe_status moe_debug_inject_fault(int kind, int n) {
+  if (kind < MOE_FAULT_NONE || kind > MOE_FAULT_CACHE_STALL || n < 0)
+    return fail(MOE_ERR_INVALID_ARG, "bad fault injection (kind %d, n %d)", kind, n);
+  g_inject_kind.store(0, std::memory_order_release);
+  g_inject_after.store(n, std::memory_order_release);
+  g_inject_kind.store(kind, std::memory_order_release);
+  return MOE_OK;
 }
 
 #pragma GCC visibility pop

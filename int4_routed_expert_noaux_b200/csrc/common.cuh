@@ -213,6 +213,50 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// sigmoid of an fp64 logit, taken in fp64 and rounded to fp32 once.
+__device__ __forceinline__ float sigmoid_f64_to_f32(double v) {
+  return (float)(1.0 / (1.0 + exp(-v)));
+}
+
+// Adaptive expert top-p over one warp's k picks (lane < k holds a picked
+// id and its unbiased score s; denom = the sum of the k scores).  A pick is
+// kept when the weight share of the picks ranked before it (descending
+// score, ties to the lower id) is below p: the kept picks are the shortest
+// weight-ordered prefix whose share reaches p (colibri summary, "--topp":
+// adaptive expert top-p; the rule is reading R16 of the layer's design).
+__device__ __forceinline__ bool topp_keep(int id, float s, float denom, int k, float p) {
+  const int lane = threadIdx.x & 31;
+  float before = 0.f;
+#pragma unroll 4
+  for (int j = 0; j < 32; ++j) {
+    const float sj = __shfl_sync(0xffffffffu, s, j);
+    const int ij = __shfl_sync(0xffffffffu, id, j);
+    const bool ahead = j < k && (sj > s || (sj == s && ij < id));
+    before += ahead ? sj / denom : 0.f;
+  }
+  return lane < k && (p >= 1.f || before < p);
+}
+
+// Output position of a pick after top-p: the kept ids ascending first, the
+// dropped picks after them in lane order.
+__device__ __forceinline__ int topp_position(int id, bool kept, int k) {
+  const int lane = threadIdx.x & 31;
+  int pos = 0;
+#pragma unroll 4
+  for (int j = 0; j < 32; ++j) {
+    const int ij = __shfl_sync(0xffffffffu, id, j);
+    const bool kj = __shfl_sync(0xffffffffu, kept ? 1 : 0, j) != 0;
+    if (j < k) pos += kept ? (kj && ij < id) : (kj || j < lane);
+  }
+  return pos;
+}
+
 __device__ __forceinline__ float silu_mul(float g, float u) {
   return g / (1.0f + __expf(-g)) * u;
 }

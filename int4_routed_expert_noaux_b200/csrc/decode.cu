@@ -52,6 +52,18 @@
 #include "async.cuh"
 #include "common.cuh"
 #include "decode.h"
+#include "device_once.h"
+
+// Timeline probes: compiled in only with -DMOE_TRACE (a profiling build);
+// slot i of CTA b gets the globaltimer at probe i.
+#ifdef MOE_TRACE
+#define TRACE_AT(i)                                                       \
+  do {                                                                    \
+    if (p.trace) p.trace[blockIdx.x * 16 + (i)] = moe::global_timer_ns(); \
+  } while (0)
+#else
+#define TRACE_AT(i) ((void)0)
+#endif
 
 namespace moe {
 
@@ -60,15 +72,17 @@ namespace {
 constexpr int kGW = 6;                   // warps per consumer group
 constexpr int kGT = kGW * 32;            // threads per consumer group
 constexpr int kGroups = 2;
-constexpr int kThreads = kGroups * kGT + 64;
+constexpr int kThreads = kGroups * kGT + 96;
 constexpr int kProducerWarp = kGroups * kGW;
 constexpr int kSelectWarp = kProducerWarp + 1;
+constexpr int kConvWarp = kProducerWarp + 2;
 constexpr int kStages = 4;
 constexpr uint32_t kStageBytes = 55296;
 constexpr int kRouterChunks = 8;         // 16-byte W chunks per thread per row
 constexpr int kMaxRR = 8;                // router rows per item
 constexpr int kMaxE = 256;
 constexpr int kMaxSlots = 33;
+constexpr int kMaxYcta = 512;            // slot partials of a CTA's own down rows
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 enum ItemType : int { kRouter = 0, kGateUp = 1, kDown = 2, kDone = 3 };
@@ -87,11 +101,14 @@ struct Smem {
   float sel_w[kMaxSlots];  // their combine weights
   int sel_ok;
   float red[kGroups][2][kGW][32];
+  double redd[kGW][kMaxRR];  // router partial sums (fp64)
   int abort_flag[kGroups];
   float norm_part[kThreads / 32];
   float inv_rms;
   float sc[kMaxE];
   float sp[kMaxE];
+  float ycta[kMaxYcta];    // [slots][ycta_rows] partial y of the CTA's own rows
+  int last_cta;
 };
 
 // The out-of-line helpers take their arguments by value: a reference to the
@@ -119,13 +136,6 @@ __device__ __forceinline__ SelArgs sel_args(const DecodeParams& p) {
   return a;
 }
 
-struct CombineArgs {
-  int k, H, has_shared;
-  const float* ypart;
-  const float* x_resid;
-  float* y;
-};
-
 __device__ __forceinline__ ItemDesc make_item(int type, int slot, int row0, int nrows) {
   ItemDesc d;
   d.type = type;
@@ -137,25 +147,40 @@ __device__ __forceinline__ ItemDesc make_item(int type, int slot, int row0, int 
   return d;
 }
 
-__device__ __forceinline__ ItemDesc decode_ticket(const DecodeParams& p, int t) {
-  // shared gate/up, routed gate/up 0..k-1, shared down, routed down 0..k-1
+// Gate/up item of ticket t, in the order: shared gate/up, routed gate/up of
+// slots 0..k-1; DONE past the last one.
+__device__ __forceinline__ ItemDesc gate_up_ticket(const DecodeParams& p, int t) {
   auto gu = [&](int slot, int b) {
     return make_item(kGateUp, slot, b * p.RG, min(p.RG, p.I - b * p.RG));
-  };
-  auto dn = [&](int slot, int b) {
-    return make_item(kDown, slot, b * p.RD, min(p.RD, p.H - b * p.RD));
   };
   if (p.has_shared) {
     if (t < p.nG) return gu(p.k, t);
     t -= p.nG;
   }
   if (t < p.k * p.nG) return gu(t / p.nG, t % p.nG);
-  t -= p.k * p.nG;
-  if (p.has_shared) {
-    if (t < p.nD) return dn(p.k, t);
-    t -= p.nD;
+  return make_item(kDone, 0, 0, 0);
+}
+
+// Down rows of CTA b: [r0, r1), whole units of A rows (A keeps every row
+// offset of the scales 16-byte aligned).
+__device__ __forceinline__ void down_rows(const DecodeParams& p, int b, int& r0, int& r1) {
+  r0 = p.A * (int)(((long long)b * p.nU) / gridDim.x);
+  r1 = p.A * (int)(((long long)(b + 1) * p.nU) / gridDim.x);
+}
+
+// This CTA's next down item: the shared expert's rows first, then slots
+// 0..k-1, each in n_db blocks of at most RD rows; DONE when all are taken.
+__device__ __forceinline__ ItemDesc next_down(const DecodeParams& p, int& dn, int r0, int r1) {
+  const int slots = p.k + p.has_shared;
+  while (dn < slots * p.n_db) {
+    const int ord = dn / p.n_db, blk = dn % p.n_db;
+    ++dn;
+    const int row0 = r0 + blk * p.RD;
+    const int nrows = min(p.RD, r1 - row0);
+    if (nrows <= 0) continue;
+    const int slot = p.has_shared ? (ord == 0 ? p.k : ord - 1) : ord;
+    return make_item(kDown, slot, row0, nrows);
   }
-  if (t < p.k * p.nD) return dn(t / p.nD, t % p.nD);
   return make_item(kDone, 0, 0, 0);
 }
 
@@ -309,24 +334,6 @@ __device__ __forceinline__ uint2 norm_bf16x4(const float* x_resid, int i0, float
   r.x = (uint32_t)f32_to_bf16_rne(v.x * inv_rms) | ((uint32_t)f32_to_bf16_rne(v.y * inv_rms) << 16);
   r.y = (uint32_t)f32_to_bf16_rne(v.z * inv_rms) | ((uint32_t)f32_to_bf16_rne(v.w * inv_rms) << 16);
   return r;
-}
-
-// Fixed-order combine of one row block of y from the per-slot partials, by
-// one warp, once every slot's down item of the block has published.
-__device__ __noinline__ void combine_block(const CombineArgs p, const float* wsel, int row0,
-                                          int nrows) {
-  const int lane = threadIdx.x & 31;
-  if (lane == 0) fence_acq_rel();  // see the other warps' partials
-  __syncwarp();
-  for (int lr = lane; lr < nrows; lr += 32) {
-    const int row = row0 + lr;
-    float acc = 0.f;
-    for (int j = 0; j < p.k; ++j)
-      acc = fmaf(wsel[j], __ldcg(p.ypart + (size_t)j * p.H + row), acc);
-    if (p.has_shared) acc += __ldcg(p.ypart + (size_t)p.k * p.H + row);
-    if (p.x_resid) acc = p.x_resid[row] + acc;  // residual stream: x + MoE(norm(x))
-    p.y[row] = acc;
-  }
 }
 
 // Order-preserving map of a float onto uint32 (larger float, larger key;
@@ -535,6 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   const int slots = p.k + p.has_shared;
 
   if (threadIdx.x == 0) {
+    TRACE_AT(0);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&S.full[s], 1);
       mbar_init(&S.empty[s], kGW);
@@ -569,12 +577,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     if (lane == 0) {
       const uint64_t policy = l2_policy_evict_first();
       bool sel_seen = false;
-      uint64_t h_seen = 0;  // bit j: slot j's h acquired
+      bool first_routed = false, first_down = false;
+      uint64_t hq_seen = 0;  // bit j: slot j's int16 h acquired
       int dones = 0;
       int rr0, rnr;
       router_rows(p, blockIdx.x, rr0, rnr);
       bool router_pending = rnr > 0;
-      int t = router_pending ? -1 : (int)atomicAdd(p.ctrl + kCtrlTicket, 1u);
+      bool tickets_over = false;
+      int dn = 0;  // this CTA's down items taken so far
+      int dr0, dr1;
+      down_rows(p, blockIdx.x, dr0, dr1);
       for (uint32_t n = 0;; ++n) {
         const int stage = (int)(n % kStages);
         ItemDesc d = make_item(kDone, 0, 0, 0);
@@ -582,18 +594,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           d = make_item(kRouter, 0, rr0, rnr);
           router_pending = false;
         } else if (dones == 0) {
-          d = decode_ticket(p, t);
-          if (d.type == kDown) {
-            // every gate/up item of the slot must have published its h rows
-            // before the slot's h is copied
-            if (!((h_seen >> d.slot) & 1ull)) {
-              if (wait_counter(p.ctrl, p.ctrl + kCtrlGuDone + d.slot, (uint32_t)p.gu_count)) {
-                h_seen |= 1ull << d.slot;
-                fence_proxy_async();  // order the h stores before the bulk read
-              } else {
-                set_error(p.ctrl, kErrTimeout, 7, n);
-                d = make_item(kDone, 0, 0, 0);
-              }
+          if (!tickets_over) {
+            d = gate_up_ticket(p, (int)atomicAdd(p.ctrl + kCtrlTicket, 1u));
+            tickets_over = d.type == kDone;
+          }
+          if (tickets_over) d = next_down(p, dn, dr0, dr1);
+          if (d.type == kDown && !((hq_seen >> d.slot) & 1ull)) {
+            // every 32-row group of the slot's h must be published as int16
+            if (wait_counter(p.ctrl, p.ctrl + kCtrlHqDone + d.slot, (uint32_t)(p.I >> 5))) {
+              hq_seen |= 1ull << d.slot;
+              fence_proxy_async();  // order the observed stores before the bulk reads
+            } else {
+              set_error(p.ctrl, kErrTimeout, 7, n);
+              d = make_item(kDone, 0, 0, 0);
             }
           }
           if (d.type == kGateUp || d.type == kDown) {
@@ -602,6 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
                 // the selection warp's result (mbarrier: release / acquire)
                 if (mbar_wait(&S.selbar, 0u, global_timer_ns() + kWaitNs) && S.sel_ok) {
                   sel_seen = true;
+                  TRACE_AT(12);
                 } else {
                   set_error(p.ctrl, kErrTimeout, 4, n);
                   d = make_item(kDone, 0, 0, 0);
@@ -635,10 +649,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         S.desc[stage] = d;
         uint8_t* dst = stages + (size_t)stage * kStageBytes;
         if (d.type == kRouter) {
+          TRACE_AT(1);
           const uint32_t bytes = (uint32_t)d.nrows * p.H * 4;
           mbar_arrive_expect_tx(&S.full[stage], bytes);
           bulk_g2s(dst, p.w_router + (size_t)d.row0 * p.H, bytes, &S.full[stage], policy);
         } else if (d.type == kGateUp) {
+          if (d.slot == 0 && !first_routed) {
+            first_routed = true;
+            TRACE_AT(6);
+          }
           const ExpertPtrs ep = p.table[d.eid];
           const uint32_t qb = (uint32_t)d.nrows * (p.H / 2), sb = (uint32_t)d.nrows * (p.H / 16);
           const size_t qoff = (size_t)d.row0 * (p.H / 2), soff = (size_t)d.row0 * (p.H / 32);
@@ -649,17 +668,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           bulk_g2s(dst + 2 * p.RG * (p.H / 2) + p.RG * (p.H / 16), ep.s_up + soff, sb,
                    &S.full[stage], policy);
         } else if (d.type == kDown) {
+          if (!first_down) {
+            first_down = true;
+            TRACE_AT(7);
+          }
           const ExpertPtrs ep = p.table[d.eid];
+          const int GD = p.I >> 5;
           const uint32_t qb = (uint32_t)d.nrows * (p.I / 2), sb = (uint32_t)d.nrows * (p.I / 16);
-          const uint32_t hb = (uint32_t)p.I * 4;
-          mbar_arrive_expect_tx(&S.full[stage], qb + sb + hb);
+          const uint32_t hb = (uint32_t)GD * 64, fb = (uint32_t)GD * 4;
+          const uint32_t tail = (uint32_t)p.RD * (p.I / 2 + p.I / 16);
+          mbar_arrive_expect_tx(&S.full[stage], qb + sb + hb + fb);
           bulk_g2s(dst, ep.q_down + (size_t)d.row0 * (p.I / 2), qb, &S.full[stage], policy);
           bulk_g2s(dst + p.RD * (p.I / 2), ep.s_down + (size_t)d.row0 * (p.I / 32), sb,
                    &S.full[stage], policy);
-          bulk_g2s(dst + p.RD * (p.I / 2) + p.RD * (p.I / 16),
-                   p.hbuf + (size_t)d.slot * p.I, hb, &S.full[stage], l2_policy_evict_last());
+          const uint64_t keep = l2_policy_evict_last();
+          bulk_g2s(dst + tail, p.hq + (size_t)d.slot * hb, hb, &S.full[stage], keep);
+          bulk_g2s(dst + tail + hb, p.hqf + (size_t)d.slot * GD, fb, &S.full[stage], keep);
         } else {
           mbar_arrive(&S.full[stage]);  // a DONE fill: one per consumer group
+          if (dones == 0) TRACE_AT(11);
           if (++dones == kGroups) {
             // leave no bulk copy in flight
             for (uint32_t m = (n >= (uint32_t)kStages ? n - kStages + 1 : 0); m < n; ++m) {
@@ -668,9 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
             }
             break;
           }
-          continue;
         }
-        t = (int)atomicAdd(p.ctrl + kCtrlTicket, 1u);
       }
     }
   } else if (warp == kSelectWarp) {
@@ -711,6 +736,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       }
     }
     if (ok) {
+      if (lane == 0) TRACE_AT(4);
 #pragma unroll
       for (int m = 0; m < kMaxE / 32; ++m) {
         const int e = lane + 32 * m;
@@ -722,6 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       }
       __syncwarp();
       run_select(sel_args(p), S);
+      if (lane == 0) TRACE_AT(5);
     } else if (lane == 0) {
       set_error(p.ctrl, kErrTimeout, 8, 0);
     }
@@ -729,6 +756,64 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     if (lane == 0) {
       S.sel_ok = ok ? 1 : 0;
       mbar_arrive(&S.selbar);
+    }
+  } else if (warp == kConvWarp) {
+    // ------------------------------------------------------------ converter
+    // Publishes 32-row groups of h as int16 words (the XQ layout the down
+    // consumers load) once their 32 rows are written.  CTA b owns groups
+    // b, b + grid, ... of the order (shared slot first, then slots 0..k-1;
+    // groups ascending), the order in which gate/up items complete.
+    const int GD = p.I >> 5, slots = p.k + p.has_shared;
+    for (int i = blockIdx.x; i < slots * GD; i += gridDim.x) {
+      const int so = i / GD, g = i % GD;
+      const int slot = p.has_shared ? (so == 0 ? p.k : so - 1) : so;
+      const uint32_t* cnt = p.ctrl + kCtrlHRows + slot * GD + g;
+      // every lane acquires the count itself (so its own loads of h below
+      // are ordered after the writers' release adds)
+      bool ok = true;
+      {
+        const uint64_t deadline = global_timer_ns() + kWaitNs;
+        for (uint32_t it = 0;; ++it) {
+          if (__all_sync(0xffffffffu, ld_acquire(cnt) >= 32u)) break;
+          if ((it & 7) == 7) {
+            const int stop = lane == 0 && (aborted(p.ctrl) || global_timer_ns() > deadline);
+            if (__shfl_sync(0xffffffffu, stop, 0)) {
+              ok = false;
+              break;
+            }
+          }
+          __nanosleep(64);
+        }
+      }
+      if (!ok) {
+        if (lane == 0 && !aborted(p.ctrl)) set_error(p.ctrl, kErrTimeout, 9, (uint32_t)i);
+        break;
+      }
+      const float hv = __ldcg(p.hbuf + (size_t)slot * p.I + g * 32 + lane);
+      // the int16 group format of the layer kernels: the largest magnitude
+      // maps into [2^14, 2^15), round to nearest even (xq_from_floats)
+      float m = fabsf(hv);
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      int ex = 0;
+      if (m > 0.f) frexpf(m, &ex);
+      const int e = 15 - ex;
+      const float sc = (m > 0.f) ? ldexpf(1.0f, e) : 0.f;
+      const float b = fmaf(hv, sc, 12582912.0f);
+      const int X = max(-32767, min(32767, (int)(__float_as_uint(b) - 0x4B400000u)));
+      // element j = 8i + r sits in word ev[2i + (r >= 4)] (r even) or
+      // od[2i + (r >= 4)] (r odd), low half for r % 4 < 2
+      const int ii = lane >> 3, r = lane & 7;
+      const int word = ((r & 1) ? 8 : 0) + 2 * ii + (r >= 4 ? 1 : 0);
+      const int half = (r & 2) ? 1 : 0;
+      uint16_t* dst = reinterpret_cast<uint16_t*>(p.hq + ((size_t)slot * GD + g) * 64);
+      dst[2 * word + half] = (uint16_t)(X & 0xFFFF);
+      if (lane == 0) p.hqf[(size_t)slot * GD + g] = (m > 0.f) ? ldexpf(1.0f, -e - 4) : 0.f;
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence();
+        red_add_release(p.ctrl + kCtrlHqDone + slot, 1u);
+      }
     }
   } else {
     // ------------------------------------------------------------ consumers
@@ -776,15 +861,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       xq_from_floats(xf, xq);
     }
     int& gabort = S.abort_flag[grp];
-    CombineArgs comb;
-    comb.k = p.k;
-    comb.H = p.H;
-    comb.has_shared = p.has_shared;
-    comb.ypart = p.ypart;
-    comb.x_resid = p.x_resid;
-    comb.y = p.y;
-    int pend_row0 = -1, pend_nrows = 0;  // this warp's last down row block
-    uint32_t pend_old = 0;               // count before this warp's add (lane 0)
+    int dr0, dr1;
+    down_rows(p, blockIdx.x, dr0, dr1);
     // Group 0 of a CTA with router rows: fill 0 is the router block.  It is
     // handled before the main loop so its bf16 inputs are dead afterwards.
     uint32_t c_first = 0;
@@ -806,23 +884,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
             xr[i] = __ldg(reinterpret_cast<const uint2*>(p.x) + cc);
           }
         }
-        const int stage = 0, rbuf = 0;
+        const int stage = 0;
         const uint32_t gpar = 0u;
         int okw = 0;
         if (lane == 0) okw = mbar_wait(&S.full[0], 0u, global_timer_ns() + kWaitNs) ? 1 : 0;
         const bool ok = __shfl_sync(0xffffffffu, okw, 0) != 0;
         if (ok) {
           mbar_test(&S.full[0], 0u);
+          if (tg == 0) TRACE_AT(2);
         } else {
           if (lane == 0) set_error(p.ctrl, kErrTimeout, 1, 0);
           gabort = 1;
         }
         const ItemDesc d = S.desc[0];
         const uint8_t* st = stages;
-        float acc[kMaxRR];
+        // fp64 sums of exact fp32 x bf16 products: the logit is exact to
+        // about 1e-13, so the selection sees scores rounded only once
+        double acc[kMaxRR];
 #pragma unroll
         for (int r = 0; r < kMaxRR; ++r) {
-          acc[r] = 0.f;
+          acc[r] = 0.0;
           if (ok && r < d.nrows) {
             const float4* wr = reinterpret_cast<const float4*>(st + (size_t)r * p.H * 4);
 #pragma unroll
@@ -830,10 +911,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
               const int cc = tg + kGT * i;
               if (cc < rchunks) {
                 const float4 wv = wr[cc];
-                acc[r] = fmaf(wv.x, bf16_bits_to_f32(xr[i].x & 0xFFFFu), acc[r]);
-                acc[r] = fmaf(wv.y, bf16_bits_to_f32(xr[i].x >> 16), acc[r]);
-                acc[r] = fmaf(wv.z, bf16_bits_to_f32(xr[i].y & 0xFFFFu), acc[r]);
-                acc[r] = fmaf(wv.w, bf16_bits_to_f32(xr[i].y >> 16), acc[r]);
+                acc[r] = fma((double)wv.x, (double)bf16_bits_to_f32(xr[i].x & 0xFFFFu), acc[r]);
+                acc[r] = fma((double)wv.y, (double)bf16_bits_to_f32(xr[i].x >> 16), acc[r]);
+                acc[r] = fma((double)wv.z, (double)bf16_bits_to_f32(xr[i].y & 0xFFFFu), acc[r]);
+                acc[r] = fma((double)wv.w, (double)bf16_bits_to_f32(xr[i].y >> 16), acc[r]);
               }
             }
           }
@@ -843,8 +924,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
 #pragma unroll
         for (int r = 0; r < kMaxRR; ++r) {
           if (r < d.nrows) {
-            const float v = warp_sum(acc[r]);
-            if (lane == 0) S.red[grp][rbuf][gw][r] = v;
+            const double v = warp_sum_f64(acc[r]);
+            if (lane == 0) S.redd[gw][r] = v;
           }
         }
         if (!group_barrier(&S.gbar[grp], gpar)) {
@@ -854,12 +935,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         if (!gabort && gw == 0) {
           // the sigmoid score of each row, tagged with this call's epoch
           if (lane < d.nrows) {
-            float v = 0.f;
-            for (int w = 0; w < kGW; ++w) v += S.red[grp][rbuf][w][lane];
-            const float sg = 1.0f / (1.0f + expf(-v));
+            double v = 0.0;
+            for (int w = 0; w < kGW; ++w) v += S.redd[w][lane];
+            const float sg = sigmoid_f64_to_f32(v);
             st_relaxed_u64(p.scores + d.row0 + lane,
                            ((uint64_t)epoch << 32) | __float_as_uint(sg));
           }
+          if (lane == 0) TRACE_AT(3);
         }
       }
     }
@@ -868,6 +950,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     // publish nothing: the instructions of both paths are fetched while the
     // first weights are still on their way, not when they have arrived.
     int warm = (grp == 1 && p.warm) ? 2 : 0;
+    bool tr_gu = false, tr_dn = false;
     uint32_t c = c_first;
     for (uint32_t it = c_first;; ++it) {  // it: group barrier phases used
       if (gabort) break;
@@ -903,6 +986,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         break;
       }
       const uint8_t* st = stages + (size_t)stage * kStageBytes;
+      if (!fake && tg == 0) {
+        if (d.type == kGateUp && d.slot == 0 && !tr_gu) {
+          tr_gu = true;
+          TRACE_AT(8 + grp * 5);
+        }
+        if (d.type == kDown && !tr_dn) {
+          tr_dn = true;
+          TRACE_AT(9 + grp * 5);
+        }
+      }
 
       if (d.type == kGateUp) {
         float v[NV_G];
@@ -930,12 +1023,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           gabort = 1;
         }
         if (gabort) break;
-        if (pend_row0 >= 0) {
-          const uint32_t last =
-              __shfl_sync(0xffffffffu, pend_old + 1 == (uint32_t)(slots * fw_d), 0);
-          if (last) combine_block(comb, S.sel_w, pend_row0, pend_nrows);
-          pend_row0 = -1;
-        }
 
         if (gw < fw_g) {
           // item row tg (= phase * NR_G + i) of this finalizer thread
@@ -951,25 +1038,35 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
             }
             p.hbuf[(size_t)d.slot * p.I + d.row0 + tg] = silu_mul(g, u);
           }
-          __syncwarp();
-          // count this warp done (nothing waits for the result)
-          if (lane == 0 && !fake) red_add_release(p.ctrl + kCtrlGuDone + d.slot, 1u);
+          // count the rows of h this warp wrote, per 32-row group of h (its
+          // rows are consecutive: at most two groups); the converter warp
+          // that owns a group publishes it once all 32 rows are in
+          const bool wrote = tg < cg.P * NR_G && tg < d.nrows;
+          const unsigned vm = __ballot_sync(0xffffffffu, wrote);
+          if (vm && !fake) {
+            const int g = (d.row0 + tg) >> 5;
+            const int g0 = __shfl_sync(0xffffffffu, g, __ffs(vm) - 1);
+            const unsigned m0 = __ballot_sync(0xffffffffu, wrote && g == g0);
+            const unsigned m1 = vm & ~m0;
+            __syncwarp();
+            if (lane == 0) {
+              uint32_t* cnt = p.ctrl + kCtrlHRows + d.slot * (p.I >> 5);
+              red_add_release(cnt + g0, (uint32_t)__popc(m0));
+              if (m1) red_add_release(cnt + g0 + 1, (uint32_t)__popc(m1));
+            }
+          }
         }
       } else {  // kDown
-        XQ hq;  // this thread's 32-row group of h, as int16 fixed point
+        XQ hq;  // this thread's 32-row group of h: int16 words and factor
         {
-          const float4* hs = reinterpret_cast<const float4*>(
-              st + (size_t)p.RD * (p.I / 2) + (size_t)p.RD * (p.I / 16)) + cd.col * 8;
-          float hv[32];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float4 t = hs[i];
-            hv[4 * i] = t.x;
-            hv[4 * i + 1] = t.y;
-            hv[4 * i + 2] = t.z;
-            hv[4 * i + 3] = t.w;
-          }
-          xq_from_floats(hv, hq);
+          const uint8_t* tail = st + (size_t)p.RD * (p.I / 2 + p.I / 16);
+          const uint4* hw = reinterpret_cast<const uint4*>(tail + (size_t)cd.col * 64);
+          const uint4 a0 = hw[0], a1 = hw[1], a2 = hw[2], a3 = hw[3];
+          hq.ev[0] = a0.x; hq.ev[1] = a0.y; hq.ev[2] = a0.z; hq.ev[3] = a0.w;
+          hq.ev[4] = a1.x; hq.ev[5] = a1.y; hq.ev[6] = a1.z; hq.ev[7] = a1.w;
+          hq.od[0] = a2.x; hq.od[1] = a2.y; hq.od[2] = a2.z; hq.od[3] = a2.w;
+          hq.od[4] = a3.x; hq.od[5] = a3.y; hq.od[6] = a3.z; hq.od[7] = a3.w;
+          hq.f = reinterpret_cast<const float*>(tail + (size_t)GD * 64)[cd.col];
         }
         float v[NR_D];
         const size_t rb = (size_t)p.I / 2;
@@ -989,12 +1086,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           gabort = 1;
         }
         if (gabort) break;
-        if (pend_row0 >= 0) {
-          const uint32_t last =
-              __shfl_sync(0xffffffffu, pend_old + 1 == (uint32_t)(slots * fw_d), 0);
-          if (last) combine_block(comb, S.sel_w, pend_row0, pend_nrows);
-          pend_row0 = -1;
-        }
 
         if (gw < fw_d && !fake) {
           if (tg < cd.P * NR_D) {
@@ -1005,39 +1096,51 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
               owner_of<NR_D, SEG_D>(ph, i, cd.wpr, w0, l0);
               float s = 0.f;
               for (int w = 0; w < cd.wpr; ++w) s += S.red[grp][rbuf][w0 + w][l0];
-              p.ypart[(size_t)d.slot * p.H + d.row0 + lr] = s;
+              // this slot's partial of one of the CTA's own rows
+              S.ycta[d.slot * p.ycta_rows + (d.row0 - dr0) + lr] = s;
             }
           }
-          __syncwarp();
-          // count this warp done; the result is looked at one item later
-          if (lane == 0)
-            pend_old = atom_add_release(p.ctrl + kCtrlRbDone + d.row0 / p.RD, 1u);
-          pend_row0 = d.row0;
-          pend_nrows = d.nrows;
         }
       }
-    }
-    // a row block completed by this warp's last down item
-    if (!gabort && pend_row0 >= 0) {
-      const uint32_t last = __shfl_sync(0xffffffffu, pend_old + 1 == (uint32_t)(slots * fw_d), 0);
-      if (last) combine_block(comb, S.sel_w, pend_row0, pend_nrows);
     }
   }
 
   // -------------------------------------------------------------- teardown
   __syncthreads();
+  {
+    // y of this CTA's own rows: the slot partials combined in slot order
+    // (sum_j w_j y_j, then the shared expert, then the residual input),
+    // the same order for every call: no atomics, bitwise repeatable
+    int r0, r1;
+    down_rows(p, blockIdx.x, r0, r1);
+    if (!aborted(p.ctrl)) {
+      for (int lr = threadIdx.x; lr < r1 - r0; lr += kThreads) {
+        float acc = 0.f;
+        for (int j = 0; j < p.k; ++j) acc = fmaf(S.sel_w[j], S.ycta[j * p.ycta_rows + lr], acc);
+        if (p.has_shared) acc += S.ycta[p.k * p.ycta_rows + lr];
+        if (p.x_resid) acc = p.x_resid[r0 + lr] + acc;  // x + MoE(norm(x))
+        p.y[r0 + lr] = acc;
+      }
+    }
+  }
   if (threadIdx.x == 0) {
+    TRACE_AT(10);
     __threadfence();
     const uint32_t old = atomicAdd(p.ctrl + kCtrlExit, 1u);
-    if (old + 1 == gridDim.x) {
-      // last CTA out: reset the counters for the next call (the error word
-      // is left for the host to read) and advance the epoch
-      __threadfence();
-      volatile uint32_t* c = p.ctrl;
+    S.last_cta = (old + 1 == gridDim.x) ? 1 : 0;
+  }
+  __syncthreads();
+  if (S.last_cta) {
+    // last CTA out: reset the counters for the next call (the error word
+    // is left for the host to read) and advance the epoch
+    __threadfence();
+    volatile uint32_t* c = p.ctrl;
+    for (int j = threadIdx.x; j < slots; j += kThreads) c[kCtrlHqDone + j] = 0;
+    for (int j = threadIdx.x; j < slots * (p.I >> 5); j += kThreads) c[kCtrlHRows + j] = 0;
+    __syncthreads();
+    if (threadIdx.x == 0) {
       c[kCtrlTicket] = 0;
       c[kCtrlAbort] = 0;
-      for (int j = 0; j < slots; ++j) c[kCtrlGuDone + j] = 0;
-      for (int b = 0; b < p.nD; ++b) c[kCtrlRbDone + b] = 0;
       c[kCtrlEpoch] = epoch;
       c[kCtrlExit] = 0;
       __threadfence();
@@ -1045,35 +1148,60 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   }
 }
 
-int g_num_sms[64] = {0};
+DeviceOnce<int> g_num_sms;
 
 int num_sms() {
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return 148;
-  if (!g_num_sms[dev]) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-    g_num_sms[dev] = n;
-  }
-  return g_num_sms[dev];
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return n;
+  g_num_sms.get(dev, &n, [dev](int* v) {
+    int m = 0;
+    if (cudaDeviceGetAttribute(&m, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || m <= 0)
+      m = 148;
+    *v = m;
+    return cudaSuccess;
+  });
+  return n;
 }
 
+// The kernel needs all of its CTAs resident at once (selection warps poll
+// every CTA's router records; down items wait on other CTAs' gate/up
+// counts), so it is launched cooperatively: a grid that cannot be
+// co-resident (another kernel holding SMs, a partitioned device) fails at
+// launch instead of running into the device-side wait limit.  The first
+// launch per device and context sets the shared-memory attribute and checks
+// that one CTA fits on an SM.
 template <int SEG_G, int SEG_D>
 cudaError_t launch_t(const DecodeParams& p, cudaStream_t st) {
-  static bool configured[64] = {false};
+  static DeviceOnce<bool> configured;
   int dev = 0;
-  cudaGetDevice(&dev);
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
   const size_t smem = decode_smem_bytes();
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<SEG_G, SEG_D>,
+  bool ok = false;
+  e = configured.get(dev, &ok, [smem](bool* v) {
+    cudaError_t r = cudaFuncSetAttribute(decode_kernel<SEG_G, SEG_D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
-  decode_kernel<SEG_G, SEG_D><<<num_sms(), kThreads, smem, st>>>(p);
-  return cudaGetLastError();
+    if (r != cudaSuccess) return r;
+    int per_sm = 0;
+    r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<SEG_G, SEG_D>,
+                                                      kThreads, smem);
+    if (r != cudaSuccess) return r;
+    if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+    *v = true;
+    return cudaSuccess;
+  });
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)num_sms());
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_kernel<SEG_G, SEG_D>, p);
 }
 
 template <int SEG_G>
@@ -1132,31 +1260,42 @@ bool decode_plan(const moe_config& c, DecodeParams& p) {
     p.sel_fast = per % q == 0 && L >= 1 && (1 << p.sel_lgL) == L && q <= kMaxE / 32;
   }
   p.RG = PG * nrg;
-  p.RD = PD * nrd;
   {
-    // a down item also carries the slot's fp32 h
-    const size_t hb = (size_t)c.inter * 4, rowb = (size_t)c.inter / 2 + c.inter / 16;
-    const int fit = (int)((kStageBytes - hb) / rowb);
-    if (fit < p.RD) p.RD = fit & ~3;
-    if (p.RD < 4 || hb % 16) return false;
+    // A down item is RD rows of q_down and s_down, then the slot's int16 h
+    // groups (GD x 64 bytes) and their factors (GD x 4 bytes, whole 16-byte
+    // units).  Rows go in units of A, so that every scale row offset is
+    // 16-byte aligned (A * GD * 2 bytes a multiple of 16).
+    if (GD % 4) return false;
+    int g8 = GD, m8 = 8;
+    while (m8) {
+      const int t = g8 % m8;
+      g8 = m8;
+      m8 = t;
+    }
+    p.A = 8 / g8;
+    const size_t tail = (size_t)GD * 64 + (size_t)GD * 4, rowb = (size_t)c.inter / 2 + c.inter / 16;
+    if (tail >= kStageBytes) return false;
+    p.RD = min(PD * nrd, (int)((kStageBytes - tail) / rowb));
+    p.RD -= p.RD % p.A;
+    if (p.RD < p.A) return false;
   }
   p.RR = (int)(kStageBytes / ((uint32_t)c.hidden * 4));
   if (p.RR > kMaxRR) p.RR = kMaxRR;
   if (p.RR < 1) return false;
   if ((size_t)p.RG * (c.hidden / 2 + c.hidden / 16) * 2 > kStageBytes) return false;
-  if ((size_t)p.RD * (c.inter / 2 + c.inter / 16) + (size_t)c.inter * 4 > kStageBytes) return false;
-  if ((p.RG * (c.hidden / 16)) % 16 || (p.RD * (c.inter / 16)) % 16) return false;
+  if ((p.RG * (c.hidden / 16)) % 16) return false;
   const int grid = num_sms();
   if ((p.E + grid - 1) / grid > p.RR) return false;  // a CTA's router rows fill one stage
   p.nR = p.E < grid ? p.E : grid;  // CTAs with at least one router row
   p.nG = (p.I + p.RG - 1) / p.RG;
-  p.nD = (p.H + p.RD - 1) / p.RD;
-  p.gu_count = p.nG * ((p.RG + 31) / 32);  // finalizer warps per item: ceil(RG / 32)
   const int slots = p.k + p.has_shared;
+  p.nU = p.H / p.A;
+  p.ycta_rows = p.A * ((p.nU + grid - 1) / grid);  // most down rows a CTA owns
+  p.n_db = (p.ycta_rows + p.RD - 1) / p.RD;
+  if (slots * p.ycta_rows > kMaxYcta) return false;
   // the control words' ranges
-  if (slots > kMaxSlots || slots > kCtrlRbDone - kCtrlGuDone) return false;
-  if (p.nD > kCtrlWords - kCtrlRbDone) return false;
-  p.n_items = p.nR + (p.k + p.has_shared) * (p.nG + p.nD);
+  if (slots > kMaxSlots || kCtrlHqDone + slots > kCtrlHRows) return false;
+  if (kCtrlHRows + slots * GD > kCtrlWords) return false;
   return true;
 }
 

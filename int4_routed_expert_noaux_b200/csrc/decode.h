@@ -22,8 +22,8 @@ enum : int {
   kCtrlExit = 4,
   kCtrlAbort = 5,
   kCtrlWhere = 8,    // [4] where the first error happened (CTA, warp, site, fill)
-  kCtrlGuDone = 16,  // [slots] finished gate/up finalizer warps of the slot
-  kCtrlRbDone = 64,  // [row blocks of hidden] finished down finalizer warps
+  kCtrlHqDone = 16,  // [slots] 32-row groups of the slot's h published as int16
+  kCtrlHRows = 64,   // [slots][inter / 32] rows of h written, per 32-row group
   kCtrlWords = (int)(kCtrlBytes / 4),
 };
 
@@ -40,8 +40,9 @@ struct DecodeParams {
   float* w_out;       // nullable
   uint32_t* ctrl;
   uint64_t* scores;   // [E]: (epoch << 32) | bits of sigmoid(logit), per expert
-  float* hbuf;        // [slots][I]
-  float* ypart;       // [slots][H]
+  float* hbuf;        // [slots][I] fp32 h
+  uint8_t* hq;        // [slots][I / 32] 64-byte int16 groups of h (XQ word order)
+  float* hqf;         // [slots][I / 32] their factors
   int H, I, E, k, n_group, topk_group, has_shared;
   float rsf;
   // selection layout: lane l owns experts l*sel_q .. l*sel_q+sel_q-1 and a
@@ -49,8 +50,11 @@ struct DecodeParams {
   int sel_fast, sel_q, sel_lgL;
   int warm;           // consumer group 1 first runs one placeholder item of each kind
   int RR, RG, RD;     // rows per router block / gate-up item / down item
-  int gu_count;       // finalizer-warp arrivals that complete one slot's h
-  int nR, nG, nD, n_items;
+  int nR, nG;         // CTAs with router rows; gate/up items per slot
+  // down rows: CTA b owns rows [A * (b * nU / grid), A * ((b + 1) * nU / grid))
+  // of every slot, nU = H / A, in n_db items of at most RD rows per slot
+  int A, nU, n_db, ycta_rows;
+  uint64_t* trace;    // timeline probes of a -DMOE_TRACE build ([grid][16]); else unused
 };
 
 // Fill the shape part of p; false if the fused kernel does not cover the

@@ -10,11 +10,11 @@ namespace moe {
 moe_status route_impl(const moe_layer* l, const uint16_t* x, int T, int32_t* idx, float* w,
                       float* scores, uint8_t* ws, const WsLayout& L, cudaStream_t st) {
   const moe_config& c = l->cfg;
-  float* logits = reinterpret_cast<float*>(ws + L.logits);
-  cudaError_t e = launch_router_logits(l->w_router, x, T, c.hidden, c.n_experts, logits, st);
+  float* sc = reinterpret_cast<float*>(ws + L.logits);
+  cudaError_t e = launch_router_scores(l->w_router, x, T, c.hidden, c.n_experts, sc, st);
   if (e == cudaSuccess)
-    e = launch_select(logits, l->bias, T, c.n_experts, c.n_group, c.topk_group, c.top_k,
-                      c.routed_scaling_factor, idx, w, scores, st);
+    e = launch_select(sc, l->bias, T, c.n_experts, c.n_group, c.topk_group, c.top_k,
+                      c.routed_scaling_factor, l->top_p, idx, w, scores, st);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "route launch");
 }
 
@@ -28,6 +28,14 @@ moe_status ffn_impl(const moe_layer* l, const uint16_t* x, int T, const int32_t*
       reinterpret_cast<float*>(ws + L.ypart), y, reinterpret_cast<uint32_t*>(ws + L.ctrl), st);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "expert launch");
 }
+
+#ifdef MOE_TRACE
+// Timeline buffer of a profiling build (-DMOE_TRACE): [grid][16] uint64.
+static uint64_t* g_trace = nullptr;
+extern "C" __attribute__((visibility("default"))) void moe_debug_set_trace(void* buf) {
+  g_trace = static_cast<uint64_t*>(buf);
+}
+#endif
 
 static moe_status launch_fused(const moe_layer* l, const uint16_t* x, const float* x_resid,
                                float norm_eps, uint16_t* xn_out, float* y, int32_t* idx_out,
@@ -51,14 +59,20 @@ static moe_status launch_fused(const moe_layer* l, const uint16_t* x, const floa
   p.scores = reinterpret_cast<uint64_t*>(ws + L.records);
   p.hbuf = reinterpret_cast<float*>(ws + L.hbuf);
   p.warm = 1;
-  p.ypart = reinterpret_cast<float*>(ws + L.ypart);
+#ifdef MOE_TRACE
+  p.trace = g_trace;
+#else
+  p.trace = nullptr;
+#endif
+  p.hq = ws + L.hq;
+  p.hqf = reinterpret_cast<float*>(ws + L.hqf);
   cudaError_t e = launch_decode(p, st);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "decode launch");
 }
 
 moe_status forward_impl(const moe_layer* l, const uint16_t* x, int T, float* y, int32_t* idx_out,
                         float* w_out, uint8_t* ws, const WsLayout& L, cudaStream_t st) {
-  if (T == 1) {
+  if (T == 1 && l->top_p >= 1.f) {
     bool used = false;
     moe_status s = launch_fused(l, x, nullptr, 0.f, nullptr, y, idx_out, w_out, ws, L, st, &used);
     if (used || s != MOE_OK) return s;
@@ -73,6 +87,8 @@ moe_status forward_impl(const moe_layer* l, const uint16_t* x, int T, float* y, 
 moe_status residual_impl(const moe_layer* l, const float* x_resid, float norm_eps, float* x_next,
                          uint16_t* xn_out, int32_t* idx_out, float* w_out, uint8_t* ws,
                          const WsLayout& L, cudaStream_t st) {
+  if (l->top_p < 1.f)
+    return fail(MOE_ERR_UNSUPPORTED, "the pre-norm step runs without adaptive top-p");
   bool used = false;
   moe_status s = launch_fused(l, nullptr, x_resid, norm_eps, xn_out, x_next, idx_out, w_out, ws,
                               L, st, &used);

@@ -11,47 +11,50 @@
 namespace moe {
 
 // ---------------------------------------------------------------------------
-// Router GEMV ("LightLX", "How it works": one router logit per routed
-// expert).  One CTA per expert row of W (fp32 [E][H]): each thread holds its
-// 16-byte chunks of the row and accumulates them against TT tokens at a
-// time; a block reduction gives the TT logits.  logits [T][E].
+// Router GEMV and sigmoid ("LightLX", "How it works": one router logit per
+// routed expert, sigmoid scores).  One CTA per expert row of W (fp32
+// [E][H]): each thread holds its 16-byte chunks of the row and accumulates
+// them against TT tokens at a time.  Every product of an fp32 weight and a
+// bf16 input is exact in fp64 and the sums are fp64, so the logit is exact
+// to about 1e-13; the sigmoid is taken in fp64 and rounded to fp32 once.
+// scores [T][E] = fp32(sigmoid(logit)).
 
 template <int TT>
-__global__ void __launch_bounds__(256) router_logits_kernel(
+__global__ void __launch_bounds__(256) router_scores_kernel(
     const float* __restrict__ w, const uint16_t* __restrict__ x, int T, int H,
-    int E, float* __restrict__ logits) {
-  __shared__ float red[TT][8];
+    int E, float* __restrict__ scores) {
+  __shared__ double red[TT][8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x;
   const float4* wr = reinterpret_cast<const float4*>(w + (size_t)e * H);
   const int nchunk = H >> 2;
   for (int t0 = 0; t0 < T; t0 += TT) {
-    float acc[TT];
+    double acc[TT];
 #pragma unroll
-    for (int t = 0; t < TT; ++t) acc[t] = 0.f;
+    for (int t = 0; t < TT; ++t) acc[t] = 0.0;
     for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
       const float4 wv = __ldg(wr + c);
 #pragma unroll
       for (int t = 0; t < TT; ++t) {
         if (t0 + t < T) {
           const uint2 xv = __ldg(reinterpret_cast<const uint2*>(x + (size_t)(t0 + t) * H) + c);
-          acc[t] = fmaf(wv.x, bf16_bits_to_f32(xv.x & 0xFFFFu), acc[t]);
-          acc[t] = fmaf(wv.y, bf16_bits_to_f32(xv.x >> 16), acc[t]);
-          acc[t] = fmaf(wv.z, bf16_bits_to_f32(xv.y & 0xFFFFu), acc[t]);
-          acc[t] = fmaf(wv.w, bf16_bits_to_f32(xv.y >> 16), acc[t]);
+          acc[t] = fma((double)wv.x, (double)bf16_bits_to_f32(xv.x & 0xFFFFu), acc[t]);
+          acc[t] = fma((double)wv.y, (double)bf16_bits_to_f32(xv.x >> 16), acc[t]);
+          acc[t] = fma((double)wv.z, (double)bf16_bits_to_f32(xv.y & 0xFFFFu), acc[t]);
+          acc[t] = fma((double)wv.w, (double)bf16_bits_to_f32(xv.y >> 16), acc[t]);
         }
       }
     }
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
-      const float s = warp_sum(acc[t]);
+      const double s = warp_sum_f64(acc[t]);
       if (lane == 0) red[t][warp] = s;
     }
     __syncthreads();
     if (threadIdx.x < TT && t0 + threadIdx.x < T) {
-      float s = 0.f;
+      double s = 0.0;
       for (int w8 = 0; w8 < (int)(blockDim.x >> 5); ++w8) s += red[threadIdx.x][w8];
-      logits[(size_t)(t0 + threadIdx.x) * E + e] = s;
+      scores[(size_t)(t0 + threadIdx.x) * E + e] = sigmoid_f64_to_f32(s);
     }
     __syncthreads();
   }
@@ -91,8 +94,8 @@ __device__ __forceinline__ ArgMax warp_argmax(ArgMax a) {
 }
 
 __global__ void __launch_bounds__(1024) select_kernel(
-    const float* __restrict__ logits, const float* __restrict__ bias, int E,
-    int n_group, int topk_group, int top_k, float rsf,
+    const float* __restrict__ scores, const float* __restrict__ bias, int E,
+    int n_group, int topk_group, int top_k, float rsf, float top_p,
     int32_t* __restrict__ idx_out, float* __restrict__ w_out,
     float* __restrict__ scores_out) {
   __shared__ float s_score[1024];
@@ -101,13 +104,13 @@ __global__ void __launch_bounds__(1024) select_kernel(
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per = E / n_group;
-  const float* lg = logits + (size_t)t * E;
+  const float* sc = scores + (size_t)t * E;
 
   if (warp < n_group) {
     const int e = warp * per + lane;
     ArgMax a{0.f, -1};
     if (lane < per) {
-      const float s = 1.0f / (1.0f + expf(-lg[e]));
+      const float s = sc[e];
       const float sp = s + bias[e];
       s_score[e] = s;
       s_sel[e] = sp;
@@ -150,17 +153,28 @@ __global__ void __launch_bounds__(1024) select_kernel(
     if (best.i >= 0 && (best.i & 31) == lane) taken |= 1u << (best.i >> 5);
     if (lane == r) my_sel = best.i;
   }
-  // rank of each selected id among the selected ids = output position
-  int rank = 0;
-  for (int j = 0; j < top_k; ++j) {
-    const int other = __shfl_sync(0xffffffffu, my_sel, j);
-    if (lane < top_k && other < my_sel) ++rank;
-  }
   const float s_mine = (lane < top_k && my_sel >= 0) ? s_score[my_sel] : 0.f;
   const float denom = warp_sum(s_mine) + 1e-20f;
-  if (lane < top_k) {
-    idx_out[(size_t)t * top_k + rank] = my_sel;
-    w_out[(size_t)t * top_k + rank] = rsf * s_mine / denom;
+  if (top_p >= 1.f) {
+    // rank of each selected id among the selected ids = output position
+    int rank = 0;
+    for (int j = 0; j < top_k; ++j) {
+      const int other = __shfl_sync(0xffffffffu, my_sel, j);
+      if (lane < top_k && other < my_sel) ++rank;
+    }
+    if (lane < top_k) {
+      idx_out[(size_t)t * top_k + rank] = my_sel;
+      w_out[(size_t)t * top_k + rank] = rsf * s_mine / denom;
+    }
+  } else {
+    // adaptive top-p: the kept picks, weights normalised over them
+    const bool kept = topp_keep(my_sel, s_mine, denom, top_k, top_p);
+    const float denom_k = warp_sum(kept ? s_mine : 0.f) + 1e-20f;
+    const int pos = topp_position(my_sel, kept, top_k);
+    if (lane < top_k) {
+      idx_out[(size_t)t * top_k + pos] = kept ? my_sel : -1;
+      w_out[(size_t)t * top_k + pos] = kept ? rsf * s_mine / denom_k : 0.f;
+    }
   }
 }
 
@@ -233,17 +247,17 @@ static int warps_for(int G) {
   return 4;
 }
 
-cudaError_t launch_router_logits(const float* w, const uint16_t* x, int T, int H, int E,
-                                 float* logits, cudaStream_t st) {
-  router_logits_kernel<8><<<E, 256, 0, st>>>(w, x, T, H, E, logits);
+cudaError_t launch_router_scores(const float* w, const uint16_t* x, int T, int H, int E,
+                                 float* scores, cudaStream_t st) {
+  router_scores_kernel<8><<<E, 256, 0, st>>>(w, x, T, H, E, scores);
   return cudaGetLastError();
 }
 
-cudaError_t launch_select(const float* logits, const float* bias, int T, int E, int n_group,
-                          int topk_group, int top_k, float rsf, int32_t* idx, float* w,
-                          float* scores, cudaStream_t st) {
-  select_kernel<<<T, 32 * n_group, 0, st>>>(logits, bias, E, n_group, topk_group, top_k, rsf,
-                                            idx, w, scores);
+cudaError_t launch_select(const float* scores, const float* bias, int T, int E, int n_group,
+                          int topk_group, int top_k, float rsf, float top_p, int32_t* idx,
+                          float* w, float* scores_out, cudaStream_t st) {
+  select_kernel<<<T, 32 * n_group, 0, st>>>(scores, bias, E, n_group, topk_group, top_k, rsf,
+                                            top_p, idx, w, scores_out);
   return cudaGetLastError();
 }
 

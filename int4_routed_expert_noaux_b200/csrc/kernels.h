@@ -9,11 +9,15 @@
 
 namespace moe {
 
-cudaError_t launch_router_logits(const float* w, const uint16_t* x, int T, int H, int E,
-                                 float* logits, cudaStream_t st);
-cudaError_t launch_select(const float* logits, const float* bias, int T, int E, int n_group,
-                          int topk_group, int top_k, float rsf, int32_t* idx, float* w,
-                          float* scores, cudaStream_t st);
+// scores [T][E] = fp32(sigmoid(W x)), the logit summed in fp64.
+cudaError_t launch_router_scores(const float* w, const uint16_t* x, int T, int H, int E,
+                                 float* scores, cudaStream_t st);
+// noaux_tc selection from the sigmoid scores, then adaptive top-p when
+// top_p < 1 (dropped slots: id -1, weight 0, after the kept ids);
+// scores_out (nullable) gets a copy of the scores.
+cudaError_t launch_select(const float* scores, const float* bias, int T, int E, int n_group,
+                          int topk_group, int top_k, float rsf, float top_p, int32_t* idx,
+                          float* w, float* scores_out, cudaStream_t st);
 // The batched expert path (union.cu): distinct experts read once for all
 // their tokens.  Scratch: xq (T * H/32 groups), hq (T * slots * I/32 groups),
 // lists (union_lists_ints ints), hbuf (T * slots * I), ypart (T * slots * H).

@@ -17,6 +17,7 @@ struct moe_layer {
   moe::ExpertPtrs* table = nullptr;  // device [E + 1]; entry E = shared
   moe::ExpertPtrs* host_table = nullptr;
   int device = 0;
+  float top_p = 1.0f;                // adaptive expert top-p (>= 1: off)
 };
 
 namespace moe {

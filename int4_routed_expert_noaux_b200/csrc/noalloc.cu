@@ -3,9 +3,7 @@
 // nothing: no cudaMalloc, no cudaFree, no library call that allocates.
 #include <cuda_runtime.h>
 
-#include <atomic>
-#include <mutex>
-
+#include "device_once.h"
 #include "layer.h"
 
 namespace moe {
@@ -14,34 +12,30 @@ namespace moe {
 // ws_layout(cfg, 1).total.  A 6144 x 2048 layer with top-8 of 256 experts
 // and one shared expert needs 357,120 bytes.
 constexpr size_t kStaticScratchBytes = 512u << 10;
-constexpr int kStaticMaxDevices = 64;
 // control words plus the router score records that follow them (8 bytes per
 // expert; the fused kernel, their only user, takes at most 256 experts)
 constexpr size_t kStaticClearBytes = kCtrlBytes + 256 * 8;
 
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
-static std::atomic<uint8_t*> g_scratch_addr[kStaticMaxDevices];
-static std::mutex g_scratch_mu;
+static DeviceOnce<uint8_t*> g_scratch_addr;
 
-// Address of g_static_scratch on `dev` (the current device), resolved once;
-// the first resolution also zero-fills the control words and the router
-// score records on `st` (the array starts zeroed at module load as well).
+// Address of g_static_scratch on `dev` (the current device), resolved once
+// per device and context; the first resolution also zero-fills the control
+// words and the router score records on `st` (the array starts zeroed at
+// module load as well).
 static moe_status scratch_address(int dev, cudaStream_t st, uint8_t** out) {
-  uint8_t* a = g_scratch_addr[dev].load(std::memory_order_acquire);
-  if (!a) {
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    a = g_scratch_addr[dev].load(std::memory_order_relaxed);
-    if (!a) {
-      void* sym = nullptr;
-      cudaError_t e = cudaGetSymbolAddress(&sym, g_static_scratch);
-      if (e != cudaSuccess) return cuda_fail(e, "scratch symbol address");
-      a = static_cast<uint8_t*>(sym);
-      e = cudaMemsetAsync(a, 0, kStaticClearBytes, st);
-      if (e != cudaSuccess) return cuda_fail(e, "scratch clear");
-      g_scratch_addr[dev].store(a, std::memory_order_release);
-    }
-  }
+  uint8_t* a = nullptr;
+  const cudaError_t e = g_scratch_addr.get(dev, &a, [st](uint8_t** v) {
+    void* sym = nullptr;
+    cudaError_t r = cudaGetSymbolAddress(&sym, g_static_scratch);
+    if (r != cudaSuccess) return r;
+    r = cudaMemsetAsync(sym, 0, kStaticClearBytes, st);
+    if (r != cudaSuccess) return r;
+    *v = static_cast<uint8_t*>(sym);
+    return cudaSuccess;
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "scratch symbol address");
   *out = a;
   return MOE_OK;
 }
@@ -74,8 +68,8 @@ moe_status moe_layer_forward_noalloc(const moe_layer* l, const void* x, float* y
   if (dev != l->device)
     return fail(MOE_ERR_INVALID_ARG, "current device %d is not the layer's device %d", dev,
                 l->device);
-  if (dev < 0 || dev >= kStaticMaxDevices)
-    return fail(MOE_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kStaticMaxDevices);
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail(MOE_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
   cudaStream_t st = (cudaStream_t)stream;
   uint8_t* ws = nullptr;
   if ((s = scratch_address(dev, st, &ws)) != MOE_OK) return s;

@@ -22,6 +22,7 @@
 
 #include "async.cuh"
 #include "common.cuh"
+#include "device_once.h"
 #include "kernels.h"
 
 namespace moe {
@@ -98,7 +99,7 @@ __global__ void __launch_bounds__(256) build_lists_kernel(const int32_t* __restr
     const int e = idx[i];
     if (e >= 0 && e < E) {
       atomicAdd(&cnt[e], 1);
-    } else {
+    } else if (e != -1) {  // -1: a slot dropped by top-p
       atomicCAS(err, 0u, (uint32_t)kErrBadExpertId);
     }
   }
@@ -436,19 +437,22 @@ cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const 
   a.R = I;
   a.in_is_pos = 0;
   a.out = hbuf;
-  static bool configured[64] = {false};
+  static DeviceOnce<bool> configured;
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    cudaError_t ce = cudaFuncSetAttribute(union_gemm_kernel<2>,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)union_smem_bytes(2));
-    if (ce == cudaSuccess)
-      ce = cudaFuncSetAttribute(union_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)union_smem_bytes(1));
-    if (ce != cudaSuccess) return ce;
-    configured[dev] = true;
-  }
+  cudaError_t ce = cudaGetDevice(&dev);
+  if (ce != cudaSuccess) return ce;
+  bool done = false;
+  ce = configured.get(dev, &done, [](bool* v) {
+    cudaError_t r = cudaFuncSetAttribute(union_gemm_kernel<2>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)union_smem_bytes(2));
+    if (r == cudaSuccess)
+      r = cudaFuncSetAttribute(union_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)union_smem_bytes(1));
+    *v = r == cudaSuccess;
+    return r;
+  });
+  if (ce != cudaSuccess) return ce;
   union_gemm_kernel<2><<<dim3((I + 31) / 32, umax), kUnionThreads, union_smem_bytes(2), st>>>(a);
   xq_table_kernel<false><<<(n_list * GD + 255) / 256, 256, 0, st>>>(hbuf, n_list, I, hq_words,
                                                                     hq_fac);

@@ -96,3 +96,15 @@ def test_lru_replay_rejects_bad_traces():
         moe.lru_replay(tr, 8, 2)
     with pytest.raises(moe.MoeError):
         moe.lru_replay(np.array([[[0, 1]]], dtype=np.int32), 8, 1)  # capacity < k
+
+
+def test_fault_injection_arguments():
+    # the injection switch is host-only: arming, disarming and bad kinds
+    # need no GPU
+    with pytest.raises(moe.MoeError) as ei:
+        moe.inject_fault(9, 0)
+    assert ei.value.status == 1
+    with pytest.raises(moe.MoeError):
+        moe.inject_fault(moe.FAULT_CACHE_COPY, -1)
+    moe.inject_fault(moe.FAULT_CACHE_COPY, 2)
+    moe.inject_fault(moe.FAULT_NONE, 0)

@@ -1,12 +1,17 @@
 """GPU parity of the hot path against the fp64 oracle, through the C ABI.
 
 Bars: expert ids bit-exact (ties to the lower index); weights within fp32
-rounding; outputs max |dy| <= 2e-3 * rms(y_oracle) per token.  Routing
-decisions are also checked in the kernel's own precision: the oracle's
-selection applied to the GPU's fp32 scores must give the GPU's ids for every
-token.  Tokens whose fp64 decision margin is below FLAG_MARGIN are reported
-and checked that way only (fp32 logits carry errors of order 1e-6 to 1e-5,
-so a smaller gap may legitimately flip)."""
+rounding; outputs max |dy| <= 2e-3 * rms(y_oracle) per token.
+
+The kernels sum the router logits in fp64 (every fp32 x bf16 product is
+exact in fp64) and round the sigmoid score to fp32 once, so a score differs
+from the oracle's by at most 2^-25 of itself, and a decision gap (k-th vs
+(k+1)-th bias-corrected score, or topk_group-th vs next group score) moves
+by less than 5e-7 between the two.  A token whose fp64 decision margin is
+at most FLAG_MARGIN = 1e-6 is flagged: its ids are checked against the
+oracle's selection run on the GPU's own fp32 scores (the kernel's precision)
+instead of the fp64 one.  Every other token must match the fp64 oracle bit
+for bit.  Each test prints its flagged count and bounds it."""
 import numpy as np
 import pytest
 
@@ -21,8 +26,21 @@ pytestmark = pytest.mark.gpu
 
 MEDIUM = synth.Shape(hidden=3072, inter=1024, n_experts=36, n_shared=1, top_k=5, n_group=4,
                      topk_group=2)
-FLAG_MARGIN = 1e-5
+FLAG_MARGIN = 1e-6
 Y_TOL = 2e-3
+SCORE_TOL = 1e-7     # fp32 rounding of an exact sigmoid: at most 2^-25 * s
+
+
+def flag_bound(n):
+    """Most flagged tokens allowed among n: a decision gap below 1e-6 comes
+    up in well under 0.5 % of tokens at these distributions, so more means
+    the margins themselves are wrong."""
+    return 2 + n // 200
+
+
+def report_flagged(what, flagged, n):
+    print(f"[parity] {what}: {flagged} of {n} tokens flagged (fp64 margin <= {FLAG_MARGIN:g})")
+    assert flagged <= flag_bound(n), (what, flagged, n)
 
 
 def needs_gpu():
@@ -79,8 +97,8 @@ def check_route(shape, dl, x_bits, gidx, gw, gsc):
     W, b = dl.host_router()
     lg = oracle.router_logits(shape, W, x_bits)
     oidx, ow, margin, osc = oracle.route(shape, lg, b)
-    # (a) sigmoid scores
-    assert np.max(np.abs(gsc.astype(np.float64) - osc)) <= 1e-5
+    # (a) sigmoid scores: the exact score rounded to fp32
+    assert np.max(np.abs(gsc.astype(np.float64) - osc)) <= SCORE_TOL
     # (b) the decision in the kernel's precision: oracle selection on the
     # GPU's fp32 scores and fp32 bias-corrected scores
     sp32 = (gsc + b[None, :]).astype(np.float32)
@@ -91,7 +109,7 @@ def check_route(shape, dl, x_bits, gidx, gw, gsc):
     # (c) bit-exact against the fp64 oracle where the decision is not a near tie
     ok = margin > FLAG_MARGIN
     assert np.array_equal(gidx[ok], oidx[ok])
-    assert np.allclose(gw[ok], ow[ok], rtol=2e-5, atol=1e-6)
+    assert np.allclose(gw[ok], ow[ok], rtol=2e-6, atol=1e-7)
     # invariants
     per = shape.n_experts // shape.n_group
     for t in range(gidx.shape[0]):
@@ -107,7 +125,7 @@ def test_route_parity(shape, T):
     dl, L = get_layer(shape)
     x_bits = synth.tokens(shape, 0, 100, T)
     gidx, gw, gsc = run_route(shape, L, x_bits)
-    check_route(shape, dl, x_bits, gidx, gw, gsc)
+    report_flagged(f"route {shape.n_experts}x{T}", check_route(shape, dl, x_bits, gidx, gw, gsc), T)
 
 
 @pytest.mark.parametrize("shape,T", [(synth.TINY, 4), (MEDIUM, 3), (synth.GLM, 2)],
@@ -140,17 +158,37 @@ def run_forward(shape, L, x_bits):
     return y.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy()
 
 
-def check_forward(shape, dl, x_bits, y, gidx, gw):
+def kernel_precision_ids(shape, b, osc):
+    """The selection as the kernels make it: the exact sigmoid scores
+    rounded to fp32, the bias added in fp32, group sums in fp32."""
+    s32 = osc.astype(np.float32)
+    sp32 = (s32 + b[None, :].astype(np.float32)).astype(np.float32)
+    didx, _, _ = oracle.select_scores(shape, s32.astype(np.float64), sp32.astype(np.float64),
+                                      round_group_f32=True)
+    return didx
+
+
+def check_forward(shape, dl, x_bits, y, gidx, gw, what=None):
+    """ids bit-exact against the fp64 oracle except flagged near-ties, whose
+    ids must equal the kernel-precision selection; weights; outputs against
+    the oracle's routes where they agree and against the oracle FFN on the
+    GPU's routes everywhere.  Returns the flagged count."""
     W, b = dl.host_router()
     lg = oracle.router_logits(shape, W, x_bits)
-    oidx, ow, margin, _ = oracle.route(shape, lg, b)
+    oidx, ow, margin, osc = oracle.route(shape, lg, b)
+    flagged = margin <= FLAG_MARGIN
     same = np.all(gidx == oidx, axis=1)
-    assert np.all(same | (margin <= FLAG_MARGIN))
-    # outputs: against the oracle's own routes where they agree, and against
-    # the oracle FFN on the GPU's routes everywhere
+    assert np.all(same | flagged)
+    if flagged.any():
+        didx = kernel_precision_ids(shape, b, osc)
+        assert np.array_equal(gidx[flagged], didx[flagged])
+    assert np.allclose(gw[same], ow[same], rtol=2e-6, atol=1e-7)
     if same.any():
         assert_y_close(y[same], oracle_y(shape, dl, x_bits[same], oidx[same], ow[same]))
     assert_y_close(y, oracle_y(shape, dl, x_bits, gidx, gw))
+    n_flag = int(flagged.sum())
+    report_flagged(what or f"forward {shape.n_experts}x{x_bits.shape[0]}", n_flag, x_bits.shape[0])
+    return n_flag
 
 
 @pytest.mark.parametrize("shape,T,first", [(synth.TINY, 1, 0), (synth.TINY, 1, 1),
