@@ -62,6 +62,8 @@ def parse():
                    help="stream: layers in pinned host memory (capped by free host RAM)")
     p.add_argument("--stream-caps", default="8,16,32,64,128", help="stream: cache slots per layer")
     p.add_argument("--stream-tokens", type=int, default=512)
+    p.add_argument("--top-p", type=float, default=1.0,
+                   help="adaptive expert top-p of every layer (>= 1: off, the headline)")
     return p.parse_args()
 
 
@@ -73,10 +75,13 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def algorithmic_bytes_per_token(shape):
-    """9 experts (8 routed + shared) + fp32 router + bias + bf16 x + fp32 y."""
+def algorithmic_bytes_per_token(shape, routed=None):
+    """routed experts (top_k, or the mean kept by top-p) + the shared one +
+    fp32 router + bias + bf16 x + fp32 y (9 experts: 197,432,320 B for the
+    GLM layer)."""
     E, H = shape.n_experts, shape.hidden
-    return ((shape.top_k + shape.n_shared) * shape.expert_bytes + E * H * 4 + E * 4 + H * 2 + H * 4)
+    r = shape.top_k if routed is None else routed
+    return int(round((r + shape.n_shared) * shape.expert_bytes + E * H * 4 + E * 4 + H * 2 + H * 4))
 
 
 DECODE_SOURCES = ("decode.cu", "decode.h", "common.cuh", "async.cuh", "forward.cu")
@@ -210,6 +215,7 @@ def config_dict(args, shape, tokens):
             "n_shared": shape.n_shared, "top_k": shape.top_k, "n_group": shape.n_group,
             "topk_group": shape.topk_group, "rsf": shape.rsf, "tokens_per_step": tokens,
             "batch": 1, "layer_copies": args.copies,
+            "top_p": getattr(args, "top_p", 1.0) if getattr(args, "top_p", 1.0) < 1.0 else None,
             "l2": "inputs larger than L2 (197 MB per token; copies rotate)",
             "parallelism": f"replicas x{args.gpus}"}
 
@@ -253,18 +259,21 @@ def main():
         dl = DeviceLayer(shape, 0, c)
         layers.append(dl)
         views.append(moe.Layer(cfg, dl.w_router, dl.bias, dl.routed, dl.shared))
+        if args.top_p < 1.0:
+            views[-1].set_top_p(args.top_p)
     torch.cuda.synchronize()
 
     n = args.tokens
     x_bits = synth.tokens(shape, 1000 * rank, 0, n)
     x = torch.from_numpy(x_bits.view(np.int16)).cuda()
     y = torch.empty((n, shape.hidden), dtype=torch.float32, device="cuda")
+    idx = torch.empty((n, shape.top_k), dtype=torch.int32, device="cuda")
     ws = moe.alloc_workspace(cfg, 1)
     stream = torch.cuda.Stream()
 
     def step(s):
         for t in range(n):
-            views[t % copies].forward(x[t:t + 1], y[t:t + 1], ws, stream=s)
+            views[t % copies].forward(x[t:t + 1], y[t:t + 1], ws, idx=idx[t:t + 1], stream=s)
 
     with torch.cuda.stream(stream):
         step(stream)
@@ -345,7 +354,9 @@ def main():
         raise RuntimeError("non-finite outputs")
 
     peak, peak_kind = peaks()
-    bytes_tok = algorithmic_bytes_per_token(shape)
+    # experts read per token: top_k, or those adaptive top-p keeps
+    kept = float((idx >= 0).sum(dim=1).float().mean().item())
+    bytes_tok = algorithmic_bytes_per_token(shape, kept)
     launch_us = ms_step * 1000.0 / n
     achieved = bytes_tok / (launch_us * 1e-6) / 1e9
     kernel = "moe_layer_forward (per token)"
@@ -375,6 +386,7 @@ def main():
                     "h2d_bytes_per_step": n * shape.hidden * 2,
                     "d2h_bytes_per_step": n * shape.hidden * 4},
             "gpu_launches": n * args.steps * launches_per_forward(),
+            "routed_experts_per_token": kept,
             "clocks": clk, "graph": graph is not None or not args.no_graph,
             "hbm_gbs": achieved,
         }

@@ -120,10 +120,10 @@ moe_status moe_layer_set_expert(moe_layer* layer, int e,
  * weights add up to at least p * routed_scaling_factor, and normalise the
  * kept weights again over the kept experts.  Routes then carry the kept ids
  * ascending followed by -1 (weight 0) for each dropped slot; -1 entries are
- * skipped by moe_expert_ffn.  p >= 1 turns it off (the default); p must be
- * > 0.  With top-p on, one-token calls take the batched path, and
- * moe_layer_forward_residual / moe_stack_forward return
- * MOE_ERR_UNSUPPORTED.  Not thread-safe against calls on the same layer. */
+ * skipped by moe_expert_ffn, and a dropped expert's bytes are not read.
+ * p >= 1 turns it off (the default); p must be > 0.  Applies to every call
+ * that routes (moe_route, moe_layer_forward, the residual and stack calls).
+ * Not thread-safe against calls on the same layer. */
 moe_status moe_layer_set_top_p(moe_layer* layer, float p);
 
 /* ---- workspace --------------------------------------------------------- */

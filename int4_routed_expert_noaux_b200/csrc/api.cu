@@ -142,6 +142,22 @@ moe_status check_ws(const moe_layer* l, int T, void* ws, size_t ws_bytes, WsLayo
   return MOE_OK;
 }
 
+static moe_status check_residual_args(const moe_layer* l, const float* x_dev,
+                                      const float* x_next_dev, const uint16_t* xn_out_dev,
+                                      const int32_t* idx_out_dev, const float* w_out_dev,
+                                      float norm_eps) {
+  if (!l) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+  moe_status s;
+  if ((s = check_device_ptr(x_dev, 16, "x")) != MOE_OK) return s;
+  if ((s = check_device_ptr(x_next_dev, 16, "x_next")) != MOE_OK) return s;
+  if (x_dev == x_next_dev) return fail(MOE_ERR_INVALID_ARG, "x and x_next must not alias");
+  if (xn_out_dev && (s = check_device_ptr(xn_out_dev, 4, "xn_out")) != MOE_OK) return s;
+  if (idx_out_dev && (s = check_device_ptr(idx_out_dev, 4, "idx_out")) != MOE_OK) return s;
+  if (w_out_dev && (s = check_device_ptr(w_out_dev, 4, "w_out")) != MOE_OK) return s;
+  if (!(norm_eps >= 0.f)) return fail(MOE_ERR_INVALID_ARG, "norm_eps must be >= 0");
+  return MOE_OK;
+}
+
 static moe_status check_call(const moe_layer* l, const void* x, int T) {
   if (!l) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
   if (T < 1 || T > kMaxTokens) return fail(MOE_ERR_INVALID_ARG, "T = %d outside 1..%d", T, kMaxTokens);
@@ -309,15 +325,9 @@ moe_status moe_layer_forward_residual(const moe_layer* l, const float* x_dev, fl
                                       float* w_out_dev, float norm_eps, void* ws, size_t ws_bytes,
                                       void* stream) {
   g_last_error[0] = 0;
-  if (!l) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
-  moe_status s;
-  if ((s = check_device_ptr(x_dev, 16, "x")) != MOE_OK) return s;
-  if ((s = check_device_ptr(x_next_dev, 16, "x_next")) != MOE_OK) return s;
-  if (x_dev == x_next_dev) return fail(MOE_ERR_INVALID_ARG, "x and x_next must not alias");
-  if (xn_out_dev && (s = check_device_ptr(xn_out_dev, 4, "xn_out")) != MOE_OK) return s;
-  if (idx_out_dev && (s = check_device_ptr(idx_out_dev, 4, "idx_out")) != MOE_OK) return s;
-  if (w_out_dev && (s = check_device_ptr(w_out_dev, 4, "w_out")) != MOE_OK) return s;
-  if (!(norm_eps >= 0.f)) return fail(MOE_ERR_INVALID_ARG, "norm_eps must be >= 0");
+  moe_status s = check_residual_args(l, x_dev, x_next_dev, xn_out_dev, idx_out_dev, w_out_dev,
+                                     norm_eps);
+  if (s != MOE_OK) return s;
   WsLayout L;
   if ((s = check_ws(l, 1, ws, ws_bytes, &L)) != MOE_OK) return s;
   return residual_impl(l, x_dev, norm_eps, x_next_dev, xn_out_dev, idx_out_dev, w_out_dev,
@@ -346,8 +356,12 @@ moe_status moe_stack_forward(const moe_layer* const* layers, int n_layers, const
     float* nxt = ((n_layers - 1 - l) % 2 == 0) ? x_out_dev : x_tmp_dev;
     if (last) nxt = x_out_dev;
     int32_t* idx = idx_out_dev ? idx_out_dev + (size_t)l * c0.top_k : nullptr;
-    moe_status s = moe_layer_forward_residual(layers[l], cur, nxt, nullptr, idx, nullptr, norm_eps,
-                                              ws, ws_bytes, stream);
+    moe_status s = check_residual_args(layers[l], cur, nxt, nullptr, idx, nullptr, norm_eps);
+    WsLayout L;
+    if (s == MOE_OK) s = check_ws(layers[l], 1, ws, ws_bytes, &L);
+    if (s != MOE_OK) return s;
+    s = residual_impl(layers[l], cur, norm_eps, nxt, nullptr, idx, nullptr, (uint8_t*)ws, L,
+                      (cudaStream_t)stream, last ? nullptr : layers[l + 1]);
     if (s != MOE_OK) return s;
     cur = nxt;
   }

@@ -50,16 +50,24 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity`, giving up at `deadline` (globaltimer ns).
-// Returns false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t deadline) {
+// Wait for phase `parity`; false if it has not completed timeout_ns after
+// the first unsuccessful probe.  The first probes follow one another at
+// once (try_wait itself suspends the thread briefly in hardware), so a
+// short wait -- the next stage landing -- ends with no added latency; a long
+// one then backs off with nanosleep so the waiting warps leave the issue
+// slots to the warps on the critical path.  The timer is read only once the
+// phase was found incomplete, then every 8 probes.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
   if (mbar_test(bar, parity)) return true;
-  uint32_t sleep_ns = 32;  // deschedule between probes: waiting warps take no issue slots
-  for (uint32_t it = 0;; ++it) {
-    __nanosleep(sleep_ns);
+  const uint64_t deadline = global_timer_ns() + timeout_ns;
+  uint32_t sleep_ns = 0;
+  for (uint32_t it = 1;; ++it) {
     if (mbar_test(bar, parity)) return true;
-    if (sleep_ns < 256) sleep_ns <<= 1;
-    if ((it & 7) == 7 && global_timer_ns() > deadline) return false;
+    if (it >= 8) {
+      sleep_ns = sleep_ns ? min(sleep_ns * 2, 256u) : 32u;
+      __nanosleep(sleep_ns);
+    }
+    if ((it & 7) == 0 && global_timer_ns() > deadline) return false;
   }
 }
 
@@ -72,6 +80,14 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "[%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst)),
       "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
       : "memory");
+}
+
+// Bulk prefetch of global memory into L2 (no shared-memory destination).
+// src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes, uint64_t policy) {
+  asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(src),
+               "r"(bytes), "l"(policy)
+               : "memory");
 }
 
 // L2 policy: evict-first (weights are streamed once per call).

@@ -247,11 +247,12 @@ __device__ __forceinline__ bool topp_keep(int id, float s, float denom, int k, f
 // dropped picks after them in lane order.
 __device__ __forceinline__ int topp_position(int id, bool kept, int k) {
   const int lane = threadIdx.x & 31;
+  const unsigned km = __ballot_sync(0xffffffffu, kept);
   int pos = 0;
-#pragma unroll 4
+#pragma unroll
   for (int j = 0; j < 32; ++j) {
     const int ij = __shfl_sync(0xffffffffu, id, j);
-    const bool kj = __shfl_sync(0xffffffffu, kept ? 1 : 0, j) != 0;
+    const bool kj = (km >> j) & 1u;
     if (j < k) pos += kept ? (kj && ij < id) : (kj || j < lane);
   }
   return pos;

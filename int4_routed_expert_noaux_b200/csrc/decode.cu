@@ -54,12 +54,16 @@
 #include "decode.h"
 #include "device_once.h"
 
-// Timeline probes: compiled in only with -DMOE_TRACE (a profiling build);
-// slot i of CTA b gets the globaltimer at probe i.
+// Timeline probes: compiled in only with -DMOE_TRACE (a profiling build).
+// Slot i < 16 of CTA b gets the SM cycle counter at probe i; slot 16 the
+// globaltimer (ns) when the CTA starts, to line the CTAs up.
 #ifdef MOE_TRACE
-#define TRACE_AT(i)                                                       \
-  do {                                                                    \
-    if (p.trace) p.trace[blockIdx.x * 16 + (i)] = moe::global_timer_ns(); \
+#define TRACE_AT(i)                                                                          \
+  do {                                                                                       \
+    if (p.trace) {                                                                           \
+      p.trace[blockIdx.x * 32 + (i)] = (uint64_t)clock64();                                  \
+      if ((i) == 0) p.trace[blockIdx.x * 32 + 16] = moe::global_timer_ns();                  \
+    }                                                                                        \
   } while (0)
 #else
 #define TRACE_AT(i) ((void)0)
@@ -98,6 +102,8 @@ struct Smem {
   uint64_t selbar;         // the selection warp has published sel_*
   ItemDesc desc[kStages];
   int sel_idx[kMaxSlots];  // selected expert ids, ascending
+  int pick_id[kMaxSlots];  // the selection's picks in pick order
+  float pick_s[kMaxSlots];
   float sel_w[kMaxSlots];  // their combine weights
   int sel_ok;
   float red[kGroups][2][kGW][32];
@@ -116,7 +122,7 @@ struct Smem {
 // whose loads miss L1 and wait on L2 while the weights stream.
 struct SelArgs {
   int E, k, n_group, topk_group, sel_q, sel_lgL, sel_fast;
-  float rsf;
+  float rsf, top_p;
   int32_t* idx_out;  // written by CTA 0 only (nullable)
   float* w_out;
 };
@@ -131,6 +137,7 @@ __device__ __forceinline__ SelArgs sel_args(const DecodeParams& p) {
   a.sel_lgL = p.sel_lgL;
   a.sel_fast = p.sel_fast;
   a.rsf = p.rsf;
+  a.top_p = p.top_p;
   a.idx_out = p.idx_out;
   a.w_out = p.w_out;
   return a;
@@ -196,6 +203,28 @@ __device__ __forceinline__ void router_rows(const DecodeParams& p, int b, int& r
   nr = (int)(((long long)(b + 1) * p.E) / p.nR) - r0;
 }
 
+// At the start of this CTA's down phase (a stack's next layer known): its
+// router rows of the next layer and shared-expert gate/up items b, b + grid,
+// ... of the next layer go to L2 with an evict-last hint, so that the next
+// layer's dependent start-up reads them from L2 instead of HBM.
+__device__ __forceinline__ void prefetch_next_layer(const DecodeParams& p) {
+  const uint64_t keep = l2_policy_evict_last();
+  int r0, nr;
+  router_rows(p, blockIdx.x, r0, nr);
+  if (nr > 0) bulk_prefetch_l2(p.pf_w_router + (size_t)r0 * p.H, (uint32_t)nr * p.H * 4, keep);
+  if (!p.has_shared) return;
+  for (int t = blockIdx.x; t < p.nG; t += gridDim.x) {
+    const int row0 = t * p.RG, nrows = min(p.RG, p.I - row0);
+    const uint32_t qb = (uint32_t)nrows * (p.H / 2), sb = (uint32_t)nrows * (p.H / 16);
+    const size_t qoff = (size_t)row0 * (p.H / 2), soff = (size_t)row0 * (p.H / 32);
+    bulk_prefetch_l2(p.pf_shared.q_gate + qoff, qb, keep);
+    bulk_prefetch_l2(p.pf_shared.q_up + qoff, qb, keep);
+    bulk_prefetch_l2(p.pf_shared.s_gate + soff, sb, keep);
+    bulk_prefetch_l2(p.pf_shared.s_up + soff, sb, keep);
+  }
+}
+
+
 // Record an error: the first one also records where it happened (CTA,
 // warp, site, fill) in the control words kCtrlWhere..kCtrlWhere+3.
 __device__ __forceinline__ void set_error(uint32_t* ctrl, uint32_t code, uint32_t site = 0,
@@ -249,6 +278,34 @@ __device__ __forceinline__ ArgMaxF am_warp(ArgMaxF a) {
     a = am_merge(a, b);
   }
   return a;
+}
+
+// The end of a selection: lane r < k holds the r-th pick (id, unbiased
+// score s).  Weights rsf * s / sum s ("LightLX", "How it works": normalised
+// sigmoid weights; colibri summary: routed_scaling_factor); with adaptive
+// top-p, the kept picks and their weights normalised over them, dropped
+// slots -1 / 0 after the kept ids.  Ids ascending to S.sel_idx / S.sel_w
+// (and, from CTA 0, to idx_out / w_out).
+__device__ __forceinline__ void publish_selection(const SelArgs& p, Smem& S, int my_sel,
+                                                  float my_s) {
+  const int lane = threadIdx.x & 31;
+  float denom = warp_sum(my_s) + 1e-20f;
+  bool kept = lane < p.k;
+  if (p.top_p < 1.f) {
+    kept = topp_keep(my_sel, my_s, denom, p.k, p.top_p);
+    denom = warp_sum(kept ? my_s : 0.f) + 1e-20f;
+  }
+  const int pos = topp_position(my_sel, kept, p.k);
+  if (lane < p.k) {
+    const int id = kept ? my_sel : -1;
+    const float wv = kept ? p.rsf * my_s / denom : 0.f;
+    S.sel_idx[pos] = id;
+    S.sel_w[pos] = wv;
+    if (blockIdx.x == 0) {
+      if (p.idx_out) p.idx_out[pos] = id;
+      if (p.w_out) p.w_out[pos] = wv;
+    }
+  }
 }
 
 // Selection for shapes whose groups do not align with lanes: one lane per
@@ -305,25 +362,8 @@ __device__ __noinline__ void run_select_generic(const SelArgs p, Smem& S) {
       }
     }
   }
-  int pos = 0;
-  for (int j = 0; j < p.k; ++j) {
-    const int other = __shfl_sync(0xffffffffu, my_sel, j);
-    if (lane < p.k && other < my_sel) ++pos;
-  }
   const float s_mine = (lane < p.k && my_sel >= 0) ? S.sc[my_sel] : 0.f;
-  float denom = s_mine;
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, o);
-  denom += 1e-20f;
-  if (lane < p.k) {
-    const float wv = p.rsf * s_mine / denom;
-    S.sel_idx[pos] = my_sel;
-    S.sel_w[pos] = wv;
-    if (blockIdx.x == 0) {
-      if (p.idx_out) p.idx_out[pos] = my_sel;
-      if (p.w_out) p.w_out[pos] = wv;
-    }
-  }
+  publish_selection(p, S, my_sel, s_mine);
 }
 
 // Four consecutive inputs of a residual (pre-norm) step, i0 % 4 == 0, as
@@ -435,19 +475,25 @@ __device__ __noinline__ void run_select(const SelArgs p, Smem& S) {
   cx(key, jid, sl, 0, 4); cx(key, jid, sl, 1, 5); cx(key, jid, sl, 2, 6); cx(key, jid, sl, 3, 7);
   cx(key, jid, sl, 2, 4); cx(key, jid, sl, 3, 5);
   cx(key, jid, sl, 1, 2); cx(key, jid, sl, 3, 4); cx(key, jid, sl, 5, 6);
-  // top_k: the best head, lowest expert id among equal heads, is popped;
-  // lane r keeps the r-th pick (lanes past k keep INT_MAX for the ordering)
-  int my_sel = 0x7FFFFFFF;
-  float my_s = 0.f;
+  // top_k: the best head is popped, k times; among equal heads (a rare,
+  // warp-uniform case) the lowest expert id.  The owner of the r-th pick
+  // leaves it in shared memory, off the dependent chain of the rounds.
+  if (lane < p.k) {
+    S.pick_id[lane] = -1;  // no candidate left (not reachable for a valid shape)
+    S.pick_s[lane] = 0.f;
+  }
+  __syncwarp();
   for (int r = 0; r < p.k; ++r) {
     const uint32_t m = __reduce_max_sync(0xffffffffu, key[0]);
-    const uint32_t cand = (key[0] == m && m != 0u) ? (uint32_t)(lane * q + jid[0]) : 0xFFFFFFFFu;
-    const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
-    const bool own = cand == win && m != 0u;
-    const int owner = __ffs(__ballot_sync(0xffffffffu, own)) - 1;
-    const float s_win = __shfl_sync(0xffffffffu, sl[0], owner & 31);
-    my_sel = (lane == r) ? (int)win : my_sel;  // no candidate left: -1
-    my_s = (lane == r) ? s_win : my_s;
+    bool own = key[0] == m && m != 0u;
+    if (__popc(__ballot_sync(0xffffffffu, own)) > 1) {
+      const uint32_t cand = own ? (uint32_t)(lane * q + jid[0]) : 0xFFFFFFFFu;
+      own = cand == __reduce_min_sync(0xffffffffu, cand);
+    }
+    if (own) {
+      S.pick_id[r] = lane * q + jid[0];
+      S.pick_s[r] = sl[0];
+    }
 #pragma unroll
     for (int j = 0; j + 1 < kQ; ++j) {  // pop the owner's head
       key[j] = own ? key[j + 1] : key[j];
@@ -456,26 +502,11 @@ __device__ __noinline__ void run_select(const SelArgs p, Smem& S) {
     }
     key[kQ - 1] = own ? 0u : key[kQ - 1];
   }
-  // ascending ids; weights from the unbiased scores
-  int pos = 0;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const int other = __shfl_sync(0xffffffffu, my_sel, j);
-    pos += (other < my_sel) ? 1 : 0;
-  }
-  float denom = (lane < p.k) ? my_s : 0.f;
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, o);
-  denom += 1e-20f;
-  if (lane < p.k) {
-    const float wv = p.rsf * my_s / denom;
-    S.sel_idx[pos] = my_sel;
-    S.sel_w[pos] = wv;
-    if (blockIdx.x == 0) {
-      if (p.idx_out) p.idx_out[pos] = my_sel;
-      if (p.w_out) p.w_out[pos] = wv;
-    }
-  }
+  __syncwarp();
+  // lane r holds the r-th pick (lanes past k: INT_MAX for the ordering)
+  const int my_sel = (lane < p.k) ? S.pick_id[lane] : 0x7FFFFFFF;
+  const float my_s = (lane < p.k) ? S.pick_s[lane] : 0.f;
+  publish_selection(p, S, my_sel, (lane < p.k) ? my_s : 0.f);
 }
 
 // Lane holding reduce-scatter value `vi` of row phase `ph` (group-local warp).
@@ -501,7 +532,7 @@ __device__ __forceinline__ bool group_barrier(uint64_t* bar, uint32_t par) {
   int ok = 1;
   if (lane == 0) {
     mbar_arrive(bar);
-    ok = mbar_wait(bar, par, global_timer_ns() + kWaitNs) ? 1 : 0;
+    ok = mbar_wait(bar, par, kWaitNs) ? 1 : 0;
   }
   ok = __shfl_sync(0xffffffffu, ok, 0);
   if (ok) mbar_test(bar, par);
@@ -541,7 +572,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slots = p.k + p.has_shared;
 
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == kProducerWarp * 32) {
+    // the producer thread sets up the barriers and sends the CTA's first
+    // fill (its router rows, the head of the dependent start-up chain)
+    // before anything else happens
     TRACE_AT(0);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&S.full[s], 1);
@@ -552,6 +586,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     S.sel_ok = 0;
     S.abort_flag[0] = S.abort_flag[1] = 0;
     fence_mbar_init();
+    int rr0, rnr;
+    router_rows(p, blockIdx.x, rr0, rnr);
+    if (rnr > 0) {
+      S.desc[0] = make_item(kRouter, 0, rr0, rnr);
+      const uint32_t bytes = (uint32_t)rnr * p.H * 4;
+      mbar_arrive_expect_tx(&S.full[0], bytes);
+      bulk_g2s(dsmem, p.w_router + (size_t)rr0 * p.H, bytes, &S.full[0], l2_policy_evict_first());
+      TRACE_AT(1);
+    }
   }
   if (p.x_resid) {
     // RMSNorm with unit gain ("LightLX", "How it works": RMSNorm of the
@@ -582,23 +625,47 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       int dones = 0;
       int rr0, rnr;
       router_rows(p, blockIdx.x, rr0, rnr);
-      bool router_pending = rnr > 0;
       bool tickets_over = false;
       int dn = 0;  // this CTA's down items taken so far
       int dr0, dr1;
       down_rows(p, blockIdx.x, dr0, dr1);
-      for (uint32_t n = 0;; ++n) {
+      // fill 0 (the router rows) went out in the prologue
+      for (uint32_t n = rnr > 0 ? 1u : 0u;; ++n) {
         const int stage = (int)(n % kStages);
         ItemDesc d = make_item(kDone, 0, 0, 0);
-        if (router_pending) {
-          d = make_item(kRouter, 0, rr0, rnr);
-          router_pending = false;
-        } else if (dones == 0) {
+        // the next item of this CTA (slots dropped by top-p are passed over)
+        while (dones == 0) {
           if (!tickets_over) {
             d = gate_up_ticket(p, (int)atomicAdd(p.ctrl + kCtrlTicket, 1u));
             tickets_over = d.type == kDone;
           }
-          if (tickets_over) d = next_down(p, dn, dr0, dr1);
+          if (tickets_over) {
+            if (dn == 0 && p.pf_w_router) prefetch_next_layer(p);
+            d = next_down(p, dn, dr0, dr1);
+          }
+          if (d.type == kDone) break;
+          if (d.slot < p.k) {
+            if (!sel_seen) {
+              // the selection warp's result (mbarrier: release / acquire)
+              if (mbar_wait(&S.selbar, 0u, kWaitNs) && S.sel_ok) {
+                sel_seen = true;
+                TRACE_AT(12);
+              } else {
+                set_error(p.ctrl, kErrTimeout, 4, n);
+                d = make_item(kDone, 0, 0, 0);
+                break;
+              }
+            }
+            d.eid = S.sel_idx[d.slot];
+            if (d.eid == -1) continue;  // dropped by top-p: no bytes read
+            if (d.eid < 0 || d.eid >= p.E) {
+              set_error(p.ctrl, kErrBadExpertId, 5, n);
+              d = make_item(kDone, 0, 0, 0);
+              break;
+            }
+          } else {
+            d.eid = p.E;  // shared expert
+          }
           if (d.type == kDown && !((hq_seen >> d.slot) & 1ull)) {
             // every 32-row group of the slot's h must be published as int16
             if (wait_counter(p.ctrl, p.ctrl + kCtrlHqDone + d.slot, (uint32_t)(p.I >> 5))) {
@@ -609,51 +676,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
               d = make_item(kDone, 0, 0, 0);
             }
           }
-          if (d.type == kGateUp || d.type == kDown) {
-            if (d.slot < p.k) {
-              if (!sel_seen) {
-                // the selection warp's result (mbarrier: release / acquire)
-                if (mbar_wait(&S.selbar, 0u, global_timer_ns() + kWaitNs) && S.sel_ok) {
-                  sel_seen = true;
-                  TRACE_AT(12);
-                } else {
-                  set_error(p.ctrl, kErrTimeout, 4, n);
-                  d = make_item(kDone, 0, 0, 0);
-                }
-              }
-              if (d.type != kDone) {
-                d.eid = S.sel_idx[d.slot];
-                if (d.eid < 0 || d.eid >= p.E) {
-                  set_error(p.ctrl, kErrBadExpertId, 5, n);
-                  d = make_item(kDone, 0, 0, 0);
-                }
-              }
-            } else {
-              d.eid = p.E;  // shared expert
-            }
-          }
+          break;
         }
         // wait until the consumers released this stage's previous contents
         if (n >= (uint32_t)kStages) {
-          const uint64_t deadline = global_timer_ns() + kWaitNs;
-          if (!mbar_wait(&S.empty[stage], ((n / kStages) - 1) & 1u, deadline)) {
+          if (!mbar_wait(&S.empty[stage], ((n / kStages) - 1) & 1u, kWaitNs)) {
             set_error(p.ctrl, kErrTimeout, 6, n);
             // stop issuing; wait (bounded) for the fills already issued
             for (uint32_t m = n - kStages; m < n; ++m) {
-              const uint64_t dl = global_timer_ns() + kWaitNs;
-              mbar_wait(&S.full[m % kStages], (m / kStages) & 1u, dl);
+              mbar_wait(&S.full[m % kStages], (m / kStages) & 1u, kWaitNs);
             }
             break;
           }
         }
         S.desc[stage] = d;
         uint8_t* dst = stages + (size_t)stage * kStageBytes;
-        if (d.type == kRouter) {
-          TRACE_AT(1);
-          const uint32_t bytes = (uint32_t)d.nrows * p.H * 4;
-          mbar_arrive_expect_tx(&S.full[stage], bytes);
-          bulk_g2s(dst, p.w_router + (size_t)d.row0 * p.H, bytes, &S.full[stage], policy);
-        } else if (d.type == kGateUp) {
+        if (d.type == kGateUp) {
           if (d.slot == 0 && !first_routed) {
             first_routed = true;
             TRACE_AT(6);
@@ -690,8 +728,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           if (++dones == kGroups) {
             // leave no bulk copy in flight
             for (uint32_t m = (n >= (uint32_t)kStages ? n - kStages + 1 : 0); m < n; ++m) {
-              const uint64_t dl = global_timer_ns() + kWaitNs;
-              mbar_wait(&S.full[m % kStages], (m / kStages) & 1u, dl);
+              mbar_wait(&S.full[m % kStages], (m / kStages) & 1u, kWaitNs);
             }
             break;
           }
@@ -764,9 +801,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     // b, b + grid, ... of the order (shared slot first, then slots 0..k-1;
     // groups ascending), the order in which gate/up items complete.
     const int GD = p.I >> 5, slots = p.k + p.has_shared;
+    bool sel_seen = false;
     for (int i = blockIdx.x; i < slots * GD; i += gridDim.x) {
       const int so = i / GD, g = i % GD;
       const int slot = p.has_shared ? (so == 0 ? p.k : so - 1) : so;
+      if (slot < p.k) {
+        // a routed slot may be dropped by top-p: its h never comes
+        if (!sel_seen) {
+          int okw = 0;
+          if (lane == 0) okw = mbar_wait(&S.selbar, 0u, kWaitNs) && S.sel_ok;
+          if (!__shfl_sync(0xffffffffu, okw, 0)) break;  // the selection warp reported it
+          mbar_test(&S.selbar, 0u);
+          sel_seen = true;
+        }
+        if (S.sel_idx[slot] == -1) continue;
+      }
       const uint32_t* cnt = p.ctrl + kCtrlHRows + slot * GD + g;
       // every lane acquires the count itself (so its own loads of h below
       // are ordered after the writers' release adds)
@@ -887,7 +936,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         const int stage = 0;
         const uint32_t gpar = 0u;
         int okw = 0;
-        if (lane == 0) okw = mbar_wait(&S.full[0], 0u, global_timer_ns() + kWaitNs) ? 1 : 0;
+        if (lane == 0) okw = mbar_wait(&S.full[0], 0u, kWaitNs) ? 1 : 0;
         const bool ok = __shfl_sync(0xffffffffu, okw, 0) != 0;
         if (ok) {
           mbar_test(&S.full[0], 0u);
@@ -928,6 +977,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
             if (lane == 0) S.redd[gw][r] = v;
           }
         }
+        if (tg == 0) TRACE_AT(15);
         if (!group_barrier(&S.gbar[grp], gpar)) {
           if (lane == 0) set_error(p.ctrl, kErrTimeout, 3, 0);
           gabort = 1;
@@ -966,7 +1016,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       bool ok = true;
       if (!fake) {
         int okw = 0;
-        if (lane == 0) okw = mbar_wait(&S.full[stage], par, global_timer_ns() + kWaitNs) ? 1 : 0;
+        if (lane == 0) okw = mbar_wait(&S.full[stage], par, kWaitNs) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, okw, 0) != 0;
         if (ok) {
           mbar_test(&S.full[stage], par);  // acquire the bulk-copied bytes in every lane
@@ -1116,7 +1166,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     if (!aborted(p.ctrl)) {
       for (int lr = threadIdx.x; lr < r1 - r0; lr += kThreads) {
         float acc = 0.f;
-        for (int j = 0; j < p.k; ++j) acc = fmaf(S.sel_w[j], S.ycta[j * p.ycta_rows + lr], acc);
+        for (int j = 0; j < p.k; ++j)
+          if (S.sel_idx[j] >= 0) acc = fmaf(S.sel_w[j], S.ycta[j * p.ycta_rows + lr], acc);
         if (p.has_shared) acc += S.ycta[p.k * p.ycta_rows + lr];
         if (p.x_resid) acc = p.x_resid[r0 + lr] + acc;  // x + MoE(norm(x))
         p.y[r0 + lr] = acc;

@@ -45,6 +45,7 @@ struct DecodeParams {
   float* hqf;         // [slots][I / 32] their factors
   int H, I, E, k, n_group, topk_group, has_shared;
   float rsf;
+  float top_p;        // adaptive expert top-p (>= 1: off); dropped slots carry id -1
   // selection layout: lane l owns experts l*sel_q .. l*sel_q+sel_q-1 and a
   // group is 2^sel_lgL consecutive lanes (sel_fast), else the generic path
   int sel_fast, sel_q, sel_lgL;
@@ -54,7 +55,12 @@ struct DecodeParams {
   // down rows: CTA b owns rows [A * (b * nU / grid), A * ((b + 1) * nU / grid))
   // of every slot, nU = H / A, in n_db items of at most RD rows per slot
   int A, nU, n_db, ycta_rows;
-  uint64_t* trace;    // timeline probes of a -DMOE_TRACE build ([grid][16]); else unused
+  uint64_t* trace;    // timeline probes of a -DMOE_TRACE build ([grid][32]); else unused
+  // The next layer of a stack (nullable): during this layer's down phase
+  // each CTA prefetches into L2 its router rows and a share of the shared
+  // expert's gate/up rows, the bytes the next layer's start-up reads first.
+  const float* pf_w_router;
+  ExpertPtrs pf_shared;
 };
 
 // Fill the shape part of p; false if the fused kernel does not cover the

@@ -30,7 +30,7 @@ moe_status ffn_impl(const moe_layer* l, const uint16_t* x, int T, const int32_t*
 }
 
 #ifdef MOE_TRACE
-// Timeline buffer of a profiling build (-DMOE_TRACE): [grid][16] uint64.
+// Timeline buffer of a profiling build (-DMOE_TRACE): [grid][32] uint64.
 static uint64_t* g_trace = nullptr;
 extern "C" __attribute__((visibility("default"))) void moe_debug_set_trace(void* buf) {
   g_trace = static_cast<uint64_t*>(buf);
@@ -40,7 +40,7 @@ extern "C" __attribute__((visibility("default"))) void moe_debug_set_trace(void*
 static moe_status launch_fused(const moe_layer* l, const uint16_t* x, const float* x_resid,
                                float norm_eps, uint16_t* xn_out, float* y, int32_t* idx_out,
                                float* w_out, uint8_t* ws, const WsLayout& L, cudaStream_t st,
-                               bool* used) {
+                               bool* used, const moe_layer* next = nullptr) {
   DecodeParams p;
   *used = false;
   if (!decode_plan(l->cfg, p)) return MOE_OK;
@@ -59,6 +59,13 @@ static moe_status launch_fused(const moe_layer* l, const uint16_t* x, const floa
   p.scores = reinterpret_cast<uint64_t*>(ws + L.records);
   p.hbuf = reinterpret_cast<float*>(ws + L.hbuf);
   p.warm = 1;
+  p.top_p = l->top_p;
+  // the next layer of a stack, when it has this layer's shape
+  const bool same = next && next->cfg.hidden == l->cfg.hidden && next->cfg.inter == l->cfg.inter &&
+                    next->cfg.n_experts == l->cfg.n_experts &&
+                    next->cfg.n_shared == l->cfg.n_shared;
+  p.pf_w_router = same ? next->w_router : nullptr;
+  p.pf_shared = same ? next->host_table[next->cfg.n_experts] : ExpertPtrs{};
 #ifdef MOE_TRACE
   p.trace = g_trace;
 #else
@@ -72,7 +79,7 @@ static moe_status launch_fused(const moe_layer* l, const uint16_t* x, const floa
 
 moe_status forward_impl(const moe_layer* l, const uint16_t* x, int T, float* y, int32_t* idx_out,
                         float* w_out, uint8_t* ws, const WsLayout& L, cudaStream_t st) {
-  if (T == 1 && l->top_p >= 1.f) {
+  if (T == 1) {
     bool used = false;
     moe_status s = launch_fused(l, x, nullptr, 0.f, nullptr, y, idx_out, w_out, ws, L, st, &used);
     if (used || s != MOE_OK) return s;
@@ -86,12 +93,10 @@ moe_status forward_impl(const moe_layer* l, const uint16_t* x, int T, float* y, 
 
 moe_status residual_impl(const moe_layer* l, const float* x_resid, float norm_eps, float* x_next,
                          uint16_t* xn_out, int32_t* idx_out, float* w_out, uint8_t* ws,
-                         const WsLayout& L, cudaStream_t st) {
-  if (l->top_p < 1.f)
-    return fail(MOE_ERR_UNSUPPORTED, "the pre-norm step runs without adaptive top-p");
+                         const WsLayout& L, cudaStream_t st, const moe_layer* next) {
   bool used = false;
   moe_status s = launch_fused(l, nullptr, x_resid, norm_eps, xn_out, x_next, idx_out, w_out, ws,
-                              L, st, &used);
+                              L, st, &used, next);
   if (s != MOE_OK) return s;
   if (!used) return fail(MOE_ERR_UNSUPPORTED, "the pre-norm step needs the fused decode kernel's shapes");
   return MOE_OK;

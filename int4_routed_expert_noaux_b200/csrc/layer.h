@@ -42,9 +42,11 @@ moe_status route_impl(const moe_layer* l, const uint16_t* x, int T, int32_t* idx
                       float* scores, uint8_t* ws, const WsLayout& L, cudaStream_t st);
 moe_status ffn_impl(const moe_layer* l, const uint16_t* x, int T, const int32_t* idx,
                     const float* w, float* y, uint8_t* ws, const WsLayout& L, cudaStream_t st);
+// next (nullable): the layer that runs after this one (a stack), whose
+// first bytes this layer's kernel prefetches into L2.
 moe_status residual_impl(const moe_layer* l, const float* x_resid, float norm_eps, float* x_next,
                          uint16_t* xn_out, int32_t* idx_out, float* w_out, uint8_t* ws,
-                         const WsLayout& L, cudaStream_t st);
+                         const WsLayout& L, cudaStream_t st, const moe_layer* next = nullptr);
 moe_status forward_impl(const moe_layer* l, const uint16_t* x, int T, float* y, int32_t* idx_out,
                         float* w_out, uint8_t* ws, const WsLayout& L, cudaStream_t st);
 
