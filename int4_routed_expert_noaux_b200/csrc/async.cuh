@@ -116,6 +116,12 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   return v;
 }
 
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
 // 64-bit relaxed load / store at gpu scope: single-copy atomic, so a record
 // that carries its own validity tag needs no fence.
 __device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {

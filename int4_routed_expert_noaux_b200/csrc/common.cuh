@@ -213,6 +213,43 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Double-float value hi + lo (|lo| <= half an ulp of hi, about 48 bits).
+struct DF {
+  float hi, lo;
+};
+
+// a += w * x with no rounding error lost: the product splits exactly into
+// p + e (e = fma(w, x, -p)), p is added to hi error-free (TwoSum), and the
+// two error terms go to lo.  The _rn intrinsics keep the compiler from
+// contracting the adds into fmas, which would break the error terms.
+__device__ __forceinline__ void df_add_prod(DF& a, float w, float x) {
+  const float p = __fmul_rn(w, x);
+  const float e = fmaf(w, x, -p);
+  const float s = __fadd_rn(a.hi, p);
+  const float bp = __fsub_rn(s, a.hi);
+  const float err = __fadd_rn(__fsub_rn(a.hi, __fsub_rn(s, bp)), __fsub_rn(p, bp));
+  a.hi = s;
+  a.lo = __fadd_rn(a.lo, __fadd_rn(err, e));
+}
+
+__device__ __forceinline__ DF df_add(DF a, DF b) {
+  const float s = __fadd_rn(a.hi, b.hi);
+  const float bp = __fsub_rn(s, a.hi);
+  const float err = __fadd_rn(__fsub_rn(a.hi, __fsub_rn(s, bp)), __fsub_rn(b.hi, bp));
+  return DF{s, __fadd_rn(__fadd_rn(a.lo, b.lo), err)};
+}
+
+__device__ __forceinline__ DF df_warp_sum(DF v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    DF u;
+    u.hi = __shfl_xor_sync(0xffffffffu, v.hi, o);
+    u.lo = __shfl_xor_sync(0xffffffffu, v.lo, o);
+    v = df_add(v, u);
+  }
+  return v;
+}
+
 __device__ __forceinline__ double warp_sum_f64(double v) {
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

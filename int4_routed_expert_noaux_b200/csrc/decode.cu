@@ -1,48 +1,47 @@
 // decode.cu -- the fused persistent decode kernel: the whole routed-MoE
 // layer for one token (router GEMV, noaux_tc selection, 8 routed + shared
-// int4 expert FFNs, weighted combine) in ONE launch.
+// int4 expert FFNs, weighted combine) in ONE cooperative launch.
 //
 // Design (sm_100a):
-//  * one CTA per SM: a producer warp, a selection warp and two consumer
-//    groups of 6 warps;
-//  * the producer claims work items from a global ticket counter, in a fixed
-//    order, and moves each item's weights HBM -> shared memory with 1-D bulk
-//    async copies (the TMA engine) into a 4-stage ring of 54 KB stages,
-//    completion tracked by mbarriers (transaction bytes).  Fill n goes to
-//    stage n % 4 and is consumed by group n % 2, so one group reduces and
-//    publishes while the other computes and two stages stay in flight;
+//  * one CTA per SM: two consumer groups of 6 warps, a producer warp, a
+//    selection warp and a converter warp;
+//  * the producer moves each work item's bytes HBM -> shared memory with
+//    1-D bulk async copies (the TMA engine) into a 4-stage ring of 54 KB
+//    stages, completion tracked by mbarriers (transaction bytes).  Fill n
+//    goes to stage n % 4 and is consumed by group n % 2, so one group reduces
+//    and publishes while the other computes and two stages stay in flight;
 //  * consumers are column-stationary: each thread owns one 16-byte chunk
 //    column of the rows it visits and keeps its 32 inputs in registers as
 //    int16 fixed point with one exponent per group; the int4 group dot
 //    product is exact in integers (dp2a); one butterfly reduce-scatter plus
 //    a cross-warp sum finishes each row; one group barrier per item;
-//  * each CTA first computes its own block of router rows (a static split
-//    of the experts over the first CTAs, the CTA's first fill) and
-//    publishes each row's sigmoid score as a 64-bit record tagged with the
-//    call's epoch (one single-copy-atomic store: no flag, no fence);
-//  * a selection warp in every CTA polls the E records until all carry this
-//    call's epoch and runs the noaux_tc selection itself (every CTA reads the
-//    same scores with the same code, so all reach the same bits); it hands
-//    the expert ids and weights to its producer and consumers through
-//    shared memory;
-//  * work items come from a global ticket counter in the order:
-//    shared-expert gate/up, routed gate/up of slots 0..k-1, shared-expert
-//    down, routed down of slots 0..k-1.  Every dependency points to an
-//    earlier ticket, so in-order claiming always makes progress; the shared
-//    expert's gate/up items keep HBM busy while the routed experts are
-//    selected, and no producer waits on a down item's inputs early on;
+//  * start-up: the producer's first fill is the CTA's block of router rows
+//    (a static split of the experts over the first CTAs).  Group 0 computes
+//    the router rows in double-float arithmetic and publishes each row's
+//    sigmoid score as a 64-bit record tagged with the call's epoch (one
+//    single-copy-atomic store: no flag, no fence);
+//  * the selection warp of every CTA polls the E records until all carry
+//    this call's epoch and runs the noaux_tc selection itself -- every CTA
+//    reads the same scores with the same code, so all reach the same bits --
+//    then loads the selected experts' tensor pointers into shared memory
+//    once;
+//  * gate/up items (8 gate + 8 up rows of one expert for the GLM shape) are
+//    dealt out statically, CTA b taking items b, b + grid, ... in the order
+//    shared expert, routed slots 0..k-1; the shared expert's items keep HBM
+//    busy while the routed experts are selected.  Finalizer warps write h
+//    rows (fp32) and count, per 32-row group of h, the rows written;
+//  * the converter warp of each CTA owns some of those groups: once a
+//    group's 32 rows are in, it publishes them as int16 words with one
+//    exponent (the layout the down consumers load) and counts the slot's
+//    published groups;
+//  * down items are static too: CTA b owns a block of output rows and, once
+//    a slot's h is published, streams that slot's down rows for it together
+//    with the slot's int16 h (4 KB); the slot partials of its rows stay in
+//    shared memory and are combined in slot order at the end (no atomics, no
+//    cross-CTA combine, bitwise repeatable);
 //  * consumer group 1 first runs one placeholder gate/up and one placeholder
 //    down item through the loop body (nothing published), so that both code
 //    paths are fetched while the first weights are in flight;
-//  * gate/up finalizer warps publish h rows (fp32) and count themselves done
-//    with a release add (nothing waits on its result); the producer waits
-//    until a slot's count is complete and bulk-copies the slot's h (8 KB for
-//    the GLM shape, from L2) into the tail of each down item's stage; down
-//    consumers convert their own 32-row group of h to int16 fixed point;
-//  * down items write per-slot partial rows; the warp whose release add
-//    completes a row block (checked one item later, off the critical path)
-//    sums the partials in slot order (deterministic, no atomics on data)
-//    into y;
 //  * every wait is bounded (1 s); a wait that runs out sets the workspace
 //    error word and the kernel winds down; the last CTA to exit resets the
 //    control counters so the next call starts clean.
@@ -55,18 +54,25 @@
 #include "device_once.h"
 
 // Timeline probes: compiled in only with -DMOE_TRACE (a profiling build).
-// Slot i < 16 of CTA b gets the SM cycle counter at probe i; slot 16 the
-// globaltimer (ns) when the CTA starts, to line the CTAs up.
+// Per CTA 128 slots: SM cycle counter at event i in slot 96 + i (i < 31),
+// the producer's per-fill wait start and issue cycles in slots 2n, 2n + 1
+// (n < 48), and the globaltimer (ns) at the CTA's start in slot 127.
 #ifdef MOE_TRACE
 #define TRACE_AT(i)                                                                          \
   do {                                                                                       \
     if (p.trace) {                                                                           \
-      p.trace[blockIdx.x * 32 + (i)] = (uint64_t)clock64();                                  \
-      if ((i) == 0) p.trace[blockIdx.x * 32 + 16] = moe::global_timer_ns();                  \
+      p.trace[blockIdx.x * 128 + 96 + (i)] = (uint64_t)clock64();                            \
+      if ((i) == 0) p.trace[blockIdx.x * 128 + 127] = moe::global_timer_ns();                \
     }                                                                                        \
+  } while (0)
+#define TRACE_FILL(n, j, tag)                                                                \
+  do {                                                                                       \
+    if (p.trace && (n) < 48)                                                                 \
+      p.trace[blockIdx.x * 128 + 2 * (n) + (j)] = (uint64_t)clock64() | ((uint64_t)(tag) << 60); \
   } while (0)
 #else
 #define TRACE_AT(i) ((void)0)
+#define TRACE_FILL(n, j, tag) ((void)0)
 #endif
 
 namespace moe {
@@ -102,6 +108,7 @@ struct Smem {
   uint64_t selbar;         // the selection warp has published sel_*
   ItemDesc desc[kStages];
   int sel_idx[kMaxSlots];  // selected expert ids, ascending
+  ExpertPtrs ep[kMaxSlots];  // the slots' expert tensors (slot k: the shared expert)
   int pick_id[kMaxSlots];  // the selection's picks in pick order
   float pick_s[kMaxSlots];
   float sel_w[kMaxSlots];  // their combine weights
@@ -125,6 +132,8 @@ struct SelArgs {
   float rsf, top_p;
   int32_t* idx_out;  // written by CTA 0 only (nullable)
   float* w_out;
+  uint64_t* trace;   // timeline probes of a -DMOE_TRACE build
+  const ExpertPtrs* table;  // nullable in a dry run
 };
 
 __device__ __forceinline__ SelArgs sel_args(const DecodeParams& p) {
@@ -140,6 +149,8 @@ __device__ __forceinline__ SelArgs sel_args(const DecodeParams& p) {
   a.top_p = p.top_p;
   a.idx_out = p.idx_out;
   a.w_out = p.w_out;
+  a.trace = p.trace;
+  a.table = p.table;
   return a;
 }
 
@@ -154,9 +165,9 @@ __device__ __forceinline__ ItemDesc make_item(int type, int slot, int row0, int 
   return d;
 }
 
-// Gate/up item of ticket t, in the order: shared gate/up, routed gate/up of
-// slots 0..k-1; DONE past the last one.
-__device__ __forceinline__ ItemDesc gate_up_ticket(const DecodeParams& p, int t) {
+// Gate/up item t, in the order: shared gate/up, routed gate/up of slots
+// 0..k-1; DONE past the last one.
+__device__ __forceinline__ ItemDesc gate_up_item(const DecodeParams& p, int t) {
   auto gu = [&](int slot, int b) {
     return make_item(kGateUp, slot, b * p.RG, min(p.RG, p.I - b * p.RG));
   };
@@ -445,6 +456,7 @@ __device__ __noinline__ void run_select(const SelArgs p, Smem& S) {
   }
   const int per = q << lgL;
   const float gs_seg = (per >= 2) ? t1 + t2 : t1;
+  if (lane == 0) TRACE_AT(17);
   // keep topk_group groups: rank by (score desc, index asc); lane g holds
   // group g (n_group <= 32), lanes past the groups hold -inf
   const int G = p.n_group;
@@ -458,6 +470,7 @@ __device__ __noinline__ void run_select(const SelArgs p, Smem& S) {
   }
   const unsigned kept_mask = __ballot_sync(0xffffffffu, lane < G && rank < p.topk_group);
   const bool kept = (kept_mask >> (lane >> lgL)) & 1u;
+  if (lane == 0) TRACE_AT(18);
   // each lane sorts its kept candidates once (a sorting network)
   uint32_t key[kQ];
   int jid[kQ];
@@ -475,6 +488,18 @@ __device__ __noinline__ void run_select(const SelArgs p, Smem& S) {
   cx(key, jid, sl, 0, 4); cx(key, jid, sl, 1, 5); cx(key, jid, sl, 2, 6); cx(key, jid, sl, 3, 7);
   cx(key, jid, sl, 2, 4); cx(key, jid, sl, 3, 5);
   cx(key, jid, sl, 1, 2); cx(key, jid, sl, 3, 4); cx(key, jid, sl, 5, 6);
+  if (lane == 0) TRACE_AT(19);
+  // the winners are among each lane's best candidates: their pointer-table
+  // entries start towards L1 now, and the loads after the selection hit it
+  if (p.table) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+      if (key[j] != 0u) {
+        const char* e = reinterpret_cast<const char*>(p.table + lane * q + jid[j]);
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(e));
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(e + sizeof(ExpertPtrs) - 1));
+      }
+  }
   // top_k: the best head is popped, k times; among equal heads (a rare,
   // warp-uniform case) the lowest expert id.  The owner of the r-th pick
   // leaves it in shared memory, off the dependent chain of the rounds.
@@ -504,6 +529,7 @@ __device__ __noinline__ void run_select(const SelArgs p, Smem& S) {
   }
   __syncwarp();
   // lane r holds the r-th pick (lanes past k: INT_MAX for the ordering)
+  if (lane == 0) TRACE_AT(20);
   const int my_sel = (lane < p.k) ? S.pick_id[lane] : 0x7FFFFFFF;
   const float my_s = (lane < p.k) ? S.pick_s[lane] : 0.f;
   publish_selection(p, S, my_sel, (lane < p.k) ? my_s : 0.f);
@@ -572,6 +598,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slots = p.k + p.has_shared;
 
+  // the producer's first-item offset (0 but in a failure test), loaded
+  // before anything else so that its round trip is over by the first fill
+  const uint32_t gu_offset =
+      threadIdx.x == kProducerWarp * 32 ? ld_relaxed_u32(p.ctrl + kCtrlTicket) : 0u;
   if (threadIdx.x == kProducerWarp * 32) {
     // the producer thread sets up the barriers and sends the CTA's first
     // fill (its router rows, the head of the dependent start-up chain)
@@ -586,6 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     S.sel_ok = 0;
     S.abort_flag[0] = S.abort_flag[1] = 0;
     fence_mbar_init();
+    if (p.has_shared) S.ep[p.k] = p.shared;  // visible to the producer: same thread
     int rr0, rnr;
     router_rows(p, blockIdx.x, rr0, rnr);
     if (rnr > 0) {
@@ -625,22 +656,41 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       int dones = 0;
       int rr0, rnr;
       router_rows(p, blockIdx.x, rr0, rnr);
-      bool tickets_over = false;
+      bool gate_up_over = false;
       int dn = 0;  // this CTA's down items taken so far
       int dr0, dr1;
       down_rows(p, blockIdx.x, dr0, dr1);
+      // Gate/up items are dealt out statically: CTA b takes items b,
+      // b + grid, ... of the order shared, routed 0..k-1.  (A shared ticket
+      // counter balances slightly better but puts an atomic's round trip to
+      // L2 -- microseconds while the weights stream -- between fills.)  The
+      // control word kCtrlTicket offsets the first item; it is 0 except in a
+      // test that starts past the last item to make a wait run out.
+      int gu_next = (int)blockIdx.x + (int)gu_offset;
       // fill 0 (the router rows) went out in the prologue
       for (uint32_t n = rnr > 0 ? 1u : 0u;; ++n) {
         const int stage = (int)(n % kStages);
         ItemDesc d = make_item(kDone, 0, 0, 0);
         // the next item of this CTA (slots dropped by top-p are passed over)
         while (dones == 0) {
-          if (!tickets_over) {
-            d = gate_up_ticket(p, (int)atomicAdd(p.ctrl + kCtrlTicket, 1u));
-            tickets_over = d.type == kDone;
+          if (!gate_up_over) {
+            d = gate_up_item(p, gu_next);
+            gate_up_over = d.type == kDone;
+            gu_next += (int)gridDim.x;
           }
-          if (tickets_over) {
-            if (dn == 0 && p.pf_w_router) prefetch_next_layer(p);
+          if (gate_up_over) {
+            if (dn == 0) {
+              if (p.pf_w_router) prefetch_next_layer(p);
+              // which slots' int16 h are complete already: one round trip
+              // for all of them instead of one per down item
+              // (relaxed loads all in flight at once, then one fence: an
+              // acquire of every count seen complete)
+              for (int j = 0; j < slots; ++j)
+                if (ld_relaxed_u32(p.ctrl + kCtrlHqDone + j) >= (uint32_t)(p.I >> 5))
+                  hq_seen |= 1ull << j;
+              fence_acq_rel();
+              fence_proxy_async();
+            }
             d = next_down(p, dn, dr0, dr1);
           }
           if (d.type == kDone) break;
@@ -679,6 +729,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           break;
         }
         // wait until the consumers released this stage's previous contents
+        TRACE_FILL(n, 0, d.type);
         if (n >= (uint32_t)kStages) {
           if (!mbar_wait(&S.empty[stage], ((n / kStages) - 1) & 1u, kWaitNs)) {
             set_error(p.ctrl, kErrTimeout, 6, n);
@@ -690,13 +741,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           }
         }
         S.desc[stage] = d;
+        TRACE_FILL(n, 1, d.slot & 15);
         uint8_t* dst = stages + (size_t)stage * kStageBytes;
         if (d.type == kGateUp) {
           if (d.slot == 0 && !first_routed) {
             first_routed = true;
             TRACE_AT(6);
           }
-          const ExpertPtrs ep = p.table[d.eid];
+          const ExpertPtrs ep = S.ep[d.slot];
           const uint32_t qb = (uint32_t)d.nrows * (p.H / 2), sb = (uint32_t)d.nrows * (p.H / 16);
           const size_t qoff = (size_t)d.row0 * (p.H / 2), soff = (size_t)d.row0 * (p.H / 32);
           mbar_arrive_expect_tx(&S.full[stage], 2 * (qb + sb));
@@ -710,7 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
             first_down = true;
             TRACE_AT(7);
           }
-          const ExpertPtrs ep = p.table[d.eid];
+          const ExpertPtrs ep = S.ep[d.slot];
           const int GD = p.I >> 5;
           const uint32_t qb = (uint32_t)d.nrows * (p.I / 2), sb = (uint32_t)d.nrows * (p.I / 16);
           const uint32_t hb = (uint32_t)GD * 64, fb = (uint32_t)GD * 4;
@@ -785,6 +837,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       }
       __syncwarp();
       run_select(sel_args(p), S);
+      __syncwarp();
+      // the selected experts' tensor pointers, one load per lane, so that
+      // no fill waits on a pointer-table load from global memory
+      if (lane < p.k) {
+        const int id = S.sel_idx[lane];
+        if (id >= 0 && id < p.E) S.ep[lane] = p.table[id];
+      }
       if (lane == 0) TRACE_AT(5);
     } else if (lane == 0) {
       set_error(p.ctrl, kErrTimeout, 8, 0);
@@ -912,27 +971,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     int& gabort = S.abort_flag[grp];
     int dr0, dr1;
     down_rows(p, blockIdx.x, dr0, dr1);
+    int rr0, rnr;
+    router_rows(p, blockIdx.x, rr0, rnr);
+    // group 0's router inputs (bf16)
+    uint2 xr[kRouterChunks];
+    const int rchunks = p.H >> 2;
+#pragma unroll
+    for (int i = 0; i < kRouterChunks; ++i) {
+      const int cc = tg + kGT * i;
+      if (grp != 0 || rnr == 0 || cc >= rchunks) {
+        xr[i] = make_uint2(0, 0);
+      } else if (p.x_resid) {
+        xr[i] = norm_bf16x4(p.x_resid, 4 * cc, inv_rms);
+      } else {
+        xr[i] = __ldg(reinterpret_cast<const uint2*>(p.x) + cc);
+      }
+    }
     // Group 0 of a CTA with router rows: fill 0 is the router block.  It is
     // handled before the main loop so its bf16 inputs are dead afterwards.
     uint32_t c_first = 0;
     {
-      int rr0, rnr;
-      router_rows(p, blockIdx.x, rr0, rnr);
       if (grp == 0 && rnr > 0) {
         c_first = 1;
-        uint2 xr[kRouterChunks];
-        const int rchunks = p.H >> 2;
-#pragma unroll
-        for (int i = 0; i < kRouterChunks; ++i) {
-          const int cc = tg + kGT * i;
-          if (cc >= rchunks) {
-            xr[i] = make_uint2(0, 0);
-          } else if (p.x_resid) {
-            xr[i] = norm_bf16x4(p.x_resid, 4 * cc, inv_rms);
-          } else {
-            xr[i] = __ldg(reinterpret_cast<const uint2*>(p.x) + cc);
-          }
-        }
         const int stage = 0;
         const uint32_t gpar = 0u;
         int okw = 0;
@@ -947,36 +1007,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         }
         const ItemDesc d = S.desc[0];
         const uint8_t* st = stages;
-        // fp64 sums of exact fp32 x bf16 products: the logit is exact to
-        // about 1e-13, so the selection sees scores rounded only once
-        double acc[kMaxRR];
+        // double-float sums of the exact fp32 x bf16 products: each product
+        // is split exactly into p + e, the p are summed error-free into
+        // (hi, lo) and the e added to lo -- about 48 bits with fp32
+        // arithmetic only, so the logit is exact to ~1e-14 and the
+        // selection sees scores rounded only once (to fp32).  Four
+        // independent chains per row (one per lane of a float4).
+        float xv[kRouterChunks][4];
 #pragma unroll
-        for (int r = 0; r < kMaxRR; ++r) {
-          acc[r] = 0.0;
-          if (ok && r < d.nrows) {
-            const float4* wr = reinterpret_cast<const float4*>(st + (size_t)r * p.H * 4);
+        for (int i = 0; i < kRouterChunks; ++i) {
+          xv[i][0] = bf16_bits_to_f32(xr[i].x & 0xFFFFu);
+          xv[i][1] = bf16_bits_to_f32(xr[i].x >> 16);
+          xv[i][2] = bf16_bits_to_f32(xr[i].y & 0xFFFFu);
+          xv[i][3] = bf16_bits_to_f32(xr[i].y >> 16);
+        }
+        const int nrr = ok ? d.nrows : 0;
+        for (int r = 0; r < nrr; ++r) {
+          const float4* wr = reinterpret_cast<const float4*>(st + (size_t)r * p.H * 4);
+          DF c0{0.f, 0.f}, c1{0.f, 0.f}, c2{0.f, 0.f}, c3{0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < kRouterChunks; ++i) {
-              const int cc = tg + kGT * i;
-              if (cc < rchunks) {
-                const float4 wv = wr[cc];
-                acc[r] = fma((double)wv.x, (double)bf16_bits_to_f32(xr[i].x & 0xFFFFu), acc[r]);
-                acc[r] = fma((double)wv.y, (double)bf16_bits_to_f32(xr[i].x >> 16), acc[r]);
-                acc[r] = fma((double)wv.z, (double)bf16_bits_to_f32(xr[i].y & 0xFFFFu), acc[r]);
-                acc[r] = fma((double)wv.w, (double)bf16_bits_to_f32(xr[i].y >> 16), acc[r]);
-              }
+          for (int i = 0; i < kRouterChunks; ++i) {
+            const int cc = tg + kGT * i;
+            if (cc < rchunks) {
+              const float4 wv = wr[cc];
+              df_add_prod(c0, wv.x, xv[i][0]);
+              df_add_prod(c1, wv.y, xv[i][1]);
+              df_add_prod(c2, wv.z, xv[i][2]);
+              df_add_prod(c3, wv.w, xv[i][3]);
             }
           }
+          const DF v = df_warp_sum(df_add(df_add(c0, c1), df_add(c2, c3)));
+          if (lane == 0) S.redd[gw][r] = (double)v.hi + (double)v.lo;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.empty[stage]);
-#pragma unroll
-        for (int r = 0; r < kMaxRR; ++r) {
-          if (r < d.nrows) {
-            const double v = warp_sum_f64(acc[r]);
-            if (lane == 0) S.redd[gw][r] = v;
-          }
-        }
         if (tg == 0) TRACE_AT(15);
         if (!group_barrier(&S.gbar[grp], gpar)) {
           if (lane == 0) set_error(p.ctrl, kErrTimeout, 3, 0);
@@ -1000,7 +1064,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     // publish nothing: the instructions of both paths are fetched while the
     // first weights are still on their way, not when they have arrived.
     int warm = (grp == 1 && p.warm) ? 2 : 0;
-    bool tr_gu = false, tr_dn = false;
     uint32_t c = c_first;
     for (uint32_t it = c_first;; ++it) {  // it: group barrier phases used
       if (gabort) break;
@@ -1036,17 +1099,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         break;
       }
       const uint8_t* st = stages + (size_t)stage * kStageBytes;
-      if (!fake && tg == 0) {
-        if (d.type == kGateUp && d.slot == 0 && !tr_gu) {
-          tr_gu = true;
-          TRACE_AT(8 + grp * 5);
-        }
-        if (d.type == kDown && !tr_dn) {
-          tr_dn = true;
-          TRACE_AT(9 + grp * 5);
-        }
-      }
-
       if (d.type == kGateUp) {
         float v[NV_G];
         const size_t rb = (size_t)p.H / 2;
@@ -1179,6 +1231,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     __threadfence();
     const uint32_t old = atomicAdd(p.ctrl + kCtrlExit, 1u);
     S.last_cta = (old + 1 == gridDim.x) ? 1 : 0;
+#ifdef MOE_TRACE
+    // per call (by epoch): the first CTA's start and the last CTA's exit
+    if (p.trace && S.last_cta) {
+      p.trace[gridDim.x * 128 + (epoch & 63) * 2 + 1] = global_timer_ns();
+      p.trace[gridDim.x * 128 + (epoch & 63) * 2 + 0] = p.trace[127];  // CTA 0's start
+    }
+#endif
   }
   __syncthreads();
   if (S.last_cta) {
@@ -1197,21 +1256,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       __threadfence();
     }
   }
-}
-
-DeviceOnce<int> g_num_sms;
-
-int num_sms() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) != cudaSuccess) return n;
-  g_num_sms.get(dev, &n, [dev](int* v) {
-    int m = 0;
-    if (cudaDeviceGetAttribute(&m, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || m <= 0)
-      m = 148;
-    *v = m;
-    return cudaSuccess;
-  });
-  return n;
 }
 
 // The kernel needs all of its CTAs resident at once (selection warps poll

@@ -29,6 +29,7 @@ enum : int {
 
 struct DecodeParams {
   const ExpertPtrs* table;
+  ExpertPtrs shared;  // the shared expert's tensors (entry E of table)
   const float* w_router;
   const float* bias;
   const uint16_t* x;  // bf16 [H] (plain step), or
@@ -55,7 +56,7 @@ struct DecodeParams {
   // down rows: CTA b owns rows [A * (b * nU / grid), A * ((b + 1) * nU / grid))
   // of every slot, nU = H / A, in n_db items of at most RD rows per slot
   int A, nU, n_db, ycta_rows;
-  uint64_t* trace;    // timeline probes of a -DMOE_TRACE build ([grid][32]); else unused
+  uint64_t* trace;    // timeline probes of a -DMOE_TRACE build ([grid][128]); else unused
   // The next layer of a stack (nullable): during this layer's down phase
   // each CTA prefetches into L2 its router rows and a share of the shared
   // expert's gate/up rows, the bytes the next layer's start-up reads first.

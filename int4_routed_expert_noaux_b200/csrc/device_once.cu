@@ -47,4 +47,18 @@ uint64_t current_context_id() {
   return (uint64_t)id;
 }
 
+int num_sms() {
+  static DeviceOnce<int> cache;
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return n;
+  cache.get(dev, &n, [dev](int* v) {
+    int m = 0;
+    if (cudaDeviceGetAttribute(&m, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || m <= 0)
+      m = 148;
+    *v = m;
+    return cudaSuccess;
+  });
+  return n;
+}
+
 }  // namespace moe

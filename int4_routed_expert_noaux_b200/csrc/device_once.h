@@ -24,6 +24,10 @@ constexpr int kMaxDevices = 64;
 // exists); 0 if it cannot be read, which only disables the reset check.
 uint64_t current_context_id();
 
+// SM count of the current device (cached per device and context; 148 if it
+// cannot be read).
+int num_sms();
+
 // One cached value per device.  get() returns the value, running fill(&v)
 // (a cudaError_t-returning callable) under a lock the first time for the
 // current device and context; a failed fill is not cached.

@@ -25,12 +25,13 @@ moe_status ffn_impl(const moe_layer* l, const uint16_t* x, int T, const int32_t*
       l->table, idx, w, x, T, c.hidden, c.inter, c.n_experts, c.top_k, c.n_shared, ws + L.xq,
       reinterpret_cast<float*>(ws + L.xqf), ws + L.hq, reinterpret_cast<float*>(ws + L.hqf),
       reinterpret_cast<int*>(ws + L.lists), reinterpret_cast<float*>(ws + L.hbuf),
-      reinterpret_cast<float*>(ws + L.ypart), y, reinterpret_cast<uint32_t*>(ws + L.ctrl), st);
+      reinterpret_cast<float*>(ws + L.ypart), y, reinterpret_cast<uint32_t*>(ws + L.ctrl),
+      L.tc_bytes ? ws + L.tc : nullptr, reinterpret_cast<int*>(ws + L.tc_exp), st);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "expert launch");
 }
 
 #ifdef MOE_TRACE
-// Timeline buffer of a profiling build (-DMOE_TRACE): [grid][32] uint64.
+// Timeline buffer of a profiling build (-DMOE_TRACE): [grid][128] uint64.
 static uint64_t* g_trace = nullptr;
 extern "C" __attribute__((visibility("default"))) void moe_debug_set_trace(void* buf) {
   g_trace = static_cast<uint64_t*>(buf);
@@ -46,6 +47,7 @@ static moe_status launch_fused(const moe_layer* l, const uint16_t* x, const floa
   if (!decode_plan(l->cfg, p)) return MOE_OK;
   *used = true;
   p.table = l->table;
+  p.shared = l->host_table[l->cfg.n_experts];
   p.w_router = l->w_router;
   p.bias = l->bias;
   p.x = x;

@@ -14,9 +14,9 @@ namespace moe {
 // Router GEMV and sigmoid ("LightLX", "How it works": one router logit per
 // routed expert, sigmoid scores).  One CTA per expert row of W (fp32
 // [E][H]): each thread holds its 16-byte chunks of the row and accumulates
-// them against TT tokens at a time.  Every product of an fp32 weight and a
-// bf16 input is exact in fp64 and the sums are fp64, so the logit is exact
-// to about 1e-13; the sigmoid is taken in fp64 and rounded to fp32 once.
+// them against TT tokens at a time.  The sums are double-float (fp32 pairs,
+// about 48 bits, every product split exactly): the logit is exact to about
+// 1e-14; the sigmoid is taken in fp64 and rounded to fp32 once.
 // scores [T][E] = fp32(sigmoid(logit)).
 
 template <int TT>
@@ -29,26 +29,26 @@ __global__ void __launch_bounds__(256) router_scores_kernel(
   const float4* wr = reinterpret_cast<const float4*>(w + (size_t)e * H);
   const int nchunk = H >> 2;
   for (int t0 = 0; t0 < T; t0 += TT) {
-    double acc[TT];
+    DF acc[TT];
 #pragma unroll
-    for (int t = 0; t < TT; ++t) acc[t] = 0.0;
+    for (int t = 0; t < TT; ++t) acc[t] = DF{0.f, 0.f};
     for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
       const float4 wv = __ldg(wr + c);
 #pragma unroll
       for (int t = 0; t < TT; ++t) {
         if (t0 + t < T) {
           const uint2 xv = __ldg(reinterpret_cast<const uint2*>(x + (size_t)(t0 + t) * H) + c);
-          acc[t] = fma((double)wv.x, (double)bf16_bits_to_f32(xv.x & 0xFFFFu), acc[t]);
-          acc[t] = fma((double)wv.y, (double)bf16_bits_to_f32(xv.x >> 16), acc[t]);
-          acc[t] = fma((double)wv.z, (double)bf16_bits_to_f32(xv.y & 0xFFFFu), acc[t]);
-          acc[t] = fma((double)wv.w, (double)bf16_bits_to_f32(xv.y >> 16), acc[t]);
+          df_add_prod(acc[t], wv.x, bf16_bits_to_f32(xv.x & 0xFFFFu));
+          df_add_prod(acc[t], wv.y, bf16_bits_to_f32(xv.x >> 16));
+          df_add_prod(acc[t], wv.z, bf16_bits_to_f32(xv.y & 0xFFFFu));
+          df_add_prod(acc[t], wv.w, bf16_bits_to_f32(xv.y >> 16));
         }
       }
     }
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
-      const double s = warp_sum_f64(acc[t]);
-      if (lane == 0) red[t][warp] = s;
+      const DF s = df_warp_sum(acc[t]);
+      if (lane == 0) red[t][warp] = (double)s.hi + (double)s.lo;
     }
     __syncthreads();
     if (threadIdx.x < TT && t0 + threadIdx.x < T) {

@@ -18,6 +18,7 @@
 // The group dot product is the exact integer one of the decode kernel
 // (dp2a over int16 inputs); only the order of the fp32 sums differs.
 #include <cuda_runtime.h>
+#include <algorithm>
 #include <stdint.h>
 
 #include "async.cuh"
@@ -78,66 +79,76 @@ __global__ void __launch_bounds__(256) xq_table_kernel(const void* __restrict__ 
 }
 
 // ---------------------------------------------------------------------------
-// lists: [0] U; u_expert [E + 1]; u_off [E + 2]; list_tok [T slots];
-// list_pos [T slots] (pos = t * slots + j: the (token, slot) row of hbuf,
-// ypart).  Out-of-range ids set the error word and are left out.
+// The expert lists of the call (layout: ListsView).  Out-of-range ids set
+// the error word and are left out; -1 (a slot dropped by top-p) is skipped.
 __global__ void __launch_bounds__(256) build_lists_kernel(const int32_t* __restrict__ idx, int T,
-                                                          int k, int E, int has_shared,
+                                                          int k, int E, int has_shared, int tc_on,
                                                           int* __restrict__ lists,
                                                           uint32_t* __restrict__ err) {
   __shared__ int cnt[kListMaxE];
   __shared__ int base[kListMaxE];
   const int slots = k + has_shared;
   const int n_list = T * slots;
-  int* u_expert = lists + 1;
-  int* u_off = u_expert + (E + 1);
-  int* list_tok = u_off + (E + 2);
-  int* list_pos = list_tok + n_list;
+  const ListsView L = lists_view(lists, E, n_list);
+  int* u_expert = const_cast<int*>(L.u_expert);
+  int* u_off = const_cast<int*>(L.u_off);
+  int* list_tok = const_cast<int*>(L.list_tok);
+  int* list_pos = const_cast<int*>(L.list_pos);
+  int* cc_u = const_cast<int*>(L.cc_u);
+  int* tc_u = const_cast<int*>(L.tc_u);
   for (int e = threadIdx.x; e <= E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
   for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
     const int e = idx[i];
     if (e >= 0 && e < E) {
       atomicAdd(&cnt[e], 1);
-    } else if (e != -1) {  // -1: a slot dropped by top-p
+    } else if (e != -1) {
       atomicCAS(err, 0u, (uint32_t)kErrBadExpertId);
     }
   }
   __syncthreads();
   if (threadIdx.x == 0 && has_shared) cnt[E] = T;
   __syncthreads();
-  // exclusive scans of (expert used, entries) over experts 0..E, ascending:
-  // thread i owns experts 2i and 2i + 1 (E + 1 <= 512)
+  // exclusive scans of (expert used, tensor-core expert, entries) over
+  // experts 0..E, ascending: thread i owns experts 2i and 2i + 1 (E + 1 <= 512)
   {
-    __shared__ int wu[8], ws[8];
+    __shared__ int wu[8], wt[8], ws[8];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int e0 = 2 * threadIdx.x, e1 = e0 + 1;
     const int c0 = e0 <= E ? cnt[e0] : 0, c1 = e1 <= E ? cnt[e1] : 0;
-    const int nu = (c0 > 0) + (c1 > 0), ns = c0 + c1;
-    int iu = nu, is = ns;  // inclusive warp scans
+    const bool t0 = tc_on && c0 >= kTcMinTok && c0 <= kTcMaxTok;
+    const bool t1 = tc_on && c1 >= kTcMinTok && c1 <= kTcMaxTok;
+    const int nu = (c0 > 0) + (c1 > 0), nt = (int)t0 + (int)t1, ns = c0 + c1;
+    int iu = nu, it = nt, is = ns;  // inclusive warp scans
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int a = __shfl_up_sync(0xffffffffu, iu, o), b = __shfl_up_sync(0xffffffffu, is, o);
+      const int a = __shfl_up_sync(0xffffffffu, iu, o), b = __shfl_up_sync(0xffffffffu, it, o),
+                c = __shfl_up_sync(0xffffffffu, is, o);
       if (lane >= o) {
         iu += a;
-        is += b;
+        it += b;
+        is += c;
       }
     }
     if (lane == 31) {
       wu[warp] = iu;
+      wt[warp] = it;
       ws[warp] = is;
     }
     __syncthreads();
-    int bu = 0, bs = 0;
+    int bu = 0, bt = 0, bs = 0;
     for (int w = 0; w < warp; ++w) {
       bu += wu[w];
+      bt += wt[w];
       bs += ws[w];
     }
-    int uu = bu + iu - nu, off = bs + is - ns;  // exclusive prefixes
+    int uu = bu + iu - nu, ut = bt + it - nt, off = bs + is - ns;  // exclusive prefixes
     if (c0 > 0) {
       u_expert[uu] = e0;
       u_off[uu] = off;
       base[e0] = off;
+      if (t0) tc_u[ut++] = uu;
+      else cc_u[uu - ut] = uu;
       ++uu;
       off += c0;
     }
@@ -145,11 +156,16 @@ __global__ void __launch_bounds__(256) build_lists_kernel(const int32_t* __restr
       u_expert[uu] = e1;
       u_off[uu] = off;
       base[e1] = off;
+      if (t1) tc_u[ut] = uu;
+      else cc_u[uu - ut] = uu;
     }
     if (threadIdx.x == blockDim.x - 1) {
-      const int U = bu + iu, total = bs + is;
+      const int U = bu + iu, n_tc = bt + it, total = bs + is;
       u_off[U] = total;
       lists[0] = U;
+      int* counts = const_cast<int*>(L.counts);
+      counts[0] = U - n_tc;
+      counts[1] = n_tc;
     }
   }
   __syncthreads();
@@ -238,154 +254,156 @@ __global__ void __launch_bounds__(kUnionThreads) union_gemm_kernel(const UnionAr
   extern __shared__ __align__(16) uint8_t usmem[];
   UStage* st = reinterpret_cast<UStage*>(usmem);
   float(*sO)[RBM][kTok + 1] = reinterpret_cast<float(*)[RBM][kTok + 1]>(usmem + kNS * sizeof(UStage));
-  const int U = a.lists[0];
-  const int u = blockIdx.y;
-  if (u >= U) return;  // uniform per CTA, before any barrier
-  const int* u_expert = a.lists + 1;
-  const int* u_off = u_expert + (a.E + 1);
-  const int* list_tok = u_off + (a.E + 2);
-  const int* list_pos = list_tok + a.n_list;
-  const int* in_idx = a.in_is_pos ? list_pos : list_tok;
-  const int e = u_expert[u];
-  const int base = u_off[u], n = u_off[u + 1] - base;
-  const int row0 = blockIdx.x * RBM;
+  const ListsView L = lists_view(a.lists, a.E, a.n_list);
+  const int* list_pos = L.list_pos;
+  const int* in_idx = a.in_is_pos ? list_pos : L.list_tok;
+  const int nb = (a.R + RBM - 1) / RBM;
+  const int items = L.counts[0] * nb;
   const int tid = threadIdx.x, lane = tid & 31;
-  const int m = (tid >> 5) * 8 + (lane & 7), q = lane >> 3;
-  const int mat = m / RBM, r = m % RBM;
-  const ExpertPtrs ep = a.table[e];
-  const int nk = (a.G + kKB - 1) / kKB;
+  // persistent: work item = (expert of the CUDA-core path, block of rows),
+  // the row blocks of an expert adjacent; the loop bounds are uniform per CTA
+  for (int item = blockIdx.x; item < items; item += gridDim.x) {
+    const int u = L.cc_u[item / nb];
+    const int e = L.u_expert[u];
+    const int base = L.u_off[u], n = L.u_off[u + 1] - base;
+    const int row0 = (item % nb) * RBM;
+    const int m = (tid >> 5) * 8 + (lane & 7), q = lane >> 3;
+    const int mat = m / RBM, r = m % RBM;
+    const ExpertPtrs ep = a.table[e];
+    const int nk = (a.G + kKB - 1) / kKB;
 
-  static_assert(64 * kKB == 4 * kUnionThreads && 64 * kKB / 2 == 2 * kUnionThreads &&
-                    kTok * kKB * 4 == 2 * kUnionThreads && kTok * kKB <= kUnionThreads,
-                "the copy assignment below");
-  // This thread's copies of every k step, as source pointers advanced by the
-  // step: weight chunks (4), scale pairs (2), token input chunks (2) and one
-  // token factor.  Row sources are fixed for the CTA, token sources per pass.
-  const int gw_ = tid & (kKB - 1), gs_ = 2 * (tid & (kKB / 2 - 1));
-  const uint8_t* wsrc[4];
-  bool wok[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int mm = (tid >> 4) + 16 * j, rr = row0 + mm % RBM;
-    const uint8_t* codes = (MATS == 2) ? ((mm / RBM) == 0 ? ep.q_gate : ep.q_up) : ep.q_down;
-    wok[j] = rr < a.R;
-    wsrc[j] = codes + ((size_t)(wok[j] ? rr : row0) * a.G + min(gw_, a.G - 1)) * 16;
-  }
-  const uint16_t* ssrc[2];
-  bool sok[2];
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int mm = (tid >> 3) + 32 * j, rr = row0 + mm % RBM;
-    const uint16_t* sc = (MATS == 2) ? ((mm / RBM) == 0 ? ep.s_gate : ep.s_up) : ep.s_down;
-    sok[j] = rr < a.R;
-    ssrc[j] = sc + (size_t)(sok[j] ? rr : row0) * a.G + min(gs_, a.G - 2);
-  }
-  const int xg_ = (tid >> 2) & (kKB - 1), xw_ = tid & 3;
-  const uint8_t* xsrc[2];
-  bool xok[2];
-  const float* fsrc = a.xq_fac;
-  bool fok = false;
-
-  // a copy that is not needed (row or token past the end, group past the
-  // step) reads nothing (source size 0) from its in-range base pointer
-  auto issue = [&](int sb, int ks) {
-    UStage& S = st[sb];
-    const int kb = ks * kKB, kbn = min(kKB, a.G - kb);
+    static_assert(64 * kKB == 4 * kUnionThreads && 64 * kKB / 2 == 2 * kUnionThreads &&
+                      kTok * kKB * 4 == 2 * kUnionThreads && kTok * kKB <= kUnionThreads,
+                  "the copy assignment below");
+    // This thread's copies of every k step, as source pointers advanced by the
+    // step: weight chunks (4), scale pairs (2), token input chunks (2) and one
+    // token factor.  Row sources are fixed for the CTA, token sources per pass.
+    const int gw_ = tid & (kKB - 1), gs_ = 2 * (tid & (kKB / 2 - 1));
+    const uint8_t* wsrc[4];
+    bool wok[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const bool ok = wok[j] && gw_ < kbn;
-      cp_async16(&S.w[(tid >> 4) + 16 * j][gw_], ok ? wsrc[j] + (size_t)kb * 16 : wsrc[j], ok);
+      const int mm = (tid >> 4) + 16 * j, rr = row0 + mm % RBM;
+      const uint8_t* codes = (MATS == 2) ? ((mm / RBM) == 0 ? ep.q_gate : ep.q_up) : ep.q_down;
+      wok[j] = rr < a.R;
+      wsrc[j] = codes + ((size_t)(wok[j] ? rr : row0) * a.G + min(gw_, a.G - 1)) * 16;
     }
+    const uint16_t* ssrc[2];
+    bool sok[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      const bool ok = sok[j] && gs_ < kbn;
-      cp_async4(&S.s[(tid >> 3) + 32 * j][gs_], ok ? ssrc[j] + kb : ssrc[j], ok);
+      const int mm = (tid >> 3) + 32 * j, rr = row0 + mm % RBM;
+      const uint16_t* sc = (MATS == 2) ? ((mm / RBM) == 0 ? ep.s_gate : ep.s_up) : ep.s_down;
+      sok[j] = rr < a.R;
+      ssrc[j] = sc + (size_t)(sok[j] ? rr : row0) * a.G + min(gs_, a.G - 2);
     }
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const bool ok = xok[j] && xg_ < kbn;
-      cp_async16(&S.x[(tid >> 6) + 4 * j][xg_][xw_], ok ? xsrc[j] + (size_t)kb * 64 : xsrc[j], ok);
-    }
-    if (tid < kTok * kKB) {
-      const bool ok = fok && (tid % kKB) < kbn;
-      cp_async4(&S.f[tid / kKB][tid % kKB], ok ? fsrc + kb : fsrc, ok);
-    }
-  };
+    const int xg_ = (tid >> 2) & (kKB - 1), xw_ = tid & 3;
+    const uint8_t* xsrc[2];
+    bool xok[2];
+    const float* fsrc = a.xq_fac;
+    bool fok = false;
 
-  for (int tc = 0; tc < n; tc += kTok) {
-    const int nt = min(kTok, n - tc);
-    // this pass's token sources
+    // a copy that is not needed (row or token past the end, group past the
+    // step) reads nothing (source size 0) from its in-range base pointer
+    auto issue = [&](int sb, int ks) {
+      UStage& S = st[sb];
+      const int kb = ks * kKB, kbn = min(kKB, a.G - kb);
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int ti = (tid >> 6) + 4 * j;
-      xok[j] = ti < nt;
-      const int rin = in_idx[base + tc + (xok[j] ? ti : 0)];
-      xsrc[j] = a.xq_words + ((size_t)rin * a.G + min(xg_, a.G - 1)) * 64 + xw_ * 16;
-    }
-    if (tid < kTok * kKB) {
-      const int ti = tid / kKB;
-      fok = ti < nt;
-      fsrc = a.xq_fac + (size_t)in_idx[base + tc + (fok ? ti : 0)] * a.G + min(tid % kKB, a.G - 1);
-    }
-    float acc[kTok];
+      for (int j = 0; j < 4; ++j) {
+        const bool ok = wok[j] && gw_ < kbn;
+        cp_async16(&S.w[(tid >> 4) + 16 * j][gw_], ok ? wsrc[j] + (size_t)kb * 16 : wsrc[j], ok);
+      }
 #pragma unroll
-    for (int ti = 0; ti < kTok; ++ti) acc[ti] = 0.f;
+      for (int j = 0; j < 2; ++j) {
+        const bool ok = sok[j] && gs_ < kbn;
+        cp_async4(&S.s[(tid >> 3) + 32 * j][gs_], ok ? ssrc[j] + kb : ssrc[j], ok);
+      }
 #pragma unroll
-    for (int s0 = 0; s0 < kNS - 1; ++s0) {
-      if (s0 < nk) issue(s0, s0);
-      cp_async_commit();
-    }
-    for (int ks = 0; ks < nk; ++ks) {
-      cp_async_wait<kNS - 2>();  // step ks has landed (this thread's copies)
-      __syncthreads();           // ... everyone's; step ks - 1 is no longer read
-      if (ks + kNS - 1 < nk) issue((ks + kNS - 1) % kNS, ks + kNS - 1);
-      cp_async_commit();
-      const UStage& S = st[ks % kNS];
-      const int kbn = min(kKB, a.G - ks * kKB);
+      for (int j = 0; j < 2; ++j) {
+        const bool ok = xok[j] && xg_ < kbn;
+        cp_async16(&S.x[(tid >> 6) + 4 * j][xg_][xw_], ok ? xsrc[j] + (size_t)kb * 64 : xsrc[j], ok);
+      }
+      if (tid < kTok * kKB) {
+        const bool ok = fok && (tid % kKB) < kbn;
+        cp_async4(&S.f[tid / kKB][tid % kKB], ok ? fsrc + kb : fsrc, ok);
+      }
+    };
+
+    for (int tc = 0; tc < n; tc += kTok) {
+      const int nt = min(kTok, n - tc);
+      // this pass's token sources
 #pragma unroll
-      for (int i = 0; i < kKB / 4; ++i) {
-        const int g = 4 * i + q;
-        if (g < kbn) {
-          uint32_t even[4], odd[4];
-          split_chunk(S.w[m][g], even, odd);  // once, for every token
-          const float sc = f16_bits_to_f32(S.s[m][g]);
+      for (int j = 0; j < 2; ++j) {
+        const int ti = (tid >> 6) + 4 * j;
+        xok[j] = ti < nt;
+        const int rin = in_idx[base + tc + (xok[j] ? ti : 0)];
+        xsrc[j] = a.xq_words + ((size_t)rin * a.G + min(xg_, a.G - 1)) * 64 + xw_ * 16;
+      }
+      if (tid < kTok * kKB) {
+        const int ti = tid / kKB;
+        fok = ti < nt;
+        fsrc = a.xq_fac + (size_t)in_idx[base + tc + (fok ? ti : 0)] * a.G + min(tid % kKB, a.G - 1);
+      }
+      float acc[kTok];
 #pragma unroll
-          for (int ti = 0; ti < kTok; ++ti) {
-            if (ti < nt) {
-              XQ xg;
-              const uint4 a0 = S.x[ti][g][0], a1 = S.x[ti][g][1], a2 = S.x[ti][g][2],
-                          a3 = S.x[ti][g][3];
-              xg.ev[0] = a0.x; xg.ev[1] = a0.y; xg.ev[2] = a0.z; xg.ev[3] = a0.w;
-              xg.ev[4] = a1.x; xg.ev[5] = a1.y; xg.ev[6] = a1.z; xg.ev[7] = a1.w;
-              xg.od[0] = a2.x; xg.od[1] = a2.y; xg.od[2] = a2.z; xg.od[3] = a2.w;
-              xg.od[4] = a3.x; xg.od[5] = a3.y; xg.od[6] = a3.z; xg.od[7] = a3.w;
-              xg.f = S.f[ti][g];
-              acc[ti] += (float)dotq_group_split(even, odd, xg) * (sc * xg.f);
+      for (int ti = 0; ti < kTok; ++ti) acc[ti] = 0.f;
+#pragma unroll
+      for (int s0 = 0; s0 < kNS - 1; ++s0) {
+        if (s0 < nk) issue(s0, s0);
+        cp_async_commit();
+      }
+      for (int ks = 0; ks < nk; ++ks) {
+        cp_async_wait<kNS - 2>();  // step ks has landed (this thread's copies)
+        __syncthreads();           // ... everyone's; step ks - 1 is no longer read
+        if (ks + kNS - 1 < nk) issue((ks + kNS - 1) % kNS, ks + kNS - 1);
+        cp_async_commit();
+        const UStage& S = st[ks % kNS];
+        const int kbn = min(kKB, a.G - ks * kKB);
+#pragma unroll
+        for (int i = 0; i < kKB / 4; ++i) {
+          const int g = 4 * i + q;
+          if (g < kbn) {
+            uint32_t even[4], odd[4];
+            split_chunk(S.w[m][g], even, odd);  // once, for every token
+            const float sc = f16_bits_to_f32(S.s[m][g]);
+#pragma unroll
+            for (int ti = 0; ti < kTok; ++ti) {
+              if (ti < nt) {
+                XQ xg;
+                const uint4 a0 = S.x[ti][g][0], a1 = S.x[ti][g][1], a2 = S.x[ti][g][2],
+                            a3 = S.x[ti][g][3];
+                xg.ev[0] = a0.x; xg.ev[1] = a0.y; xg.ev[2] = a0.z; xg.ev[3] = a0.w;
+                xg.ev[4] = a1.x; xg.ev[5] = a1.y; xg.ev[6] = a1.z; xg.ev[7] = a1.w;
+                xg.od[0] = a2.x; xg.od[1] = a2.y; xg.od[2] = a2.z; xg.od[3] = a2.w;
+                xg.od[4] = a3.x; xg.od[5] = a3.y; xg.od[6] = a3.z; xg.od[7] = a3.w;
+                xg.f = S.f[ti][g];
+                acc[ti] += (float)dotq_group_split(even, odd, xg) * (sc * xg.f);
+              }
             }
           }
         }
       }
-    }
-    cp_async_wait<0>();
-    // the four column quarters of a row are lanes l, l + 8, l + 16, l + 24
+      cp_async_wait<0>();
+      // the four column quarters of a row are lanes l, l + 8, l + 16, l + 24
 #pragma unroll
-    for (int ti = 0; ti < kTok; ++ti) {
-      acc[ti] += __shfl_xor_sync(0xffffffffu, acc[ti], 8);
-      acc[ti] += __shfl_xor_sync(0xffffffffu, acc[ti], 16);
-    }
-    if (q == 0) {
-#pragma unroll
-      for (int ti = 0; ti < kTok; ++ti) sO[mat][r][ti] = acc[ti];
-    }
-    __syncthreads();
-    for (int i = tid; i < RBM * nt; i += kUnionThreads) {
-      const int rr = i % RBM, ti = i / RBM;
-      if (row0 + rr < a.R) {
-        const float v = (MATS == 2) ? silu_mul(sO[0][rr][ti], sO[1][rr][ti]) : sO[0][rr][ti];
-        a.out[(size_t)list_pos[base + tc + ti] * a.R + row0 + rr] = v;
+      for (int ti = 0; ti < kTok; ++ti) {
+        acc[ti] += __shfl_xor_sync(0xffffffffu, acc[ti], 8);
+        acc[ti] += __shfl_xor_sync(0xffffffffu, acc[ti], 16);
       }
+      if (q == 0) {
+#pragma unroll
+        for (int ti = 0; ti < kTok; ++ti) sO[mat][r][ti] = acc[ti];
+      }
+      __syncthreads();
+      for (int i = tid; i < RBM * nt; i += kUnionThreads) {
+        const int rr = i % RBM, ti = i / RBM;
+        if (row0 + rr < a.R) {
+          const float v = (MATS == 2) ? silu_mul(sO[0][rr][ti], sO[1][rr][ti]) : sO[0][rr][ti];
+          a.out[(size_t)list_pos[base + tc + ti] * a.R + row0 + rr] = v;
+        }
+      }
+      __syncthreads();  // sO and the stages are rewritten by the next pass
     }
-    __syncthreads();  // sO and the stages are rewritten by the next pass
   }
 }
 
@@ -411,21 +429,22 @@ __global__ void __launch_bounds__(256) union_combine_kernel(
 }  // namespace
 
 size_t union_lists_ints(int T, int k, int E, int has_shared) {
-  return 1 + (size_t)(E + 1) + (E + 2) + 2 * (size_t)T * (k + has_shared);
+  return 1 + (size_t)(E + 1) + (E + 2) + 2 * (size_t)T * (k + has_shared) + 2 + 2 * (size_t)(E + 1);
 }
 
 cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const float* w,
                              const uint16_t* x, int T, int H, int I, int E, int k, int has_shared,
                              uint8_t* xq_words, float* xq_fac, uint8_t* hq_words, float* hq_fac,
                              int* lists, float* hbuf, float* ypart, float* y, uint32_t* err,
-                             cudaStream_t st) {
+                             uint8_t* tc_bpack, int* tc_rowexp, cudaStream_t st) {
   if (E + 1 > kListMaxE) return cudaErrorInvalidValue;
+  const bool tc = tc_bpack && T >= 16 && tc_shape_ok(H, I);
   const int slots = k + has_shared;
   const int G = H / 32, GD = I / 32;
   const int n_list = T * slots;
   const int umax = (E < T * k ? E : T * k) + has_shared;
   xq_table_kernel<true><<<(T * G + 255) / 256, 256, 0, st>>>(x, T, H, xq_words, xq_fac);
-  build_lists_kernel<<<1, 256, 0, st>>>(idx, T, k, E, has_shared, lists, err);
+  build_lists_kernel<<<1, 256, 0, st>>>(idx, T, k, E, has_shared, tc ? 1 : 0, lists, err);
   UnionArgs a;
   a.table = table;
   a.lists = lists;
@@ -437,23 +456,42 @@ cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const 
   a.R = I;
   a.in_is_pos = 0;
   a.out = hbuf;
-  static DeviceOnce<bool> configured;
+  // blocks per SM of union_gemm<2> (low half) and union_gemm<1> (high half)
+  static DeviceOnce<uint32_t> configured;
   int dev = 0;
   cudaError_t ce = cudaGetDevice(&dev);
   if (ce != cudaSuccess) return ce;
-  bool done = false;
-  ce = configured.get(dev, &done, [](bool* v) {
+  uint32_t occ = 0;
+  ce = configured.get(dev, &occ, [](uint32_t* v) {
     cudaError_t r = cudaFuncSetAttribute(union_gemm_kernel<2>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)union_smem_bytes(2));
     if (r == cudaSuccess)
       r = cudaFuncSetAttribute(union_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)union_smem_bytes(1));
-    *v = r == cudaSuccess;
+    int o2 = 0, o1 = 0;
+    if (r == cudaSuccess)
+      r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o2, union_gemm_kernel<2>, kUnionThreads,
+                                                        union_smem_bytes(2));
+    if (r == cudaSuccess)
+      r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o1, union_gemm_kernel<1>, kUnionThreads,
+                                                        union_smem_bytes(1));
+    if (r == cudaSuccess && (o2 < 1 || o1 < 1)) r = cudaErrorInvalidConfiguration;
+    *v = (uint32_t)o2 | ((uint32_t)o1 << 16);
     return r;
   });
   if (ce != cudaSuccess) return ce;
-  union_gemm_kernel<2><<<dim3((I + 31) / 32, umax), kUnionThreads, union_smem_bytes(2), st>>>(a);
+  // persistent grids: at most one wave, and no more CTAs than work items
+  const int sms = num_sms();
+  const int nb2 = (I + 31) / 32, nb1 = (H + 63) / 64;
+  const int grid2 = std::min((int)(occ & 0xFFFFu) * sms, umax * nb2);
+  const int grid1 = std::min((int)(occ >> 16) * sms, umax * nb1);
+  union_gemm_kernel<2><<<grid2, kUnionThreads, union_smem_bytes(2), st>>>(a);
+  if (tc) {
+    const cudaError_t e = launch_tc_ffn_step(2, table, lists, E, n_list, T, k, has_shared, x, H,
+                                             I, T, tc_rowexp, tc_bpack, hbuf, err, st);
+    if (e != cudaSuccess) return e;
+  }
   xq_table_kernel<false><<<(n_list * GD + 255) / 256, 256, 0, st>>>(hbuf, n_list, I, hq_words,
                                                                     hq_fac);
   a.xq_words = hq_words;
@@ -462,7 +500,12 @@ cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const 
   a.R = H;
   a.in_is_pos = 1;
   a.out = ypart;
-  union_gemm_kernel<1><<<dim3((H + 63) / 64, umax), kUnionThreads, union_smem_bytes(1), st>>>(a);
+  union_gemm_kernel<1><<<grid1, kUnionThreads, union_smem_bytes(1), st>>>(a);
+  if (tc) {
+    const cudaError_t e = launch_tc_ffn_step(1, table, lists, E, n_list, T, k, has_shared, hbuf,
+                                             I, H, n_list, tc_rowexp, tc_bpack, ypart, err, st);
+    if (e != cudaSuccess) return e;
+  }
   union_combine_kernel<<<dim3((H + 255) / 256, T), 256, 0, st>>>(idx, w, ypart, T, H, k, E,
                                                                  has_shared, y);
   return cudaGetLastError();

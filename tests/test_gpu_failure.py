@@ -13,9 +13,9 @@ from test_gpu_parity import get_layer, to_dev_bf16  # noqa: E402
 pytestmark = pytest.mark.gpu
 
 # Tiny layer (hidden 256, inter 128, top-2 + shared): a gate/up item covers
-# 96 rows of inter, so each slot has 2 gate/up items and the fused kernel's
-# dynamic tickets start with 2 shared + 2 * 2 routed gate/up tickets.
-TINY_GATE_UP_TICKETS = 6
+# 96 rows of inter, so each slot has 2 gate/up items: 2 shared + 2 * 2 routed
+# gate/up items in all.
+TINY_GATE_UP_ITEMS = 6
 
 
 def test_wait_runs_out_and_reports_timeout():
@@ -29,10 +29,10 @@ def test_wait_runs_out_and_reports_timeout():
     moe.ws_check(ws_ref)
 
     ws = moe.alloc_workspace(cfg, 1)
-    # the ticket counter starts past every gate/up item: producers claim down
-    # items whose h is never published, and wait for it (a count nothing
-    # raises) until the limit
-    ws[:4096].view(torch.int32)[1] = TINY_GATE_UP_TICKETS
+    # control word 1 offsets the first gate/up item of every CTA: past the
+    # last one, the producers go on to down items whose h is never
+    # published, and wait for it (a count nothing raises) until the limit
+    ws[:4096].view(torch.int32)[1] = TINY_GATE_UP_ITEMS
     y = torch.zeros((1, shape.hidden), dtype=torch.float32, device="cuda")
     L.forward(x, y, ws)
     with pytest.raises(moe.MoeError) as e:
@@ -40,7 +40,7 @@ def test_wait_runs_out_and_reports_timeout():
     assert moe.STATUS_NAMES[e.value.status] == "MOE_ERR_TIMEOUT"
     words = ws[:4096].view(torch.int32).cpu().numpy()
     assert words[0] == 0  # cleared by ws_check
-    assert words[1] == 0  # the ticket counter was reset on the way out
+    assert words[1] == 0  # the offset word was reset on the way out
     # the same workspace serves the next call normally
     y2 = torch.empty_like(y_ref)
     L.forward(x, y2, ws)
