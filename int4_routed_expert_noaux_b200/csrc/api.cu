@@ -128,12 +128,14 @@ WsLayout ws_layout(const moe_config* c, int T) {
   off = align_up(off + (size_t)T * slots * (c->inter / 32) * 4, 256);
   L.lists = off;
   off = align_up(off + union_lists_ints(T, k, c->n_experts, c->n_shared) * 4, 256);
-  // packed inputs of the tensor-core path (calls of 16 tokens or more)
+  // packed inputs and tensor-map slots of the tensor-core path
   L.tc = off;
   L.tc_bytes = tc_bpack_bytes(T, k, c->n_shared, c->hidden, c->inter);
   off = align_up(off + L.tc_bytes, 256);
   L.tc_exp = off;
   if (L.tc_bytes) off = align_up(off + tc_rowexp_ints(T, k, c->n_shared) * 4, 256);
+  L.tc_maps = off;
+  if (L.tc_bytes) off = align_up(off + tc_maps_bytes(), 256);
   L.total = off;
   return L;
 }

@@ -26,7 +26,8 @@ moe_status ffn_impl(const moe_layer* l, const uint16_t* x, int T, const int32_t*
       reinterpret_cast<float*>(ws + L.xqf), ws + L.hq, reinterpret_cast<float*>(ws + L.hqf),
       reinterpret_cast<int*>(ws + L.lists), reinterpret_cast<float*>(ws + L.hbuf),
       reinterpret_cast<float*>(ws + L.ypart), y, reinterpret_cast<uint32_t*>(ws + L.ctrl),
-      L.tc_bytes ? ws + L.tc : nullptr, reinterpret_cast<int*>(ws + L.tc_exp), st);
+      L.tc_bytes ? ws + L.tc : nullptr, reinterpret_cast<int*>(ws + L.tc_exp),
+      L.tc_bytes ? ws + L.tc_maps : nullptr, st);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "expert launch");
 }
 

@@ -13,11 +13,12 @@ namespace moe {
 // ---------------------------------------------------------------------------
 // Router GEMV and sigmoid ("LightLX", "How it works": one router logit per
 // routed expert, sigmoid scores).  One CTA per expert row of W (fp32
-// [E][H]): each thread holds its 16-byte chunks of the row and accumulates
-// them against TT tokens at a time.  The sums are double-float (fp32 pairs,
-// about 48 bits, every product split exactly): the logit is exact to about
-// 1e-14; the sigmoid is taken in fp64 and rounded to fp32 once.
-// scores [T][E] = fp32(sigmoid(logit)).
+// [E][H]): each thread takes 8-input chunks of the row (the row's chunk c
+// and the tokens' chunk c) and accumulates them against TT tokens at a
+// time in fp64: every product of an fp32 weight and a bf16 input is exact
+// in fp64 (32 significant bits), so the logit carries only the fp64
+// rounding of the sums (about 1e-16 relative); the sigmoid is taken in fp64
+// and rounded to fp32 once.  scores [T][E] = fp32(sigmoid(logit)).
 
 template <int TT>
 __global__ void __launch_bounds__(256) router_scores_kernel(
@@ -27,28 +28,31 @@ __global__ void __launch_bounds__(256) router_scores_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x;
   const float4* wr = reinterpret_cast<const float4*>(w + (size_t)e * H);
-  const int nchunk = H >> 2;
+  const int nchunk = H >> 3;
   for (int t0 = 0; t0 < T; t0 += TT) {
-    DF acc[TT];
+    double acc[TT];
 #pragma unroll
-    for (int t = 0; t < TT; ++t) acc[t] = DF{0.f, 0.f};
+    for (int t = 0; t < TT; ++t) acc[t] = 0.0;
     for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
-      const float4 wv = __ldg(wr + c);
+      const float4 wa = __ldg(wr + 2 * c), wb = __ldg(wr + 2 * c + 1);
+      const double wd[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
       for (int t = 0; t < TT; ++t) {
         if (t0 + t < T) {
-          const uint2 xv = __ldg(reinterpret_cast<const uint2*>(x + (size_t)(t0 + t) * H) + c);
-          df_add_prod(acc[t], wv.x, bf16_bits_to_f32(xv.x & 0xFFFFu));
-          df_add_prod(acc[t], wv.y, bf16_bits_to_f32(xv.x >> 16));
-          df_add_prod(acc[t], wv.z, bf16_bits_to_f32(xv.y & 0xFFFFu));
-          df_add_prod(acc[t], wv.w, bf16_bits_to_f32(xv.y >> 16));
+          const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + t) * H) + c);
+          const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            acc[t] = fma(wd[2 * j], (double)bf16_bits_to_f32(xs[j] & 0xFFFFu), acc[t]);
+            acc[t] = fma(wd[2 * j + 1], (double)bf16_bits_to_f32(xs[j] >> 16), acc[t]);
+          }
         }
       }
     }
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
-      const DF s = df_warp_sum(acc[t]);
-      if (lane == 0) red[t][warp] = (double)s.hi + (double)s.lo;
+      const double s = warp_sum_f64(acc[t]);
+      if (lane == 0) red[t][warp] = s;
     }
     __syncthreads();
     if (threadIdx.x < TT && t0 + threadIdx.x < T) {

@@ -23,16 +23,21 @@ cudaError_t launch_select(const float* scores, const float* bias, int T, int E, 
 // lists (union_lists_ints ints), hbuf (T * slots * I), ypart (T * slots * H).
 size_t union_lists_ints(int T, int k, int E, int has_shared);
 
-// Distinct experts with kTcMinTok..kTcMaxTok tokens take the tensor-core
-// path when it is on.
-constexpr int kTcMinTok = 16, kTcMaxTok = 64;
+// Distinct experts with tc_min_tokens()..kTcMaxTok tokens take the
+// tensor-core path when it is on (16 tokens at least: below that the
+// contraction is too thin for the tensor cores to pay); the workspace holds
+// the packed inputs for any threshold down to kTcMinTokFloor.
+constexpr int kTcMinTokFloor = 16, kTcMaxTok = 64, kTcMinTokDefault = 16;
+int tc_min_tokens();
 
 // The per-call expert lists (build_lists_kernel), ints:
 //   [0] U (distinct experts, the shared one last); u_expert [E + 1];
 //   u_off [E + 2] (entries of expert slot u: u_off[u] .. u_off[u + 1]);
 //   list_tok [n_list], list_pos [n_list] (token and (token, slot) row of
 //   each entry); n_cc, n_tc; cc_u [E + 1], tc_u [E + 1] (the expert slots of
-//   the CUDA-core and of the tensor-core path, ascending).
+//   the CUDA-core and of the tensor-core path, ascending); tc_roff [E + 2]
+//   (first packed input row of each tensor-core expert: its token count
+//   rounded up to 16, summed over the ones before it).
 struct ListsView {
   const int* u_expert;
   const int* u_off;
@@ -41,6 +46,7 @@ struct ListsView {
   const int* counts;  // [0] n_cc, [1] n_tc
   const int* cc_u;
   const int* tc_u;
+  const int* tc_roff;
 };
 
 __host__ __device__ __forceinline__ ListsView lists_view(const int* lists, int E, int n_list) {
@@ -52,26 +58,30 @@ __host__ __device__ __forceinline__ ListsView lists_view(const int* lists, int E
   v.counts = v.list_pos + n_list;
   v.cc_u = v.counts + 2;
   v.tc_u = v.cc_u + (E + 1);
+  v.tc_roff = v.tc_u + (E + 1);
   return v;
 }
 // tc_bpack (nullable, tc_bpack_bytes(T, k, has_shared, H, I) bytes): the
 // packed inputs of the tensor-core path (tc_union.cu), taken by every
-// distinct expert with 16 to 64 tokens when the shape allows it; the other
-// experts run on the CUDA-core union kernels.
+// distinct expert with tc_min_tokens() to 64 tokens when the shape allows
+// it; the other experts run on the CUDA-core union kernels.  tc_maps
+// (tc_maps_bytes(), 128-byte aligned): the path's tensor-map slots.
 cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const float* w,
                              const uint16_t* x, int T, int H, int I, int E, int k, int has_shared,
                              uint8_t* xq_words, float* xq_fac, uint8_t* hq_words, float* hq_fac,
                              int* lists, float* hbuf, float* ypart, float* y, uint32_t* err,
-                             uint8_t* tc_bpack, int* tc_rowexp, cudaStream_t st);
+                             uint8_t* tc_bpack, int* tc_rowexp, uint8_t* tc_maps,
+                             cudaStream_t st);
 // The tensor-core path (tc_union.cu): packed inputs and per-row exponents.
 size_t tc_bpack_bytes(int T, int k, int has_shared, int H, int I);
 size_t tc_rowexp_ints(int T, int k, int has_shared);
 bool tc_shape_ok(int H, int I);
 int tc_max_experts(int T, int k, int has_shared);
+size_t tc_maps_bytes();
 cudaError_t launch_tc_ffn_step(int mats, const ExpertPtrs* table, const int* lists, int E,
                                int n_list, int T, int k, int has_shared, const void* in, int K,
-                               int R, int in_rows, int* row_exp, uint8_t* bpack, float* out,
-                               uint32_t* err, cudaStream_t st);
+                               int R, int in_rows, int* row_exp, uint8_t* bpack, uint8_t* maps,
+                               float* out, uint32_t* err, cudaStream_t st);
 
 cudaError_t launch_gemv_int4(const uint8_t* q, const uint16_t* s, int rows, int cols,
                              const float* x, float* y, cudaStream_t st);

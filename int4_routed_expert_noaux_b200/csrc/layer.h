@@ -26,7 +26,8 @@ constexpr int kMaxTokens = 64;
 
 // Byte offsets inside a workspace.
 struct WsLayout {
-  size_t ctrl, records, logits, idx, w, hbuf, ypart, xq, xqf, hq, hqf, lists, tc, tc_bytes, tc_exp, total;
+  size_t ctrl, records, logits, idx, w, hbuf, ypart, xq, xqf, hq, hqf, lists, tc, tc_bytes, tc_exp,
+      tc_maps, total;
 };
 
 WsLayout ws_layout(const moe_config* c, int T);

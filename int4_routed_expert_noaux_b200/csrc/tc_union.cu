@@ -1,40 +1,50 @@
 // tc_union.cu -- the batched (verify) expert path on the 5th-generation
-// tensor cores, for every distinct expert that 16 to 64 of the call's
-// tokens route to: each expert's weights stream from HBM once for all its
-// tokens (colibri summary, "Principales fonctionnalites implementees":
-// batch-union of the experts of the draft tokens; "LightLX", "How it
-// works": the MTP verify step), and the products run as tcgen05 MMAs.
+// tensor cores, for every distinct expert that a few (tc_min_tokens()) to
+// 64 of the call's tokens route to: each expert's weights stream from HBM
+// once for all its tokens (colibri summary, "Principales fonctionnalites
+// implementees": batch-union of the experts of the draft tokens; "LightLX",
+// "How it works": the MTP verify step), and the products run as tcgen05
+// MMAs.
 //
-// Per (expert, tile of 128 weight rows) one CTA.  Two converter warpgroups
-// split the 32-input scale groups of the K range in halves, one thread per
-// weight row (= tensor-memory lane):
-//   - the thread's row of int4 codes and fp16 scales comes into shared
-//     memory by cp.async, kWS stages of two groups ahead, and only that
-//     thread reads it back;
-//   - it forms the group's 32 weights code * scale as an fp16 pair hi + lo
-//     (hi = fp16(code * scale) rounded, lo = code * scale - hi exactly: an
-//     fma of fp16 values whose exact result has at most 4 significant bits),
-//     so hi + lo is the weight to about 2^-22, and stores the 32 hi and 32
-//     lo halves to a slot of a ring of A operands in tensor memory;
-//   - a producer thread brings each group's packed token inputs (B operand,
-//     fp16, K-major canonical layout; the down projection's h as fp16 hi and
-//     lo tiles) into a ring of shared-memory slots by bulk async copies;
-//   - an issuer thread runs per group the M=128 K=16 fp16 MMAs A_hi B and
-//     A_lo B (and A_hi B_lo for the down projection) for both K halves into
-//     its warpgroup's fp32 accumulator in tensor memory, which holds the
-//     whole K range: no per-group epilogue; one commit per group frees the
-//     group's ring slot.
-// At the end each warpgroup's accumulator is read back (tcgen05.ld) and the
-// two are added in a fixed order through shared memory; gate/up tiles hold
-// 64 gate and 64 up rows of the same indices, so h = silu(g) * u is formed
-// in the tile.
+// A persistent CTA per SM takes (expert, tile of 128 weight rows) work items
+// in turn.  Per CTA:
+//   - a weight producer warp points the item's tensor maps at the expert's
+//     matrices (tensormap.replace on a copy of a template, published to a
+//     per-CTA global slot) and streams the tile's int4 codes and fp16
+//     scales with 2-D TMA loads: 128 rows x 8 groups per stage, codes
+//     128-byte swizzled so that each thread's row reads without bank
+//     conflicts;
+//   - two converter warpgroups split the 32-input groups of the K range in
+//     halves, one thread per weight row (= tensor-memory lane); a thread
+//     forms the group's 32 weights code * scale as an fp16 pair hi + lo,
+//     both exact (the scale split into its top 7 and low 4 significant
+//     bits, each times a 4-bit code), so hi + lo is the weight exactly, and
+//     stores the 32 hi and 32 lo halves to a slot of a ring of A operands
+//     in tensor memory;
+//   - an input producer warp brings each group's packed token inputs (B
+//     operand, fp16, K-major canonical layout; the down projection's h as
+//     fp16 hi and lo tiles) into a ring of shared-memory slots by bulk
+//     async copies;
+//   - four issuer warps (one thread each, taking the groups in turn) run per
+//     group the M=128 K=16 fp16 MMAs A_hi B and A_lo B (and A_hi B_lo for
+//     the down projection) for both K halves into the issuer's fp32
+//     accumulator in tensor memory, which holds its share of the whole K
+//     range: no per-group epilogue; one commit per group frees the group's
+//     ring slot.
+// At the end of an item the four accumulators are read back (tcgen05.ld)
+// and added in a fixed order; gate/up tiles hold 64 gate and 64 up rows of
+// the same indices, interleaved by 16 so that a warp holds both rows of an
+// index, and h = silu(g) * u is formed in the tile.
 //
 // Within a group the MMA's K order is a fixed permutation of the 32 inputs
 // (the order the nibble pairs come out of a word); the packed inputs use the
-// same permutation (tc_perm).
+// same permutation.
+#include <cuda.h>
 #include <cuda_runtime.h>
-#include <algorithm>
 #include <stdint.h>
+
+#include <algorithm>
+#include <atomic>
 
 #include "async.cuh"
 #include "common.cuh"
@@ -45,55 +55,74 @@ namespace moe {
 
 namespace {
 
-// Per-step timeline of CTA 0's first work item in a -DMOE_TRACE profiling
+// Per-step timeline of CTA 0's second work item in a -DMOE_TRACE profiling
 // build (row 7: the end of each of CTA 0's items).
 #ifdef MOE_TRACE
-__device__ uint64_t g_tc_trace[8][256];
+__device__ uint64_t g_tc_trace[14][256];
 #define TC_TRACE(kind, st)                                                          \
   do {                                                                              \
-    if (blockIdx.x == 0 && it == 0 && (st) < 256)                                   \
+    if (blockIdx.x == 0 && it == 1 && (st) < 256)                                   \
       g_tc_trace[kind][st] = (uint64_t)clock64();                                   \
   } while (0)
+#define TC_TRACE_AT(kind, i) (g_tc_trace[kind][i] = (uint64_t)clock64())
 #define TC_TRACE_ITEM()                                                             \
   do {                                                                              \
     if (blockIdx.x == 0 && it < 256) g_tc_trace[7][it] = (uint64_t)clock64();       \
   } while (0)
 #else
 #define TC_TRACE(kind, st) ((void)0)
+#define TC_TRACE_AT(kind, i) ((void)0)
 #define TC_TRACE_ITEM() ((void)0)
 #endif
 
 constexpr int kWG = 2;                    // converter warpgroups (K halves)
 constexpr int kConvThreads = kWG * 128;
-constexpr int kTcThreads = kConvThreads + 32;  // + one warp: B producer (lane 0), issuer (lane 1)
-constexpr int kWS = 8;                    // code stages per warpgroup (2 groups each)
-constexpr int kR = 12;                    // ring slots (A in tensor memory, B in shared memory)
+// + six warps, separate so that one's waits (nanosleep back-off) never
+// hold up another's issue.  Four MMA issuers: a thread stalls about 90
+// cycles on each tcgen05.mma it issues (and more on its commit), while the
+// tensor cores finish an M=128 N<=64 K=16 MMA in about 45, so issuer j
+// takes the ring steps st = j (mod 4) -- warpgroup j % 2's groups -- into an
+// accumulator of its own.
+constexpr int kWProdWarp = kConvThreads / 32;  // weight tiles (TMA), tensor maps
+constexpr int kBProdWarp = kWProdWarp + 1;     // packed inputs
+constexpr int kIssueWarp = kWProdWarp + 2;     // MMA issuer j: warp kIssueWarp + j
+constexpr int kIssuers = 2 * kWG;
+constexpr int kTcThreads = kConvThreads + 32 * (2 + kIssuers);
+constexpr int kGS = 8;                    // groups per weight stage: 128 bytes of codes a row
+constexpr int kSW = 3;                    // weight stages per warpgroup
+constexpr int kR = 8;                     // ring slots (A in tensor memory, B in shared memory)
 constexpr int kNmax = 64;                 // most tokens per expert on this path
-constexpr int kColD = 0;                  // tensor memory: D of warpgroup w at w * kNmax
-constexpr int kColA = kWG * kNmax;        // then kR slots of 32 columns (hi 16, lo 16)
+constexpr int kColD = 0;                  // tensor memory: D of issuer j at j * kNmax
+constexpr int kColA = kIssuers * kNmax;   // then kR slots of 32 columns (hi 16, lo 16)
+constexpr int kMaps = 4;                  // tensor maps of an item (codes, scales) x matrices
+constexpr int kMapSets = 4;               // map sets per CTA, used by items in turn
+constexpr int kTcMaxCtas = 256;           // per-CTA tensor-map slots in the workspace
+static_assert(kMapSets - 1 >= 3, "a map set outlives the loads through it");
+constexpr uint32_t kWStageBytes = 128 * 128 + 128 * 16;
 constexpr uint64_t kTcWaitNs = 1000000000ull;
 static_assert(kColA + kR * 32 <= 512, "tensor memory columns");
+static_assert(kTcMaxTok == kNmax, "the token bound of the path");
 
-struct TcSmem {
-  uint4 w[kWG][kWS][128][2];              // codes: [wg][stage][row][group of the pair]
-  uint32_t sc[kWG][kWS][128];             // the two groups' fp16 scales
-  uint8_t b[kR][kNmax * 64 * 2];          // B of one group (down: hi then lo)
+struct __align__(1024) TcSmem {
+  uint8_t wc[kWG][kSW][128 * 128];        // code tiles: 128 rows x 8 groups, 128-byte swizzled
+  uint8_t wsc[kWG][kSW][128 * 16];        // scale tiles: 128 rows x 8 fp16
+  uint8_t b[kR][kNmax * 128];             // packed inputs of one group (down: hi then lo)
+  CUtensorMap tm[kMaps];                  // the item's tensor maps, before publishing
+  uint64_t w_full[kWG][kSW];              // a weight stage landed
+  uint64_t w_empty[kWG][kSW];             // the warpgroup's 4 warps read it
   uint64_t a_full[kR];                    // converters wrote the slot's A (4 warps)
   uint64_t b_full[kR];                    // the slot's B landed
   uint64_t slot_free[kR];                 // the MMAs reading the slot finished
-  uint64_t fin;                           // all MMAs finished
+  uint64_t fin;                           // all MMAs of the item finished (4 issuers)
+  uint64_t d_free;                        // the item's accumulators were read (8 warps)
   uint32_t tmem_base;
   int abort_flag;
 };
-static_assert(sizeof(uint4) * kWG * kWS * 128 * 2 >= sizeof(float) * kWG * 128 * kNmax,
-              "the partial sums reuse the code stages");
+static_assert(sizeof(TcSmem) + 1024 <= 232448, "shared memory per CTA");
 
-// MMA-K index k of a group holds input tc_perm(k): the converter makes the
-// pair of TMEM column 4i + j from nibbles j and j + 4 of word i.
-__device__ __forceinline__ int tc_perm(int k) {
-  const int i = k >> 3, r = k & 7;
-  return 8 * i + (r >> 1) + 4 * (r & 1);
-}
+// The MMA-K order of a group's 32 inputs: K index 8 i + 2 j + h holds input
+// 8 i + j + 4 h (the converter makes the pair of TMEM column 4 i + j from
+// nibbles j and j + 4 of word i; tc_pack_kernel packs the inputs alike).
 
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   // canonical K-major layout without swizzle: LBO = byte distance of core
@@ -142,57 +171,87 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&v)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                 "=r"(v[6]), "=r"(v[7])
+               : "r"(taddr)
+               : "memory");
+}
+
+// 2-D tiled TMA load of box (x, y) of a tensor map in global memory.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar, uint64_t policy) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-      "%15}, [%16];"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-        "=r"(v[14]), "=r"(v[15])
-      : "r"(taddr)
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
       : "memory");
 }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
+// Tensor-map updates: the global address of a map held in shared memory;
+// its copy to global memory with a release of the tensormap proxy (whole
+// warp); the acquire before the first load through it.
+__device__ __forceinline__ void tmap_set_address(CUtensorMap* smem_map, const void* addr) {
+  asm volatile("tensormap.replace.tile.global_address.shared::cta.b1024.b64 [%0], %1;" ::"r"(
+                   smem_addr(smem_map)),
+               "l"(addr)
                : "memory");
 }
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src)
+__device__ __forceinline__ void tmap_publish(CUtensorMap* gmem_map, const CUtensorMap* smem_map) {
+  asm volatile(
+      "tensormap.cp_fenceproxy.global.shared::cta.tensormap::generic.release.gpu.sync.aligned"
+      " [%0], [%1], 128;" ::"l"(gmem_map),
+      "r"(smem_addr(smem_map))
+      : "memory");
+}
+__device__ __forceinline__ void tmap_acquire(const CUtensorMap* gmem_map) {
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(gmem_map)
                : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// The 32 weights of one 16-byte chunk times its fp16 scale s2 (both halves)
-// as fp16 pairs: hi[4i + j] holds the weights of nibbles j and j + 4 of
-// word i rounded to fp16, lo[4i + j] the exact remainders.
-__device__ __forceinline__ void weights_hi_lo(const uint4 w, uint32_t s2, uint32_t (&hl)[32]) {
+// A group's fp16 scale s split for weights_hi_lo, as f16x2 pairs (both
+// halves equal): s_hi = s with its 4 low mantissa bits cleared (at most 7
+// significant bits), s_lo = s - s_hi (at most 4), and -24 times each (exact:
+// 24 has 2 significant bits).
+struct GroupScale {
+  uint32_t s1, s2, c1, c2;
+};
+
+__device__ __forceinline__ GroupScale group_scale(uint32_t sh) {
+  GroupScale g;
+  const uint32_t s = sh | (sh << 16);
+  g.s1 = s & 0xFFF0FFF0u;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(g.s2) : "r"(s), "r"(g.s1));
+  asm("{ .reg .b32 m; mov.b32 m, 0xCE00CE00; mul.rn.f16x2 %0, %1, m; }" : "=r"(g.c1) : "r"(g.s1));
+  asm("{ .reg .b32 m; mov.b32 m, 0xCE00CE00; mul.rn.f16x2 %0, %1, m; }" : "=r"(g.c2) : "r"(g.s2));
+  return g;
+}
+
+// The 32 weights code * s of one 16-byte chunk as fp16 pairs: hi[4i + j]
+// holds code * s_hi of nibbles j and j + 4 of word i, lo[4i + j] code * s_lo.
+// Both products are exact in fp16 (a code of at most 4 significant bits
+// times 7 or 4), so hi + lo = code * s.  Each is one fma on v = fp16(16 + u),
+// u = nibble ^ 8 = code + 8 (a shift and one bit operation put u in the
+// mantissa under the exponent of 16): v * s_x - 24 * s_x = code * s_x.
+__device__ __forceinline__ void weights_hi_lo(const uint4 w, const GroupScale& gs,
+                                              uint32_t (&hl)[32]) {
   const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      // fp16(1024 + (n ^ 8)) in both halves, minus 1032: the exact code
-      const uint32_t v = ((ws[i] >> (4 * j)) & 0x000F000Fu) ^ 0x64086408u;
-      uint32_t q, hi, lo;
-      asm("{ .reg .b32 c; mov.b32 c, 0x64086408; sub.rn.f16x2 %0, %1, c; }" : "=r"(q) : "r"(v));
-      asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(q), "r"(s2));
-      asm("{ .reg .b32 n; xor.b32 n, %3, 0x80008000; fma.rn.f16x2 %0, %1, %2, n; }"
-          : "=r"(lo)
-          : "r"(q), "r"(s2), "r"(hi));
+      // nibbles j and j + 4 to bits 6..9 of their halves
+      const uint32_t t = j < 2 ? ws[i] << (6 - 4 * j) : ws[i] >> (4 * j - 6);
+      const uint32_t v = (t & 0x03C003C0u) ^ 0x4E004E00u;
+      uint32_t hi, lo;
+      asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(hi) : "r"(v), "r"(gs.s1), "r"(gs.c1));
+      asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(lo) : "r"(v), "r"(gs.s2), "r"(gs.c2));
       hl[4 * i + j] = hi;
       hl[16 + 4 * i + j] = lo;
     }
   }
 }
-
-static_assert(kTcMaxTok == kNmax, "the token bound of the path");
 
 struct TcArgs {
   const ExpertPtrs* table;
@@ -201,37 +260,63 @@ struct TcArgs {
   int K, G;          // inputs of a weight row and its 32-input groups
   int R;             // rows of one weight matrix
   int mats;          // 2: gate/up tiles (64 + 64 rows), 1: down tiles (128 rows)
-  const uint8_t* bpack;  // packed B per path expert: [rank][G][B bytes of a group at kNmax]
+  const uint8_t* bpack;  // packed B: expert rank r from row tc_roff[r], [G][its rows][64 or 128 B]
   const int* row_exp;    // power-of-two scale of each input row (tc_rowscale_kernel)
   float* out;        // [T slots][R] (h for gate/up, partial y for down)
   uint32_t* err;     // kErrTimeout when a wait ran out
+  CUtensorMap* maps; // [grid][kMapSets][kMaps] global slots for the tensor maps
 };
 
-__host__ __device__ __forceinline__ size_t tc_group_bytes(int mats) {
-  return (size_t)kNmax * 64 * (mats == 2 ? 1 : 2);
+// Waits (bounded) in lane 0 and makes every lane an observer of the phase:
+// false (the same in all lanes) when the wait ran out.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int lane,
+                                          volatile int* abort_flag) {
+  int ok = 0;
+  if (lane == 0 && !*abort_flag) {
+    ok = mbar_wait(bar, parity, kTcWaitNs) ? 1 : 0;
+    if (!ok) *abort_flag = 1;
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) mbar_test(bar, parity);
+  return ok != 0;
 }
 
-__global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const TcArgs a) {
-  extern __shared__ __align__(1024) uint8_t tsmem[];
-  TcSmem& S = *reinterpret_cast<TcSmem*>(tsmem);
+// tm_codes / tm_scales: templates of the item's maps (dimensions, strides,
+// boxes: codes uint8 [R][K/2], box 128 bytes x tile rows, 128-byte swizzle;
+// scales uint16 [R][G], box 8 x tile rows); each item points copies of them
+// at its expert's matrices.
+__global__ void __launch_bounds__(kTcThreads, 1)
+    tc_gemm_kernel(const TcArgs a, const __grid_constant__ CUtensorMap tm_codes,
+                   const __grid_constant__ CUtensorMap tm_scales) {
+  extern __shared__ uint8_t tsmem_raw[];
+  // 1024-byte alignment for the swizzled code tiles
+  TcSmem& S = *reinterpret_cast<TcSmem*>(tsmem_raw + ((1024u - (smem_addr(tsmem_raw) & 1023u)) & 1023u));
   const ListsView L = lists_view(a.lists, a.E, a.n_list);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile_rows = a.mats == 2 ? 64 : 128;
   const int tiles = a.R / tile_rows;
   const int items = L.counts[1] * tiles;
   if ((int)blockIdx.x >= items) return;  // uniform per CTA, before any barrier
-  const int ng = a.G / kWG;              // groups per warpgroup (G % 4 == 0)
+  const int ng = a.G / kWG;              // groups per warpgroup (a multiple of kGS)
+  const int nst = ng / kGS;              // weight stages per warpgroup and item
   const int steps = kWG * ng;            // step s of an item: warpgroup s % kWG, its group s / kWG
-  const size_t gbytes = tc_group_bytes(a.mats);
+  const int mb = a.mats == 2 ? 64 : 128;  // bytes of a packed input row of one group
+  const int nmaps = a.mats == 2 ? 4 : 2;
   volatile int* abort_flag = &S.abort_flag;
 
   if (tid == 0) {
+    for (int w = 0; w < kWG; ++w)
+      for (int s = 0; s < kSW; ++s) {
+        mbar_init(&S.w_full[w][s], 1);
+        mbar_init(&S.w_empty[w][s], 4);
+      }
     for (int i = 0; i < kR; ++i) {
       mbar_init(&S.a_full[i], 4);
       mbar_init(&S.b_full[i], 1);
       mbar_init(&S.slot_free[i], 1);
     }
-    mbar_init(&S.fin, 1);
+    mbar_init(&S.fin, kIssuers);
+    mbar_init(&S.d_free, kConvThreads / 32);
     S.abort_flag = 0;
     fence_mbar_init();
   }
@@ -246,25 +331,98 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const TcArgs a) 
   const uint32_t tmem = S.tmem_base;
 
   // Persistent: work item = (expert of the path, tile of weight rows), the
-  // tiles of an expert adjacent.  The ring of A/B slots runs on across
-  // items (ring step gs + st); an item's accumulators are read back before
-  // the next item's first MMAs overwrite them.
-  int gs = 0, it = 0;
-  for (int item = blockIdx.x; item < items; item += gridDim.x, gs += steps, ++it) {
-    const int rank = item / tiles;
-    const int u = L.tc_u[rank];
-    const int e = L.u_expert[u];
-    const int base = L.u_off[u], n = L.u_off[u + 1] - base;
-    const int N = (n + 15) & ~15;
-    const int r0 = (item % tiles) * tile_rows;
-    if (warp == kConvThreads / 32) {
+  // tiles of an expert adjacent.  Each role runs its own loop over the
+  // CTA's items; the rings run on across items (ring step it * steps + st,
+  // weight stage it * nst + j), so the producers stream the next item's
+  // tiles while the converters finish this one's epilogue.  An item's first
+  // MMAs wait until the previous item's accumulators were read (d_free).
+  int w_last[kWG][kSW];  // weight producer: last use issued per stage buffer
+  int b_last[kR];        // input producer: the same per ring slot
+  for (int w = 0; w < kWG; ++w)
+    for (int s = 0; s < kSW; ++s) w_last[w][s] = -1;
+  for (int i = 0; i < kR; ++i) b_last[i] = -1;
+  const int* list_tok = L.list_tok;
+  const int* list_pos = L.list_pos;
+
+  if (warp == kWProdWarp) {
+    // ------------------------------------------------ weight producer
+    const uint64_t stream = l2_policy_evict_first();
+    for (int item = blockIdx.x, it = 0; item < items; item += gridDim.x, ++it) {
+      if (!__shfl_sync(0xffffffffu, lane == 0 ? !*abort_flag : 0, 0)) break;
+      const int e = L.u_expert[L.tc_u[item / tiles]];
+      const int r0 = (item % tiles) * tile_rows;
+      // the item's tensor maps: templates re-pointed at the expert, in map
+      // set it % kMapSets of the CTA.  A set is rewritten kMapSets items
+      // later; by then every load through it has landed (this producer has
+      // issued at least kMapSets - 1 >= kSW stages of the items between,
+      // each after the stage kSW before it was consumed).
+      CUtensorMap* gm = a.maps + ((size_t)blockIdx.x * kMapSets + (it % kMapSets)) * kMaps;
+      const ExpertPtrs ep = a.table[e];
+      if (lane < 8 * nmaps) {  // the templates into shared memory, 16 bytes a lane
+        const int j = lane >> 3, part = lane & 7;
+        const CUtensorMap* src = (j & 1) ? &tm_scales : &tm_codes;
+        reinterpret_cast<uint4*>(&S.tm[j])[part] = reinterpret_cast<const uint4*>(src)[part];
+      }
+      __syncwarp();
       if (lane == 0) {
-        // -------------------------------------------------- B producer
-        const uint8_t* bsrc = a.bpack + ((size_t)rank * a.G) * gbytes;
-        const uint32_t bcopy = (uint32_t)N * 64 * (a.mats == 2 ? 1 : 2);
-        const uint64_t keep = l2_policy_evict_last();
-        for (int st = 0; st < steps && !*abort_flag; ++st) {
-          const int q = gs + st, slot = q % kR, use = q / kR;
+        tmap_set_address(&S.tm[0], a.mats == 2 ? (const void*)ep.q_gate : (const void*)ep.q_down);
+        tmap_set_address(&S.tm[1], a.mats == 2 ? (const void*)ep.s_gate : (const void*)ep.s_down);
+        if (a.mats == 2) {
+          tmap_set_address(&S.tm[2], ep.q_up);
+          tmap_set_address(&S.tm[3], ep.s_up);
+        }
+      }
+      __syncwarp();
+      for (int j = 0; j < nmaps; ++j) tmap_publish(gm + j, &S.tm[j]);
+      int ok = 1;
+      if (lane == 0) {
+        for (int j = 0; j < nmaps; ++j) tmap_acquire(gm + j);
+        if (blockIdx.x == 0 && it < 256) TC_TRACE_AT(12, it);
+        for (int j = 0; j < nst && ok; ++j) {
+          for (int w = 0; w < kWG; ++w) {
+            const int q = it * nst + j, sb = q % kSW, use = q / kSW;
+            if (use > 0 &&
+                !mbar_wait(&S.w_empty[w][sb], (uint32_t)((use - 1) & 1), kTcWaitNs)) {
+              *abort_flag = 1;
+              ok = 0;
+              break;
+            }
+            const int g = w * ng + j * kGS;  // first group of the stage
+            if (w == 0) TC_TRACE(13, j);
+            uint64_t* bar = &S.w_full[w][sb];
+            mbar_arrive_expect_tx(bar, kWStageBytes);
+            w_last[w][sb] = use;
+            if (a.mats == 2) {
+              // tile rows 32 qd .. + 15: gate rows r0 + 16 qd ..; the next
+              // 16: the up rows of the same indices
+              for (int qd = 0; qd < 4; ++qd) {
+                const int y = r0 + 16 * qd;
+                tma_load_2d(S.wc[w][sb] + (32 * qd) * 128, gm + 0, g * 16, y, bar, stream);
+                tma_load_2d(S.wc[w][sb] + (32 * qd + 16) * 128, gm + 2, g * 16, y, bar, stream);
+                tma_load_2d(S.wsc[w][sb] + (32 * qd) * 16, gm + 1, g, y, bar, stream);
+                tma_load_2d(S.wsc[w][sb] + (32 * qd + 16) * 16, gm + 3, g, y, bar, stream);
+              }
+            } else {
+              tma_load_2d(S.wc[w][sb], gm + 0, g * 16, r0, bar, stream);
+              tma_load_2d(S.wsc[w][sb], gm + 1, g, r0, bar, stream);
+            }
+          }
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+    }
+  } else if (warp == kBProdWarp) {
+    if (lane == 0) {
+      // ---------------------------------------------- input producer
+      const uint64_t keep = l2_policy_evict_last();
+      for (int item = blockIdx.x, it = 0; item < items && !*abort_flag;
+           item += gridDim.x, ++it) {
+        const int rank = item / tiles;
+        const int roff = L.tc_roff[rank], N = L.tc_roff[rank + 1] - roff;
+        const uint32_t bcopy = (uint32_t)(N * mb);
+        const uint8_t* bsrc = a.bpack + (size_t)roff * a.G * mb;
+        for (int st = 0; st < steps; ++st) {
+          const int q = it * steps + st, slot = q % kR, use = q / kR;
           if (use > 0 && !mbar_wait(&S.slot_free[slot], (uint32_t)((use - 1) & 1), kTcWaitNs)) {
             *abort_flag = 1;
             break;
@@ -272,13 +430,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const TcArgs a) 
           const int g = (st % kWG) * ng + st / kWG;
           TC_TRACE(0, st);
           mbar_arrive_expect_tx(&S.b_full[slot], bcopy);
-          bulk_g2s(S.b[slot], bsrc + (size_t)g * gbytes, bcopy, &S.b_full[slot], keep);
+          b_last[slot] = use;
+          bulk_g2s(S.b[slot], bsrc + (size_t)g * bcopy, bcopy, &S.b_full[slot], keep);
         }
-      } else if (lane == 1) {
-        // -------------------------------------------------- MMA issuer
+      }
+    }
+  } else if (warp >= kIssueWarp) {
+    if (lane == 0) {
+      // ---------------------------------------------- MMA issuers
+      const int j = warp - kIssueWarp;
+      const uint32_t d = tmem + (uint32_t)(kColD + j * kNmax);
+      for (int item = blockIdx.x, it = 0; item < items; item += gridDim.x, ++it) {
+        const int rank = item / tiles;
+        const int N = L.tc_roff[rank + 1] - L.tc_roff[rank];
         const uint32_t idesc = umma_idesc_f16(128, N);
-        for (int st = 0; st < steps; ++st) {
-          const int q = gs + st, slot = q % kR, use = q / kR;
+        // the previous item's accumulators have been read
+        if (*abort_flag ||
+            (it > 0 && !mbar_wait(&S.d_free, (uint32_t)((it - 1) & 1), kTcWaitNs))) {
+          *abort_flag = 1;
+          tc_commit(&S.fin);
+          break;
+        }
+        tc_fence_after();
+        for (int st = j; st < steps; st += kIssuers) {
+          const int q = it * steps + st, slot = q % kR, use = q / kR;
           if (*abort_flag || !mbar_wait(&S.a_full[slot], (uint32_t)(use & 1), kTcWaitNs)) {
             *abort_flag = 1;
             break;
@@ -290,14 +465,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const TcArgs a) 
           }
           TC_TRACE(2, st);
           tc_fence_after();
-          const int w = st % kWG, i = st / kWG;
-          const uint32_t d = tmem + (uint32_t)(kColD + w * kNmax);
           const uint32_t ahi = tmem + (uint32_t)(kColA + slot * 32), alo = ahi + 16;
           const uint32_t bhi = smem_addr(S.b[slot]), blo = bhi + (uint32_t)N * 64;
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk) {
             const uint64_t dh = umma_desc(bhi + kk * 256, 128, 512);
-            tc_mma(d, ahi + kk * 8, dh, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+            tc_mma(d, ahi + kk * 8, dh, idesc, (st >= kIssuers || kk > 0) ? 1u : 0u);
             tc_mma(d, alo + kk * 8, dh, idesc, 1u);
             if (a.mats == 1)
               tc_mma(d, ahi + kk * 8, umma_desc(blo + kk * 256, 128, 512), idesc, 1u);
@@ -305,126 +478,132 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const TcArgs a) 
           tc_commit(&S.slot_free[slot]);
           TC_TRACE(3, st);
         }
-        // every MMA of the item has finished when this arrives
+        // every MMA of this issuer's item has finished when this arrives
         tc_commit(&S.fin);
+        if (*abort_flag) break;
       }
-    } else {
-      // ---------------------------------------------------- converters
-      const int wg = warp >> 2, row = (warp & 3) * 32 + lane;  // row = tensor-memory lane
-      const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-      const ExpertPtrs ep = a.table[e];
-      const int mrow = r0 + (a.mats == 2 ? (row & 63) : row);
-      const uint8_t* codes = (a.mats == 2 ? (row < 64 ? ep.q_gate : ep.q_up) : ep.q_down) +
-                             (size_t)mrow * (a.K / 2);
-      const uint16_t* scales = (a.mats == 2 ? (row < 64 ? ep.s_gate : ep.s_up) : ep.s_down) +
-                               (size_t)mrow * a.G;
-      const int g0 = wg * ng;  // this warpgroup's groups [g0, g0 + ng), g0 even
-      auto issue_stage = [&](int j) {
-        const int gl = 2 * j;
-        if (gl < ng) {
-          const int s = j % kWS;
-          cp_async16(&S.w[wg][s][row][0], codes + (size_t)(g0 + gl) * 16);
-          cp_async16(&S.w[wg][s][row][1], codes + (size_t)(g0 + gl + 1) * 16);
-          cp_async4(&S.sc[wg][s][row], scales + g0 + gl);  // one aligned word: two scales
-        }
-      };
-#pragma unroll 1
-      for (int j = 0; j < kWS - 1; ++j) {
-        issue_stage(j);
-        cp_async_commit();
-      }
-      for (int i = 0; i < ng; ++i) {
-        if ((i & 1) == 0) {
-          cp_async_wait<kWS - 2>();  // this thread's stage i / 2 has landed
-          issue_stage(i / 2 + kWS - 1);
-          cp_async_commit();
-        }
-        const int s = (i >> 1) % kWS;
-        const uint4 w = S.w[wg][s][row][i & 1];
-        const uint32_t sp = S.sc[wg][s][row];
-        const uint32_t sh = (i & 1) ? (sp >> 16) : (sp & 0xFFFFu);  // fp16 scale of group g0 + i
-        uint32_t hl[32];
-        weights_hi_lo(w, sh | (sh << 16), hl);
-        const int st = i * kWG + wg, q = gs + st, slot = q % kR, use = q / kR;
-        if (row == 0) TC_TRACE(4, st);
-        // the slot's previous MMAs (ring step q - kR) have finished
-        if (use > 0) {
-          int okw = 0;
-          if (lane == 0 && !*abort_flag) {
-            okw = mbar_wait(&S.slot_free[slot], (uint32_t)((use - 1) & 1), kTcWaitNs) ? 1 : 0;
-            if (!okw) *abort_flag = 1;
-          }
-          okw = __shfl_sync(0xffffffffu, okw, 0);
-          if (!okw) break;
-          mbar_test(&S.slot_free[slot], (uint32_t)((use - 1) & 1));
-          tc_fence_after();
-        }
-        if (row == 0) TC_TRACE(5, st);
-        tmem_st32(tmem + lane_base + (uint32_t)(kColA + slot * 32), hl);
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-        if (row == 0) TC_TRACE(6, st);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.a_full[slot]);
-      }
-      cp_async_wait<0>();
     }
-    // -------------------------------------------------------- epilogue
-    __syncthreads();
-    if (tid == kConvThreads) {  // one wait for the item's last commit (bounded)
-      if (!mbar_wait(&S.fin, (uint32_t)(it & 1), kTcWaitNs)) *abort_flag = 1;
-      TC_TRACE_ITEM();
-    }
-    __syncthreads();
-    tc_fence_after();
-    const bool aborted = *abort_flag != 0;  // uniform: nobody writes it until the next item
-    float* red = reinterpret_cast<float*>(&S.w[0][0][0][0]);  // [wg][row][kNmax]
-    if (warp < kConvThreads / 32 && !aborted) {
-      const int wg = warp >> 2, row = (warp & 3) * 32 + lane;
-      const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-      const uint32_t d = tmem + lane_base + (uint32_t)(kColD + wg * kNmax);
+  } else {
+    // ---------------------------------------------------- converters
+    const int wg = warp >> 2, row = (warp & 3) * 32 + lane;  // row = tensor-memory lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t swz = (uint32_t)(row & 7);
+    for (int item = blockIdx.x, it = 0; item < items; item += gridDim.x, ++it) {
+      const int rank = item / tiles;
+      const int u = L.tc_u[rank];
+      const int base = L.u_off[u], n = L.u_off[u + 1] - base;
+      const int N = L.tc_roff[rank + 1] - L.tc_roff[rank];
+      const int r0 = (item % tiles) * tile_rows;
+      bool ok = true;
+      for (int j = 0; j < nst && ok; ++j) {
+        const int q = it * nst + j, sb = q % kSW, use = q / kSW;
+        if (!warp_wait(&S.w_full[wg][sb], (uint32_t)(use & 1), lane, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* crow = &S.wc[wg][sb][row * 128];
+        const uint4 sc8 = *reinterpret_cast<const uint4*>(&S.wsc[wg][sb][row * 16]);
+        const uint32_t spair[4] = {sc8.x, sc8.y, sc8.z, sc8.w};
 #pragma unroll
-      for (int c = 0; c < kNmax / 16; ++c) {
-        if (c * 16 < N) {
-          uint32_t dv[16];
-          tmem_ld16(d + (uint32_t)(c * 16), dv);
+        for (int c = 0; c < kGS; ++c) {
+          const uint4 w = *reinterpret_cast<const uint4*>(crow + (((uint32_t)c ^ swz) << 4));
+          const uint32_t sh = (c & 1) ? (spair[c >> 1] >> 16) : (spair[c >> 1] & 0xFFFFu);
+          uint32_t hl[32];
+          weights_hi_lo(w, group_scale(sh), hl);
+          const int i = j * kGS + c;  // group of this warpgroup
+          const int st = i * kWG + wg, qs = it * steps + st, slot = qs % kR, suse = qs / kR;
+          if (row == 0) TC_TRACE(4, st);
+          // the slot's previous MMAs (ring step qs - kR) have finished
+          if (suse > 0) {
+            if (!warp_wait(&S.slot_free[slot], (uint32_t)((suse - 1) & 1), lane, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          if (row == 0) TC_TRACE(5, st);
+          tmem_st32(tmem + lane_base + (uint32_t)(kColA + slot * 32), hl);
+          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+          if (row == 0) TC_TRACE(6, st);
+          if (lane == 0) TC_TRACE(8 + (warp & 3), st);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.a_full[slot]);
+        }
+        // the stage's codes and scales are read (every lane's loads retired)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.w_empty[wg][sb]);
+      }
+      // ------------------------------------------------------ epilogue
+      // Thread (wg, row) takes tokens [wg * N/2, (wg + 1) * N/2) of its
+      // row: the four issuers' accumulators, added in a fixed order (the
+      // K halves of warpgroup 0, then of warpgroup 1).
+      if (!ok || !warp_wait(&S.fin, (uint32_t)(it & 1), lane, abort_flag)) break;
+      if (row == 0 && wg == 0) TC_TRACE_ITEM();
+      tc_fence_after();
+      const int half = N >> 1, t0 = wg * half;
+      float sum[kNmax / 2];
+      const uint32_t dl = tmem + lane_base + (uint32_t)(kColD + t0);
+#pragma unroll
+      for (int c = 0; c < kNmax / 2; c += 8) {
+        if (c < half) {
+          uint32_t v0[8], v1[8], v2[8], v3[8];
+          tmem_ld8(dl + (uint32_t)(0 * kNmax + c), v0);
+          tmem_ld8(dl + (uint32_t)(2 * kNmax + c), v2);
+          tmem_ld8(dl + (uint32_t)(1 * kNmax + c), v1);
+          tmem_ld8(dl + (uint32_t)(3 * kNmax + c), v3);
           asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-          for (int t = 0; t < 16; ++t)
-            red[((size_t)wg * 128 + row) * kNmax + c * 16 + t] = __uint_as_float(dv[t]);
+          for (int t = 0; t < 8; ++t)
+            sum[c + t] = (__uint_as_float(v0[t]) + __uint_as_float(v2[t])) +
+                         (__uint_as_float(v1[t]) + __uint_as_float(v3[t]));
+        }
+      }
+      // the accumulators may be overwritten by the next item's MMAs
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.d_free);
+      if (a.mats == 2) {
+        // h = silu(gate) * up: lane m < 16 of quarter q holds gate row
+        // r0 + 16 q + m, lane m + 16 the up row of the same index
+        const int hrow = r0 + 16 * (warp & 3) + (lane & 15);
+#pragma unroll
+        for (int c = 0; c < kNmax / 2; ++c) {
+          if (c < half) {
+            const float up = __shfl_down_sync(0xffffffffu, sum[c], 16);
+            const int t = t0 + c;
+            if (lane < 16 && t < n) {
+              const float f = ldexpf(1.0f, a.row_exp[list_tok[base + t]]);
+              a.out[(size_t)list_pos[base + t] * a.R + hrow] = silu_mul(sum[c] * f, up * f);
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kNmax / 2; ++c) {
+          const int t = t0 + c;
+          if (c < half && t < n)
+            a.out[(size_t)list_pos[base + t] * a.R + r0 + row] =
+                sum[c] * ldexpf(1.0f, a.row_exp[list_pos[base + t]]);
         }
       }
     }
-    tc_fence_before();
-    __syncthreads();
-    if (aborted) {
-      if (tid == 0) atomicCAS(a.err, 0u, (uint32_t)kErrTimeout);
-      break;
-    }
-    const int* list_tok = L.list_tok;
-    const int* list_pos = L.list_pos;
-    if (a.mats == 2) {
-      // h = silu(gate) * up for the tile's 64 rows, every token
-      for (int idx = tid; idx < 64 * n; idx += kTcThreads) {
-        const int rr = idx % 64, t = idx / 64;
-        float gsum = 0.f, usum = 0.f;
-        for (int w = 0; w < kWG; ++w) {
-          gsum += red[((size_t)w * 128 + rr) * kNmax + t];
-          usum += red[((size_t)w * 128 + rr + 64) * kNmax + t];
-        }
-        const float f = ldexpf(1.0f, a.row_exp[list_tok[base + t]]);
-        a.out[(size_t)list_pos[base + t] * a.R + r0 + rr] = silu_mul(gsum * f, usum * f);
-      }
-    } else {
-      for (int idx = tid; idx < 128 * n; idx += kTcThreads) {
-        const int rr = idx % 128, t = idx / 128;
-        float ysum = 0.f;
-        for (int w = 0; w < kWG; ++w) ysum += red[((size_t)w * 128 + rr) * kNmax + t];
-        a.out[(size_t)list_pos[base + t] * a.R + r0 + rr] =
-            ysum * ldexpf(1.0f, a.row_exp[list_pos[base + t]]);
-      }
-    }
-    __syncthreads();  // red (the code stages) is rewritten by the next item
+  }
+  // A wait that ran out leaves the rest of the call's results unwritten
+  // and reports it.  Copies may still be in flight into this CTA's shared
+  // memory: each producer waits (bounded) for the last one it issued into
+  // every buffer before the CTA exits.
+  __syncthreads();
+  if (*abort_flag) {
+    if (tid == 0) atomicCAS(a.err, 0u, (uint32_t)kErrTimeout);
+    if (warp == kWProdWarp && lane == 0)
+      for (int w = 0; w < kWG; ++w)
+        for (int s = 0; s < kSW; ++s)
+          if (w_last[w][s] >= 0)
+            mbar_wait(&S.w_full[w][s], (uint32_t)(w_last[w][s] & 1), kTcWaitNs);
+    if (warp == kBProdWarp && lane == 0)
+      for (int i = 0; i < kR; ++i)
+        if (b_last[i] >= 0) mbar_wait(&S.b_full[i], (uint32_t)(b_last[i] & 1), kTcWaitNs);
   }
   __syncthreads();
   if (warp == 0) {
@@ -437,6 +616,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const TcArgs a) 
 // divided by 2^e (e >= 0, the least with max |v| / 2^e <= 2^14) before it is
 // rounded to fp16 and the row's results are multiplied back, so that no
 // input overflows fp16; e is 0 for every row of ordinary size.
+// 16-byte loads (K a multiple of 8), several in flight per thread.
 template <bool kF32>
 __global__ void __launch_bounds__(256) tc_rowscale_kernel(const void* in, int K, int rows,
                                                           int* row_exp) {
@@ -444,10 +624,23 @@ __global__ void __launch_bounds__(256) tc_rowscale_kernel(const void* in, int K,
   const int r = blockIdx.x;
   if (r >= rows) return;
   float m = 0.f;
-  for (int k = threadIdx.x; k < K; k += blockDim.x) {
-    const float v = kF32 ? static_cast<const float*>(in)[(size_t)r * K + k]
-                         : bf16_bits_to_f32(static_cast<const uint16_t*>(in)[(size_t)r * K + k]);
-    m = fmaxf(m, fabsf(v));
+  if (kF32) {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(in) + (size_t)r * K);
+#pragma unroll 4
+    for (int c = threadIdx.x; c < K / 4; c += blockDim.x) {
+      const float4 v = p[c];
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+  } else {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(in) + (size_t)r * K);
+#pragma unroll 4
+    for (int c = threadIdx.x; c < K / 8; c += blockDim.x) {
+      const uint4 v = p[c];
+      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32(u[j] & 0xFFFFu)), fabsf(bf16_bits_to_f32(u[j] >> 16))));
+    }
   }
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -469,11 +662,15 @@ __device__ __forceinline__ uint16_t f32_to_f16_rne(float f) {
 }
 
 // Packs the inputs of every path expert: for expert rank r and group g, the
-// B operand of its MMAs, rows = its tokens (zero rows up to a multiple of
-// 16), in the canonical K-major layout [N/8][4][8 rows][8 inputs] of fp16,
-// inputs in the MMA order tc_perm, each row divided by 2^row_exp.
+// B operand of its MMAs, rows = its tokens (zero rows up to N, a multiple of
+// 16), at byte (tc_roff[r] * G + g * N) * (64, down: 128), in the canonical
+// K-major layout [N/8][4][8 rows][8 inputs] of fp16, inputs in the MMA order,
+// each row divided by 2^row_exp.
 // Gate/up: x (bf16 -> fp16, exact within fp16's range).  Down: h (fp32) as
 // an fp16 hi tile then an fp16 lo (h - hi) tile.
+// One thread per (group, row): the row's 32 inputs of the group in 16-byte
+// loads, out as 4 core-matrix rows of 16 bytes (chunk cb holds inputs
+// 8 cb + {0, 4, 1, 5, 2, 6, 3, 7}).
 template <bool kDown>
 __global__ void __launch_bounds__(256) tc_pack_kernel(const int* lists, int E, int n_list,
                                                       const void* in, int K, int G,
@@ -485,83 +682,154 @@ __global__ void __launch_bounds__(256) tc_pack_kernel(const int* lists, int E, i
   const int* list_tok = L.list_tok;
   const int* list_pos = L.list_pos;
   const int base = L.u_off[u], n = L.u_off[u + 1] - base;
-  const int N = (n + 15) & ~15;
-  const size_t gbytes = tc_group_bytes(kDown ? 1 : 2);
-  // one thread per (group, row, core column): 8 inputs -> 16 bytes (x2 for down)
-  const int per_group = N * 4;
-  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < G * per_group;
+  const int roff = L.tc_roff[rank], N = L.tc_roff[rank + 1] - roff;
+  const size_t gbytes = (size_t)N * (kDown ? 128 : 64);
+  uint8_t* dst0 = bpack + (size_t)roff * G * (kDown ? 128 : 64);
+  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < G * N;
        idx += gridDim.x * blockDim.x) {
-    const int g = idx / per_group, rem = idx % per_group;
-    const int nr = rem / 4, cb = rem % 4;
-    uint16_t hi[8], lo[8];
-    const int in_row = nr < n ? (kDown ? list_pos[base + nr] : list_tok[base + nr]) : 0;
-    const int ex = nr < n ? row_exp[in_row] : 0;
+    const int g = idx / N, nr = idx % N;
+    float v[32];
+    if (nr < n) {
+      const int in_row = kDown ? list_pos[base + nr] : list_tok[base + nr];
+      const float sc = ldexpf(1.0f, -row_exp[in_row]);
+      if (kDown) {
+        const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(in) +
+                                                          (size_t)in_row * K + g * 32);
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      hi[kk] = 0;
-      lo[kk] = 0;
-      if (nr < n) {
-        const int kin = g * 32 + tc_perm(cb * 8 + kk);
-        if (kDown) {
-          const float v = ldexpf(static_cast<const float*>(in)[(size_t)in_row * K + kin], -ex);
-          const uint16_t h16 = f32_to_f16_rne(v);
-          hi[kk] = h16;
-          lo[kk] = f32_to_f16_rne(v - f16_bits_to_f32(h16));
-        } else {
-          const float v = bf16_bits_to_f32(static_cast<const uint16_t*>(in)[(size_t)in_row * K + kin]);
-          hi[kk] = f32_to_f16_rne(ldexpf(v, -ex));
+        for (int j = 0; j < 8; ++j) {
+          const float4 f = p[j];
+          v[4 * j] = f.x * sc;
+          v[4 * j + 1] = f.y * sc;
+          v[4 * j + 2] = f.z * sc;
+          v[4 * j + 3] = f.w * sc;
+        }
+      } else {
+        const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(in) +
+                                                        (size_t)in_row * K + g * 32);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 q = p[j];
+          const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            v[8 * j + 2 * h] = bf16_bits_to_f32(w4[h] & 0xFFFFu) * sc;
+            v[8 * j + 2 * h + 1] = bf16_bits_to_f32(w4[h] >> 16) * sc;
+          }
         }
       }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = 0.f;
     }
     // core matrix (nr / 8, cb) at ((nr / 8) * 4 + cb) * 128 bytes, row nr % 8
-    uint8_t* dst = bpack + ((size_t)rank * G + g) * gbytes +
-                   ((size_t)((nr >> 3) * 4 + cb)) * 128 + (size_t)(nr & 7) * 16;
-    uint4 vh;
-    vh.x = hi[0] | ((uint32_t)hi[1] << 16);
-    vh.y = hi[2] | ((uint32_t)hi[3] << 16);
-    vh.z = hi[4] | ((uint32_t)hi[5] << 16);
-    vh.w = hi[6] | ((uint32_t)hi[7] << 16);
-    *reinterpret_cast<uint4*>(dst) = vh;
-    if (kDown) {
-      uint4 vl;
-      vl.x = lo[0] | ((uint32_t)lo[1] << 16);
-      vl.y = lo[2] | ((uint32_t)lo[3] << 16);
-      vl.z = lo[4] | ((uint32_t)lo[5] << 16);
-      vl.w = lo[6] | ((uint32_t)lo[7] << 16);
-      *reinterpret_cast<uint4*>(dst + (size_t)N * 64) = vl;
+    uint8_t* dst = dst0 + (size_t)g * gbytes + (size_t)(nr >> 3) * 512 + (size_t)(nr & 7) * 16;
+#pragma unroll
+    for (int cb = 0; cb < 4; ++cb) {
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        // MMA-K order: the pair (8 cb + h, 8 cb + h + 4)
+        const float a0 = v[8 * cb + h], a1 = v[8 * cb + h + 4];
+        const uint16_t h0 = f32_to_f16_rne(a0), h1 = f32_to_f16_rne(a1);
+        hi[h] = h0 | ((uint32_t)h1 << 16);
+        if (kDown) {
+          const uint16_t l0 = f32_to_f16_rne(a0 - f16_bits_to_f32(h0));
+          const uint16_t l1 = f32_to_f16_rne(a1 - f16_bits_to_f32(h1));
+          lo[h] = l0 | ((uint32_t)l1 << 16);
+        }
+      }
+      *reinterpret_cast<uint4*>(dst + cb * 128) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      if (kDown)
+        *reinterpret_cast<uint4*>(dst + cb * 128 + (size_t)N * 64) =
+            make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
   }
 }
 
+// cuTensorMapEncodeTiled, reached through the runtime's driver entry points
+// (no link-time dependency on libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static const EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return (EncodeTiledFn) nullptr;
+    }
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// A 2-D map over a row-major matrix [rows][inner] of elements of `bytes`
+// bytes; base is any 16-byte aligned address (the kernel re-points it).
+bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, int bytes, void* base, uint64_t inner,
+               uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  const EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * (uint64_t)bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+std::atomic<int> g_tc_min{kTcMinTokDefault};
+
 }  // namespace
+
+int tc_min_tokens() { return g_tc_min.load(std::memory_order_relaxed); }
 
 #ifdef MOE_TRACE
 extern "C" __attribute__((visibility("default"))) int moe_debug_tc_trace(void* host_dst) {
   return (int)cudaMemcpyFromSymbol(host_dst, g_tc_trace, sizeof(g_tc_trace));
 }
+
+// Profiling builds: the least token count of a tensor-core expert.
+extern "C" __attribute__((visibility("default"))) int moe_debug_set_tc_min(int n) {
+  if (n < kTcMinTokFloor || n > kTcMaxTok + 1) return -1;
+  g_tc_min.store(n, std::memory_order_relaxed);
+  return 0;
+}
 #endif
 
 // Most experts a call of T tokens can have on the path: each routed one
-// takes kTcMinTok of the T * k entries at least.
+// takes kTcMinTokFloor of the T * k entries at least.
 int tc_max_experts(int T, int k, int has_shared) {
-  return T < kTcMinTok ? 0 : (T * k) / kTcMinTok + has_shared;
+  if (T < kTcMinTokFloor) return 0;
+  return std::min((T * k) / kTcMinTokFloor + has_shared, T * k + has_shared);
 }
 
+// Packed input rows: each path expert's tokens rounded up to 16.
 size_t tc_bpack_bytes(int T, int k, int has_shared, int H, int I) {
-  if (T < kTcMinTok) return 0;
   const size_t experts = (size_t)tc_max_experts(T, k, has_shared);
-  const size_t gu = (size_t)(H / 32) * tc_group_bytes(2), dn = (size_t)(I / 32) * tc_group_bytes(1);
-  return experts * (gu > dn ? gu : dn);
+  if (experts == 0) return 0;
+  const size_t rows = (size_t)T * (k + has_shared) + 15 * experts;
+  const size_t gu = (size_t)(H / 32) * 64, dn = (size_t)(I / 32) * 128;
+  return rows * (gu > dn ? gu : dn);
 }
 
 size_t tc_rowexp_ints(int T, int k, int has_shared) { return (size_t)T * (k + has_shared); }
 
-bool tc_shape_ok(int H, int I) { return H % 128 == 0 && I % 128 == 0; }
+size_t tc_maps_bytes() { return (size_t)kTcMaxCtas * kMapSets * kMaps * sizeof(CUtensorMap); }
+
+// Weight stages of 8 groups per warpgroup half of K: K a multiple of 512.
+bool tc_shape_ok(int H, int I) {
+  return H % 512 == 0 && I % 512 == 0 && encode_tiled() != nullptr;
+}
 
 cudaError_t launch_tc_ffn_step(int mats, const ExpertPtrs* table, const int* lists, int E,
                                int n_list, int T, int k, int has_shared, const void* in, int K,
-                               int R, int in_rows, int* row_exp, uint8_t* bpack, float* out,
-                               uint32_t* err, cudaStream_t st) {
+                               int R, int in_rows, int* row_exp, uint8_t* bpack, uint8_t* maps,
+                               float* out, uint32_t* err, cudaStream_t st) {
   static DeviceOnce<bool> configured;
   int dev = 0;
   cudaError_t ce = cudaGetDevice(&dev);
@@ -570,7 +838,7 @@ cudaError_t launch_tc_ffn_step(int mats, const ExpertPtrs* table, const int* lis
   ce = configured.get(dev, &done, [](bool* v) {
     const cudaError_t r = cudaFuncSetAttribute(tc_gemm_kernel,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)sizeof(TcSmem));
+                                               (int)sizeof(TcSmem) + 1024);
     *v = r == cudaSuccess;
     return r;
   });
@@ -578,6 +846,16 @@ cudaError_t launch_tc_ffn_step(int mats, const ExpertPtrs* table, const int* lis
   const int G = K / 32;
   const int tcmax = tc_max_experts(T, k, has_shared);
   if (tcmax == 0) return cudaSuccess;
+  // templates: the matrices the weight rows of a tile come from are [R][K];
+  // a box is 8 groups of 16 (gate/up: gate and up rows interleave in the
+  // tile by 16) or 128 rows
+  const int tile_rows = mats == 2 ? 64 : 128, box_rows = mats == 2 ? 16 : 128;
+  CUtensorMap tm_codes, tm_scales;
+  if (!encode_2d(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, bpack, (uint64_t)K / 2,
+                 (uint64_t)R, 128, (uint32_t)box_rows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, bpack, (uint64_t)G, (uint64_t)R,
+                 kGS, (uint32_t)box_rows, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
   if (mats == 2) {
     tc_rowscale_kernel<false><<<in_rows, 256, 0, st>>>(in, K, in_rows, row_exp);
     tc_pack_kernel<false><<<dim3(16, tcmax), 256, 0, st>>>(lists, E, n_list, in, K, G, row_exp,
@@ -600,11 +878,12 @@ cudaError_t launch_tc_ffn_step(int mats, const ExpertPtrs* table, const int* lis
   a.row_exp = row_exp;
   a.out = out;
   a.err = err;
+  a.maps = reinterpret_cast<CUtensorMap*>(maps);
   // persistent: one CTA per SM (its shared memory and 512 tensor-memory
   // columns), no more CTAs than the call can have work items
-  const int tiles = mats == 2 ? R / 64 : R / 128;
-  const int grid = std::min(num_sms(), tcmax * tiles);
-  tc_gemm_kernel<<<grid, kTcThreads, sizeof(TcSmem), st>>>(a);
+  const int tiles = R / tile_rows;
+  const int grid = std::min(std::min(num_sms(), kTcMaxCtas), tcmax * tiles);
+  tc_gemm_kernel<<<grid, kTcThreads, sizeof(TcSmem) + 1024, st>>>(a, tm_codes, tm_scales);
   return cudaGetLastError();
 }
 

@@ -32,6 +32,7 @@ namespace {
 
 constexpr int kUnionThreads = 256;
 constexpr int kListMaxE = 257;   // routed experts + shared
+constexpr int kListMaxIds = 64 * 32;  // T * top_k at most
 
 // ---------------------------------------------------------------------------
 template <bool kBf16>
@@ -82,11 +83,12 @@ __global__ void __launch_bounds__(256) xq_table_kernel(const void* __restrict__ 
 // The expert lists of the call (layout: ListsView).  Out-of-range ids set
 // the error word and are left out; -1 (a slot dropped by top-p) is skipped.
 __global__ void __launch_bounds__(256) build_lists_kernel(const int32_t* __restrict__ idx, int T,
-                                                          int k, int E, int has_shared, int tc_on,
+                                                          int k, int E, int has_shared, int tc_min,
                                                           int* __restrict__ lists,
                                                           uint32_t* __restrict__ err) {
   __shared__ int cnt[kListMaxE];
   __shared__ int base[kListMaxE];
+  __shared__ int sid[kListMaxIds];
   const int slots = k + has_shared;
   const int n_list = T * slots;
   const ListsView L = lists_view(lists, E, n_list);
@@ -96,59 +98,80 @@ __global__ void __launch_bounds__(256) build_lists_kernel(const int32_t* __restr
   int* list_pos = const_cast<int*>(L.list_pos);
   int* cc_u = const_cast<int*>(L.cc_u);
   int* tc_u = const_cast<int*>(L.tc_u);
-  for (int e = threadIdx.x; e <= E; e += blockDim.x) cnt[e] = 0;
-  __syncthreads();
+  int* tc_roff = const_cast<int*>(L.tc_roff);
+  // the ids into shared memory; warp 0 counts them 32 at a time: the lanes
+  // holding one id find each other (match.any) and the lowest adds their
+  // number (no atomics, which correlated tokens would serialise on a few ids)
   for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
     const int e = idx[i];
-    if (e >= 0 && e < E) {
-      atomicAdd(&cnt[e], 1);
-    } else if (e != -1) {
-      atomicCAS(err, 0u, (uint32_t)kErrBadExpertId);
+    sid[i] = e;
+    if ((e < 0 || e >= E) && e != -1) atomicCAS(err, 0u, (uint32_t)kErrBadExpertId);
+  }
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    for (int i0 = 0; i0 < T * k; i0 += 32) {
+      const int e = i0 + lane < T * k ? sid[i0 + lane] : -1;
+      const uint32_t peers = __match_any_sync(0xffffffffu, e);
+      if (e >= 0 && e < E && lane == __ffs(peers) - 1) cnt[e] += __popc(peers);
+      __syncwarp();
     }
   }
   __syncthreads();
   if (threadIdx.x == 0 && has_shared) cnt[E] = T;
   __syncthreads();
-  // exclusive scans of (expert used, tensor-core expert, entries) over
-  // experts 0..E, ascending: thread i owns experts 2i and 2i + 1 (E + 1 <= 512)
+  // exclusive scans of (expert used, tensor-core expert, entries, packed
+  // rows) over experts 0..E, ascending: thread i owns experts 2i and 2i + 1
+  // (E + 1 <= 512); tc_min 0: no tensor-core experts
   {
-    __shared__ int wu[8], wt[8], ws[8];
+    __shared__ int wu[8], wt[8], ws[8], wp[8];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int e0 = 2 * threadIdx.x, e1 = e0 + 1;
     const int c0 = e0 <= E ? cnt[e0] : 0, c1 = e1 <= E ? cnt[e1] : 0;
-    const bool t0 = tc_on && c0 >= kTcMinTok && c0 <= kTcMaxTok;
-    const bool t1 = tc_on && c1 >= kTcMinTok && c1 <= kTcMaxTok;
-    const int nu = (c0 > 0) + (c1 > 0), nt = (int)t0 + (int)t1, ns = c0 + c1;
-    int iu = nu, it = nt, is = ns;  // inclusive warp scans
+    const bool t0 = tc_min > 0 && c0 >= tc_min && c0 <= kTcMaxTok;
+    const bool t1 = tc_min > 0 && c1 >= tc_min && c1 <= kTcMaxTok;
+    const int p0 = t0 ? (c0 + 15) & ~15 : 0, p1 = t1 ? (c1 + 15) & ~15 : 0;
+    const int nu = (c0 > 0) + (c1 > 0), nt = (int)t0 + (int)t1, ns = c0 + c1, np = p0 + p1;
+    int iu = nu, it = nt, is = ns, ip = np;  // inclusive warp scans
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int a = __shfl_up_sync(0xffffffffu, iu, o), b = __shfl_up_sync(0xffffffffu, it, o),
-                c = __shfl_up_sync(0xffffffffu, is, o);
+                c = __shfl_up_sync(0xffffffffu, is, o), d = __shfl_up_sync(0xffffffffu, ip, o);
       if (lane >= o) {
         iu += a;
         it += b;
         is += c;
+        ip += d;
       }
     }
     if (lane == 31) {
       wu[warp] = iu;
       wt[warp] = it;
       ws[warp] = is;
+      wp[warp] = ip;
     }
     __syncthreads();
-    int bu = 0, bt = 0, bs = 0;
+    int bu = 0, bt = 0, bs = 0, bp = 0;
     for (int w = 0; w < warp; ++w) {
       bu += wu[w];
       bt += wt[w];
       bs += ws[w];
+      bp += wp[w];
     }
-    int uu = bu + iu - nu, ut = bt + it - nt, off = bs + is - ns;  // exclusive prefixes
+    // exclusive prefixes
+    int uu = bu + iu - nu, ut = bt + it - nt, off = bs + is - ns, poff = bp + ip - np;
     if (c0 > 0) {
       u_expert[uu] = e0;
       u_off[uu] = off;
       base[e0] = off;
-      if (t0) tc_u[ut++] = uu;
-      else cc_u[uu - ut] = uu;
+      if (t0) {
+        tc_roff[ut] = poff;
+        tc_u[ut++] = uu;
+        poff += p0;
+      } else {
+        cc_u[uu - ut] = uu;
+      }
       ++uu;
       off += c0;
     }
@@ -156,8 +179,12 @@ __global__ void __launch_bounds__(256) build_lists_kernel(const int32_t* __restr
       u_expert[uu] = e1;
       u_off[uu] = off;
       base[e1] = off;
-      if (t1) tc_u[ut] = uu;
-      else cc_u[uu - ut] = uu;
+      if (t1) {
+        tc_roff[ut] = poff;
+        tc_u[ut] = uu;
+      } else {
+        cc_u[uu - ut] = uu;
+      }
     }
     if (threadIdx.x == blockDim.x - 1) {
       const int U = bu + iu, n_tc = bt + it, total = bs + is;
@@ -166,20 +193,28 @@ __global__ void __launch_bounds__(256) build_lists_kernel(const int32_t* __restr
       int* counts = const_cast<int*>(L.counts);
       counts[0] = U - n_tc;
       counts[1] = n_tc;
+      tc_roff[n_tc] = bp + ip;
     }
   }
   __syncthreads();
-  // each expert appends its entries in (token, slot) order
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    if (cnt[e] == 0) continue;
-    int pos = base[e];
-    for (int i = 0; i < T * k; ++i) {
-      if (idx[i] == e) {
+  // the entries in (token, slot) order, placed by warp 0 32 at a time: an
+  // entry's place is its expert's next free one plus its rank among the
+  // lanes holding the same id
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    for (int i0 = 0; i0 < T * k; i0 += 32) {
+      const int i = i0 + lane;
+      const int e = i < T * k ? sid[i] : -1;
+      const uint32_t peers = __match_any_sync(0xffffffffu, e);
+      if (e >= 0 && e < E) {
+        const int pos = base[e] + __popc(peers & ((1u << lane) - 1u));
         const int t = i / k, j = i % k;
         list_tok[pos] = t;
         list_pos[pos] = t * slots + j;
-        ++pos;
       }
+      __syncwarp();
+      if (e >= 0 && e < E && lane == __ffs(peers) - 1) base[e] += __popc(peers);
+      __syncwarp();
     }
   }
   if (has_shared) {
@@ -429,22 +464,26 @@ __global__ void __launch_bounds__(256) union_combine_kernel(
 }  // namespace
 
 size_t union_lists_ints(int T, int k, int E, int has_shared) {
-  return 1 + (size_t)(E + 1) + (E + 2) + 2 * (size_t)T * (k + has_shared) + 2 + 2 * (size_t)(E + 1);
+  return 1 + (size_t)(E + 1) + (E + 2) + 2 * (size_t)T * (k + has_shared) + 2 +
+         2 * (size_t)(E + 1) + (E + 2);
 }
 
 cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const float* w,
                              const uint16_t* x, int T, int H, int I, int E, int k, int has_shared,
                              uint8_t* xq_words, float* xq_fac, uint8_t* hq_words, float* hq_fac,
                              int* lists, float* hbuf, float* ypart, float* y, uint32_t* err,
-                             uint8_t* tc_bpack, int* tc_rowexp, cudaStream_t st) {
-  if (E + 1 > kListMaxE) return cudaErrorInvalidValue;
-  const bool tc = tc_bpack && T >= 16 && tc_shape_ok(H, I);
+                             uint8_t* tc_bpack, int* tc_rowexp, uint8_t* tc_maps,
+                             cudaStream_t st) {
+  if (E + 1 > kListMaxE || T * k > kListMaxIds) return cudaErrorInvalidValue;
+  const int tc_min = tc_min_tokens();
+  const bool tc = tc_bpack && tc_maps && T >= tc_min && tc_shape_ok(H, I);
   const int slots = k + has_shared;
   const int G = H / 32, GD = I / 32;
   const int n_list = T * slots;
   const int umax = (E < T * k ? E : T * k) + has_shared;
   xq_table_kernel<true><<<(T * G + 255) / 256, 256, 0, st>>>(x, T, H, xq_words, xq_fac);
-  build_lists_kernel<<<1, 256, 0, st>>>(idx, T, k, E, has_shared, tc ? 1 : 0, lists, err);
+  build_lists_kernel<<<1, 256, 0, st>>>(idx, T, k, E, has_shared, tc ? tc_min : 0, lists,
+                                         err);
   UnionArgs a;
   a.table = table;
   a.lists = lists;
@@ -489,7 +528,7 @@ cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const 
   union_gemm_kernel<2><<<grid2, kUnionThreads, union_smem_bytes(2), st>>>(a);
   if (tc) {
     const cudaError_t e = launch_tc_ffn_step(2, table, lists, E, n_list, T, k, has_shared, x, H,
-                                             I, T, tc_rowexp, tc_bpack, hbuf, err, st);
+                                             I, T, tc_rowexp, tc_bpack, tc_maps, hbuf, err, st);
     if (e != cudaSuccess) return e;
   }
   xq_table_kernel<false><<<(n_list * GD + 255) / 256, 256, 0, st>>>(hbuf, n_list, I, hq_words,
@@ -503,7 +542,8 @@ cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const 
   union_gemm_kernel<1><<<grid1, kUnionThreads, union_smem_bytes(1), st>>>(a);
   if (tc) {
     const cudaError_t e = launch_tc_ffn_step(1, table, lists, E, n_list, T, k, has_shared, hbuf,
-                                             I, H, n_list, tc_rowexp, tc_bpack, ypart, err, st);
+                                             I, H, n_list, tc_rowexp, tc_bpack, tc_maps, ypart,
+                                             err, st);
     if (e != cudaSuccess) return e;
   }
   union_combine_kernel<<<dim3((H + 255) / 256, T), 256, 0, st>>>(idx, w, ypart, T, H, k, E,
