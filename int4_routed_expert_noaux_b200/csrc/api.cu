@@ -9,7 +9,6 @@
 
 #include "common.cuh"
 #include "kernels.h"
-#include "kernels.h"
 #include "layer.h"
 #include "moe.h"
 
@@ -106,9 +105,9 @@ WsLayout ws_layout(const moe_config* c, int T) {
   // from call to call: a region that no other call writes
   L.records = off;
   off = align_up(off + (size_t)c->n_experts * 8, 256);
-  // fp32 router logits of the step kernels
+  // fp64 router logits of the step kernels, in K slices
   L.logits = off;
-  off = align_up(off + (size_t)T * c->n_experts * 4, 256);
+  off = align_up(off + (size_t)kRouterMaxSlices * T * c->n_experts * 8, 256);
   L.idx = off;
   off = align_up(off + (size_t)T * k * 4, 256);
   L.w = off;

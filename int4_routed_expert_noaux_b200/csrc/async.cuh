@@ -50,6 +50,21 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// One probe that suspends the thread in hardware until phase `parity`
+// completes or about `hint_ns` pass (whichever is first): a waiting thread
+// takes no issue slots and wakes as soon as the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity,
+                                                   uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; "
+      "selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for phase `parity`; false if it has not completed timeout_ns after
 // the first unsuccessful probe.  The first probes follow one another at
 // once (try_wait itself suspends the thread briefly in hardware), so a

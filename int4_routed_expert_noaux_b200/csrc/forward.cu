@@ -10,11 +10,11 @@ namespace moe {
 moe_status route_impl(const moe_layer* l, const uint16_t* x, int T, int32_t* idx, float* w,
                       float* scores, uint8_t* ws, const WsLayout& L, cudaStream_t st) {
   const moe_config& c = l->cfg;
-  float* sc = reinterpret_cast<float*>(ws + L.logits);
-  cudaError_t e = launch_router_scores(l->w_router, x, T, c.hidden, c.n_experts, sc, st);
+  double* part = reinterpret_cast<double*>(ws + L.logits);
+  cudaError_t e = launch_router_partial(l->w_router, x, T, c.hidden, c.n_experts, part, st);
   if (e == cudaSuccess)
-    e = launch_select(sc, l->bias, T, c.n_experts, c.n_group, c.topk_group, c.top_k,
-                      c.routed_scaling_factor, l->top_p, idx, w, scores, st);
+    e = launch_select(part, c.hidden, l->bias, T, c.n_experts, c.n_group, c.topk_group,
+                      c.top_k, c.routed_scaling_factor, l->top_p, idx, w, scores, st);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "route launch");
 }
 

@@ -11,56 +11,61 @@
 namespace moe {
 
 // ---------------------------------------------------------------------------
-// Router GEMV and sigmoid ("LightLX", "How it works": one router logit per
-// routed expert, sigmoid scores).  One CTA per expert row of W (fp32
-// [E][H]): each thread takes 8-input chunks of the row (the row's chunk c
-// and the tokens' chunk c) and accumulates them against TT tokens at a
-// time in fp64: every product of an fp32 weight and a bf16 input is exact
-// in fp64 (32 significant bits), so the logit carries only the fp64
-// rounding of the sums (about 1e-16 relative); the sigmoid is taken in fp64
-// and rounded to fp32 once.  scores [T][E] = fp32(sigmoid(logit)).
+// Router GEMV ("LightLX", "How it works": one router logit per routed
+// expert) on the FP64 tensor cores: part[ks][t][e] = the sum over slice ks
+// of the K range (H / KS inputs) of w[e][k] x[t][k], by mma m8n8k4 in fp64
+// -- every product of an fp32 weight and a bf16 input is exact in fp64, the
+// sums are rounded in fp64 (about 1e-16 relative).  The selection kernel
+// adds the KS slices in order and takes the sigmoid in fp64.
+// CTA (ks, 8-expert tile); warp w: tokens 8w .. 8w + 7.  Within a 16-input
+// block the inputs are dealt to the MMA's K index as k = 4 (lane mod 4) + j
+// at step j, the same for the A (x) and B (w) fragments, so that each lane
+// loads 4 consecutive inputs once.
 
-template <int TT>
-__global__ void __launch_bounds__(256) router_scores_kernel(
-    const float* __restrict__ w, const uint16_t* __restrict__ x, int T, int H,
-    int E, float* __restrict__ scores) {
-  __shared__ double red[TT][8];
+__device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, double b) {
+  asm volatile(
+      "mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+      : "+d"(d0), "+d"(d1)
+      : "d"(a), "d"(b));
+}
+
+__global__ void __launch_bounds__(256) router_partial_kernel(
+    const float* __restrict__ w, const uint16_t* __restrict__ x, int T, int H, int E, int KS,
+    double* __restrict__ part) {
+  const int ks = blockIdx.x, e0 = blockIdx.y * 8;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x;
-  const float4* wr = reinterpret_cast<const float4*>(w + (size_t)e * H);
-  const int nchunk = H >> 3;
-  for (int t0 = 0; t0 < T; t0 += TT) {
-    double acc[TT];
-#pragma unroll
-    for (int t = 0; t < TT; ++t) acc[t] = 0.0;
-    for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
-      const float4 wa = __ldg(wr + 2 * c), wb = __ldg(wr + 2 * c + 1);
-      const double wd[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-#pragma unroll
-      for (int t = 0; t < TT; ++t) {
-        if (t0 + t < T) {
-          const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + t) * H) + c);
-          const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            acc[t] = fma(wd[2 * j], (double)bf16_bits_to_f32(xs[j] & 0xFFFFu), acc[t]);
-            acc[t] = fma(wd[2 * j + 1], (double)bf16_bits_to_f32(xs[j] >> 16), acc[t]);
-          }
-        }
-      }
+  const int t0 = warp * 8;
+  if (t0 >= T) return;
+  const int len = H / KS, k0 = ks * len;
+  const int r = lane >> 2, c = lane & 3;  // A row (token) and B column (expert); K index
+  // rows past T or E read row 0: their results land in D rows / columns
+  // that are not stored
+  const uint16_t* xr = x + (size_t)(t0 + r < T ? t0 + r : 0) * H + k0 + 4 * c;
+  const float* wr = w + (size_t)(e0 + r < E ? e0 + r : 0) * H + k0 + 4 * c;
+  // four accumulators (one per step j), added in order at the end: four
+  // independent MMA chains instead of one; the next block's loads are in
+  // flight while this block's MMAs run
+  double d[4][2] = {{0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}};
+  uint2 xv = __ldg(reinterpret_cast<const uint2*>(xr));
+  float4 wv = __ldg(reinterpret_cast<const float4*>(wr));
+  for (int kb = 0; kb < len; kb += 16) {
+    const uint2 xc = xv;
+    const float4 wc = wv;
+    if (kb + 16 < len) {
+      xv = __ldg(reinterpret_cast<const uint2*>(xr + kb + 16));
+      wv = __ldg(reinterpret_cast<const float4*>(wr + kb + 16));
     }
-#pragma unroll
-    for (int t = 0; t < TT; ++t) {
-      const double s = warp_sum_f64(acc[t]);
-      if (lane == 0) red[t][warp] = s;
-    }
-    __syncthreads();
-    if (threadIdx.x < TT && t0 + threadIdx.x < T) {
-      double s = 0.0;
-      for (int w8 = 0; w8 < (int)(blockDim.x >> 5); ++w8) s += red[threadIdx.x][w8];
-      scores[(size_t)(t0 + threadIdx.x) * E + e] = sigmoid_f64_to_f32(s);
-    }
-    __syncthreads();
+    dmma_8x8x4(d[0][0], d[0][1], (double)bf16_bits_to_f32(xc.x & 0xFFFFu), (double)wc.x);
+    dmma_8x8x4(d[1][0], d[1][1], (double)bf16_bits_to_f32(xc.x >> 16), (double)wc.y);
+    dmma_8x8x4(d[2][0], d[2][1], (double)bf16_bits_to_f32(xc.y & 0xFFFFu), (double)wc.z);
+    dmma_8x8x4(d[3][0], d[3][1], (double)bf16_bits_to_f32(xc.y >> 16), (double)wc.w);
+  }
+  // D[row = lane / 4][col = 2 (lane mod 4) + i]: token t0 + row, expert e0 + col
+  const int t = t0 + r, e = e0 + 2 * c;
+  if (t < T) {
+    double* pr = part + ((size_t)ks * T + t) * E;
+    if (e < E) pr[e] = ((d[0][0] + d[1][0]) + d[2][0]) + d[3][0];
+    if (e + 1 < E) pr[e + 1] = ((d[0][1] + d[1][1]) + d[2][1]) + d[3][1];
   }
 }
 
@@ -98,7 +103,7 @@ __device__ __forceinline__ ArgMax warp_argmax(ArgMax a) {
 }
 
 __global__ void __launch_bounds__(1024) select_kernel(
-    const float* __restrict__ scores, const float* __restrict__ bias, int E,
+    const double* __restrict__ part, int KS, int T, const float* __restrict__ bias, int E,
     int n_group, int topk_group, int top_k, float rsf, float top_p,
     int32_t* __restrict__ idx_out, float* __restrict__ w_out,
     float* __restrict__ scores_out) {
@@ -108,13 +113,23 @@ __global__ void __launch_bounds__(1024) select_kernel(
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per = E / n_group;
-  const float* sc = scores + (size_t)t * E;
 
   if (warp < n_group) {
     const int e = warp * per + lane;
     ArgMax a{0.f, -1};
     if (lane < per) {
-      const float s = sc[e];
+      // the logit: the K slices added in order; the sigmoid in fp64,
+      // rounded to fp32 once
+      double lg = 0.0;
+      for (int k0 = 0; k0 < KS; k0 += 8) {  // 8 loads in flight at a time
+        double pk[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          pk[j] = k0 + j < KS ? part[((size_t)(k0 + j) * T + t) * E + e] : 0.0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) lg += pk[j];
+      }
+      const float s = sigmoid_f64_to_f32(lg);
       const float sp = s + bias[e];
       s_score[e] = s;
       s_sel[e] = sp;
@@ -251,17 +266,29 @@ static int warps_for(int G) {
   return 4;
 }
 
-cudaError_t launch_router_scores(const float* w, const uint16_t* x, int T, int H, int E,
-                                 float* scores, cudaStream_t st) {
-  router_scores_kernel<8><<<E, 256, 0, st>>>(w, x, T, H, E, scores);
+// Slices of the router's K range: more for fewer tokens (a CTA's warps
+// take 8 tokens each), so that every call keeps the SMs busy.
+int router_slices(int H, int T) {
+  const int want = T <= 8 ? 32 : T <= 16 ? 16 : 8;
+  for (int ks = want; ks > 1; ks >>= 1)
+    if (H % (16 * ks) == 0) return ks;
+  return 1;
+}
+
+cudaError_t launch_router_partial(const float* w, const uint16_t* x, int T, int H, int E,
+                                  double* part, cudaStream_t st) {
+  if (H % 16 != 0 || T < 1 || T > 64) return cudaErrorInvalidValue;
+  const int ks = router_slices(H, T);
+  router_partial_kernel<<<dim3(ks, (E + 7) / 8), 32 * ((T + 7) / 8), 0, st>>>(w, x, T, H, E, ks,
+                                                                            part);
   return cudaGetLastError();
 }
 
-cudaError_t launch_select(const float* scores, const float* bias, int T, int E, int n_group,
-                          int topk_group, int top_k, float rsf, float top_p, int32_t* idx,
-                          float* w, float* scores_out, cudaStream_t st) {
-  select_kernel<<<T, 32 * n_group, 0, st>>>(scores, bias, E, n_group, topk_group, top_k, rsf,
-                                            top_p, idx, w, scores_out);
+cudaError_t launch_select(const double* part, int H, const float* bias, int T, int E,
+                          int n_group, int topk_group, int top_k, float rsf, float top_p,
+                          int32_t* idx, float* w, float* scores_out, cudaStream_t st) {
+  select_kernel<<<T, 32 * n_group, 0, st>>>(part, router_slices(H, T), T, bias, E, n_group,
+                                            topk_group, top_k, rsf, top_p, idx, w, scores_out);
   return cudaGetLastError();
 }
 

@@ -9,15 +9,20 @@
 
 namespace moe {
 
-// scores [T][E] = fp32(sigmoid(W x)), the logit summed in fp64.
-cudaError_t launch_router_scores(const float* w, const uint16_t* x, int T, int H, int E,
-                                 float* scores, cudaStream_t st);
-// noaux_tc selection from the sigmoid scores, then adaptive top-p when
-// top_p < 1 (dropped slots: id -1, weight 0, after the kept ids);
-// scores_out (nullable) gets a copy of the scores.
-cudaError_t launch_select(const float* scores, const float* bias, int T, int E, int n_group,
-                          int topk_group, int top_k, float rsf, float top_p, int32_t* idx,
-                          float* w, float* scores_out, cudaStream_t st);
+// Router logits in K slices: part [router_slices(H, T)][T][E] (fp64), each
+// the sum of W x over a slice of the inputs (1 <= T <= 64, H a multiple of
+// 16).
+constexpr int kRouterMaxSlices = 32;
+int router_slices(int H, int T);
+cudaError_t launch_router_partial(const float* w, const uint16_t* x, int T, int H, int E,
+                                  double* part, cudaStream_t st);
+// noaux_tc selection from the logits (slices added in order, sigmoid in
+// fp64 rounded to fp32), then adaptive top-p when top_p < 1 (dropped slots:
+// id -1, weight 0, after the kept ids); scores_out (nullable) gets the
+// fp32 sigmoid scores.
+cudaError_t launch_select(const double* part, int H, const float* bias, int T, int E,
+                          int n_group, int topk_group, int top_k, float rsf, float top_p,
+                          int32_t* idx, float* w, float* scores_out, cudaStream_t st);
 // The batched expert path (union.cu): distinct experts read once for all
 // their tokens.  Scratch: xq (T * H/32 groups), hq (T * slots * I/32 groups),
 // lists (union_lists_ints ints), hbuf (T * slots * I), ypart (T * slots * H).
@@ -64,8 +69,8 @@ __host__ __device__ __forceinline__ ListsView lists_view(const int* lists, int E
 // tc_bpack (nullable, tc_bpack_bytes(T, k, has_shared, H, I) bytes): the
 // packed inputs of the tensor-core path (tc_union.cu), taken by every
 // distinct expert with tc_min_tokens() to 64 tokens when the shape allows
-// it; the other experts run on the CUDA-core union kernels.  tc_maps
-// (tc_maps_bytes(), 128-byte aligned): the path's tensor-map slots.
+// it (tc_shape_ok); the other experts run on the CUDA-core union kernels.
+// tc_maps (tc_maps_bytes(), 128-byte aligned): the path's tensor-map slots.
 cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const float* w,
                              const uint16_t* x, int T, int H, int I, int E, int k, int has_shared,
                              uint8_t* xq_words, float* xq_fac, uint8_t* hq_words, float* hq_fac,

@@ -50,6 +50,7 @@
 #include "common.cuh"
 #include "device_once.h"
 #include "kernels.h"
+#include "tile_stream.cuh"
 
 namespace moe {
 
@@ -58,16 +59,21 @@ namespace {
 // Per-step timeline of CTA 0's second work item in a -DMOE_TRACE profiling
 // build (row 7: the end of each of CTA 0's items).
 #ifdef MOE_TRACE
-__device__ uint64_t g_tc_trace[14][256];
+__device__ uint64_t g_tc_trace[16][256];
+__device__ int g_tc_trace_mats = 1;  // the launch traced: 2 gate/up, 1 down
 #define TC_TRACE(kind, st)                                                          \
   do {                                                                              \
-    if (blockIdx.x == 0 && it == 1 && (st) < 256)                                   \
+    if (blockIdx.x == 0 && it == 1 && (st) < 256 && a.mats == g_tc_trace_mats)      \
       g_tc_trace[kind][st] = (uint64_t)clock64();                                   \
   } while (0)
-#define TC_TRACE_AT(kind, i) (g_tc_trace[kind][i] = (uint64_t)clock64())
+#define TC_TRACE_AT(kind, i)                                                        \
+  do {                                                                              \
+    if (a.mats == g_tc_trace_mats) g_tc_trace[kind][i] = (uint64_t)clock64();       \
+  } while (0)
 #define TC_TRACE_ITEM()                                                             \
   do {                                                                              \
-    if (blockIdx.x == 0 && it < 256) g_tc_trace[7][it] = (uint64_t)clock64();       \
+    if (blockIdx.x == 0 && it < 256 && a.mats == g_tc_trace_mats)                   \
+      g_tc_trace[7][it] = (uint64_t)clock64();                                      \
   } while (0)
 #else
 #define TC_TRACE(kind, st) ((void)0)
@@ -75,48 +81,31 @@ __device__ uint64_t g_tc_trace[14][256];
 #define TC_TRACE_ITEM() ((void)0)
 #endif
 
-constexpr int kWG = 2;                    // converter warpgroups (K halves)
 constexpr int kConvThreads = kWG * 128;
-// + six warps, separate so that one's waits (nanosleep back-off) never
-// hold up another's issue.  Four MMA issuers: a thread stalls about 90
-// cycles on each tcgen05.mma it issues (and more on its commit), while the
-// tensor cores finish an M=128 N<=64 K=16 MMA in about 45, so issuer j
-// takes the ring steps st = j (mod 4) -- warpgroup j % 2's groups -- into an
-// accumulator of its own.
+// + six warps, separate so that one's waits never hold up another's issue.
+// Four MMA issuers: a thread stalls about 90 cycles on each tcgen05.mma it
+// issues (and more on its commit), while the tensor cores finish an M=128
+// N<=64 K=16 MMA in about 45, so issuer j takes the ring steps st = j
+// (mod 4) -- warpgroup j % 2's groups -- into an accumulator of its own.
 constexpr int kWProdWarp = kConvThreads / 32;  // weight tiles (TMA), tensor maps
 constexpr int kBProdWarp = kWProdWarp + 1;     // packed inputs
 constexpr int kIssueWarp = kWProdWarp + 2;     // MMA issuer j: warp kIssueWarp + j
 constexpr int kIssuers = 2 * kWG;
 constexpr int kTcThreads = kConvThreads + 32 * (2 + kIssuers);
-constexpr int kGS = 8;                    // groups per weight stage: 128 bytes of codes a row
-constexpr int kSW = 3;                    // weight stages per warpgroup
-constexpr int kR = 8;                     // ring slots (A in tensor memory, B in shared memory)
+constexpr int kBRing = 64 * 1024;         // shared memory of the B ring
 constexpr int kNmax = 64;                 // most tokens per expert on this path
-constexpr int kColD = 0;                  // tensor memory: D of issuer j at j * kNmax
-constexpr int kColA = kIssuers * kNmax;   // then kR slots of 32 columns (hi 16, lo 16)
-constexpr int kMaps = 4;                  // tensor maps of an item (codes, scales) x matrices
-constexpr int kMapSets = 4;               // map sets per CTA, used by items in turn
-constexpr int kTcMaxCtas = 256;           // per-CTA tensor-map slots in the workspace
-static_assert(kMapSets - 1 >= 3, "a map set outlives the loads through it");
-constexpr uint32_t kWStageBytes = 128 * 128 + 128 * 16;
-constexpr uint64_t kTcWaitNs = 1000000000ull;
-static_assert(kColA + kR * 32 <= 512, "tensor memory columns");
+// Tensor memory: the accumulator of issuer j at columns j * Ncap (Ncap: the
+// call's most padded tokens of an expert), then the ring's A slots of 32
+// columns (hi 16, lo 16).  The ring has as many slots as tensor memory and
+// the B ring's shared memory hold at Ncap: 8 at 64 tokens, 12 at 32.
 static_assert(kTcMaxTok == kNmax, "the token bound of the path");
 
-struct __align__(1024) TcSmem {
-  uint8_t wc[kWG][kSW][128 * 128];        // code tiles: 128 rows x 8 groups, 128-byte swizzled
-  uint8_t wsc[kWG][kSW][128 * 16];        // scale tiles: 128 rows x 8 fp16
-  uint8_t b[kR][kNmax * 128];             // packed inputs of one group (down: hi then lo)
-  CUtensorMap tm[kMaps];                  // the item's tensor maps, before publishing
-  uint64_t w_full[kWG][kSW];              // a weight stage landed
-  uint64_t w_empty[kWG][kSW];             // the warpgroup's 4 warps read it
-  uint64_t a_full[kR];                    // converters wrote the slot's A (4 warps)
-  uint64_t b_full[kR];                    // the slot's B landed
-  uint64_t slot_free[kR];                 // the MMAs reading the slot finished
+struct __align__(1024) TcSmem : StreamSmem {
+  uint8_t b[kBRing];                      // B ring: slot s at s * Ncap * (64 or 128) bytes
+  uint64_t a_full[kRmax];                 // converters wrote the slot's A (4 warps)
   uint64_t fin;                           // all MMAs of the item finished (4 issuers)
   uint64_t d_free;                        // the item's accumulators were read (8 warps)
   uint32_t tmem_base;
-  int abort_flag;
 };
 static_assert(sizeof(TcSmem) + 1024 <= 232448, "shared memory per CTA");
 
@@ -179,37 +168,6 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&v)[8]) {
                : "memory");
 }
 
-// 2-D tiled TMA load of box (x, y) of a tensor map in global memory.
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
-      : "memory");
-}
-
-// Tensor-map updates: the global address of a map held in shared memory;
-// its copy to global memory with a release of the tensormap proxy (whole
-// warp); the acquire before the first load through it.
-__device__ __forceinline__ void tmap_set_address(CUtensorMap* smem_map, const void* addr) {
-  asm volatile("tensormap.replace.tile.global_address.shared::cta.b1024.b64 [%0], %1;" ::"r"(
-                   smem_addr(smem_map)),
-               "l"(addr)
-               : "memory");
-}
-__device__ __forceinline__ void tmap_publish(CUtensorMap* gmem_map, const CUtensorMap* smem_map) {
-  asm volatile(
-      "tensormap.cp_fenceproxy.global.shared::cta.tensormap::generic.release.gpu.sync.aligned"
-      " [%0], [%1], 128;" ::"l"(gmem_map),
-      "r"(smem_addr(smem_map))
-      : "memory");
-}
-__device__ __forceinline__ void tmap_acquire(const CUtensorMap* gmem_map) {
-  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(gmem_map)
-               : "memory");
-}
-
 // A group's fp16 scale s split for weights_hi_lo, as f16x2 pairs (both
 // halves equal): s_hi = s with its 4 low mantissa bits cleared (at most 7
 // significant bits), s_lo = s - s_hi (at most 4), and -24 times each (exact:
@@ -267,20 +225,6 @@ struct TcArgs {
   CUtensorMap* maps; // [grid][kMapSets][kMaps] global slots for the tensor maps
 };
 
-// Waits (bounded) in lane 0 and makes every lane an observer of the phase:
-// false (the same in all lanes) when the wait ran out.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int lane,
-                                          volatile int* abort_flag) {
-  int ok = 0;
-  if (lane == 0 && !*abort_flag) {
-    ok = mbar_wait(bar, parity, kTcWaitNs) ? 1 : 0;
-    if (!ok) *abort_flag = 1;
-  }
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  if (ok) mbar_test(bar, parity);
-  return ok != 0;
-}
-
 // tm_codes / tm_scales: templates of the item's maps (dimensions, strides,
 // boxes: codes uint8 [R][K/2], box 128 bytes x tile rows, 128-byte swizzle;
 // scales uint16 [R][G], box 8 x tile rows); each item points copies of them
@@ -301,8 +245,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int nst = ng / kGS;              // weight stages per warpgroup and item
   const int steps = kWG * ng;            // step s of an item: warpgroup s % kWG, its group s / kWG
   const int mb = a.mats == 2 ? 64 : 128;  // bytes of a packed input row of one group
-  const int nmaps = a.mats == 2 ? 4 : 2;
   volatile int* abort_flag = &S.abort_flag;
+  // the call's most padded tokens of an expert (every warp reduces it)
+  int ncap = 16;
+  for (int r = lane; r < L.counts[1]; r += 32) ncap = max(ncap, L.tc_roff[r + 1] - L.tc_roff[r]);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) ncap = max(ncap, __shfl_xor_sync(0xffffffffu, ncap, o));
+  // (a multiple of kBG: a B copy fills kBG consecutive slots)
+  const int kR =
+      min(kRmax, min((512 - kIssuers * ncap) / 32, kBRing / (ncap * mb))) / kBG * kBG;
+  const uint32_t colA = (uint32_t)(kIssuers * ncap);
+  const int bstride = ncap * mb;  // bytes of a B ring slot
 
   if (tid == 0) {
     for (int w = 0; w < kWG; ++w)
@@ -310,11 +263,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mbar_init(&S.w_full[w][s], 1);
         mbar_init(&S.w_empty[w][s], 4);
       }
-    for (int i = 0; i < kR; ++i) {
+    for (int i = 0; i < kRmax; ++i) {
       mbar_init(&S.a_full[i], 4);
-      mbar_init(&S.b_full[i], 1);
+
       mbar_init(&S.slot_free[i], 1);
     }
+    for (int i = 0; i < kRmax / kBG; ++i) mbar_init(&S.b_full[i], 1);
     mbar_init(&S.fin, kIssuers);
     mbar_init(&S.d_free, kConvThreads / 32);
     S.abort_flag = 0;
@@ -337,136 +291,65 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // tiles while the converters finish this one's epilogue.  An item's first
   // MMAs wait until the previous item's accumulators were read (d_free).
   int w_last[kWG][kSW];  // weight producer: last use issued per stage buffer
-  int b_last[kR];        // input producer: the same per ring slot
+  int b_last[kRmax / kBG];  // input producer: the same per B run
   for (int w = 0; w < kWG; ++w)
     for (int s = 0; s < kSW; ++s) w_last[w][s] = -1;
-  for (int i = 0; i < kR; ++i) b_last[i] = -1;
+  for (int i = 0; i < kRmax / kBG; ++i) b_last[i] = -1;
   const int* list_tok = L.list_tok;
   const int* list_pos = L.list_pos;
 
+  StreamGeom geom;
+  geom.items = items;
+  geom.tiles = tiles;
+  geom.tile_rows = tile_rows;
+  geom.mats = a.mats;
+  geom.ng = ng;
+  geom.nst = nst;
+  geom.steps = steps;
   if (warp == kWProdWarp) {
-    // ------------------------------------------------ weight producer
-    const uint64_t stream = l2_policy_evict_first();
-    for (int item = blockIdx.x, it = 0; item < items; item += gridDim.x, ++it) {
-      if (!__shfl_sync(0xffffffffu, lane == 0 ? !*abort_flag : 0, 0)) break;
-      const int e = L.u_expert[L.tc_u[item / tiles]];
-      const int r0 = (item % tiles) * tile_rows;
-      // the item's tensor maps: templates re-pointed at the expert, in map
-      // set it % kMapSets of the CTA.  A set is rewritten kMapSets items
-      // later; by then every load through it has landed (this producer has
-      // issued at least kMapSets - 1 >= kSW stages of the items between,
-      // each after the stage kSW before it was consumed).
-      CUtensorMap* gm = a.maps + ((size_t)blockIdx.x * kMapSets + (it % kMapSets)) * kMaps;
-      const ExpertPtrs ep = a.table[e];
-      if (lane < 8 * nmaps) {  // the templates into shared memory, 16 bytes a lane
-        const int j = lane >> 3, part = lane & 7;
-        const CUtensorMap* src = (j & 1) ? &tm_scales : &tm_codes;
-        reinterpret_cast<uint4*>(&S.tm[j])[part] = reinterpret_cast<const uint4*>(src)[part];
-      }
-      __syncwarp();
-      if (lane == 0) {
-        tmap_set_address(&S.tm[0], a.mats == 2 ? (const void*)ep.q_gate : (const void*)ep.q_down);
-        tmap_set_address(&S.tm[1], a.mats == 2 ? (const void*)ep.s_gate : (const void*)ep.s_down);
-        if (a.mats == 2) {
-          tmap_set_address(&S.tm[2], ep.q_up);
-          tmap_set_address(&S.tm[3], ep.s_up);
-        }
-      }
-      __syncwarp();
-      for (int j = 0; j < nmaps; ++j) tmap_publish(gm + j, &S.tm[j]);
-      int ok = 1;
-      if (lane == 0) {
-        for (int j = 0; j < nmaps; ++j) tmap_acquire(gm + j);
-        if (blockIdx.x == 0 && it < 256) TC_TRACE_AT(12, it);
-        for (int j = 0; j < nst && ok; ++j) {
-          for (int w = 0; w < kWG; ++w) {
-            const int q = it * nst + j, sb = q % kSW, use = q / kSW;
-            if (use > 0 &&
-                !mbar_wait(&S.w_empty[w][sb], (uint32_t)((use - 1) & 1), kTcWaitNs)) {
-              *abort_flag = 1;
-              ok = 0;
-              break;
-            }
-            const int g = w * ng + j * kGS;  // first group of the stage
-            if (w == 0) TC_TRACE(13, j);
-            uint64_t* bar = &S.w_full[w][sb];
-            mbar_arrive_expect_tx(bar, kWStageBytes);
-            w_last[w][sb] = use;
-            if (a.mats == 2) {
-              // tile rows 32 qd .. + 15: gate rows r0 + 16 qd ..; the next
-              // 16: the up rows of the same indices
-              for (int qd = 0; qd < 4; ++qd) {
-                const int y = r0 + 16 * qd;
-                tma_load_2d(S.wc[w][sb] + (32 * qd) * 128, gm + 0, g * 16, y, bar, stream);
-                tma_load_2d(S.wc[w][sb] + (32 * qd + 16) * 128, gm + 2, g * 16, y, bar, stream);
-                tma_load_2d(S.wsc[w][sb] + (32 * qd) * 16, gm + 1, g, y, bar, stream);
-                tma_load_2d(S.wsc[w][sb] + (32 * qd + 16) * 16, gm + 3, g, y, bar, stream);
-              }
-            } else {
-              tma_load_2d(S.wc[w][sb], gm + 0, g * 16, r0, bar, stream);
-              tma_load_2d(S.wsc[w][sb], gm + 1, g, r0, bar, stream);
-            }
-          }
-        }
-      }
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-    }
+    stream_weights(S, geom, a.table, L.u_expert, L.tc_u, a.maps, tm_codes, tm_scales, lane,
+                   abort_flag, w_last);
   } else if (warp == kBProdWarp) {
-    if (lane == 0) {
-      // ---------------------------------------------- input producer
-      const uint64_t keep = l2_policy_evict_last();
-      for (int item = blockIdx.x, it = 0; item < items && !*abort_flag;
-           item += gridDim.x, ++it) {
-        const int rank = item / tiles;
-        const int roff = L.tc_roff[rank], N = L.tc_roff[rank + 1] - roff;
-        const uint32_t bcopy = (uint32_t)(N * mb);
-        const uint8_t* bsrc = a.bpack + (size_t)roff * a.G * mb;
-        for (int st = 0; st < steps; ++st) {
-          const int q = it * steps + st, slot = q % kR, use = q / kR;
-          if (use > 0 && !mbar_wait(&S.slot_free[slot], (uint32_t)((use - 1) & 1), kTcWaitNs)) {
-            *abort_flag = 1;
-            break;
-          }
-          const int g = (st % kWG) * ng + st / kWG;
-          TC_TRACE(0, st);
-          mbar_arrive_expect_tx(&S.b_full[slot], bcopy);
-          b_last[slot] = use;
-          bulk_g2s(S.b[slot], bsrc + (size_t)g * bcopy, bcopy, &S.b_full[slot], keep);
-        }
-      }
-    }
+    if (lane == 0)
+      stream_inputs(S, S.b, geom, L.tc_roff, a.bpack, a.G, mb, bstride, kR, abort_flag, b_last);
   } else if (warp >= kIssueWarp) {
     if (lane == 0) {
       // ---------------------------------------------- MMA issuers
       const int j = warp - kIssueWarp;
-      const uint32_t d = tmem + (uint32_t)(kColD + j * kNmax);
+      const uint32_t d = tmem + (uint32_t)(j * ncap);
+      RingPos pos;  // ring step it * steps + st
+      pos.advance(j, kR);
       for (int item = blockIdx.x, it = 0; item < items; item += gridDim.x, ++it) {
         const int rank = item / tiles;
         const int N = L.tc_roff[rank + 1] - L.tc_roff[rank];
         const uint32_t idesc = umma_idesc_f16(128, N);
         // the previous item's accumulators have been read
         if (*abort_flag ||
-            (it > 0 && !mbar_wait(&S.d_free, (uint32_t)((it - 1) & 1), kTcWaitNs))) {
+            (it > 0 && !stream_wait(&S.d_free, (uint32_t)((it - 1) & 1)))) {
           *abort_flag = 1;
           tc_commit(&S.fin);
           break;
         }
         tc_fence_after();
         for (int st = j; st < steps; st += kIssuers) {
-          const int q = it * steps + st, slot = q % kR, use = q / kR;
-          if (*abort_flag || !mbar_wait(&S.a_full[slot], (uint32_t)(use & 1), kTcWaitNs)) {
+          const int slot = pos.slot, use = pos.use;
+          pos.advance(kIssuers, kR);
+          if (*abort_flag || !stream_wait(&S.a_full[slot], (uint32_t)(use & 1))) {
             *abort_flag = 1;
             break;
           }
           TC_TRACE(1, st);
-          if (!mbar_wait(&S.b_full[slot], (uint32_t)(use & 1), kTcWaitNs)) {
+          if (!stream_wait(&S.b_full[slot / kBG], (uint32_t)(use & 1))) {
             *abort_flag = 1;
             break;
           }
           TC_TRACE(2, st);
           tc_fence_after();
-          const uint32_t ahi = tmem + (uint32_t)(kColA + slot * 32), alo = ahi + 16;
-          const uint32_t bhi = smem_addr(S.b[slot]), blo = bhi + (uint32_t)N * 64;
+          const uint32_t ahi = tmem + colA + (uint32_t)(slot * 32), alo = ahi + 16;
+          // step q's inputs: kBG steps of N rows each from the run's first slot
+          const uint32_t bhi = smem_addr(S.b + (slot / kBG * kBG) * bstride) +
+                               (uint32_t)((slot % kBG) * N * mb),
+                         blo = bhi + (uint32_t)N * 64;
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk) {
             const uint64_t dh = umma_desc(bhi + kk * 256, 128, 512);
@@ -488,6 +371,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int wg = warp >> 2, row = (warp & 3) * 32 + lane;  // row = tensor-memory lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t swz = (uint32_t)(row & 7);
+    RingPos pos;  // ring step of this warpgroup's next group
+    pos.advance(wg, kR);
     for (int item = blockIdx.x, it = 0; item < items; item += gridDim.x, ++it) {
       const int rank = item / tiles;
       const int u = L.tc_u[rank];
@@ -511,7 +396,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           uint32_t hl[32];
           weights_hi_lo(w, group_scale(sh), hl);
           const int i = j * kGS + c;  // group of this warpgroup
-          const int st = i * kWG + wg, qs = it * steps + st, slot = qs % kR, suse = qs / kR;
+          [[maybe_unused]] const int st = i * kWG + wg;  // the item's ring step (traces)
+          const int slot = pos.slot, suse = pos.use;
+          pos.advance(kWG, kR);
           if (row == 0) TC_TRACE(4, st);
           // the slot's previous MMAs (ring step qs - kR) have finished
           if (suse > 0) {
@@ -522,7 +409,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_after();
           }
           if (row == 0) TC_TRACE(5, st);
-          tmem_st32(tmem + lane_base + (uint32_t)(kColA + slot * 32), hl);
+          tmem_st32(tmem + lane_base + colA + (uint32_t)(slot * 32), hl);
           asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
           if (row == 0) TC_TRACE(6, st);
           if (lane == 0) TC_TRACE(8 + (warp & 3), st);
@@ -543,15 +430,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_after();
       const int half = N >> 1, t0 = wg * half;
       float sum[kNmax / 2];
-      const uint32_t dl = tmem + lane_base + (uint32_t)(kColD + t0);
+      const uint32_t dl = tmem + lane_base + (uint32_t)t0;
 #pragma unroll
       for (int c = 0; c < kNmax / 2; c += 8) {
         if (c < half) {
           uint32_t v0[8], v1[8], v2[8], v3[8];
-          tmem_ld8(dl + (uint32_t)(0 * kNmax + c), v0);
-          tmem_ld8(dl + (uint32_t)(2 * kNmax + c), v2);
-          tmem_ld8(dl + (uint32_t)(1 * kNmax + c), v1);
-          tmem_ld8(dl + (uint32_t)(3 * kNmax + c), v3);
+          tmem_ld8(dl + (uint32_t)(0 * ncap + c), v0);
+          tmem_ld8(dl + (uint32_t)(2 * ncap + c), v2);
+          tmem_ld8(dl + (uint32_t)(1 * ncap + c), v1);
+          tmem_ld8(dl + (uint32_t)(3 * ncap + c), v3);
           asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
           for (int t = 0; t < 8; ++t)
@@ -563,47 +450,50 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.d_free);
-      if (a.mats == 2) {
-        // h = silu(gate) * up: lane m < 16 of quarter q holds gate row
-        // r0 + 16 q + m, lane m + 16 the up row of the same index
-        const int hrow = r0 + 16 * (warp & 3) + (lane & 15);
+      // 8 tokens at a time: their output rows and input scales first (the
+      // lists are read-only in this kernel: non-coherent loads, which the
+      // stores before them do not hold back), then the outputs
+      const int orow = a.mats == 2 ? r0 + 16 * (warp & 3) + (lane & 15) : r0 + row;
 #pragma unroll
-        for (int c = 0; c < kNmax / 2; ++c) {
-          if (c < half) {
-            const float up = __shfl_down_sync(0xffffffffu, sum[c], 16);
-            const int t = t0 + c;
-            if (lane < 16 && t < n) {
-              const float f = ldexpf(1.0f, a.row_exp[list_tok[base + t]]);
-              a.out[(size_t)list_pos[base + t] * a.R + hrow] = silu_mul(sum[c] * f, up * f);
+      for (int c0 = 0; c0 < kNmax / 2; c0 += 8) {
+        if (c0 < half) {
+          int pos[8];
+          float f[8];
+#pragma unroll
+          for (int u8 = 0; u8 < 8; ++u8) {
+            const int t = t0 + c0 + u8;
+            pos[u8] = 0;
+            f[u8] = 0.f;
+            if (t < n) {
+              pos[u8] = __ldg(list_pos + base + t);
+              const int in_row = a.mats == 2 ? __ldg(list_tok + base + t) : pos[u8];
+              f[u8] = ldexpf(1.0f, __ldg(a.row_exp + in_row));
             }
           }
-        }
-      } else {
 #pragma unroll
-        for (int c = 0; c < kNmax / 2; ++c) {
-          const int t = t0 + c;
-          if (c < half && t < n)
-            a.out[(size_t)list_pos[base + t] * a.R + r0 + row] =
-                sum[c] * ldexpf(1.0f, a.row_exp[list_pos[base + t]]);
+          for (int u8 = 0; u8 < 8; ++u8) {
+            const int t = t0 + c0 + u8;
+            if (a.mats == 2) {
+              // h = silu(gate) * up: lane m < 16 of quarter q holds gate row
+              // r0 + 16 q + m, lane m + 16 the up row of the same index
+              const float up = __shfl_down_sync(0xffffffffu, sum[c0 + u8], 16);
+              if (lane < 16 && t < n)
+                a.out[(size_t)pos[u8] * a.R + orow] =
+                    silu_mul(sum[c0 + u8] * f[u8], up * f[u8]);
+            } else if (t < n) {
+              a.out[(size_t)pos[u8] * a.R + orow] = sum[c0 + u8] * f[u8];
+            }
+          }
         }
       }
     }
   }
   // A wait that ran out leaves the rest of the call's results unwritten
-  // and reports it.  Copies may still be in flight into this CTA's shared
-  // memory: each producer waits (bounded) for the last one it issued into
-  // every buffer before the CTA exits.
+  // and reports it (after the producers drained their copies).
   __syncthreads();
   if (*abort_flag) {
     if (tid == 0) atomicCAS(a.err, 0u, (uint32_t)kErrTimeout);
-    if (warp == kWProdWarp && lane == 0)
-      for (int w = 0; w < kWG; ++w)
-        for (int s = 0; s < kSW; ++s)
-          if (w_last[w][s] >= 0)
-            mbar_wait(&S.w_full[w][s], (uint32_t)(w_last[w][s] & 1), kTcWaitNs);
-    if (warp == kBProdWarp && lane == 0)
-      for (int i = 0; i < kR; ++i)
-        if (b_last[i] >= 0) mbar_wait(&S.b_full[i], (uint32_t)(b_last[i] & 1), kTcWaitNs);
+    stream_drain(S, warp, lane, kWProdWarp, kBProdWarp, kR, w_last, b_last);
   }
   __syncthreads();
   if (warp == 0) {
@@ -663,7 +553,9 @@ __device__ __forceinline__ uint16_t f32_to_f16_rne(float f) {
 
 // Packs the inputs of every path expert: for expert rank r and group g, the
 // B operand of its MMAs, rows = its tokens (zero rows up to N, a multiple of
-// 16), at byte (tc_roff[r] * G + g * N) * (64, down: 128), in the canonical
+// 16), at byte (tc_roff[r] * G + s * N) * (64, down: 128) where s is the
+// group's ring step (2 (g mod G/2) + g div G/2: the two warpgroups' groups
+// alternate, so consecutive steps' inputs are contiguous), in the canonical
 // K-major layout [N/8][4][8 rows][8 inputs] of fp16, inputs in the MMA order,
 // each row divided by 2^row_exp.
 // Gate/up: x (bf16 -> fp16, exact within fp16's range).  Down: h (fp32) as
@@ -721,8 +613,10 @@ __global__ void __launch_bounds__(256) tc_pack_kernel(const int* lists, int E, i
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = 0.f;
     }
+    // group g's tile at its ring step (warpgroup g / (G/2), its group g % (G/2));
     // core matrix (nr / 8, cb) at ((nr / 8) * 4 + cb) * 128 bytes, row nr % 8
-    uint8_t* dst = dst0 + (size_t)g * gbytes + (size_t)(nr >> 3) * 512 + (size_t)(nr & 7) * 16;
+    const int half_g = G / kWG, step = kWG * (g % half_g) + g / half_g;
+    uint8_t* dst = dst0 + (size_t)step * gbytes + (size_t)(nr >> 3) * 512 + (size_t)(nr & 7) * 16;
 #pragma unroll
     for (int cb = 0; cb < 4; ++cb) {
       uint32_t hi[4], lo[4];
@@ -746,42 +640,6 @@ __global__ void __launch_bounds__(256) tc_pack_kernel(const int* lists, int E, i
   }
 }
 
-// cuTensorMapEncodeTiled, reached through the runtime's driver entry points
-// (no link-time dependency on libcuda).
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_tiled() {
-  static const EncodeTiledFn fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
-                                         &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess) {
-      cudaGetLastError();
-      return (EncodeTiledFn) nullptr;
-    }
-    return reinterpret_cast<EncodeTiledFn>(p);
-  }();
-  return fn;
-}
-
-// A 2-D map over a row-major matrix [rows][inner] of elements of `bytes`
-// bytes; base is any 16-byte aligned address (the kernel re-points it).
-bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, int bytes, void* base, uint64_t inner,
-               uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
-  const EncodeTiledFn fn = encode_tiled();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {inner, rows};
-  const cuuint64_t strides[1] = {inner * (uint64_t)bytes};
-  const cuuint32_t box[2] = {box_inner, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 std::atomic<int> g_tc_min{kTcMinTokDefault};
 
 }  // namespace
@@ -791,6 +649,10 @@ int tc_min_tokens() { return g_tc_min.load(std::memory_order_relaxed); }
 #ifdef MOE_TRACE
 extern "C" __attribute__((visibility("default"))) int moe_debug_tc_trace(void* host_dst) {
   return (int)cudaMemcpyFromSymbol(host_dst, g_tc_trace, sizeof(g_tc_trace));
+}
+
+extern "C" __attribute__((visibility("default"))) int moe_debug_tc_trace_mats(int mats) {
+  return (int)cudaMemcpyToSymbol(g_tc_trace_mats, &mats, sizeof(int));
 }
 
 // Profiling builds: the least token count of a tensor-core expert.
@@ -819,11 +681,11 @@ size_t tc_bpack_bytes(int T, int k, int has_shared, int H, int I) {
 
 size_t tc_rowexp_ints(int T, int k, int has_shared) { return (size_t)T * (k + has_shared); }
 
-size_t tc_maps_bytes() { return (size_t)kTcMaxCtas * kMapSets * kMaps * sizeof(CUtensorMap); }
+size_t tc_maps_bytes() { return stream_maps_bytes(); }
 
 // Weight stages of 8 groups per warpgroup half of K: K a multiple of 512.
 bool tc_shape_ok(int H, int I) {
-  return H % 512 == 0 && I % 512 == 0 && encode_tiled() != nullptr;
+  return H % 512 == 0 && I % 512 == 0 && tensor_maps_available();
 }
 
 cudaError_t launch_tc_ffn_step(int mats, const ExpertPtrs* table, const int* lists, int E,
@@ -882,7 +744,7 @@ cudaError_t launch_tc_ffn_step(int mats, const ExpertPtrs* table, const int* lis
   // persistent: one CTA per SM (its shared memory and 512 tensor-memory
   // columns), no more CTAs than the call can have work items
   const int tiles = R / tile_rows;
-  const int grid = std::min(std::min(num_sms(), kTcMaxCtas), tcmax * tiles);
+  const int grid = std::min(std::min(num_sms(), kStreamMaxCtas), tcmax * tiles);
   tc_gemm_kernel<<<grid, kTcThreads, sizeof(TcSmem) + 1024, st>>>(a, tm_codes, tm_scales);
   return cudaGetLastError();
 }
