@@ -397,6 +397,15 @@ def launches_per_forward():
     return 1
 
 
+def launches_per_verify_call(T, shape):
+    """Kernels of one T-token moe_layer_forward: router, selection, x groups,
+    expert lists, gate/up, h groups, down, combine; plus row scales, packing
+    and the tensor-core kernel for both projections when 16 or more tokens
+    can share an expert (the tensor-core path's shapes: H, I multiples of 512)."""
+    tc = T >= 16 and shape.hidden % 512 == 0 and shape.inter % 512 == 0
+    return 8 + (6 if tc else 0)
+
+
 def max_over_ranks(value, dist=None, device="cuda"):
     """The largest value over all ranks (every rank gets it): a multi-GPU
     time is the slowest rank's."""
@@ -502,7 +511,7 @@ def run_mode(args, shape):
                              "frac": achieved / peak, "traffic": None, "peak_source": peak_kind,
                              "kernel": "moe_layer_forward (T tokens)",
                              "algorithmic_bytes_per_launch": byts / calls, "launch_us": call_us},
-                "gpu_launches": calls * args.steps * 8})
+                "gpu_launches": calls * args.steps * launches_per_verify_call(T, shape)})
         return
 
     if args.mode == "stack":
