@@ -172,7 +172,11 @@ moe_status moe_expert_ffn(const moe_layer* layer, const void* x_dev, int T,
 /* Steps 1-5 for T tokens.  idx_out_dev / w_out_dev nullable.  T == 1 runs the
  * single fused persistent decode kernel; T > 1 runs the batched path, which
  * reads every distinct selected expert once for all tokens routed to it.
- * 1 <= T <= 64. */
+ * 1 <= T <= 64.
+ * The fused kernel (T == 1 here, moe_layer_forward_residual,
+ * moe_stack_forward, moe_layer_forward_noalloc) needs the whole device: one
+ * CTA on every SM at once, launched cooperatively.  When SMs are held by
+ * other work the launch fails (MOE_ERR_CUDA) instead of waiting. */
 moe_status moe_layer_forward(const moe_layer* layer, const void* x_dev, int T,
                              float* y_dev, int32_t* idx_out_dev,
                              float* w_out_dev, void* ws_dev, size_t ws_bytes,

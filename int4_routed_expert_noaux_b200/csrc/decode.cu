@@ -600,8 +600,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
 
   // the producer's first-item offset (0 but in a failure test), loaded
   // before anything else so that its round trip is over by the first fill
-  const uint32_t gu_offset =
-      threadIdx.x == kProducerWarp * 32 ? ld_relaxed_u32(p.ctrl + kCtrlTicket) : 0u;
   if (threadIdx.x == kProducerWarp * 32) {
     // the producer thread sets up the barriers and sends the CTA's first
     // fill (its router rows, the head of the dependent start-up chain)
@@ -627,6 +625,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       TRACE_AT(1);
     }
   }
+  // Programmatic dependent launch: the next call on the stream may start its
+  // prologue (barriers, its router rows' fill: inputs no call writes) as
+  // this grid's CTAs leave their SMs; everything an earlier call writes --
+  // the control words, x of a stack's next layer -- is read after the wait.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the producer's first-item offset (0 but in a failure test)
+  const uint32_t gu_offset =
+      threadIdx.x == kProducerWarp * 32 ? ld_relaxed_u32(p.ctrl + kCtrlTicket) : 0u;
   if (p.x_resid) {
     // RMSNorm with unit gain ("LightLX", "How it works": RMSNorm of the
     // upstream model): every CTA forms the same fixed-order sum of squares.
@@ -1262,9 +1269,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
 // every CTA's router records; down items wait on other CTAs' gate/up
 // counts), so it is launched cooperatively: a grid that cannot be
 // co-resident (another kernel holding SMs, a partitioned device) fails at
-// launch instead of running into the device-side wait limit.  The first
-// launch per device and context sets the shared-memory attribute and checks
-// that one CTA fits on an SM.
+// launch instead of running into the device-side wait limit.  It is also a
+// programmatic dependent launch: its prologue may overlap the end of the
+// previous call on the stream (the kernel waits on griddepcontrol before it
+// reads anything an earlier call writes).  The first launch per device and
+// context sets the shared-memory attribute and checks that one CTA fits on
+// an SM.
 template <int SEG_G, int SEG_D>
 cudaError_t launch_t(const DecodeParams& p, cudaStream_t st) {
   static DeviceOnce<bool> configured;
@@ -1291,11 +1301,13 @@ cudaError_t launch_t(const DecodeParams& p, cudaStream_t st) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, decode_kernel<SEG_G, SEG_D>, p);
 }
 
