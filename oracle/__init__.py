@@ -59,6 +59,8 @@ def lib():
         L.orc_rmsnorm.argtypes = [p, i, d, p]
         L.orc_lru_sim.restype = i
         L.orc_lru_sim.argtypes = [i, i, i, i, i, p, p, p]
+        L.orc_lru_sim_pinned.restype = i
+        L.orc_lru_sim_pinned.argtypes = [i, i, i, i, i, p, i, p, p, p]
         _lib = L
     return _lib
 
@@ -240,6 +242,21 @@ def lru_sim(trace, n_experts, capacity):
     hits = np.zeros((L,), dtype=np.uint64)
     misses = np.zeros((L,), dtype=np.uint64)
     rc = lib().orc_lru_sim(L, n_experts, capacity, k, T, _p(tr), _p(hits), _p(misses))
+    if rc != 0:
+        raise ValueError("bad LRU simulation arguments")
+    return hits, misses
+
+
+def lru_sim_pinned(trace, n_experts, capacity, pinned):
+    """trace [T][L][k] int32, pinned [L][n_pin] -> (hits[L], misses[L]):
+    the LRU with each layer's pinned experts held for the whole trace."""
+    tr = _c(trace, np.int32)
+    T, L, k = tr.shape
+    pn = _c(np.asarray(pinned).reshape(L, -1), np.int32)
+    hits = np.zeros((L,), dtype=np.uint64)
+    misses = np.zeros((L,), dtype=np.uint64)
+    rc = lib().orc_lru_sim_pinned(L, n_experts, capacity, k, T, _p(tr), pn.shape[1], _p(pn),
+                                  _p(hits), _p(misses))
     if rc != 0:
         raise ValueError("bad LRU simulation arguments")
     return hits, misses

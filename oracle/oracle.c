@@ -441,3 +441,72 @@ int orc_lru_sim(int n_layers, int n_experts, int capacity, int k, int T,
   free(slot_id); free(stamp);
   return 0;
 }
+
+/* Per-layer LRU with a pinned hot-store (colibri summary, "Learning cache et
+ * attentes selon le materiel": the most used experts are pinned at start-up;
+ * reading R19).  The n_pin experts pinned[l][..] of layer l occupy n_pin of
+ * the capacity slots for the whole trace and always hit; every other id runs
+ * the LRU rule of orc_lru_sim over the remaining capacity - n_pin slots,
+ * which start empty. */
+int orc_lru_sim_pinned(int n_layers, int n_experts, int capacity, int k, int T,
+                       const int32_t* trace, int n_pin, const int32_t* pinned,
+                       uint64_t* hits, uint64_t* misses) {
+  if (n_layers <= 0 || k <= 0 || T < 0 || !trace || n_pin < 0 || capacity - n_pin < k ||
+      (n_pin > 0 && !pinned))
+    return -1;
+  const int free_slots = capacity - n_pin;
+  int32_t* slot_id = (int32_t*)malloc(sizeof(int32_t) * (size_t)free_slots);
+  uint64_t* stamp = (uint64_t*)malloc(sizeof(uint64_t) * (size_t)free_slots);
+  char* is_pinned = (char*)malloc((size_t)n_experts);
+  int rc = 0;
+  for (int l = 0; l < n_layers && rc == 0; ++l) {
+    uint64_t clock = 0, h = 0, m = 0;
+    memset(is_pinned, 0, (size_t)n_experts);
+    for (int j = 0; j < n_pin; ++j) {
+      const int32_t e = pinned[(size_t)l * n_pin + j];
+      if (e < 0 || e >= n_experts || is_pinned[e]) { rc = -1; break; }
+      is_pinned[e] = 1;
+    }
+    for (int i = 0; i < free_slots; ++i) { slot_id[i] = -1; stamp[i] = 0; }
+    for (int t = 0; t < T && rc == 0; ++t) {
+      const int32_t* ids = trace + ((size_t)t * n_layers + l) * (size_t)k;
+      for (int j = 0; j < k; ++j)
+        if (ids[j] < 0 || ids[j] >= n_experts) rc = -1;
+      if (rc) break;
+      /* pinned ids hit; cached ids hit and are touched, ascending */
+      for (int j = 0; j < k; ++j) {
+        if (is_pinned[ids[j]]) { ++h; continue; }
+        for (int i = 0; i < free_slots; ++i)
+          if (slot_id[i] == ids[j]) { stamp[i] = ++clock; ++h; break; }
+      }
+      /* the other ids, ascending: lowest empty slot, else the least
+       * recently used slot not holding one of this call's ids */
+      for (int j = 0; j < k; ++j) {
+        if (is_pinned[ids[j]]) continue;
+        int found = 0;
+        for (int i = 0; i < free_slots; ++i)
+          if (slot_id[i] == ids[j]) { found = 1; break; }
+        if (found) continue;
+        int victim = -1;
+        for (int i = 0; i < free_slots && victim < 0; ++i)
+          if (slot_id[i] < 0) victim = i;
+        if (victim < 0) {
+          for (int i = 0; i < free_slots; ++i) {
+            int current = 0;
+            for (int jj = 0; jj < k; ++jj)
+              if (slot_id[i] == ids[jj]) current = 1;
+            if (current) continue;
+            if (victim < 0 || stamp[i] < stamp[victim]) victim = i;
+          }
+        }
+        slot_id[victim] = ids[j];
+        stamp[victim] = ++clock;
+        ++m;
+      }
+    }
+    hits[l] = h;
+    misses[l] = m;
+  }
+  free(slot_id); free(stamp); free(is_pinned);
+  return rc;
+}

@@ -145,6 +145,11 @@ void orc_rmsnorm(const double* x, int n, double eps, double* out);
  * (per layer).  Returns 0, or -1 when capacity < k or args are bad. */
 int orc_lru_sim(int n_layers, int n_experts, int capacity, int k, int T,
                 const int32_t* trace, uint64_t* hits, uint64_t* misses);
+/* orc_lru_sim with n_pin experts per layer (pinned [L][n_pin]) pinned for
+ * the whole trace: they always hit and hold n_pin of the slots. */
+int orc_lru_sim_pinned(int n_layers, int n_experts, int capacity, int k, int T,
+                       const int32_t* trace, int n_pin, const int32_t* pinned,
+                       uint64_t* hits, uint64_t* misses);
 
 #ifdef __cplusplus
 }

@@ -542,6 +542,46 @@ def test_lru_invariants_on_zipf_trace():
     assert np.all(m128 <= m8)
 
 
+def test_lru_pinned_hand_worked():
+    # capacity 3, k 2, expert 0 pinned: the LRU part has 2 slots.
+    # t0 {0,1}: 0 pinned hit; 1 -> empty slot            h1 m1
+    # t1 {0,2}: 0 hit; 2 -> empty slot                   h1 m1   [1@1 2@2]
+    # t2 {1,2}: both hit, touched 1 then 2               h2 m0   [1@3 2@4]
+    # t3 {0,3}: 0 hit; 3 evicts the LRU of {1,2}: 1      h1 m1   [3@5 2@4]
+    # t4 {1,3}: 3 hit; 1 evicts the LRU not in {1,3}: 2  h1 m1
+    trace = np.array([[[0, 1]], [[0, 2]], [[1, 2]], [[0, 3]], [[1, 3]]], dtype=np.int32)
+    h, m = oracle.lru_sim_pinned(trace, 4, 3, np.array([[0]]))
+    assert h.tolist() == [6] and m.tolist() == [4]
+    # the same trace unpinned: 0 is evicted at t2 (the LRU then) and misses at t3
+    h, m = oracle.lru_sim(trace, 4, 3)
+    assert h.tolist() == [5] and m.tolist() == [5]
+    # fewer than k free slots left is refused
+    with pytest.raises(ValueError):
+        oracle.lru_sim_pinned(trace, 4, 3, np.array([[0, 1]]))
+
+
+def test_lru_pinned_special_cases():
+    tr = synth.zipf_trace(3, 2, 64, 4, 300)
+    # nothing pinned: the plain LRU
+    for cap in (4, 9, 32):
+        h0, m0 = oracle.lru_sim_pinned(tr, 64, cap, np.zeros((2, 0), dtype=np.int32))
+        h1, m1 = oracle.lru_sim(tr, 64, cap)
+        assert np.array_equal(h0, h1) and np.array_equal(m0, m1)
+    # pinned experts never miss; with room for every other id seen, only
+    # the first access of each unpinned id misses
+    pinned = np.array([[0, 5, 17], [2, 3, 40]], dtype=np.int32)
+    for l in range(2):
+        other = np.setdiff1d(np.unique(tr[:, l, :]), pinned[l])
+        cap = 3 + len(other)
+        h, m = oracle.lru_sim_pinned(tr[:, l:l + 1, :], 64, cap, pinned[l:l + 1])
+        assert int(m[0]) == len(other)
+        assert int(h[0]) + int(m[0]) == 300 * 4
+    # a trace made only of pinned ids never misses
+    only = np.tile(np.array([[[0, 5]]], dtype=np.int32), (10, 1, 1))
+    h, m = oracle.lru_sim_pinned(only, 64, 4, np.array([[0, 5]]))
+    assert m.tolist() == [0] and h.tolist() == [20]
+
+
 # ---------------------------------------------------------------------------
 # byte figures printed on the pages (P1-P4)
 
