@@ -283,6 +283,24 @@ moe_status moe_cache_layer(moe_cache* cache, int layer,
 moe_status moe_cache_acquire(moe_cache* cache, int layer,
                              const int32_t* ids_host, int n,
                              void* compute_stream);
+/* Hot-store (colibri summary, "Learning cache et attentes selon le
+ * materiel": routed experts are logged and the most used are pinned at
+ * start-up).  Makes ids_host[0..n) (ascending, distinct) the pinned set of
+ * `layer`: each is made resident as by moe_cache_acquire (copies on the copy
+ * stream, compute_stream waits for them, the pointer table is updated on
+ * it) and its slot is never chosen as a victim afterwards; the previously
+ * pinned experts not in ids become ordinary LRU entries.  n = 0 unpins all.
+ * 0 <= n <= slots_per_layer - top_k, n <= 32.  Counts its bytes in
+ * bytes_h2d but not as hits, misses or usage.  Transactional like
+ * moe_cache_acquire.  With p experts pinned, an acquire takes at most
+ * slots_per_layer - p ids. */
+moe_status moe_cache_pin(moe_cache* cache, int layer, const int32_t* ids_host,
+                         int n, void* compute_stream);
+/* The usage log of `layer`: counts_host[e] (n_experts entries, caller-owned
+ * host memory) = how many committed moe_cache_acquire calls of the layer
+ * named expert e.  The ranking a caller pins by is its own choice. */
+moe_status moe_cache_usage(const moe_cache* cache, int layer,
+                           uint64_t* counts_host);
 /* Mark the end of the compute that reads `layer`'s slots on compute_stream. */
 moe_status moe_cache_release(moe_cache* cache, int layer, void* compute_stream);
 /* Cumulative counters of a layer (any pointer nullable). */
@@ -302,6 +320,14 @@ moe_status moe_cache_wait(moe_cache* cache, int timeout_ms);
 moe_status moe_lru_replay(int n_layers, int n_experts, int capacity, int k,
                           int T, const int32_t* trace, uint64_t* hits,
                           uint64_t* misses);
+/* moe_lru_replay with the hot-store: before the first call, experts
+ * pinned[l][0..n_pinned) (ascending) of each layer l are loaded and pinned
+ * as by moe_cache_pin (their loads are not counted); n_pinned <= capacity -
+ * k. */
+moe_status moe_lru_replay_pinned(int n_layers, int n_experts, int capacity,
+                                 int k, int T, const int32_t* trace,
+                                 int n_pinned, const int32_t* pinned,
+                                 uint64_t* hits, uint64_t* misses);
 
 /* ---- diagnostics ------------------------------------------------------- */
 

@@ -106,6 +106,12 @@ def lib():
         L.moe_debug_inject_fault.argtypes = [i, i]
         L.moe_lru_replay.restype = st
         L.moe_lru_replay.argtypes = [i, i, i, i, i, p, p, p]
+        L.moe_lru_replay_pinned.restype = st
+        L.moe_lru_replay_pinned.argtypes = [i, i, i, i, i, p, i, p, p, p]
+        L.moe_cache_pin.restype = st
+        L.moe_cache_pin.argtypes = [p, i, p, i, p]
+        L.moe_cache_usage.restype = st
+        L.moe_cache_usage.argtypes = [p, i, p]
         L.moe_debug_gemv_int4.restype = st
         L.moe_debug_gemv_int4.argtypes = [p, p, i, i, p, p, p]
         _lib = L
@@ -226,15 +232,22 @@ def stack_forward(layers, x_in, x_out, x_tmp, ws, idx=None, eps=NORM_EPS, stream
           "moe_stack_forward")
 
 
-def lru_replay(trace, n_experts, capacity):
-    """The cache's LRU rule on a host trace [T][L][k] -> (hits[L], misses[L])."""
+def lru_replay(trace, n_experts, capacity, pinned=None):
+    """The cache's LRU rule on a host trace [T][L][k] -> (hits[L], misses[L]).
+    pinned: optional [L][n_pinned] ascending ids pinned before the first call."""
     import numpy as np
     tr = np.ascontiguousarray(trace, dtype=np.int32)
     T, Lyr, k = tr.shape
     hits = np.zeros(Lyr, dtype=np.uint64)
     misses = np.zeros(Lyr, dtype=np.uint64)
-    check(lib().moe_lru_replay(Lyr, n_experts, capacity, k, T, tr.ctypes.data, hits.ctypes.data,
-                               misses.ctypes.data), "moe_lru_replay")
+    if pinned is None:
+        check(lib().moe_lru_replay(Lyr, n_experts, capacity, k, T, tr.ctypes.data,
+                                   hits.ctypes.data, misses.ctypes.data), "moe_lru_replay")
+    else:
+        pn = np.ascontiguousarray(pinned, dtype=np.int32).reshape(Lyr, -1)
+        check(lib().moe_lru_replay_pinned(Lyr, n_experts, capacity, k, T, tr.ctypes.data,
+                                          pn.shape[1], pn.ctypes.data, hits.ctypes.data,
+                                          misses.ctypes.data), "moe_lru_replay_pinned")
     return hits, misses
 
 
@@ -286,6 +299,20 @@ class Cache:
         a = np.ascontiguousarray(ids, dtype=np.int32)
         check(lib().moe_cache_acquire(self.handle, int(l), a.ctypes.data, a.size, _stream(stream)),
               "moe_cache_acquire")
+
+    def pin(self, l, ids, stream=None):
+        """Make ids (ascending) the pinned hot-store of layer l."""
+        import numpy as np
+        a = np.ascontiguousarray(ids, dtype=np.int32)
+        check(lib().moe_cache_pin(self.handle, int(l), a.ctypes.data if a.size else None, a.size,
+                                  _stream(stream)), "moe_cache_pin")
+
+    def usage(self, l):
+        """Usage log of layer l: uint64 [n_experts] acquire counts."""
+        import numpy as np
+        out = np.zeros(self.cfg.n_experts, dtype=np.uint64)
+        check(lib().moe_cache_usage(self.handle, int(l), out.ctypes.data), "moe_cache_usage")
+        return out
 
     def release(self, l, stream=None):
         check(lib().moe_cache_release(self.handle, int(l), _stream(stream)), "moe_cache_release")

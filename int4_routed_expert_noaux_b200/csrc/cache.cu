@@ -7,7 +7,13 @@
 // Replacement rule, per layer and per call: ids already cached are hits and
 // are touched in ascending id order; then every missing id, in ascending
 // order, takes an empty slot (the lowest) or else the least recently used
-// slot whose expert is not among the call's ids.
+// slot that is not pinned and whose expert is not among the call's ids.
+//
+// Hot-store (colibri summary, "Learning cache et attentes selon le
+// materiel": routed experts are logged and the most used ones are pinned at
+// start-up): every acquire counts its ids in a per-layer usage log, and
+// moe_cache_pin pins a chosen set of experts in their slots, so that the LRU
+// never evicts them; the remaining slots (at least top_k) run the rule above.
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
@@ -27,7 +33,7 @@ namespace moe {
 class LruPolicy {
  public:
   LruPolicy(int n_experts, int slots)
-      : slot_expert_(slots, -1), stamp_(slots, 0), expert_slot_(n_experts, -1) {}
+      : slot_expert_(slots, -1), stamp_(slots, 0), pinned_(slots, 0), expert_slot_(n_experts, -1) {}
 
   struct Load {
     int expert, slot, evicted;
@@ -39,6 +45,13 @@ class LruPolicy {
     if (old >= 0) expert_slot_[old] = -1;
     slot_expert_[slot] = -1;
     stamp_[slot] = 0;
+    pinned_[slot] = 0;
+  }
+
+  int pinned_count() const {
+    int n = 0;
+    for (char p : pinned_) n += p;
+    return n;
   }
 
   // ids ascending, distinct.  Fills loads (misses) and returns the hit count.
@@ -52,34 +65,58 @@ class LruPolicy {
         ++hits;
       }
     }
-    for (int j = 0; j < n; ++j) {
-      const int e = ids[j];
-      if (expert_slot_[e] >= 0) continue;
-      int victim = -1;
-      for (int s = 0; s < (int)slot_expert_.size() && victim < 0; ++s)
-        if (slot_expert_[s] < 0) victim = s;
-      if (victim < 0) {
-        for (int s = 0; s < (int)slot_expert_.size(); ++s) {
-          bool current = false;
-          for (int jj = 0; jj < n; ++jj)
-            if (slot_expert_[s] == ids[jj]) current = true;
-          if (current) continue;
-          if (victim < 0 || stamp_[s] < stamp_[victim]) victim = s;
-        }
-      }
-      const int old = slot_expert_[victim];
-      if (old >= 0) expert_slot_[old] = -1;
-      slot_expert_[victim] = e;
-      expert_slot_[e] = victim;
-      stamp_[victim] = ++clock_;
-      loads.push_back(Load{e, victim, old});
-    }
+    for (int j = 0; j < n; ++j)
+      if (expert_slot_[ids[j]] < 0) load(ids[j], ids, n, loads);
     return hits;
   }
 
+  // Make ids (ascending, distinct) the pinned set: cached ones are pinned
+  // where they are, missing ones are loaded (as by access) and pinned; every
+  // other slot becomes an ordinary LRU slot.  The caller keeps
+  // n <= slots - top_k, so that a call of top_k ids always finds a victim.
+  void pin(const int32_t* ids, int n, std::vector<Load>& loads) {
+    loads.clear();
+    for (char& p : pinned_) p = 0;
+    for (int j = 0; j < n; ++j) {
+      const int s = expert_slot_[ids[j]];
+      if (s >= 0) {
+        pinned_[s] = 1;
+        stamp_[s] = ++clock_;
+      }
+    }
+    for (int j = 0; j < n; ++j)
+      if (expert_slot_[ids[j]] < 0) pinned_[load(ids[j], ids, n, loads)] = 1;
+  }
+
  private:
+  // Put expert e in the lowest empty slot, else in the least recently used
+  // slot that is not pinned and does not hold one of ids; returns the slot.
+  int load(int e, const int32_t* ids, int n, std::vector<Load>& loads) {
+    int victim = -1;
+    for (int s = 0; s < (int)slot_expert_.size() && victim < 0; ++s)
+      if (slot_expert_[s] < 0) victim = s;
+    if (victim < 0) {
+      for (int s = 0; s < (int)slot_expert_.size(); ++s) {
+        if (pinned_[s]) continue;
+        bool current = false;
+        for (int jj = 0; jj < n; ++jj)
+          if (slot_expert_[s] == ids[jj]) current = true;
+        if (current) continue;
+        if (victim < 0 || stamp_[s] < stamp_[victim]) victim = s;
+      }
+    }
+    const int old = slot_expert_[victim];
+    if (old >= 0) expert_slot_[old] = -1;
+    slot_expert_[victim] = e;
+    expert_slot_[e] = victim;
+    stamp_[victim] = ++clock_;
+    loads.push_back(Load{e, victim, old});
+    return victim;
+  }
+
   std::vector<int> slot_expert_;
   std::vector<uint64_t> stamp_;
+  std::vector<char> pinned_;
   std::vector<int> expert_slot_;
   uint64_t clock_ = 0;
 };
@@ -140,6 +177,7 @@ struct moe_cache {
   std::vector<LruPolicy> lru;
   std::vector<moe_layer*> views;       // per layer, created by moe_cache_layer
   std::vector<uint64_t> hits, misses, bytes;
+  std::vector<uint64_t> usage;         // [L][E]: times each expert was acquired
   std::vector<LruPolicy::Load> loads;  // scratch
 };
 
@@ -179,17 +217,108 @@ ExpertPtrs slot_ptrs(const moe_cache* c, int layer, int slot) {
 
 }  // namespace
 
+namespace {
+
+moe_status check_ids(const moe_cache* c, const int32_t* ids, int n) {
+  for (int j = 0; j < n; ++j)
+    if (ids[j] < 0 || ids[j] >= c->cfg.n_experts || (j && ids[j] <= ids[j - 1]))
+      return fail(MOE_ERR_INVALID_ARG, "ids must be ascending, distinct and in range");
+  return MOE_OK;
+}
+
+// Enqueues the copies of c->loads, which were planned on `plan` (a copy of
+// the layer's replacement state), and then commits plan, the counters and
+// the pointer table -- only once every copy of every load is enqueued.
+// `acquire_ids` (n of them, nullable) are the ids of an acquire: they count
+// as hits / misses and in the usage log; a pin counts only its bytes.
+moe_status commit_loads(moe_cache* c, int layer, cudaStream_t cs, const LruPolicy& plan,
+                        int hits, const int32_t* acquire_ids, int n, const char* who) {
+  cudaError_t ce = cudaSuccess;
+  if (!c->loads.empty()) {
+    // A victim slot may still be read by compute enqueued earlier for this
+    // layer: that of the last release, or -- acquired again with no release
+    // in between -- everything enqueued on the compute stream so far.
+    if (c->acquired[layer]) {
+      ce = cudaEventRecord(c->used[layer], cs);
+      if (ce == cudaSuccess) c->used_valid[layer] = true;
+    }
+    if (ce == cudaSuccess && c->used_valid[layer])
+      ce = cudaStreamWaitEvent(c->copy_stream, c->used[layer], 0);
+    if (ce == cudaSuccess && g_inject_kind.load(std::memory_order_acquire) == MOE_FAULT_CACHE_STALL) {
+      const int ms = g_inject_after.exchange(0);
+      g_inject_kind.store(0, std::memory_order_release);
+      ce = cudaLaunchHostFunc(c->copy_stream, hold_stream, reinterpret_cast<void*>((intptr_t)ms));
+    }
+  }
+  TableUpdate u;
+  u.n = 0;
+  int reached = 0;  // loads whose slot a copy may have written
+  for (const LruPolicy::Load& ld : c->loads) {
+    if (ce != cudaSuccess) break;
+    const moe_expert& he = c->host[(size_t)layer * c->cfg.n_experts + ld.expert];
+    const ExpertPtrs d = slot_ptrs(c, layer, ld.slot);
+    const void* src[6] = {he.q_gate, he.q_up, he.s_gate, he.s_up, he.q_down, he.s_down};
+    void* dst[6] = {(void*)d.q_gate, (void*)d.q_up, (void*)d.s_gate,
+                    (void*)d.s_up, (void*)d.q_down, (void*)d.s_down};
+    const size_t sz[6] = {c->off[1] - c->off[0], c->off[2] - c->off[1], c->off[3] - c->off[2],
+                          c->off[4] - c->off[3], c->off[5] - c->off[4],
+                          c->expert_bytes - c->off[5]};
+    ++reached;
+    for (int t = 0; t < 6 && ce == cudaSuccess; ++t)
+      ce = inject(MOE_FAULT_CACHE_COPY)
+               ? cudaErrorInvalidValue
+               : cudaMemcpyAsync(dst[t], src[t], sz[t], cudaMemcpyHostToDevice, c->copy_stream);
+    u.ids[u.n] = ld.expert;
+    u.ptrs[u.n] = d;
+    ++u.n;
+  }
+  if (!c->loads.empty()) {
+    if (ce == cudaSuccess) ce = cudaEventRecord(c->copied[layer], c->copy_stream);
+    if (ce == cudaSuccess) ce = cudaStreamWaitEvent(cs, c->copied[layer], 0);
+    if (ce == cudaSuccess) {
+      table_update_kernel<<<1, kMaxTableUpdates, 0, cs>>>(c->views[layer]->table, u);
+      ce = cudaGetLastError();
+    }
+  }
+  if (ce != cudaSuccess) {
+    // Roll back: the layer keeps its committed state, except that a slot a
+    // copy may have reached no longer counts as holding anything.
+    for (int i = 0; i < reached; ++i) c->lru[layer].invalidate(c->loads[i].slot);
+    return cuda_fail(ce, who);
+  }
+  c->lru[layer] = plan;
+  moe_layer* view = c->views[layer];
+  for (int i = 0; i < u.n; ++i) view->host_table[u.ids[i]] = u.ptrs[i];
+  c->bytes[layer] += (uint64_t)u.n * c->expert_bytes;
+  if (acquire_ids) {
+    c->hits[layer] += hits;
+    c->misses[layer] += u.n;
+    uint64_t* use = c->usage.data() + (size_t)layer * c->cfg.n_experts;
+    for (int j = 0; j < n; ++j) ++use[acquire_ids[j]];
+    c->acquired[layer] = true;
+  }
+  return MOE_OK;
+}
+
+}  // namespace
+
 extern "C" {
 #pragma GCC visibility push(default)
 
-moe_status moe_lru_replay(int n_layers, int n_experts, int capacity, int k, int T,
-                          const int32_t* trace, uint64_t* hits, uint64_t* misses) {
-  if (n_layers < 1 || n_experts < 1 || k < 1 || capacity < k || T < 0 || !trace || !hits ||
-      !misses)
+moe_status moe_lru_replay_pinned(int n_layers, int n_experts, int capacity, int k, int T,
+                                 const int32_t* trace, int n_pinned, const int32_t* pinned,
+                                 uint64_t* hits, uint64_t* misses) {
+  if (n_layers < 1 || n_experts < 1 || k < 1 || T < 0 || !trace || !hits || !misses ||
+      n_pinned < 0 || capacity - n_pinned < k || (n_pinned > 0 && !pinned))
     return fail(MOE_ERR_INVALID_ARG, "bad LRU replay arguments");
   std::vector<LruPolicy::Load> loads;
   for (int l = 0; l < n_layers; ++l) {
     LruPolicy lru(n_experts, capacity);
+    const int32_t* pin = pinned ? pinned + (size_t)l * n_pinned : nullptr;
+    for (int j = 0; j < n_pinned; ++j)
+      if (pin[j] < 0 || pin[j] >= n_experts || (j && pin[j] <= pin[j - 1]))
+        return fail(MOE_ERR_INVALID_ARG, "pinned ids must be ascending and in range");
+    lru.pin(pin, n_pinned, loads);
     uint64_t h = 0, m = 0;
     for (int t = 0; t < T; ++t) {
       const int32_t* ids = trace + ((size_t)t * n_layers + l) * k;
@@ -203,6 +332,12 @@ moe_status moe_lru_replay(int n_layers, int n_experts, int capacity, int k, int 
     misses[l] = m;
   }
   return MOE_OK;
+}
+
+moe_status moe_lru_replay(int n_layers, int n_experts, int capacity, int k, int T,
+                          const int32_t* trace, uint64_t* hits, uint64_t* misses) {
+  return moe_lru_replay_pinned(n_layers, n_experts, capacity, k, T, trace, 0, nullptr, hits,
+                               misses);
 }
 
 moe_status moe_cache_create(const moe_config* cfg, int n_layers, int slots_per_layer,
@@ -255,6 +390,7 @@ moe_status moe_cache_create(const moe_config* cfg, int n_layers, int slots_per_l
   for (int l = 0; l < n_layers; ++l) c->lru.emplace_back(cfg->n_experts, slots_per_layer);
   c->views.assign(n_layers, nullptr);
   c->hits.assign(n_layers, 0);
+  c->usage.assign((size_t)n_layers * cfg->n_experts, 0);
   c->misses.assign(n_layers, 0);
   c->bytes.assign(n_layers, 0);
   *out = c;
@@ -305,77 +441,40 @@ moe_status moe_cache_acquire(moe_cache* c, int layer, const int32_t* ids_host, i
   if (!c->views[layer]) return fail(MOE_ERR_INVALID_ARG, "create the layer view first (moe_cache_layer)");
   if (n < 1 || n > c->slots || n > kMaxTableUpdates)
     return fail(MOE_ERR_INVALID_ARG, "n = %d outside 1..min(slots, %d)", n, kMaxTableUpdates);
-  for (int j = 0; j < n; ++j)
-    if (ids_host[j] < 0 || ids_host[j] >= c->cfg.n_experts || (j && ids_host[j] <= ids_host[j - 1]))
-      return fail(MOE_ERR_INVALID_ARG, "ids must be ascending, distinct and in range");
-  cudaStream_t cs = (cudaStream_t)compute_stream;
+  moe_status st = check_ids(c, ids_host, n);
+  if (st != MOE_OK) return st;
+  if (n > c->slots - c->lru[layer].pinned_count())
+    return fail(MOE_ERR_INVALID_ARG, "n = %d exceeds the layer's unpinned slots", n);
   // The replacement is planned on a copy of the layer's state and committed
   // (with the counters and the pointer table) only once every copy of every
   // miss is enqueued.
   LruPolicy plan = c->lru[layer];
   const int hits = plan.access(ids_host, n, c->loads);
-  if (c->loads.empty()) {
-    c->lru[layer] = plan;
-    c->hits[layer] += hits;
-    c->acquired[layer] = true;
-    return MOE_OK;
-  }
-  cudaError_t ce = cudaSuccess;
-  // A victim slot may still be read by compute enqueued earlier for this
-  // layer: that of the last release, or -- acquired again with no release
-  // in between -- everything enqueued on the compute stream so far.
-  if (c->acquired[layer]) {
-    ce = cudaEventRecord(c->used[layer], cs);
-    if (ce == cudaSuccess) c->used_valid[layer] = true;
-  }
-  if (ce == cudaSuccess && c->used_valid[layer])
-    ce = cudaStreamWaitEvent(c->copy_stream, c->used[layer], 0);
-  if (ce == cudaSuccess && g_inject_kind.load(std::memory_order_acquire) == MOE_FAULT_CACHE_STALL) {
-    const int ms = g_inject_after.exchange(0);
-    g_inject_kind.store(0, std::memory_order_release);
-    ce = cudaLaunchHostFunc(c->copy_stream, hold_stream, reinterpret_cast<void*>((intptr_t)ms));
-  }
-  TableUpdate u;
-  u.n = 0;
-  int reached = 0;  // loads whose slot a copy may have written
-  for (const LruPolicy::Load& ld : c->loads) {
-    if (ce != cudaSuccess) break;
-    const moe_expert& he = c->host[(size_t)layer * c->cfg.n_experts + ld.expert];
-    const ExpertPtrs d = slot_ptrs(c, layer, ld.slot);
-    const void* src[6] = {he.q_gate, he.q_up, he.s_gate, he.s_up, he.q_down, he.s_down};
-    void* dst[6] = {(void*)d.q_gate, (void*)d.q_up, (void*)d.s_gate,
-                    (void*)d.s_up, (void*)d.q_down, (void*)d.s_down};
-    const size_t sz[6] = {c->off[1] - c->off[0], c->off[2] - c->off[1], c->off[3] - c->off[2],
-                          c->off[4] - c->off[3], c->off[5] - c->off[4],
-                          c->expert_bytes - c->off[5]};
-    ++reached;
-    for (int t = 0; t < 6 && ce == cudaSuccess; ++t)
-      ce = inject(MOE_FAULT_CACHE_COPY)
-               ? cudaErrorInvalidValue
-               : cudaMemcpyAsync(dst[t], src[t], sz[t], cudaMemcpyHostToDevice, c->copy_stream);
-    u.ids[u.n] = ld.expert;
-    u.ptrs[u.n] = d;
-    ++u.n;
-  }
-  if (ce == cudaSuccess) ce = cudaEventRecord(c->copied[layer], c->copy_stream);
-  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(cs, c->copied[layer], 0);
-  if (ce == cudaSuccess) {
-    table_update_kernel<<<1, kMaxTableUpdates, 0, cs>>>(c->views[layer]->table, u);
-    ce = cudaGetLastError();
-  }
-  if (ce != cudaSuccess) {
-    // Roll back: the layer keeps its committed state, except that a slot a
-    // copy may have reached no longer counts as holding anything.
-    for (int i = 0; i < reached; ++i) c->lru[layer].invalidate(c->loads[i].slot);
-    return cuda_fail(ce, "moe_cache_acquire");
-  }
-  c->lru[layer] = plan;
-  moe_layer* view = c->views[layer];
-  for (int i = 0; i < u.n; ++i) view->host_table[u.ids[i]] = u.ptrs[i];
-  c->hits[layer] += hits;
-  c->misses[layer] += u.n;
-  c->bytes[layer] += (uint64_t)u.n * c->expert_bytes;
-  c->acquired[layer] = true;
+  return commit_loads(c, layer, (cudaStream_t)compute_stream, plan, hits, ids_host, n,
+                      "moe_cache_acquire");
+}
+
+moe_status moe_cache_pin(moe_cache* c, int layer, const int32_t* ids_host, int n,
+                         void* compute_stream) {
+  if (!c || (n > 0 && !ids_host)) return fail(MOE_ERR_INVALID_ARG, "cache or ids is NULL");
+  if (layer < 0 || layer >= c->n_layers) return fail(MOE_ERR_INVALID_ARG, "layer out of range");
+  if (!c->views[layer]) return fail(MOE_ERR_INVALID_ARG, "create the layer view first (moe_cache_layer)");
+  if (n < 0 || n > c->slots - c->cfg.top_k || n > kMaxTableUpdates)
+    return fail(MOE_ERR_INVALID_ARG, "n = %d outside 0..min(slots - top_k, %d)", n,
+                kMaxTableUpdates);
+  moe_status st = check_ids(c, ids_host, n);
+  if (st != MOE_OK) return st;
+  LruPolicy plan = c->lru[layer];
+  plan.pin(ids_host, n, c->loads);
+  return commit_loads(c, layer, (cudaStream_t)compute_stream, plan, 0, nullptr, 0,
+                      "moe_cache_pin");
+}
+
+moe_status moe_cache_usage(const moe_cache* c, int layer, uint64_t* counts) {
+  if (!c || !counts) return fail(MOE_ERR_INVALID_ARG, "cache or counts is NULL");
+  if (layer < 0 || layer >= c->n_layers) return fail(MOE_ERR_INVALID_ARG, "layer out of range");
+  memcpy(counts, c->usage.data() + (size_t)layer * c->cfg.n_experts,
+         sizeof(uint64_t) * c->cfg.n_experts);
   return MOE_OK;
 }
 

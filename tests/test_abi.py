@@ -90,6 +90,39 @@ def test_library_lru_matches_oracle_lru():
             assert np.array_equal(h1, h2) and np.array_equal(m1, m2), (seed, cap)
 
 
+def hot_set(counts, n):
+    """The n most used experts (ties to the lower id), ascending."""
+    order = np.lexsort((np.arange(len(counts)), -np.asarray(counts, dtype=np.int64)))
+    return np.sort(order[:n])
+
+
+def test_library_pinned_lru_matches_oracle():
+    # the hot-store: pin the experts most used in the first half of a Zipf
+    # trace, replay the whole trace in the library and in the oracle
+    import oracle
+    for seed, (L, E, k, T) in enumerate([(3, 256, 8, 300), (2, 16, 2, 200), (1, 64, 6, 500)]):
+        tr = synth.zipf_trace(seed, L, E, k, T)
+        for cap in sorted({k + 1, 2 * k, 4 * k, E // 2, E}):
+            for n_pin in sorted({1, (cap - k) // 2, cap - k}):
+                if n_pin < 1 or cap - n_pin < k or cap > E:
+                    continue
+                pinned = np.stack([hot_set(np.bincount(tr[:T // 2, l, :].ravel(), minlength=E),
+                                           n_pin) for l in range(L)])
+                h1, m1 = moe.lru_replay(tr, E, cap, pinned=pinned)
+                h2, m2 = oracle.lru_sim_pinned(tr, E, cap, pinned)
+                assert np.array_equal(h1, h2) and np.array_equal(m1, m2), (seed, cap, n_pin)
+
+
+def test_pinned_lru_replay_rejects_bad_arguments():
+    tr = np.array([[[0, 1]], [[1, 2]]], dtype=np.int32)
+    with pytest.raises(moe.MoeError):
+        moe.lru_replay(tr, 8, 3, pinned=np.array([[0, 1]]))    # 3 - 2 < k
+    with pytest.raises(moe.MoeError):
+        moe.lru_replay(tr, 8, 4, pinned=np.array([[1, 0]]))    # not ascending
+    with pytest.raises(moe.MoeError):
+        moe.lru_replay(tr, 8, 4, pinned=np.array([[0, 9]]))    # out of range
+
+
 def test_lru_replay_rejects_bad_traces():
     tr = np.array([[[3, 1]]], dtype=np.int32)  # not ascending
     with pytest.raises(moe.MoeError):
