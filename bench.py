@@ -58,9 +58,12 @@ def parse():
     p.add_argument("--correlated", action="store_true",
                    help="verify: draft tokens x0 + 0.05 eps (heavily shared experts)")
     p.add_argument("--stack-layers", type=int, default=24)
-    p.add_argument("--stream-layers", type=int, default=8,
-                   help="stream: layers in pinned host memory (capped by free host RAM)")
+    p.add_argument("--stream-layers", type=int, default=75,
+                   help="stream: at most this many layers in pinned host memory (75, the "
+                        "model's MoE layers; fewer when host memory is smaller)")
     p.add_argument("--stream-caps", default="8,16,32,64,128", help="stream: cache slots per layer")
+    p.add_argument("--stream-router-caps", default="32,128",
+                   help="stream: cache sizes also run with the device router's ids")
     p.add_argument("--stream-tokens", type=int, default=512)
     p.add_argument("--top-p", type=float, default=1.0,
                    help="adaptive expert top-p of every layer (>= 1: off, the headline)")
@@ -462,6 +465,215 @@ def _line(args, shape, extra):
     print(json.dumps(base), flush=True)
 
 
+# Share of the host's free memory the streamed store may pin; the rest stays
+# with the operating system, the CUDA driver and this process.
+STREAM_HOST_FRACTION = 0.75
+
+
+def host_free_bytes():
+    """Free host memory: psutil's available figure, bounded by the cgroup's
+    remaining limit where there is one."""
+    import psutil
+    free = psutil.virtual_memory().available
+    for lim_path, use_path in (("/sys/fs/cgroup/memory.max", "/sys/fs/cgroup/memory.current"),
+                               ("/sys/fs/cgroup/memory/memory.limit_in_bytes",
+                                "/sys/fs/cgroup/memory/memory.usage_in_bytes")):
+        try:
+            lim = int(open(lim_path).read().strip())
+            use = int(open(use_path).read().strip())
+        except (OSError, ValueError):
+            continue
+        free = min(free, max(0, lim - use))
+    return free
+
+
+class HostStore:
+    """Routed experts of L layers in page-locked host memory (numpy buffers
+    registered with cudaHostRegister, so that no allocator rounds them up),
+    filled by the device generator and copied back, laid out as
+    synth.layers.expert_offsets per expert."""
+
+    def __init__(self, shape, n_layers):
+        import torch
+        from synth.layers import DeviceLayer, expert_offsets
+        E, B = shape.n_experts, shape.expert_bytes
+        offs = expert_offsets(shape)
+        self.layer_bytes = E * B
+        self.bufs, self.experts = [], []
+        cudart = torch.cuda.cudart()
+        for l in range(n_layers):
+            raw = np.empty(self.layer_bytes + 4096, dtype=np.uint8)
+            base = (raw.ctypes.data + 4095) // 4096 * 4096
+            view = raw[base - raw.ctypes.data: base - raw.ctypes.data + self.layer_bytes]
+            rc = int(cudart.cudaHostRegister(base, self.layer_bytes, 0))
+            if rc != 0:
+                self.close()
+                raise RuntimeError(f"cudaHostRegister failed ({rc}) at layer {l}")
+            self.bufs.append((raw, base, view))
+            dl = DeviceLayer(shape, 0, l)
+            torch.from_numpy(view).copy_(dl.slab[: self.layer_bytes])
+            del dl
+            self.experts.append([{k: base + e * B + o for k, o in offs.items()}
+                                 for e in range(E)])
+        torch.cuda.synchronize()
+
+    def close(self):
+        import torch
+        cudart = torch.cuda.cudart()
+        for raw, base, view in self.bufs:
+            cudart.cudaHostUnregister(base)
+        self.bufs = []
+
+
+def hot_set(counts, n):
+    """The n most used experts of a usage log (ties to the lower id), ascending."""
+    order = np.lexsort((np.arange(len(counts)), -np.asarray(counts, dtype=np.int64)))
+    return np.sort(order[:n])
+
+
+def run_stream(args, shape, cfg, stream):
+    """Host-streamed experts: an LRU cache per layer in HBM over a pinned host
+    store of as many layers as STREAM_HOST_FRACTION of the free host memory
+    holds.  Per cache size: the Zipf trace with plain LRU, the same trace with
+    the hot-store (experts pinned at start-up from the usage log of an earlier
+    session of the same popularity), and, with --stream-router, ids from the
+    device router of each layer read back to the host before the acquire."""
+    import torch
+    import int4_routed_expert_noaux_b200 as moe
+    import synth
+    from synth.layers import DeviceLayer
+    E, H, k = shape.n_experts, shape.hidden, shape.top_k
+    layer_bytes = E * shape.expert_bytes
+    free = host_free_bytes()
+    L = max(1, min(args.stream_layers, int(free * STREAM_HOST_FRACTION) // layer_bytes))
+    t0 = time.time()
+    store = HostStore(shape, L)
+    fill_s = time.time() - t0
+    dls = [DeviceLayer(shape, 0, l, routed=False) for l in range(L)]
+    # measured host->device bandwidth of the store (2 GiB copies)
+    probe = torch.empty(min(layer_bytes, 2 << 30), dtype=torch.uint8, device="cuda")
+    src = torch.from_numpy(store.bufs[0][2][: probe.numel()])
+    hb_ms = _timed(stream, lambda: probe.copy_(src, non_blocking=True), 3, 1)
+    h2d_gbs = 3 * probe.numel() / (hb_ms / 1000.0) / 1e9
+    del probe, src
+    Tn = args.stream_tokens
+    # tokens [0, Tn) are the earlier session whose usage log the hot-store
+    # pins from; tokens [Tn, 2 Tn) are the measured trace
+    full = synth.zipf_trace(5, L, E, k, 2 * Tn)
+    learn, trace = full[:Tn], np.ascontiguousarray(full[Tn:])
+    usage = [np.bincount(learn[:, l].ravel(), minlength=E) for l in range(L)]
+    xb = synth.tokens(shape, 0, 0, Tn)
+    x = torch.from_numpy(xb.view(np.int16)).cuda()
+    ids_dev = torch.from_numpy(trace).cuda()
+    w = torch.full((1, k), shape.rsf / k, dtype=torch.float32, device="cuda")
+    y = torch.empty((1, H), dtype=torch.float32, device="cuda")
+    ws = moe.alloc_workspace(cfg, 1)
+    ridx = torch.empty((1, k), dtype=torch.int32, device="cuda")
+    rw = torch.empty((1, k), dtype=torch.float32, device="cuda")
+    ids_host = torch.empty((1, k), dtype=torch.int32, pin_memory=True)
+    ev_ids = torch.cuda.Event()
+    caps = [int(v) for v in args.stream_caps.split(",")]
+    router_caps = [int(v) for v in args.stream_router_caps.split(",") if v]
+
+    def pins_for(cap):
+        """Experts to pin per layer: the hottest n of the usage log, n chosen
+        among five candidates by replaying the earlier session."""
+        best_n, best_h = 0, -1
+        for n in sorted({0, (cap - k) // 4, (cap - k) // 2, 3 * (cap - k) // 4, cap - k}):
+            pinned = np.stack([hot_set(usage[l], n) for l in range(L)])
+            h, _ = moe.lru_replay(learn, E, cap, pinned=pinned if n else None)
+            if int(h.sum()) > best_h:
+                best_n, best_h = n, int(h.sum())
+        return best_n, [hot_set(usage[l], best_n) for l in range(L)]
+
+    def one(cap, arm):
+        try:
+            cache = moe.Cache(cfg, store.experts, cap)
+        except moe.MoeError as e:
+            print(json.dumps({"mode": "stream", "cache_slots_per_layer": cap,
+                              "skipped": str(e)}), flush=True)
+            return
+        views = [cache.layer(l, dls[l].w_router, dls[l].bias, dls[l].shared) for l in range(L)]
+        n_pin = 0
+        if arm == "hot-store":
+            n_pin, pins = pins_for(cap)
+            for l in range(L):
+                if n_pin:
+                    cache.pin(l, pins[l], stream=stream)
+        cache.sync()
+        torch.cuda.synchronize()
+        before = [cache.stats(l) for l in range(L)]
+        miss_calls = 0  # acquires with a miss: each adds one pointer-table update kernel
+        m_last = [b[1] for b in before]
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for t in range(Tn):
+                for l in range(L):
+                    if arm == "router":
+                        views[l].route(x[t:t + 1], ridx, rw, ws, stream=stream)
+                        ids_host.copy_(ridx, non_blocking=True)
+                        ev_ids.record(stream)
+                        ev_ids.synchronize()
+                        cache.acquire(l, ids_host.numpy()[0], stream=stream)
+                        views[l].expert_ffn(x[t:t + 1], ridx, rw, y, ws, stream=stream)
+                    else:
+                        cache.acquire(l, trace[t, l], stream=stream)
+                        views[l].expert_ffn(x[t:t + 1], ids_dev[t, l:l + 1], w, y, ws,
+                                            stream=stream)
+                    cache.release(l, stream=stream)
+                    m_now = cache.stats(l)[1]
+                    miss_calls += m_now != m_last[l]
+                    m_last[l] = m_now
+            ev1.record(stream)
+        stream.synchronize()
+        cache.sync()
+        ms = ev0.elapsed_time(ev1)
+        moe.ws_check(ws, stream)
+        hits = misses = moved = 0
+        for l in range(L):
+            h, m, b = cache.stats(l)
+            hits += h - before[l][0]
+            misses += m - before[l][1]
+            moved += b - before[l][2]
+        link = moved / (ms / 1000.0) / 1e9
+        routing = {"lru": "Zipf trace, plain LRU",
+                   "hot-store": f"Zipf trace, {n_pin} experts per layer pinned from the usage "
+                                "log of an earlier session, LRU on the other slots",
+                   "router": "device router of each layer (ids read back to the host), "
+                             "plain LRU"}[arm]
+        # moe_expert_ffn of one token: x groups, expert lists, gate/up, h
+        # groups, down, combine; moe_route adds the router and the selection
+        per_call = 6 + (2 if arm == "router" else 0)
+        _line(args, shape, {
+            "value": Tn / (ms / 1000.0), "ms_per_step": ms,
+            "config": {"workload": f"{L} GLM-5.2-shaped MoE layers in pinned host memory "
+                                   f"({L * layer_bytes / 1e9:.1f} GB), per-layer cache in HBM",
+                       "layers": L, "host_free_bytes": free,
+                       "host_fraction_pinned": STREAM_HOST_FRACTION,
+                       "host_fill_s": round(fill_s, 1), "cache_slots_per_layer": cap,
+                       "policy": arm, "pinned_per_layer": n_pin, "tokens": Tn,
+                       "routing": routing, "hit_rate": hits / max(1, hits + misses),
+                       "expert_bytes": shape.expert_bytes},
+            "roofline": {"bound": "h2d", "achieved": link, "peak": h2d_gbs, "unit": "GB/s",
+                         "frac": link / h2d_gbs, "traffic": moved, "peak_source":
+                         "measured pinned host->device copy, same run",
+                         "kernel": "expert loads (cudaMemcpyAsync, side stream)"},
+            "gpu_launches": Tn * L * per_call + miss_calls})
+        cache.close()
+
+    try:
+        for cap in caps:
+            one(cap, "lru")
+            if cap - k >= 1:
+                one(cap, "hot-store")
+        for cap in router_caps:
+            one(cap, "router")
+    finally:
+        store.close()
+
+
 def run_mode(args, shape):
     import torch
     import int4_routed_expert_noaux_b200 as moe
@@ -550,71 +762,8 @@ def run_mode(args, shape):
         return
 
     if args.mode == "stream":
-        import psutil
-        stride = synth.expert_stride(shape)
-        layer_bytes = E * stride
-        avail = psutil.virtual_memory().available
-        L = max(1, min(args.stream_layers, int(avail * 0.25) // layer_bytes))
-        host, keep = [], []
-        for l in range(L):
-            buf = torch.empty(layer_bytes, dtype=torch.uint8).pin_memory()
-            keep.append(buf)
-            base = buf.data_ptr()
-            experts = []
-            for e in range(E):
-                offs = synth.expert_into(shape, 0, l, e, base + e * stride)
-                experts.append({k: base + e * stride + o for k, o in offs.items()})
-            host.append(experts)
-        dls = [DeviceLayer(shape, 0, l, routed=False) for l in range(L)]
-        # measured host->device bandwidth of pinned memory (>= 1 GB copies)
-        probe = torch.empty(min(layer_bytes, 2 << 30), dtype=torch.uint8, device="cuda")
-        hb_ms = _timed(stream, lambda: probe.copy_(keep[0][:probe.numel()], non_blocking=True), 3, 1)
-        h2d_gbs = 3 * probe.numel() / (hb_ms / 1000.0) / 1e9
-        del probe
-        trace = synth.zipf_trace(5, L, E, shape.top_k, args.stream_tokens)
-        xb = synth.tokens(shape, 0, 0, args.stream_tokens)
-        x = torch.from_numpy(xb.view(np.int16)).cuda()
-        ids_dev = torch.from_numpy(trace.astype(np.int32)).cuda()
-        w = torch.full((1, shape.top_k), shape.rsf / shape.top_k, dtype=torch.float32, device="cuda")
-        y = torch.empty((1, H), dtype=torch.float32, device="cuda")
-        ws = moe.alloc_workspace(cfg, 1)
-        for cap in [int(v) for v in args.stream_caps.split(",")]:
-            cache = moe.Cache(cfg, host, cap)
-            views = [cache.layer(l, dls[l].w_router, dls[l].bias, dls[l].shared) for l in range(L)]
-            torch.cuda.synchronize()
-            ev0 = torch.cuda.Event(enable_timing=True)
-            ev1 = torch.cuda.Event(enable_timing=True)
-            with torch.cuda.stream(stream):
-                ev0.record(stream)
-                for t in range(args.stream_tokens):
-                    for l in range(L):
-                        cache.acquire(l, trace[t, l], stream=stream)
-                        views[l].expert_ffn(x[t:t + 1], ids_dev[t, l:l + 1], w, y, ws, stream=stream)
-                        cache.release(l, stream=stream)
-                ev1.record(stream)
-            stream.synchronize()
-            cache.sync()
-            ms = ev0.elapsed_time(ev1)
-            moe.ws_check(ws, stream)
-            hits = misses = moved = 0
-            for l in range(L):
-                h, m, b = cache.stats(l)
-                hits, misses, moved = hits + h, misses + m, moved + b
-            link = moved / (ms / 1000.0) / 1e9
-            _line(args, shape, {
-                "value": args.stream_tokens / (ms / 1000.0), "ms_per_step": ms,
-                "config": {"workload": f"{L} GLM-5.2-shaped MoE layers in pinned host memory, "
-                                       "per-layer LRU cache in HBM, Zipf(1.1) trace",
-                           "layers": L, "cache_slots_per_layer": cap,
-                           "tokens": args.stream_tokens, "routing": "trace; weights rsf/k",
-                           "hit_rate": hits / max(1, hits + misses),
-                           "host_bytes_per_layer": layer_bytes},
-                "roofline": {"bound": "h2d", "achieved": link, "peak": h2d_gbs, "unit": "GB/s",
-                             "frac": link / h2d_gbs, "traffic": moved, "peak_source":
-                             "measured pinned cudaMemcpyAsync, same run",
-                             "kernel": "expert loads (cudaMemcpyAsync, side stream)"},
-                "gpu_launches": args.stream_tokens * L * 7})
-            cache.close()
+        run_stream(args, shape, cfg, stream)
+        return
         return
 
 

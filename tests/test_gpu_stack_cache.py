@@ -246,3 +246,114 @@ def test_cache_reacquire_without_release():
     for y_c, y_r, _ in outs:
         assert torch.equal(y_c, y_r)
     cache.close()
+
+
+# ---------------------------------------------------------------------------
+# hot-store: pinned experts over the LRU (reading R19)
+
+def hot_set(counts, n):
+    """The n most used experts (ties to the lower id), ascending."""
+    order = np.lexsort((np.arange(len(counts)), -np.asarray(counts, dtype=np.int64)))
+    return np.sort(order[:n])
+
+
+WIDE = synth.Shape(hidden=256, inter=128, n_experts=64, n_shared=1, top_k=2, n_group=4,
+                   topk_group=2)
+
+
+@pytest.mark.parametrize("shape,L,T,cap,n_pin", [(synth.TINY, 3, 40, 6, 3), (WIDE, 2, 30, 48, 40)],
+                         ids=["tiny", "64-experts-40-pinned"])
+def test_cache_hot_store_matches_resident_and_oracle(shape, L, T, cap, n_pin):
+    # A learning pass over the first half of a Zipf trace fills the usage
+    # log; a fresh cache pins each layer's most used experts, then runs the
+    # whole trace.  Outputs are bitwise the resident ones, the counters are
+    # the oracle's pinned LRU, and the usage log counts the trace's ids.
+    # (40 pinned experts take two pointer-table updates.)
+    needs_gpu()
+    cfg = moe.Config.from_shape(shape)
+    host = [[pinned_expert(shape, 0, l, e) for e in range(shape.n_experts)] for l in range(L)]
+    dls = [DeviceLayer(shape, 0, l) for l in range(L)]
+    resident = [moe.Layer(cfg, d.w_router, d.bias, d.routed, d.shared) for d in dls]
+    trace = synth.zipf_trace(7, L, shape.n_experts, shape.top_k, T)
+    learn = moe.Cache(cfg, host, cap)
+    for l in range(L):
+        learn.layer(l, dls[l].w_router, dls[l].bias, dls[l].shared)
+    for t in range(T // 2):
+        for l in range(L):
+            learn.acquire(l, trace[t, l])
+            learn.release(l)
+    learn.sync()
+    usage = [learn.usage(l) for l in range(L)]
+    for l in range(L):
+        assert np.array_equal(usage[l], np.bincount(trace[:T // 2, l].ravel(),
+                                                    minlength=shape.n_experts))
+    learn.close()
+    pinned = np.stack([hot_set(usage[l], n_pin) for l in range(L)])
+
+    cache = moe.Cache(cfg, host, cap)
+    views = [cache.layer(l, dls[l].w_router, dls[l].bias, dls[l].shared) for l in range(L)]
+    for l in range(L):
+        cache.pin(l, pinned[l])
+    x = torch.from_numpy(synth.tokens(shape, 0, 70, T).view(np.int16)).cuda()
+    wts = torch.tensor([[1.25, 1.25]], dtype=torch.float32, device="cuda")
+    ws, ws2 = moe.alloc_workspace(cfg, 1), moe.alloc_workspace(cfg, 1)
+    y_s = torch.empty((T, L, shape.hidden), dtype=torch.float32, device="cuda")
+    y_r = torch.empty_like(y_s)
+    for t in range(T):
+        for l in range(L):
+            idx = torch.from_numpy(trace[t, l].reshape(1, -1).copy()).cuda()
+            cache.acquire(l, trace[t, l])
+            views[l].expert_ffn(x[t:t + 1], idx, wts, y_s[t, l:l + 1], ws)
+            cache.release(l)
+            resident[l].expert_ffn(x[t:t + 1], idx, wts, y_r[t, l:l + 1], ws2)
+    moe.ws_check(ws)
+    moe.ws_check(ws2)
+    cache.sync()
+    assert torch.equal(y_s, y_r)
+    h_ref, m_ref = oracle.lru_sim_pinned(trace, shape.n_experts, cap, pinned)
+    for l in range(L):
+        h, m, b = cache.stats(l)
+        assert (h, m) == (int(h_ref[l]), int(m_ref[l]))
+        assert b == (m + n_pin) * shape.expert_bytes
+        assert np.array_equal(cache.usage(l), np.bincount(trace[:, l].ravel(),
+                                                          minlength=shape.n_experts))
+    cache.close()
+
+
+def test_cache_pin_changes_and_limits():
+    # Re-pinning mid-run, unpinning, the slot limits, and a failed copy
+    # during a pin (rolled back; the next acquire is bitwise correct).
+    shape, cfg, host, dls, resident = tiny_cache_setup(cap=4)
+    cache = moe.Cache(cfg, host, 4)
+    view = cache.layer(0, dls[0].w_router, dls[0].bias, dls[0].shared)
+    x = torch.from_numpy(synth.tokens(shape, 0, 63, 1).view(np.int16)).cuda()
+    with pytest.raises(moe.MoeError):
+        cache.pin(0, [1, 2, 3])           # 4 slots - top_k 2 = at most 2 pinned
+    with pytest.raises(moe.MoeError):
+        cache.pin(0, [3, 1])              # not ascending
+    cache.pin(0, [3, 7])
+    with pytest.raises(moe.MoeError):
+        cache.acquire(0, [0, 1, 2])       # 3 ids, 2 unpinned slots
+    outs = []
+    for ids, pin in (([3, 9], None), ([0, 7], [0, 9]), ([4, 9], []), ([3, 5], [5, 11])):
+        if pin is not None:
+            cache.pin(0, pin)
+        cache.acquire(0, ids)
+        outs.append(ffn_pair(shape, cfg, view, resident[0], ids, x))
+        cache.release(0)
+    torch.cuda.synchronize()
+    for y_c, y_r, _ in outs:
+        assert torch.equal(y_c, y_r)
+    before = cache.stats(0)
+    moe.inject_fault(moe.FAULT_CACHE_COPY, 2)
+    with pytest.raises(moe.MoeError) as ei:
+        cache.pin(0, [12, 13])            # both missing: the third copy fails
+    assert ei.value.status == 2
+    assert cache.stats(0) == before
+    cache.sync()
+    cache.acquire(0, [12, 13])
+    y_c, y_r, keep = ffn_pair(shape, cfg, view, resident[0], [12, 13], x)
+    cache.release(0)
+    torch.cuda.synchronize()
+    assert torch.equal(y_c, y_r)
+    cache.close()
