@@ -45,7 +45,7 @@ def parse():
     p.add_argument("--tokens", type=int, default=1000, help="tokens per step")
     p.add_argument("--copies", type=int, default=8, help="rotating layer copies")
     p.add_argument("--no-graph", action="store_true", help="launch eagerly instead of a CUDA graph")
-    p.add_argument("--cpu-sample", type=int, default=6, help="tokens in the CPU-baseline sample")
+    p.add_argument("--cpu-sample", type=int, default=64, help="tokens in the CPU-baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--small", action="store_true", help="tiny layer (smoke/profiling only)")
     p.add_argument("--experts", type=int, default=0,

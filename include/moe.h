@@ -290,7 +290,7 @@ moe_status moe_cache_acquire(moe_cache* cache, int layer,
  * stream, compute_stream waits for them, the pointer table is updated on
  * it) and its slot is never chosen as a victim afterwards; the previously
  * pinned experts not in ids become ordinary LRU entries.  n = 0 unpins all.
- * 0 <= n <= slots_per_layer - top_k, n <= 32.  Counts its bytes in
+ * 0 <= n <= slots_per_layer - top_k.  Counts its bytes in
  * bytes_h2d but not as hits, misses or usage.  Transactional like
  * moe_cache_acquire.  With p experts pinned, an acquire takes at most
  * slots_per_layer - p ids. */

@@ -250,8 +250,9 @@ moe_status commit_loads(moe_cache* c, int layer, cudaStream_t cs, const LruPolic
       ce = cudaLaunchHostFunc(c->copy_stream, hold_stream, reinterpret_cast<void*>((intptr_t)ms));
     }
   }
-  TableUpdate u;
-  u.n = 0;
+  // pointer-table entries of the loads, kMaxTableUpdates per update kernel
+  std::vector<TableUpdate> ups((c->loads.size() + kMaxTableUpdates - 1) / kMaxTableUpdates);
+  for (TableUpdate& u : ups) u.n = 0;
   int reached = 0;  // loads whose slot a copy may have written
   for (const LruPolicy::Load& ld : c->loads) {
     if (ce != cudaSuccess) break;
@@ -268,6 +269,7 @@ moe_status commit_loads(moe_cache* c, int layer, cudaStream_t cs, const LruPolic
       ce = inject(MOE_FAULT_CACHE_COPY)
                ? cudaErrorInvalidValue
                : cudaMemcpyAsync(dst[t], src[t], sz[t], cudaMemcpyHostToDevice, c->copy_stream);
+    TableUpdate& u = ups[(reached - 1) / kMaxTableUpdates];
     u.ids[u.n] = ld.expert;
     u.ptrs[u.n] = d;
     ++u.n;
@@ -275,8 +277,8 @@ moe_status commit_loads(moe_cache* c, int layer, cudaStream_t cs, const LruPolic
   if (!c->loads.empty()) {
     if (ce == cudaSuccess) ce = cudaEventRecord(c->copied[layer], c->copy_stream);
     if (ce == cudaSuccess) ce = cudaStreamWaitEvent(cs, c->copied[layer], 0);
-    if (ce == cudaSuccess) {
-      table_update_kernel<<<1, kMaxTableUpdates, 0, cs>>>(c->views[layer]->table, u);
+    for (size_t i = 0; i < ups.size() && ce == cudaSuccess; ++i) {
+      table_update_kernel<<<1, kMaxTableUpdates, 0, cs>>>(c->views[layer]->table, ups[i]);
       ce = cudaGetLastError();
     }
   }
@@ -288,11 +290,12 @@ moe_status commit_loads(moe_cache* c, int layer, cudaStream_t cs, const LruPolic
   }
   c->lru[layer] = plan;
   moe_layer* view = c->views[layer];
-  for (int i = 0; i < u.n; ++i) view->host_table[u.ids[i]] = u.ptrs[i];
-  c->bytes[layer] += (uint64_t)u.n * c->expert_bytes;
+  for (const TableUpdate& u : ups)
+    for (int i = 0; i < u.n; ++i) view->host_table[u.ids[i]] = u.ptrs[i];
+  c->bytes[layer] += (uint64_t)c->loads.size() * c->expert_bytes;
   if (acquire_ids) {
     c->hits[layer] += hits;
-    c->misses[layer] += u.n;
+    c->misses[layer] += c->loads.size();
     uint64_t* use = c->usage.data() + (size_t)layer * c->cfg.n_experts;
     for (int j = 0; j < n; ++j) ++use[acquire_ids[j]];
     c->acquired[layer] = true;
@@ -459,9 +462,8 @@ moe_status moe_cache_pin(moe_cache* c, int layer, const int32_t* ids_host, int n
   if (!c || (n > 0 && !ids_host)) return fail(MOE_ERR_INVALID_ARG, "cache or ids is NULL");
   if (layer < 0 || layer >= c->n_layers) return fail(MOE_ERR_INVALID_ARG, "layer out of range");
   if (!c->views[layer]) return fail(MOE_ERR_INVALID_ARG, "create the layer view first (moe_cache_layer)");
-  if (n < 0 || n > c->slots - c->cfg.top_k || n > kMaxTableUpdates)
-    return fail(MOE_ERR_INVALID_ARG, "n = %d outside 0..min(slots - top_k, %d)", n,
-                kMaxTableUpdates);
+  if (n < 0 || n > c->slots - c->cfg.top_k)
+    return fail(MOE_ERR_INVALID_ARG, "n = %d outside 0..slots - top_k", n);
   moe_status st = check_ids(c, ids_host, n);
   if (st != MOE_OK) return st;
   LruPolicy plan = c->lru[layer];

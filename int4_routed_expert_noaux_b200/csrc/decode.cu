@@ -114,7 +114,7 @@ struct Smem {
   float sel_w[kMaxSlots];  // their combine weights
   int sel_ok;
   float red[kGroups][2][kGW][32];
-  double redd[kGW][kMaxRR];  // router partial sums (fp64)
+  double redd[kGroups * kGW][kMaxRR];  // router partial sums (fp64), per group and warp
   int abort_flag[kGroups];
   float norm_part[kThreads / 32];
   float inv_rms;
@@ -212,6 +212,16 @@ __device__ __forceinline__ void router_rows(const DecodeParams& p, int b, int& r
   }
   r0 = (int)(((long long)b * p.E) / p.nR);
   nr = (int)(((long long)(b + 1) * p.E) / p.nR) - r0;
+}
+
+// The CTA's router rows go out as one fill per consumer group (fill g is
+// consumed by group g): group 0 takes the first ceil(nr / 2) rows, group 1
+// the rest, so that a CTA with two rows computes them at the same time.
+__device__ __forceinline__ int router_fills(int nr) { return nr >= 2 ? 2 : (nr > 0 ? 1 : 0); }
+__device__ __forceinline__ void router_fill_rows(int r0, int nr, int g, int& f0, int& fn) {
+  const int a = router_fills(nr) == 2 ? (nr + 1) / 2 : nr;
+  f0 = g == 0 ? r0 : r0 + a;
+  fn = g == 0 ? a : nr - a;
 }
 
 // At the start of this CTA's down phase (a stack's next layer known): its
@@ -617,13 +627,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     if (p.has_shared) S.ep[p.k] = p.shared;  // visible to the producer: same thread
     int rr0, rnr;
     router_rows(p, blockIdx.x, rr0, rnr);
-    if (rnr > 0) {
-      S.desc[0] = make_item(kRouter, 0, rr0, rnr);
-      const uint32_t bytes = (uint32_t)rnr * p.H * 4;
-      mbar_arrive_expect_tx(&S.full[0], bytes);
-      bulk_g2s(dsmem, p.w_router + (size_t)rr0 * p.H, bytes, &S.full[0], l2_policy_evict_first());
-      TRACE_AT(1);
+    for (int g = 0; g < router_fills(rnr); ++g) {
+      int f0, fn;
+      router_fill_rows(rr0, rnr, g, f0, fn);
+      S.desc[g] = make_item(kRouter, 0, f0, fn);
+      const uint32_t bytes = (uint32_t)fn * p.H * 4;
+      mbar_arrive_expect_tx(&S.full[g], bytes);
+      bulk_g2s(dsmem + (size_t)g * kStageBytes, p.w_router + (size_t)f0 * p.H, bytes, &S.full[g],
+               l2_policy_evict_first());
     }
+    if (rnr > 0) TRACE_AT(1);
   }
   // Programmatic dependent launch: the next call on the stream may start its
   // prologue (barriers, its router rows' fill: inputs no call writes) as
@@ -674,8 +687,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       // control word kCtrlTicket offsets the first item; it is 0 except in a
       // test that starts past the last item to make a wait run out.
       int gu_next = (int)blockIdx.x + (int)gu_offset;
-      // fill 0 (the router rows) went out in the prologue
-      for (uint32_t n = rnr > 0 ? 1u : 0u;; ++n) {
+      // fills 0 (and 1) -- the router rows -- went out in the prologue
+      for (uint32_t n = (uint32_t)router_fills(rnr);; ++n) {
         const int stage = (int)(n % kStages);
         ItemDesc d = make_item(kDone, 0, 0, 0);
         // the next item of this CTA (slots dropped by top-p are passed over)
@@ -928,6 +941,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       if (lane == 0) {
         __threadfence();
         red_add_release(p.ctrl + kCtrlHqDone + slot, 1u);
+        if (slot == p.k) TRACE_AT(21);
       }
     }
   } else {
@@ -986,7 +1000,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
 #pragma unroll
     for (int i = 0; i < kRouterChunks; ++i) {
       const int cc = tg + kGT * i;
-      if (grp != 0 || rnr == 0 || cc >= rchunks) {
+      if (grp >= router_fills(rnr) || cc >= rchunks) {
         xr[i] = make_uint2(0, 0);
       } else if (p.x_resid) {
         xr[i] = norm_bf16x4(p.x_resid, 4 * cc, inv_rms);
@@ -994,26 +1008,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         xr[i] = __ldg(reinterpret_cast<const uint2*>(p.x) + cc);
       }
     }
-    // Group 0 of a CTA with router rows: fill 0 is the router block.  It is
+    // Group g of a CTA with router rows: fill g is its router block.  It is
     // handled before the main loop so its bf16 inputs are dead afterwards.
     uint32_t c_first = 0;
     {
-      if (grp == 0 && rnr > 0) {
+      if (grp < router_fills(rnr)) {
         c_first = 1;
-        const int stage = 0;
+        const int stage = grp;
         const uint32_t gpar = 0u;
         int okw = 0;
-        if (lane == 0) okw = mbar_wait(&S.full[0], 0u, kWaitNs) ? 1 : 0;
+        if (lane == 0) okw = mbar_wait(&S.full[stage], 0u, kWaitNs) ? 1 : 0;
         const bool ok = __shfl_sync(0xffffffffu, okw, 0) != 0;
         if (ok) {
-          mbar_test(&S.full[0], 0u);
-          if (tg == 0) TRACE_AT(2);
+          mbar_test(&S.full[stage], 0u);
+          if (tg == 0 && grp == 0) TRACE_AT(2);
         } else {
           if (lane == 0) set_error(p.ctrl, kErrTimeout, 1, 0);
           gabort = 1;
         }
-        const ItemDesc d = S.desc[0];
-        const uint8_t* st = stages;
+        const ItemDesc d = S.desc[stage];
+        const uint8_t* st = stages + (size_t)stage * kStageBytes;
         // double-float sums of the exact fp32 x bf16 products: each product
         // is split exactly into p + e, the p are summed error-free into
         // (hi, lo) and the e added to lo -- about 48 bits with fp32
@@ -1044,11 +1058,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
             }
           }
           const DF v = df_warp_sum(df_add(df_add(c0, c1), df_add(c2, c3)));
-          if (lane == 0) S.redd[gw][r] = (double)v.hi + (double)v.lo;
+          if (lane == 0) S.redd[grp * kGW + gw][r] = (double)v.hi + (double)v.lo;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.empty[stage]);
-        if (tg == 0) TRACE_AT(15);
+        if (tg == 0 && grp == 0) TRACE_AT(15);
         if (!group_barrier(&S.gbar[grp], gpar)) {
           if (lane == 0) set_error(p.ctrl, kErrTimeout, 3, 0);
           gabort = 1;
@@ -1057,20 +1071,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           // the sigmoid score of each row, tagged with this call's epoch
           if (lane < d.nrows) {
             double v = 0.0;
-            for (int w = 0; w < kGW; ++w) v += S.redd[w][lane];
+            for (int w = 0; w < kGW; ++w) v += S.redd[grp * kGW + w][lane];
             const float sg = sigmoid_f64_to_f32(v);
             st_relaxed_u64(p.scores + d.row0 + lane,
                            ((uint64_t)epoch << 32) | __float_as_uint(sg));
           }
-          if (lane == 0) TRACE_AT(3);
+          if (lane == 0 && grp == 0) TRACE_AT(3);
         }
       }
     }
-    // Group 1 starts with two placeholder items (a gate/up, then a down
-    // item) that run the real loop body on whatever the stage holds and
-    // publish nothing: the instructions of both paths are fetched while the
-    // first weights are still on their way, not when they have arrived.
-    int warm = (grp == 1 && p.warm) ? 2 : 0;
+    // Group 1 of a CTA whose router rows all went to group 0 starts with two
+    // placeholder items (a gate/up, then a down item) that run the real loop
+    // body on whatever the stage holds and publish nothing: the instructions
+    // of both paths are fetched while the first weights are still on their
+    // way, not when they have arrived.  (A group that had router rows has
+    // spent that time on them; placeholders would only delay its first item.)
+    int warm = (grp == 1 && p.warm && c_first == 0) ? 2 : 0;
     uint32_t c = c_first;
     for (uint32_t it = c_first;; ++it) {  // it: group barrier phases used
       if (gabort) break;
@@ -1162,6 +1178,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
               uint32_t* cnt = p.ctrl + kCtrlHRows + d.slot * (p.I >> 5);
               red_add_release(cnt + g0, (uint32_t)__popc(m0));
               if (m1) red_add_release(cnt + g0 + 1, (uint32_t)__popc(m1));
+              if (d.slot == p.k) TRACE_AT(22);
             }
           }
         }
