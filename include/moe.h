@@ -169,6 +169,23 @@ moe_status moe_expert_ffn(const moe_layer* layer, const void* x_dev, int T,
                           float* y_dev, void* ws_dev, size_t ws_bytes,
                           void* stream);
 
+/* moe_expert_ffn for a subset of the slots, so that the experts of a token
+ * can run in several calls (a streamed cache runs the resident experts first
+ * and each copied one once its copy is done: colibri summary, "Principales
+ * fonctionnalites implementees", the next expert block read while another is
+ * multiplied).  slot_mask bit j (j < top_k) runs routed slot j of every
+ * token, bit top_k the shared expert; the partial outputs of the other slots
+ * in the workspace are left as they are.  combine != 0 then writes y from the
+ * partial outputs of every slot -- those of this call and of earlier calls on
+ * the same workspace with the same x, idx and T -- in the fixed slot order,
+ * so that calls covering every slot once give y bitwise equal to one
+ * moe_expert_ffn call.  combine == 0 leaves y unwritten.  Other arguments
+ * and errors as moe_expert_ffn. */
+moe_status moe_expert_ffn_part(const moe_layer* layer, const void* x_dev, int T,
+                               const int32_t* idx_dev, const float* w_dev,
+                               float* y_dev, uint64_t slot_mask, int combine,
+                               void* ws_dev, size_t ws_bytes, void* stream);
+
 /* Steps 1-5 for T tokens.  idx_out_dev / w_out_dev nullable.  T == 1 runs the
  * single fused persistent decode kernel; T > 1 runs the batched path, which
  * reads every distinct selected expert once for all tokens routed to it.
@@ -283,6 +300,39 @@ moe_status moe_cache_layer(moe_cache* cache, int layer,
 moe_status moe_cache_acquire(moe_cache* cache, int layer,
                              const int32_t* ids_host, int n,
                              void* compute_stream);
+/* moe_cache_acquire with one completion per copied expert instead of one
+ * for the call: the replacement, counters, usage log and the pointer-table
+ * update on compute_stream are those of moe_cache_acquire, but compute_stream
+ * does not wait for the copies.  missed_host[j] (n int32, caller-owned) is
+ * set to 1 when ids_host[j] was copied by this call, else 0; before compute
+ * on compute_stream reads a copied expert, the caller calls
+ * moe_cache_wait_expert for it (a hit needs no wait: this call makes
+ * compute_stream wait for any copy of a hit's slot still pending), so the
+ * resident experts can run while the copies are on the link.
+ * Transactional and with the limits of moe_cache_acquire. */
+moe_status moe_cache_acquire_split(moe_cache* cache, int layer,
+                                   const int32_t* ids_host, int n,
+                                   void* compute_stream, int32_t* missed_host);
+/* Make compute_stream wait until the copy that loaded `expert` into
+ * `layer`'s cache is done (MOE_ERR_INVALID_ARG if the expert is not in the
+ * cache). */
+moe_status moe_cache_wait_expert(moe_cache* cache, int layer, int expert,
+                                 void* compute_stream);
+/* One token of `layer` through the cache, the resident experts first:
+ * moe_cache_acquire_split of the token's top_k ids (ids_host, ascending,
+ * distinct; the same ids as idx_dev, which the kernels read), then
+ * moe_expert_ffn_part of the hits and the shared expert at once, then, for
+ * each copied expert in slot order, moe_cache_wait_expert and its own
+ * moe_expert_ffn_part; the last call combines.  y_dev is bitwise that of
+ * moe_expert_ffn on the resident layer.  x_dev bf16 [1][hidden], idx_dev
+ * int32 [1][top_k], w_dev fp32 [1][top_k], y_dev fp32 [1][hidden], a
+ * workspace of moe_workspace_bytes(cfg, 1).  n_copied (nullable): how many
+ * experts were copied.  Errors as the calls it makes; on an error after the
+ * acquire the caller still releases the layer. */
+moe_status moe_cache_expert_ffn(moe_cache* cache, int layer, const void* x_dev,
+                                const int32_t* ids_host, const int32_t* idx_dev,
+                                const float* w_dev, float* y_dev, void* ws_dev,
+                                size_t ws_bytes, void* stream, int* n_copied);
 /* Hot-store (colibri summary, "Learning cache et attentes selon le
  * materiel": routed experts are logged and the most used are pinned at
  * start-up).  Makes ids_host[0..n) (ascending, distinct) the pinned set of

@@ -78,6 +78,8 @@ def lib():
         L.moe_route.argtypes = [p, p, i, p, p, p, p, sz, p]
         L.moe_expert_ffn.restype = st
         L.moe_expert_ffn.argtypes = [p, p, i, p, p, p, p, sz, p]
+        L.moe_expert_ffn_part.restype = st
+        L.moe_expert_ffn_part.argtypes = [p, p, i, p, p, p, ctypes.c_uint64, i, p, sz, p]
         L.moe_layer_forward.restype = st
         L.moe_layer_forward.argtypes = [p, p, i, p, p, p, p, sz, p]
         L.moe_layer_forward_noalloc.restype = st
@@ -94,6 +96,12 @@ def lib():
         L.moe_cache_layer.argtypes = [p, i, p, p, p, ctypes.POINTER(p)]
         L.moe_cache_acquire.restype = st
         L.moe_cache_acquire.argtypes = [p, i, p, i, p]
+        L.moe_cache_acquire_split.restype = st
+        L.moe_cache_acquire_split.argtypes = [p, i, p, i, p, p]
+        L.moe_cache_wait_expert.restype = st
+        L.moe_cache_wait_expert.argtypes = [p, i, i, p]
+        L.moe_cache_expert_ffn.restype = st
+        L.moe_cache_expert_ffn.argtypes = [p, i, p, p, p, p, p, p, sz, p, p]
         L.moe_cache_release.restype = st
         L.moe_cache_release.argtypes = [p, i, p]
         L.moe_cache_stats.restype = st
@@ -198,6 +206,14 @@ class Layer:
         check(lib().moe_expert_ffn(self.handle, _ptr(x), T, _ptr(idx), _ptr(w), _ptr(y),
                                    _ptr(ws), ws.numel(), _stream(stream)), "moe_expert_ffn")
 
+    def expert_ffn_part(self, x, idx, w, y, ws, slot_mask, combine, stream=None):
+        """moe_expert_ffn for the slots in slot_mask (bit top_k: the shared
+        expert); combine: write y from every slot's partial output."""
+        T = x.shape[0]
+        check(lib().moe_expert_ffn_part(self.handle, _ptr(x), T, _ptr(idx), _ptr(w), _ptr(y),
+                                        int(slot_mask), int(bool(combine)), _ptr(ws),
+                                        ws.numel(), _stream(stream)), "moe_expert_ffn_part")
+
     def forward(self, x, y, ws, idx=None, w=None, stream=None):
         T = x.shape[0]
         check(lib().moe_layer_forward(self.handle, _ptr(x), T, _ptr(y), _ptr(idx), _ptr(w),
@@ -260,6 +276,7 @@ class _LayerView:
 
     route = Layer.route
     expert_ffn = Layer.expert_ffn
+    expert_ffn_part = Layer.expert_ffn_part
     forward = Layer.forward
     set_top_p = Layer.set_top_p
 
@@ -299,6 +316,33 @@ class Cache:
         a = np.ascontiguousarray(ids, dtype=np.int32)
         check(lib().moe_cache_acquire(self.handle, int(l), a.ctypes.data, a.size, _stream(stream)),
               "moe_cache_acquire")
+
+    def acquire_split(self, l, ids, stream=None):
+        """acquire without waiting for the copies: returns a bool array, True
+        where ids[j] was copied (wait_expert before computing it)."""
+        import numpy as np
+        a = np.ascontiguousarray(ids, dtype=np.int32)
+        missed = np.zeros(a.size, dtype=np.int32)
+        check(lib().moe_cache_acquire_split(self.handle, int(l), a.ctypes.data, a.size,
+                                            _stream(stream), missed.ctypes.data),
+              "moe_cache_acquire_split")
+        return missed.astype(bool)
+
+    def wait_expert(self, l, expert, stream=None):
+        check(lib().moe_cache_wait_expert(self.handle, int(l), int(expert), _stream(stream)),
+              "moe_cache_wait_expert")
+
+    def expert_ffn(self, l, x, idx, w, ids_host, y, ws, stream=None):
+        """moe_cache_expert_ffn: one token of layer l through the cache, the
+        resident experts first, each copied one once its copy is done.
+        Returns the number of copied experts."""
+        import numpy as np
+        a = np.ascontiguousarray(ids_host, dtype=np.int32)
+        n = ctypes.c_int()
+        check(lib().moe_cache_expert_ffn(self.handle, int(l), _ptr(x), a.ctypes.data, _ptr(idx),
+                                         _ptr(w), _ptr(y), _ptr(ws), ws.numel(), _stream(stream),
+                                         ctypes.byref(n)), "moe_cache_expert_ffn")
+        return n.value
 
     def pin(self, l, ids, stream=None):
         """Make ids (ascending) the pinned hot-store of layer l."""

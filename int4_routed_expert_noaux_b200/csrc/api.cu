@@ -312,6 +312,21 @@ moe_status moe_expert_ffn(const moe_layer* l, const void* x, int T, const int32_
   return ffn_impl(l, (const uint16_t*)x, T, idx, w, y, (uint8_t*)ws, L, (cudaStream_t)stream);
 }
 
+moe_status moe_expert_ffn_part(const moe_layer* l, const void* x, int T, const int32_t* idx,
+                               const float* w, float* y, uint64_t slot_mask, int combine,
+                               void* ws, size_t ws_bytes, void* stream) {
+  g_last_error[0] = 0;
+  moe_status s = check_call(l, x, T);
+  if (s != MOE_OK) return s;
+  if ((s = check_device_ptr(idx, 4, "idx")) != MOE_OK) return s;
+  if ((s = check_device_ptr(w, 4, "w")) != MOE_OK) return s;
+  if ((s = check_device_ptr(y, 16, "y")) != MOE_OK) return s;
+  WsLayout L;
+  if ((s = check_ws(l, T, ws, ws_bytes, &L)) != MOE_OK) return s;
+  return ffn_impl(l, (const uint16_t*)x, T, idx, w, y, (uint8_t*)ws, L, (cudaStream_t)stream,
+                  slot_mask, combine != 0);
+}
+
 moe_status moe_layer_forward(const moe_layer* l, const void* x, int T, float* y,
                              int32_t* idx_out, float* w_out, void* ws, size_t ws_bytes,
                              void* stream) {

@@ -48,6 +48,8 @@ class LruPolicy {
     pinned_[slot] = 0;
   }
 
+  int slot_of(int expert) const { return expert_slot_[expert]; }
+
   int pinned_count() const {
     int n = 0;
     for (char p : pinned_) n += p;
@@ -172,6 +174,7 @@ struct moe_cache {
   cudaStream_t copy_stream = nullptr;
   std::vector<cudaEvent_t> copied;     // per layer: loads of the last acquire done
   std::vector<cudaEvent_t> used;       // per layer: compute of the last release done
+  std::vector<cudaEvent_t> slot_ev;    // [L][slots]: the copies of the slot's latest load done
   std::vector<bool> used_valid;
   std::vector<bool> acquired;          // per layer: acquired, not yet released
   std::vector<LruPolicy> lru;
@@ -232,7 +235,8 @@ moe_status check_ids(const moe_cache* c, const int32_t* ids, int n) {
 // `acquire_ids` (n of them, nullable) are the ids of an acquire: they count
 // as hits / misses and in the usage log; a pin counts only its bytes.
 moe_status commit_loads(moe_cache* c, int layer, cudaStream_t cs, const LruPolicy& plan,
-                        int hits, const int32_t* acquire_ids, int n, const char* who) {
+                        int hits, const int32_t* acquire_ids, int n, const char* who,
+                        bool split = false) {
   cudaError_t ce = cudaSuccess;
   if (!c->loads.empty()) {
     // A victim slot may still be read by compute enqueued earlier for this
@@ -269,14 +273,19 @@ moe_status commit_loads(moe_cache* c, int layer, cudaStream_t cs, const LruPolic
       ce = inject(MOE_FAULT_CACHE_COPY)
                ? cudaErrorInvalidValue
                : cudaMemcpyAsync(dst[t], src[t], sz[t], cudaMemcpyHostToDevice, c->copy_stream);
+    // this expert's own completion, for compute that waits per expert
+    if (ce == cudaSuccess)
+      ce = cudaEventRecord(c->slot_ev[(size_t)layer * c->slots + ld.slot], c->copy_stream);
     TableUpdate& u = ups[(reached - 1) / kMaxTableUpdates];
     u.ids[u.n] = ld.expert;
     u.ptrs[u.n] = d;
     ++u.n;
   }
   if (!c->loads.empty()) {
-    if (ce == cudaSuccess) ce = cudaEventRecord(c->copied[layer], c->copy_stream);
-    if (ce == cudaSuccess) ce = cudaStreamWaitEvent(cs, c->copied[layer], 0);
+    if (!split) {
+      if (ce == cudaSuccess) ce = cudaEventRecord(c->copied[layer], c->copy_stream);
+      if (ce == cudaSuccess) ce = cudaStreamWaitEvent(cs, c->copied[layer], 0);
+    }
     for (size_t i = 0; i < ups.size() && ce == cudaSuccess; ++i) {
       table_update_kernel<<<1, kMaxTableUpdates, 0, cs>>>(c->views[layer]->table, ups[i]);
       ce = cudaGetLastError();
@@ -379,12 +388,15 @@ moe_status moe_cache_create(const moe_config* cfg, int n_layers, int slots_per_l
   if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&c->copy_stream, cudaStreamNonBlocking);
   c->copied.assign(n_layers, nullptr);
   c->used.assign(n_layers, nullptr);
+  c->slot_ev.assign((size_t)n_layers * slots_per_layer, nullptr);
   c->used_valid.assign(n_layers, false);
   c->acquired.assign(n_layers, false);
   for (int l = 0; l < n_layers && ce == cudaSuccess; ++l) {
     ce = cudaEventCreateWithFlags(&c->copied[l], cudaEventDisableTiming);
     if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->used[l], cudaEventDisableTiming);
   }
+  for (size_t i = 0; i < c->slot_ev.size() && ce == cudaSuccess; ++i)
+    ce = cudaEventCreateWithFlags(&c->slot_ev[i], cudaEventDisableTiming);
   if (ce != cudaSuccess) {
     s = cuda_fail(ce, "moe_cache_create");
     moe_cache_destroy(c);
@@ -407,6 +419,8 @@ void moe_cache_destroy(moe_cache* c) {
   for (cudaEvent_t e : c->copied)
     if (e) cudaEventDestroy(e);
   for (cudaEvent_t e : c->used)
+    if (e) cudaEventDestroy(e);
+  for (cudaEvent_t e : c->slot_ev)
     if (e) cudaEventDestroy(e);
   if (c->copy_stream) cudaStreamDestroy(c->copy_stream);
   if (c->dev_slots) cudaFree(c->dev_slots);
@@ -455,6 +469,85 @@ moe_status moe_cache_acquire(moe_cache* c, int layer, const int32_t* ids_host, i
   const int hits = plan.access(ids_host, n, c->loads);
   return commit_loads(c, layer, (cudaStream_t)compute_stream, plan, hits, ids_host, n,
                       "moe_cache_acquire");
+}
+
+moe_status moe_cache_acquire_split(moe_cache* c, int layer, const int32_t* ids_host, int n,
+                                   void* compute_stream, int32_t* missed_host) {
+  if (!c || !ids_host || !missed_host) return fail(MOE_ERR_INVALID_ARG, "cache, ids or missed is NULL");
+  if (layer < 0 || layer >= c->n_layers) return fail(MOE_ERR_INVALID_ARG, "layer out of range");
+  if (!c->views[layer]) return fail(MOE_ERR_INVALID_ARG, "create the layer view first (moe_cache_layer)");
+  if (n < 1 || n > c->slots || n > kMaxTableUpdates)
+    return fail(MOE_ERR_INVALID_ARG, "n = %d outside 1..min(slots, %d)", n, kMaxTableUpdates);
+  moe_status st = check_ids(c, ids_host, n);
+  if (st != MOE_OK) return st;
+  if (n > c->slots - c->lru[layer].pinned_count())
+    return fail(MOE_ERR_INVALID_ARG, "n = %d exceeds the layer's unpinned slots", n);
+  cudaStream_t cs = (cudaStream_t)compute_stream;
+  LruPolicy plan = c->lru[layer];
+  const int hits = plan.access(ids_host, n, c->loads);
+  st = commit_loads(c, layer, cs, plan, hits, ids_host, n, "moe_cache_acquire_split", true);
+  if (st != MOE_OK) return st;
+  // a hit's slot may hold a load whose copies no compute has waited for
+  // yet: the compute stream waits for the slot's latest load (long done,
+  // as a rule); the misses are left to moe_cache_wait_expert
+  for (int j = 0; j < n; ++j) {
+    bool missed = false;
+    for (const LruPolicy::Load& ld : c->loads) missed = missed || ld.expert == ids_host[j];
+    missed_host[j] = missed ? 1 : 0;
+    if (!missed) {
+      const int s = c->lru[layer].slot_of(ids_host[j]);
+      const cudaError_t ce = cudaStreamWaitEvent(cs, c->slot_ev[(size_t)layer * c->slots + s], 0);
+      if (ce != cudaSuccess) return cuda_fail(ce, "moe_cache_acquire_split");
+    }
+  }
+  return MOE_OK;
+}
+
+moe_status moe_cache_wait_expert(moe_cache* c, int layer, int expert, void* compute_stream) {
+  if (!c) return fail(MOE_ERR_INVALID_ARG, "cache is NULL");
+  if (layer < 0 || layer >= c->n_layers) return fail(MOE_ERR_INVALID_ARG, "layer out of range");
+  if (expert < 0 || expert >= c->cfg.n_experts)
+    return fail(MOE_ERR_INVALID_ARG, "expert %d out of range", expert);
+  const int s = c->lru[layer].slot_of(expert);
+  if (s < 0) return fail(MOE_ERR_INVALID_ARG, "expert %d is not in layer %d's cache", expert, layer);
+  const cudaError_t ce = cudaStreamWaitEvent((cudaStream_t)compute_stream,
+                                             c->slot_ev[(size_t)layer * c->slots + s], 0);
+  return ce == cudaSuccess ? MOE_OK : cuda_fail(ce, "moe_cache_wait_expert");
+}
+
+moe_status moe_cache_expert_ffn(moe_cache* c, int layer, const void* x_dev,
+                                const int32_t* ids_host, const int32_t* idx_dev,
+                                const float* w_dev, float* y_dev, void* ws_dev, size_t ws_bytes,
+                                void* stream, int* n_copied) {
+  if (!c || !ids_host) return fail(MOE_ERR_INVALID_ARG, "cache or ids is NULL");
+  if (layer < 0 || layer >= c->n_layers) return fail(MOE_ERR_INVALID_ARG, "layer out of range");
+  const int k = c->cfg.top_k;
+  int32_t missed[kMaxTableUpdates];
+  moe_status s = moe_cache_acquire_split(c, layer, ids_host, k, stream, missed);
+  if (s != MOE_OK) return s;
+  const moe_layer* view = c->views[layer];
+  uint64_t hit_mask = c->cfg.n_shared ? 1ull << k : 0ull;
+  int n_miss = 0;
+  for (int j = 0; j < k; ++j) {
+    if (missed[j]) ++n_miss;
+    else hit_mask |= 1ull << j;
+  }
+  // the resident experts (and the shared one) while the copies are on the link
+  if (hit_mask)
+    s = moe_expert_ffn_part(view, x_dev, 1, idx_dev, w_dev, y_dev, hit_mask, n_miss == 0, ws_dev,
+                            ws_bytes, stream);
+  // then each copied expert as soon as its own copy is done; the last call
+  // combines every slot in the fixed order
+  for (int j = 0, m = 0; j < k && s == MOE_OK; ++j) {
+    if (!missed[j]) continue;
+    ++m;
+    s = moe_cache_wait_expert(c, layer, ids_host[j], stream);
+    if (s == MOE_OK)
+      s = moe_expert_ffn_part(view, x_dev, 1, idx_dev, w_dev, y_dev, 1ull << j, m == n_miss,
+                              ws_dev, ws_bytes, stream);
+  }
+  if (s == MOE_OK && n_copied) *n_copied = n_miss;
+  return s;
 }
 
 moe_status moe_cache_pin(moe_cache* c, int layer, const int32_t* ids_host, int n,

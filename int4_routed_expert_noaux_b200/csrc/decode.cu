@@ -267,11 +267,11 @@ __device__ __forceinline__ bool aborted(const uint32_t* ctrl) {
 __device__ bool wait_counter(uint32_t* ctrl, const uint32_t* p, uint32_t target) {
   if (ld_acquire(p) >= target) return true;
   const uint64_t deadline = global_timer_ns() + kWaitNs;
-  uint32_t sleep_ns = 64;  // back off so that polling warps leave issue slots free
+  // one polling thread: a short constant pause, so that the wait ends within
+  // tens of nanoseconds of the count (no growing back-off on this path)
   for (uint32_t it = 0;; ++it) {
-    __nanosleep(sleep_ns);
+    __nanosleep(32);
     if (ld_acquire(p) >= target) return true;
-    if (sleep_ns < 512) sleep_ns <<= 1;
     if ((it & 7) == 7) {
       if (aborted(ctrl) || global_timer_ns() > deadline) return false;
     }
@@ -857,6 +857,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       }
       __syncwarp();
       run_select(sel_args(p), S);
+      if (lane == 0) TRACE_AT(24);
       __syncwarp();
       // the selected experts' tensor pointers, one load per lane, so that
       // no fill waits on a pointer-table load from global memory

@@ -19,7 +19,8 @@ moe_status route_impl(const moe_layer* l, const uint16_t* x, int T, int32_t* idx
 }
 
 moe_status ffn_impl(const moe_layer* l, const uint16_t* x, int T, const int32_t* idx,
-                    const float* w, float* y, uint8_t* ws, const WsLayout& L, cudaStream_t st) {
+                    const float* w, float* y, uint8_t* ws, const WsLayout& L, cudaStream_t st,
+                    uint64_t slot_mask, bool combine) {
   const moe_config& c = l->cfg;
   cudaError_t e = launch_union_ffn(
       l->table, idx, w, x, T, c.hidden, c.inter, c.n_experts, c.top_k, c.n_shared, ws + L.xq,
@@ -27,7 +28,7 @@ moe_status ffn_impl(const moe_layer* l, const uint16_t* x, int T, const int32_t*
       reinterpret_cast<int*>(ws + L.lists), reinterpret_cast<float*>(ws + L.hbuf),
       reinterpret_cast<float*>(ws + L.ypart), y, reinterpret_cast<uint32_t*>(ws + L.ctrl),
       L.tc_bytes ? ws + L.tc : nullptr, reinterpret_cast<int*>(ws + L.tc_exp),
-      L.tc_bytes ? ws + L.tc_maps : nullptr, st);
+      L.tc_bytes ? ws + L.tc_maps : nullptr, st, slot_mask, combine);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "expert launch");
 }
 

@@ -76,7 +76,11 @@ cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const 
                              uint8_t* xq_words, float* xq_fac, uint8_t* hq_words, float* hq_fac,
                              int* lists, float* hbuf, float* ypart, float* y, uint32_t* err,
                              uint8_t* tc_bpack, int* tc_rowexp, uint8_t* tc_maps,
-                             cudaStream_t st);
+                             cudaStream_t st, uint64_t slot_mask = ~0ull, bool combine = true);
+// slot_mask: bit j (j < k) computes routed slot j of every token, bit k the
+// shared expert; the rows of the other slots in ypart are left as they are.
+// combine: y from every slot's ypart row (including rows an earlier call on
+// the same workspace computed), in the fixed slot order.
 // The tensor-core path (tc_union.cu): packed inputs and per-row exponents.
 size_t tc_bpack_bytes(int T, int k, int has_shared, int H, int I);
 size_t tc_rowexp_ints(int T, int k, int has_shared);

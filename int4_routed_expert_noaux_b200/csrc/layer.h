@@ -42,7 +42,8 @@ ExpertPtrs to_ptrs(const moe_expert& e);
 moe_status route_impl(const moe_layer* l, const uint16_t* x, int T, int32_t* idx, float* w,
                       float* scores, uint8_t* ws, const WsLayout& L, cudaStream_t st);
 moe_status ffn_impl(const moe_layer* l, const uint16_t* x, int T, const int32_t* idx,
-                    const float* w, float* y, uint8_t* ws, const WsLayout& L, cudaStream_t st);
+                    const float* w, float* y, uint8_t* ws, const WsLayout& L, cudaStream_t st,
+                    uint64_t slot_mask = ~0ull, bool combine = true);
 // next (nullable): the layer that runs after this one (a stack), whose
 // first bytes this layer's kernel prefetches into L2.
 moe_status residual_impl(const moe_layer* l, const float* x_resid, float norm_eps, float* x_next,

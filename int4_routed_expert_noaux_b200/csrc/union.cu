@@ -83,15 +83,19 @@ __global__ void __launch_bounds__(256) xq_table_kernel(const void* __restrict__ 
 // The expert lists of the call (layout: ListsView).  Out-of-range ids set
 // the error word and are left out; -1 (a slot dropped by top-p) is skipped.
 __global__ void __launch_bounds__(256) build_lists_kernel(const int32_t* __restrict__ idx, int T,
-                                                          int k, int E, int has_shared, int tc_min,
+                                                          int k, int E, int has_shared,
+                                                          uint64_t slot_mask, int tc_min,
                                                           int* __restrict__ lists,
                                                           uint32_t* __restrict__ err) {
   __shared__ int cnt[kListMaxE];
   __shared__ int base[kListMaxE];
   __shared__ int sid[kListMaxIds];
-  const int slots = k + has_shared;
+  const int slots = k + has_shared;  // the layout of h and ypart rows: (token, slot)
   const int n_list = T * slots;
   const ListsView L = lists_view(lists, E, n_list);
+  // the slots this call computes: routed slot j when bit j of slot_mask is
+  // set, the shared expert when bit k is (the others keep their rows)
+  const bool shared_on = has_shared && ((slot_mask >> k) & 1ull);
   int* u_expert = const_cast<int*>(L.u_expert);
   int* u_off = const_cast<int*>(L.u_off);
   int* list_tok = const_cast<int*>(L.list_tok);
@@ -104,7 +108,7 @@ __global__ void __launch_bounds__(256) build_lists_kernel(const int32_t* __restr
   // number (no atomics, which correlated tokens would serialise on a few ids)
   for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
     const int e = idx[i];
-    sid[i] = e;
+    sid[i] = ((slot_mask >> (i % k)) & 1ull) ? e : -1;
     if ((e < 0 || e >= E) && e != -1) atomicCAS(err, 0u, (uint32_t)kErrBadExpertId);
   }
   for (int e = threadIdx.x; e <= E; e += blockDim.x) cnt[e] = 0;
@@ -119,7 +123,7 @@ __global__ void __launch_bounds__(256) build_lists_kernel(const int32_t* __restr
     }
   }
   __syncthreads();
-  if (threadIdx.x == 0 && has_shared) cnt[E] = T;
+  if (threadIdx.x == 0 && shared_on) cnt[E] = T;
   __syncthreads();
   // exclusive scans of (expert used, tensor-core expert, entries, packed
   // rows) over experts 0..E, ascending: thread i owns experts 2i and 2i + 1
@@ -217,7 +221,7 @@ __global__ void __launch_bounds__(256) build_lists_kernel(const int32_t* __restr
       __syncwarp();
     }
   }
-  if (has_shared) {
+  if (shared_on) {
     for (int t = threadIdx.x; t < T; t += blockDim.x) {
       list_tok[base[E] + t] = t;
       list_pos[base[E] + t] = t * slots + k;
@@ -473,7 +477,7 @@ cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const 
                              uint8_t* xq_words, float* xq_fac, uint8_t* hq_words, float* hq_fac,
                              int* lists, float* hbuf, float* ypart, float* y, uint32_t* err,
                              uint8_t* tc_bpack, int* tc_rowexp, uint8_t* tc_maps,
-                             cudaStream_t st) {
+                             cudaStream_t st, uint64_t slot_mask, bool combine) {
   if (E + 1 > kListMaxE || T * k > kListMaxIds) return cudaErrorInvalidValue;
   const int tc_min = tc_min_tokens();
   const bool tc = tc_bpack && tc_maps && T >= tc_min && tc_shape_ok(H, I);
@@ -482,8 +486,8 @@ cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const 
   const int n_list = T * slots;
   const int umax = (E < T * k ? E : T * k) + has_shared;
   xq_table_kernel<true><<<(T * G + 255) / 256, 256, 0, st>>>(x, T, H, xq_words, xq_fac);
-  build_lists_kernel<<<1, 256, 0, st>>>(idx, T, k, E, has_shared, tc ? tc_min : 0, lists,
-                                         err);
+  build_lists_kernel<<<1, 256, 0, st>>>(idx, T, k, E, has_shared, slot_mask, tc ? tc_min : 0,
+                                         lists, err);
   UnionArgs a;
   a.table = table;
   a.lists = lists;
@@ -546,8 +550,9 @@ cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const 
                                              err, st);
     if (e != cudaSuccess) return e;
   }
-  union_combine_kernel<<<dim3((H + 255) / 256, T), 256, 0, st>>>(idx, w, ypart, T, H, k, E,
-                                                                 has_shared, y);
+  if (combine)
+    union_combine_kernel<<<dim3((H + 255) / 256, T), 256, 0, st>>>(idx, w, ypart, T, H, k, E,
+                                                                   has_shared, y);
   return cudaGetLastError();
 }
 

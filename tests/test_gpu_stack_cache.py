@@ -357,3 +357,82 @@ def test_cache_pin_changes_and_limits():
     torch.cuda.synchronize()
     assert torch.equal(y_c, y_r)
     cache.close()
+
+
+# ---------------------------------------------------------------------------
+# the experts of a token in several calls, and compute that waits per expert
+
+@pytest.mark.parametrize("shape,T", [(synth.TINY, 1), (synth.TINY, 6), (synth.GLM, 1)],
+                         ids=["tiny-1", "tiny-6", "glm-1"])
+def test_expert_ffn_parts_match_one_call(shape, T):
+    # slots computed in three calls, in a scrambled order, then combined:
+    # y is bitwise that of one moe_expert_ffn call, and a call with
+    # combine = 0 leaves y alone
+    from test_gpu_parity import get_layer, to_dev_bf16
+    dl, L = get_layer(shape)
+    cfg = moe.Config.from_shape(shape)
+    k = shape.top_k
+    x = to_dev_bf16(synth.tokens(shape, 0, 90, T))
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    ws = moe.alloc_workspace(cfg, T)
+    L.route(x, idx, w, ws)
+    y_ref = torch.empty((T, shape.hidden), dtype=torch.float32, device="cuda")
+    L.expert_ffn(x, idx, w, y_ref, ws)
+    ws2 = moe.alloc_workspace(cfg, T)
+    y = torch.full((T, shape.hidden), 7.0, dtype=torch.float32, device="cuda")
+    rng = np.random.default_rng(3)
+    order = rng.permutation(k + 1)          # slot k: the shared expert
+    parts = np.array_split(order, 3)
+    for n, part in enumerate(parts):
+        mask = sum(1 << int(j) for j in part)
+        L.expert_ffn_part(x, idx, w, y, ws2, mask, n == len(parts) - 1)
+        if n < len(parts) - 1:
+            torch.cuda.synchronize()
+            assert torch.all(y == 7.0)
+    moe.ws_check(ws2)
+    assert torch.equal(y, y_ref)
+
+
+@pytest.mark.parametrize("cap", [2, 5], ids=["cap-k", "cap5"])
+def test_cache_expert_ffn_waits_per_expert(cap):
+    # moe_cache_expert_ffn (hits and the shared expert first, each copied
+    # expert after its own copy): bitwise the resident output, and the
+    # oracle's LRU counts
+    needs_gpu()
+    shape = synth.TINY
+    L, T = 3, 30
+    cfg = moe.Config.from_shape(shape)
+    host = [[pinned_expert(shape, 0, l, e) for e in range(shape.n_experts)] for l in range(L)]
+    dls = [DeviceLayer(shape, 0, l) for l in range(L)]
+    resident = [moe.Layer(cfg, d.w_router, d.bias, d.routed, d.shared) for d in dls]
+    cache = moe.Cache(cfg, host, cap)
+    for l in range(L):
+        cache.layer(l, dls[l].w_router, dls[l].bias, dls[l].shared)
+    trace = synth.zipf_trace(9, L, shape.n_experts, shape.top_k, T)
+    x = torch.from_numpy(synth.tokens(shape, 0, 80, T).view(np.int16)).cuda()
+    wts = torch.tensor([[1.25, 0.75]], dtype=torch.float32, device="cuda")
+    ws, ws2 = moe.alloc_workspace(cfg, 1), moe.alloc_workspace(cfg, 1)
+    y_s = torch.empty((T, L, shape.hidden), dtype=torch.float32, device="cuda")
+    y_r = torch.empty_like(y_s)
+    copied = 0
+    for t in range(T):
+        for l in range(L):
+            idx = torch.from_numpy(trace[t, l].reshape(1, -1).copy()).cuda()
+            copied += cache.expert_ffn(l, x[t:t + 1], idx, wts, trace[t, l], y_s[t, l:l + 1], ws)
+            cache.release(l)
+            resident[l].expert_ffn(x[t:t + 1], idx, wts, y_r[t, l:l + 1], ws2)
+    moe.ws_check(ws)
+    moe.ws_check(ws2)
+    cache.sync()
+    assert torch.equal(y_s, y_r)
+    h_ref, m_ref = oracle.lru_sim(trace, shape.n_experts, cap)
+    assert copied == int(m_ref.sum())
+    for l in range(L):
+        h, m, b = cache.stats(l)
+        assert (h, m) == (int(h_ref[l]), int(m_ref[l]))
+    absent = [e for e in range(shape.n_experts) if e not in trace[:, 0]]
+    if absent:  # an expert layer 0 never loaded is not in its cache
+        with pytest.raises(moe.MoeError):
+            cache.wait_expert(0, absent[0])
+    cache.close()
