@@ -15,33 +15,37 @@
 //    int16 fixed point with one exponent per group; the int4 group dot
 //    product is exact in integers (dp2a); one butterfly reduce-scatter plus
 //    a cross-warp sum finishes each row; one group barrier per item;
-//  * start-up: the producer's first fill is the CTA's block of router rows
-//    (a static split of the experts over the first CTAs).  Group 0 computes
-//    the router rows in double-float arithmetic and publishes each row's
-//    sigmoid score as a 64-bit record tagged with the call's epoch (one
-//    single-copy-atomic store: no flag, no fence);
+//  * start-up: the producer's first fills are the CTA's block of router
+//    rows (a static split of the experts over the CTAs), one fill per
+//    consumer group.  The groups compute the router rows in double-float
+//    arithmetic and publish each row's sigmoid score as a 64-bit record
+//    tagged with the call's epoch (one single-copy-atomic store: no flag, no
+//    fence);
 //  * the selection warp of every CTA polls the E records until all carry
 //    this call's epoch and runs the noaux_tc selection itself -- every CTA
-//    reads the same scores with the same code, so all reach the same bits --
-//    then loads the selected experts' tensor pointers into shared memory
-//    once;
+//    reads the same scores with the same code, so all reach the same bits.
+//    The routed experts are handled in pick order (descending score): each
+//    pick's barrier is released as soon as the pick is final, so the
+//    producer streams pick 0 while the later picks are still being found;
 //  * gate/up items (8 gate + 8 up rows of one expert for the GLM shape) are
 //    dealt out statically, CTA b taking items b, b + grid, ... in the order
-//    shared expert, routed slots 0..k-1; the shared expert's items keep HBM
+//    shared expert, routed picks 0..k-1; the shared expert's items keep HBM
 //    busy while the routed experts are selected.  Finalizer warps write h
 //    rows (fp32) and count, per 32-row group of h, the rows written;
 //  * the converter warp of each CTA owns some of those groups: once a
 //    group's 32 rows are in, it publishes them as int16 words with one
-//    exponent (the layout the down consumers load) and counts the slot's
+//    exponent (the layout the down consumers load) and counts the pick's
 //    published groups;
 //  * down items are static too: CTA b owns a block of output rows and, once
-//    a slot's h is published, streams that slot's down rows for it together
-//    with the slot's int16 h (4 KB); the slot partials of its rows stay in
-//    shared memory and are combined in slot order at the end (no atomics, no
-//    cross-CTA combine, bitwise repeatable);
-//  * consumer group 1 first runs one placeholder gate/up and one placeholder
-//    down item through the loop body (nothing published), so that both code
-//    paths are fetched while the first weights are in flight;
+//    a pick's h is published, streams that pick's down rows for it together
+//    with the pick's int16 h (4 KB); the partials of its rows stay in shared
+//    memory and are combined at the end in slot order (ascending expert id,
+//    as the outputs are laid out): no atomics, no cross-CTA combine, bitwise
+//    repeatable;
+//  * consumer group 1 of a CTA without a second router fill first runs one
+//    placeholder gate/up and one placeholder down item through the loop
+//    body (nothing published), so that both code paths are fetched while
+//    the first weights are in flight;
 //  * every wait is bounded (1 s); a wait that runs out sets the workspace
 //    error word and the kernel winds down; the last CTA to exit resets the
 //    control counters so the next call starts clean.
@@ -105,13 +109,15 @@ struct Smem {
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t gbar[kGroups];  // per-group item barrier (one arrival per warp)
-  uint64_t selbar;         // the selection warp has published sel_*
+  uint64_t pickbar[kMaxSlots];  // pick r of the selection is final (one arrival)
   ItemDesc desc[kStages];
-  int sel_idx[kMaxSlots];  // selected expert ids, ascending
-  ExpertPtrs ep[kMaxSlots];  // the slots' expert tensors (slot k: the shared expert)
-  int pick_id[kMaxSlots];  // the selection's picks in pick order
+  int sel_idx[kMaxSlots];  // selected expert ids, ascending (the slot order)
+  ExpertPtrs ep[kMaxSlots];  // the picks' expert tensors (index k: the shared expert)
+  int pick_id[kMaxSlots];  // the selection's picks in pick order (descending score)
   float pick_s[kMaxSlots];
-  float sel_w[kMaxSlots];  // their combine weights
+  int pick_kept[kMaxSlots];  // pick r kept by top-p (valid once the whole selection is out)
+  int slot_pick[kMaxSlots];  // the pick that is slot j
+  float sel_w[kMaxSlots];  // the slots' combine weights
   int sel_ok;
   float red[kGroups][2][kGW][32];
   double redd[kGroups * kGW][kMaxRR];  // router partial sums (fp64), per group and warp
@@ -120,7 +126,7 @@ struct Smem {
   float inv_rms;
   float sc[kMaxE];
   float sp[kMaxE];
-  float ycta[kMaxYcta];    // [slots][ycta_rows] partial y of the CTA's own rows
+  float ycta[kMaxYcta];    // [picks + shared][ycta_rows] partial y of the CTA's own rows
   int last_cta;
 };
 
@@ -134,6 +140,7 @@ struct SelArgs {
   float* w_out;
   uint64_t* trace;   // timeline probes of a -DMOE_TRACE build
   const ExpertPtrs* table;  // nullable in a dry run
+  int early_picks;  // each pick's barrier arrives as soon as the pick is final
 };
 
 __device__ __forceinline__ SelArgs sel_args(const DecodeParams& p) {
@@ -151,6 +158,8 @@ __device__ __forceinline__ SelArgs sel_args(const DecodeParams& p) {
   a.w_out = p.w_out;
   a.trace = p.trace;
   a.table = p.table;
+  // with every pick kept (no top-p), pick r is final once it is popped
+  a.early_picks = p.sel_fast && !(p.top_p < 1.f);
   return a;
 }
 
@@ -322,11 +331,17 @@ __device__ __forceinline__ void publish_selection(const SelArgs& p, Smem& S, int
     const float wv = kept ? p.rsf * my_s / denom : 0.f;
     S.sel_idx[pos] = id;
     S.sel_w[pos] = wv;
+    if (!p.early_picks) S.pick_id[lane] = my_sel;
+    S.pick_kept[lane] = kept ? 1 : 0;
+    S.slot_pick[pos] = lane;
     if (blockIdx.x == 0) {
       if (p.idx_out) p.idx_out[pos] = id;
       if (p.w_out) p.w_out[pos] = wv;
     }
   }
+  // the picks are final now (unless each went out as it was popped): lane r
+  // releases its own pick_id / pick_kept
+  if (!p.early_picks && lane < p.k) mbar_arrive(&S.pickbar[lane]);
 }
 
 // Selection for shapes whose groups do not align with lanes: one lane per
@@ -529,6 +544,12 @@ __device__ __noinline__ void run_select(const SelArgs p, Smem& S) {
       S.pick_id[r] = lane * q + jid[0];
       S.pick_s[r] = sl[0];
     }
+    if (p.early_picks) {
+      // pick r is final: the producer may start streaming its expert while
+      // the remaining picks are found
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.pickbar[r]);
+    }
 #pragma unroll
     for (int j = 0; j + 1 < kQ; ++j) {  // pop the owner's head
       key[j] = own ? key[j + 1] : key[j];
@@ -620,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       mbar_init(&S.empty[s], kGW);
     }
     for (int g = 0; g < kGroups; ++g) mbar_init(&S.gbar[g], kGW);
-    mbar_init(&S.selbar, 1);
+    for (int r = 0; r < kMaxSlots; ++r) mbar_init(&S.pickbar[r], 1);
     S.sel_ok = 0;
     S.abort_flag[0] = S.abort_flag[1] = 0;
     fence_mbar_init();
@@ -671,6 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     if (lane == 0) {
       const uint64_t policy = l2_policy_evict_first();
       bool sel_seen = false;
+      uint64_t pick_seen = 0, pick_dropped = 0;  // bit r: pick r acquired / dropped by top-p
       bool first_routed = false, first_down = false;
       uint64_t hq_seen = 0;  // bit j: slot j's int16 h acquired
       int dones = 0;
@@ -681,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       int dr0, dr1;
       down_rows(p, blockIdx.x, dr0, dr1);
       // Gate/up items are dealt out statically: CTA b takes items b,
-      // b + grid, ... of the order shared, routed 0..k-1.  (A shared ticket
+      // b + grid, ... of the order shared, routed picks 0..k-1.  (A shared ticket
       // counter balances slightly better but puts an atomic's round trip to
       // L2 -- microseconds while the weights stream -- between fills.)  The
       // control word kCtrlTicket offsets the first item; it is 0 except in a
@@ -715,19 +737,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           }
           if (d.type == kDone) break;
           if (d.slot < p.k) {
-            if (!sel_seen) {
-              // the selection warp's result (mbarrier: release / acquire)
-              if (mbar_wait(&S.selbar, 0u, kWaitNs) && S.sel_ok) {
-                sel_seen = true;
-                TRACE_AT(12);
+            // routed items go in pick order (descending score): pick r's
+            // items can stream as soon as pick r is final, before the later
+            // picks are found
+            if (!((pick_seen >> d.slot) & 1ull)) {
+              // the selection warp's pick (mbarrier: release / acquire)
+              if (mbar_wait(&S.pickbar[d.slot], 0u, kWaitNs) && S.sel_ok) {
+                pick_seen |= 1ull << d.slot;
+                if (!sel_seen) {
+                  sel_seen = true;
+                  TRACE_AT(12);
+                }
+                const int id = S.pick_id[d.slot];
+                if (p.top_p < 1.f && !S.pick_kept[d.slot]) {
+                  pick_dropped |= 1ull << d.slot;
+                } else if (id >= 0 && id < p.E) {
+                  S.ep[d.slot] = p.table[id];  // the pick's tensors, once
+                }
               } else {
                 set_error(p.ctrl, kErrTimeout, 4, n);
                 d = make_item(kDone, 0, 0, 0);
                 break;
               }
             }
-            d.eid = S.sel_idx[d.slot];
-            if (d.eid == -1) continue;  // dropped by top-p: no bytes read
+            if ((pick_dropped >> d.slot) & 1ull) continue;  // dropped by top-p: no bytes read
+            d.eid = S.pick_id[d.slot];
             if (d.eid < 0 || d.eid >= p.E) {
               set_error(p.ctrl, kErrBadExpertId, 5, n);
               d = make_item(kDone, 0, 0, 0);
@@ -845,7 +879,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       }
     }
     if (ok) {
-      if (lane == 0) TRACE_AT(4);
+      if (lane == 0) {
+        TRACE_AT(4);
+        S.sel_ok = 1;  // before any pick goes out
+      }
 #pragma unroll
       for (int m = 0; m < kMaxE / 32; ++m) {
         const int e = lane + 32 * m;
@@ -856,45 +893,36 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         }
       }
       __syncwarp();
+      // every pick barrier gets its one arrival in here: as each pick is
+      // popped, or all at the end of the selection
       run_select(sel_args(p), S);
-      if (lane == 0) TRACE_AT(24);
-      __syncwarp();
-      // the selected experts' tensor pointers, one load per lane, so that
-      // no fill waits on a pointer-table load from global memory
-      if (lane < p.k) {
-        const int id = S.sel_idx[lane];
-        if (id >= 0 && id < p.E) S.ep[lane] = p.table[id];
-      }
       if (lane == 0) TRACE_AT(5);
     } else if (lane == 0) {
       set_error(p.ctrl, kErrTimeout, 8, 0);
-    }
-    __syncwarp();
-    if (lane == 0) {
-      S.sel_ok = ok ? 1 : 0;
-      mbar_arrive(&S.selbar);
+      S.sel_ok = 0;
+      for (int r = 0; r < p.k; ++r) mbar_arrive(&S.pickbar[r]);  // reported, not selected
     }
   } else if (warp == kConvWarp) {
     // ------------------------------------------------------------ converter
     // Publishes 32-row groups of h as int16 words (the XQ layout the down
     // consumers load) once their 32 rows are written.  CTA b owns groups
-    // b, b + grid, ... of the order (shared slot first, then slots 0..k-1;
-    // groups ascending), the order in which gate/up items complete.
+    // b, b + grid, ... of the order (the shared expert first, then picks
+    // 0..k-1; groups ascending), the order in which gate/up items complete.
     const int GD = p.I >> 5, slots = p.k + p.has_shared;
-    bool sel_seen = false;
+    uint64_t pick_seen = 0;
     for (int i = blockIdx.x; i < slots * GD; i += gridDim.x) {
       const int so = i / GD, g = i % GD;
-      const int slot = p.has_shared ? (so == 0 ? p.k : so - 1) : so;
+      const int slot = p.has_shared ? (so == 0 ? p.k : so - 1) : so;  // routed: a pick
       if (slot < p.k) {
-        // a routed slot may be dropped by top-p: its h never comes
-        if (!sel_seen) {
+        // a routed pick may be dropped by top-p: its h never comes
+        if (!((pick_seen >> slot) & 1ull)) {
           int okw = 0;
-          if (lane == 0) okw = mbar_wait(&S.selbar, 0u, kWaitNs) && S.sel_ok;
+          if (lane == 0) okw = mbar_wait(&S.pickbar[slot], 0u, kWaitNs) && S.sel_ok;
           if (!__shfl_sync(0xffffffffu, okw, 0)) break;  // the selection warp reported it
-          mbar_test(&S.selbar, 0u);
-          sel_seen = true;
+          mbar_test(&S.pickbar[slot], 0u);
+          pick_seen |= 1ull << slot;
         }
-        if (S.sel_idx[slot] == -1) continue;
+        if (p.top_p < 1.f && !S.pick_kept[slot]) continue;
       }
       const uint32_t* cnt = p.ctrl + kCtrlHRows + slot * GD + g;
       // every lane acquires the count itself (so its own loads of h below
@@ -1235,7 +1263,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   // -------------------------------------------------------------- teardown
   __syncthreads();
   {
-    // y of this CTA's own rows: the slot partials combined in slot order
+    // y of this CTA's own rows: the partials combined in slot order
     // (sum_j w_j y_j, then the shared expert, then the residual input),
     // the same order for every call: no atomics, bitwise repeatable
     int r0, r1;
@@ -1244,7 +1272,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       for (int lr = threadIdx.x; lr < r1 - r0; lr += kThreads) {
         float acc = 0.f;
         for (int j = 0; j < p.k; ++j)
-          if (S.sel_idx[j] >= 0) acc = fmaf(S.sel_w[j], S.ycta[j * p.ycta_rows + lr], acc);
+          if (S.sel_idx[j] >= 0)
+            acc = fmaf(S.sel_w[j], S.ycta[S.slot_pick[j] * p.ycta_rows + lr], acc);
         if (p.has_shared) acc += S.ycta[p.k * p.ycta_rows + lr];
         if (p.x_resid) acc = p.x_resid[r0 + lr] + acc;  // x + MoE(norm(x))
         p.y[r0 + lr] = acc;
@@ -1357,6 +1386,8 @@ bool phases(int G, int& P) {
 
 }  // namespace
 
+static_assert((size_t)kStages * kStageBytes + sizeof(Smem) <= 232448,
+              "one CTA's dynamic shared memory must fit the 227 KB limit");
 size_t decode_smem_bytes() { return (size_t)kStages * kStageBytes + sizeof(Smem); }
 
 bool decode_plan(const moe_config& c, DecodeParams& p) {
