@@ -506,6 +506,33 @@ __device__ __noinline__ void run_select(const SelArgs p, Smem& S) {
     jid[j] = j;
     sl[j] = sc[j];
   }
+  // Pick 0, the best kept candidate (ties: the lower expert id), goes out
+  // before the lists are sorted, so that its expert starts streaming while
+  // the other picks are found; round 0 below pops the same candidate.
+  if (p.early_picks) {
+    uint32_t bk = 0u;
+    int bj = 0;
+    float bsl = 0.f;
+#pragma unroll
+    for (int j = 0; j < kQ; ++j)
+      if (key[j] > bk) {
+        bk = key[j];
+        bj = j;
+        bsl = sl[j];
+      }
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    bool own = bk == m && m != 0u;
+    if (__popc(__ballot_sync(0xffffffffu, own)) > 1) {
+      const uint32_t cand = own ? (uint32_t)(lane * q + bj) : 0xFFFFFFFFu;
+      own = cand == __reduce_min_sync(0xffffffffu, cand);
+    }
+    if (own) {
+      S.pick_id[0] = lane * q + bj;
+      S.pick_s[0] = bsl;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.pickbar[0]);
+  }
   static_assert(kQ == 8, "the network below sorts 8 candidates");
   cx(key, jid, sl, 0, 1); cx(key, jid, sl, 2, 3); cx(key, jid, sl, 4, 5); cx(key, jid, sl, 6, 7);
   cx(key, jid, sl, 0, 2); cx(key, jid, sl, 1, 3); cx(key, jid, sl, 4, 6); cx(key, jid, sl, 5, 7);
@@ -528,7 +555,7 @@ __device__ __noinline__ void run_select(const SelArgs p, Smem& S) {
   // top_k: the best head is popped, k times; among equal heads (a rare,
   // warp-uniform case) the lowest expert id.  The owner of the r-th pick
   // leaves it in shared memory, off the dependent chain of the rounds.
-  if (lane < p.k) {
+  if (lane < p.k && !(p.early_picks && lane == 0)) {
     S.pick_id[lane] = -1;  // no candidate left (not reachable for a valid shape)
     S.pick_s[lane] = 0.f;
   }
@@ -540,11 +567,11 @@ __device__ __noinline__ void run_select(const SelArgs p, Smem& S) {
       const uint32_t cand = own ? (uint32_t)(lane * q + jid[0]) : 0xFFFFFFFFu;
       own = cand == __reduce_min_sync(0xffffffffu, cand);
     }
-    if (own) {
+    if (own && !(p.early_picks && r == 0)) {  // pick 0 went out already
       S.pick_id[r] = lane * q + jid[0];
       S.pick_s[r] = sl[0];
     }
-    if (p.early_picks) {
+    if (p.early_picks && r > 0) {
       // pick r is final: the producer may start streaming its expert while
       // the remaining picks are found
       __syncwarp();
