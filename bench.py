@@ -323,17 +323,35 @@ def main():
     ms_step = ms / args.steps
     value = job_rate(n * args.steps, world, ms)
 
-    # e2e: host buffers, per-token pinned H2D of x and D2H of y in the timed region
+    # e2e: host buffers, per-token pinned H2D of x and D2H of y in the timed
+    # region.  The copies run on their own streams, double-buffered: token
+    # t + 1's input goes up while token t computes, and token t's output
+    # comes down while token t + 1 computes.
     x_host = torch.from_numpy(x_bits.view(np.int16)).pin_memory()
     y_host = torch.empty((n, shape.hidden), dtype=torch.float32).pin_memory()
-    xd = torch.empty((1, shape.hidden), dtype=torch.int16, device="cuda")
-    yd = torch.empty((1, shape.hidden), dtype=torch.float32, device="cuda")
+    xd = [torch.empty((1, shape.hidden), dtype=torch.int16, device="cuda") for _ in range(2)]
+    yd = [torch.empty((1, shape.hidden), dtype=torch.float32, device="cuda") for _ in range(2)]
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_k = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
     def e2e_step():
         for t in range(n):
-            xd.copy_(x_host[t:t + 1], non_blocking=True)
-            views[t % copies].forward(xd, yd, ws, stream=stream)
-            y_host[t:t + 1].copy_(yd, non_blocking=True)
+            b = t & 1
+            up.wait_event(ev_k[b])            # x buffer b: token t - 2 has computed
+            with torch.cuda.stream(up):
+                xd[b].copy_(x_host[t:t + 1], non_blocking=True)
+                ev_in[b].record(up)
+            stream.wait_event(ev_in[b])
+            stream.wait_event(ev_out[b])      # y buffer b: token t - 2 is down
+            views[t % copies].forward(xd[b], yd[b], ws, stream=stream)
+            ev_k[b].record(stream)
+            down.wait_event(ev_k[b])
+            with torch.cuda.stream(down):
+                y_host[t:t + 1].copy_(yd[b], non_blocking=True)
+                ev_out[b].record(down)
+        stream.wait_event(ev_out[(n - 1) & 1])  # the step ends with its last output on the host
 
     with torch.cuda.stream(stream):
         e2e_step()
