@@ -436,3 +436,41 @@ def test_cache_expert_ffn_waits_per_expert(cap):
         with pytest.raises(moe.MoeError):
             cache.wait_expert(0, absent[0])
     cache.close()
+
+
+def test_cache_argument_checks():
+    # every refused argument returns MOE_ERR_INVALID_ARG (status 1) before
+    # anything is allocated or copied, and leaves the cache usable
+    shape, cfg, host, dls, resident = tiny_cache_setup(cap=4, L=2)
+    for bad_cap in (shape.top_k - 1, shape.n_experts + 1):
+        with pytest.raises(moe.MoeError) as ei:
+            moe.Cache(cfg, host, bad_cap)
+        assert ei.value.status == 1
+    pageable = [[{k: torch.from_numpy(v.numpy().copy()) for k, v in e.items()}
+                 for e in layer] for layer in host]
+    with pytest.raises(moe.MoeError) as ei:
+        moe.Cache(cfg, pageable, 4)  # not page-locked host memory
+    assert ei.value.status == 1
+    cache = moe.Cache(cfg, host, 4)
+    with pytest.raises(moe.MoeError):
+        cache.acquire(0, [1, 5])     # no layer view yet
+    view = cache.layer(0, dls[0].w_router, dls[0].bias, dls[0].shared)
+    for ids in ([5, 1], [1, 1], [1, shape.n_experts], [-1, 3], [0, 1, 2, 3, 4]):
+        with pytest.raises(moe.MoeError) as ei:
+            cache.acquire(0, ids)
+        assert ei.value.status == 1
+    with pytest.raises(moe.MoeError):
+        cache.acquire(2, [1, 5])     # layer out of range
+    with pytest.raises(moe.MoeError):
+        cache.usage(5)
+    with pytest.raises(moe.MoeError):
+        cache.wait(-1)
+    assert cache.stats(0) == (0, 0, 0)
+    # still usable
+    x = torch.from_numpy(synth.tokens(shape, 0, 64, 1).view(np.int16)).cuda()
+    cache.acquire(0, [1, 5])
+    y_c, y_r, keep = ffn_pair(shape, cfg, view, resident[0], [1, 5], x)
+    cache.release(0)
+    torch.cuda.synchronize()
+    assert torch.equal(y_c, y_r)
+    cache.close()
