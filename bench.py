@@ -18,6 +18,7 @@ With --gpus N (torchrun) each rank runs its own replica of the workload
 workload on the host cores: there is no other implementation to run.
 """
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -50,11 +51,15 @@ def parse():
     p.add_argument("--small", action="store_true", help="tiny layer (smoke/profiling only)")
     p.add_argument("--experts", type=int, default=0,
                    help="routed experts per layer (profiling only; default: the shape's 256)")
-    p.add_argument("--mode", default="layer", choices=["layer", "verify", "stack", "stream"],
+    p.add_argument("--mode", default="layer",
+                   choices=["layer", "verify", "stack", "stream", "timeline"],
                    help="layer: batch-1 decode of one layer (the headline); verify: T-token "
                         "calls; stack: one token through 24 layers; stream: host-streamed "
-                        "experts through the LRU cache")
+                        "experts through the LRU cache; timeline: per-phase times of the "
+                        "one-token kernel from its probe build")
     p.add_argument("--verify-T", default="2,3,4,8,32", help="tokens per verify call")
+    p.add_argument("--timeline-sm-mhz", type=float, default=1965.0,
+                   help="timeline: SM clock that converts clock64 probes to time")
     p.add_argument("--correlated", action="store_true",
                    help="verify: draft tokens x0 + 0.05 eps (heavily shared experts)")
     p.add_argument("--stack-layers", type=int, default=24)
@@ -235,6 +240,9 @@ def main():
         shape = dataclasses.replace(shape, n_experts=args.experts)
     if args.impl == "reference":
         run_reference(args, shape)
+        return
+    if args.mode == "timeline":
+        run_timeline(args, shape)
         return
     if args.mode != "layer":
         run_mode(args, shape)
@@ -690,6 +698,88 @@ def run_stream(args, shape, cfg, stream):
             one(cap, "router")
     finally:
         store.close()
+
+
+# Probe points of the one-token kernel's -DMOE_TRACE build (TRACE_AT indices).
+TIMELINE_PHASES = {0: "entry", 1: "router fill issued", 2: "router rows landed",
+                   15: "router dot products done", 3: "records published",
+                   4: "all records seen", 17: "group scores", 18: "groups ranked",
+                   19: "candidate lists sorted", 12: "producer has pick 0",
+                   6: "first routed gate/up fill issued", 20: "all picks found",
+                   5: "selection published", 22: "last shared gate/up item finalised",
+                   21: "shared h group published", 7: "first down fill issued",
+                   11: "last fill issued", 10: "exit"}
+
+
+def run_timeline(args, shape):
+    """Per-phase times of the one-token kernel: the probe build of the same
+    sources records clock64 at fixed points of every CTA (and globaltimer at
+    entry); CUDA-graph replay of 64 tokens over 8 layer copies; medians over
+    CTAs, then over replays."""
+    import torch
+    import int4_routed_expert_noaux_b200 as moe
+    from int4_routed_expert_noaux_b200 import build as B
+    import synth
+    from synth.layers import DeviceLayer
+    moe.LIB_PATH = B.build(trace=True)
+    L = moe.lib()
+    L.moe_debug_set_trace.argtypes = [ctypes.c_void_p]
+    L.moe_debug_set_trace.restype = None
+    torch.cuda.set_device(0)
+    cfg = moe.Config.from_shape(shape)
+    copies = max(1, args.copies)
+    dls = [DeviceLayer(shape, 0, c) for c in range(copies)]
+    views = [moe.Layer(cfg, d.w_router, d.bias, d.routed, d.shared) for d in dls]
+    n = 64
+    x = torch.from_numpy(synth.tokens(shape, 0, 0, n).view(np.int16)).cuda()
+    y = torch.empty((n, shape.hidden), dtype=torch.float32, device="cuda")
+    ws = moe.alloc_workspace(cfg, 1)
+    nsm = torch.cuda.get_device_properties(0).multi_processor_count
+    tr = torch.zeros(nsm * 128 + 128, dtype=torch.int64, device="cuda")
+    L.moe_debug_set_trace(ctypes.c_void_p(tr.data_ptr()))
+    stream = torch.cuda.Stream()
+
+    def step():
+        for t in range(n):
+            views[t % copies].forward(x[t:t + 1], y[t:t + 1], ws, stream=stream)
+    g = _graph(stream, step)
+    clocks = Clocks(0)
+    f_ghz = []
+    acc = {i: [] for i in TIMELINE_PHASES}
+    per_call = []
+    for rep in range(8):
+        tr.zero_()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        per_call.append(e0.elapsed_time(e1) * 1000.0 / n)
+        if rep < 2:
+            continue
+        raw = tr.cpu().numpy()[: nsm * 128].reshape(nsm, 128).astype(np.float64)
+        gt0, c0 = raw[:, 127], raw[:, 96]  # each CTA's entry: globaltimer ns, clock64
+        f_ghz.append(args.timeline_sm_mhz / 1000.0)
+        t0 = gt0.min()
+        for i in TIMELINE_PHASES:
+            v = raw[:, 96 + i]
+            m = v != 0
+            if m.any():
+                acc[i].append(np.median((gt0[m] + (v[m] - c0[m]) / f_ghz[-1] - t0) / 1000.0))
+    clk = clocks.stop()
+    moe.ws_check(ws, stream)
+    L.moe_debug_set_trace(None)
+    phases = {TIMELINE_PHASES[i]: round(float(np.median(v)), 2)
+              for i, v in sorted(acc.items(), key=lambda kv: np.median(kv[1]) if kv[1] else 1e9)
+              if v}
+    print(json.dumps({"mode": "timeline", "workload": "one GLM-5.2-shaped layer per token, "
+                      f"{copies} rotating layer copies, CUDA-graph replay of {n} tokens",
+                      "library": "probe build (-DMOE_TRACE) of the same sources",
+                      "us_per_token_probe_build": round(float(np.median(per_call[2:])), 2),
+                      "phases_us_median_over_ctas": phases,
+                      "clock_mhz_assumed": args.timeline_sm_mhz, "clocks": clk}), flush=True)
 
 
 def run_mode(args, shape):

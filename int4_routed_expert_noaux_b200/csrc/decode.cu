@@ -139,7 +139,7 @@ struct SelArgs {
   int32_t* idx_out;  // written by CTA 0 only (nullable)
   float* w_out;
   uint64_t* trace;   // timeline probes of a -DMOE_TRACE build
-  const ExpertPtrs* table;  // nullable in a dry run
+  const ExpertPtrs* table;  // nullable (no pointer-table prefetch)
   int early_picks;  // each pick's barrier arrives as soon as the pick is final
 };
 
