@@ -102,10 +102,103 @@ __device__ __forceinline__ ArgMax warp_argmax(ArgMax a) {
   return a;
 }
 
+// A score as an unsigned key in the same order (larger float, larger key);
+// 0 is below every score's key.
+__device__ __forceinline__ uint32_t sel_key(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+constexpr int kSelQ = 8;  // candidates per lane (E <= 256)
+
+// Compare-exchange of a lane's candidate list: position a before b in the
+// order (key descending, expert index ascending).
+__device__ __forceinline__ void sel_cx(uint32_t (&key)[kSelQ], int (&jid)[kSelQ], int a, int b) {
+  const bool sw = key[b] > key[a] || (key[b] == key[a] && jid[b] < jid[a]);
+  const uint32_t ka = key[a], kb = key[b];
+  const int ja = jid[a], jb = jid[b];
+  key[a] = sw ? kb : ka;
+  key[b] = sw ? ka : kb;
+  jid[a] = sw ? jb : ja;
+  jid[b] = sw ? ja : jb;
+}
+
+// Group-limited top-k of one token by one warp, when the groups align with
+// lanes: lane l owns experts l*q .. l*q+q-1 and a group is 2^lgL
+// consecutive lanes.  Group score = the two largest bias-corrected scores;
+// the topk_group best groups (ties: lower index) are kept; the top_k best
+// kept experts (ties: lower id) are popped from per-lane sorted lists, one
+// warp-wide max per pick.  Lane r < top_k receives the r-th pick.
+// Branch-free: no data-dependent guard around a warp collective.
+__device__ __forceinline__ int select_fast_warp(const float* s_sel, int E, int q, int lgL,
+                                                int n_group, int topk_group, int top_k) {
+  const int lane = threadIdx.x & 31;
+  const int L = 1 << lgL;
+  const int nmine = max(0, min(q, E - lane * q));
+  float sp[kSelQ];
+#pragma unroll
+  for (int j = 0; j < kSelQ; ++j) sp[j] = (j < nmine) ? s_sel[lane * q + j] : -INFINITY;
+  float t1 = -INFINITY, t2 = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < kSelQ; ++j) {
+    t2 = fmaxf(t2, fminf(t1, sp[j]));
+    t1 = fmaxf(t1, sp[j]);
+  }
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float p1 = __shfl_xor_sync(0xffffffffu, t1, o);
+    const float p2 = __shfl_xor_sync(0xffffffffu, t2, o);
+    const float n2 = fmaxf(fminf(t1, p1), fmaxf(t2, p2));
+    const float n1 = fmaxf(t1, p1);
+    t1 = (o < L) ? n1 : t1;
+    t2 = (o < L) ? n2 : t2;
+  }
+  const float gs_seg = ((q << lgL) >= 2) ? t1 + t2 : t1;
+  float gs = __shfl_sync(0xffffffffu, gs_seg, (lane < n_group ? lane : 0) << lgL);
+  gs = (lane < n_group) ? gs : -INFINITY;
+  int rank = 0;
+#pragma unroll
+  for (int h = 0; h < 32; ++h) {
+    const float o = __shfl_sync(0xffffffffu, gs, h);
+    rank += (o > gs || (o == gs && h < lane)) ? 1 : 0;
+  }
+  const unsigned kept_mask = __ballot_sync(0xffffffffu, lane < n_group && rank < topk_group);
+  const bool kept = (kept_mask >> (lane >> lgL)) & 1u;
+  uint32_t key[kSelQ];
+  int jid[kSelQ];
+#pragma unroll
+  for (int j = 0; j < kSelQ; ++j) {
+    key[j] = (j < nmine && kept) ? sel_key(sp[j]) : 0u;
+    jid[j] = j;
+  }
+  sel_cx(key, jid, 0, 1); sel_cx(key, jid, 2, 3); sel_cx(key, jid, 4, 5); sel_cx(key, jid, 6, 7);
+  sel_cx(key, jid, 0, 2); sel_cx(key, jid, 1, 3); sel_cx(key, jid, 4, 6); sel_cx(key, jid, 5, 7);
+  sel_cx(key, jid, 1, 2); sel_cx(key, jid, 5, 6);
+  sel_cx(key, jid, 0, 4); sel_cx(key, jid, 1, 5); sel_cx(key, jid, 2, 6); sel_cx(key, jid, 3, 7);
+  sel_cx(key, jid, 2, 4); sel_cx(key, jid, 3, 5);
+  sel_cx(key, jid, 1, 2); sel_cx(key, jid, 3, 4); sel_cx(key, jid, 5, 6);
+  int my_sel = -1;
+  for (int r = 0; r < top_k; ++r) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, key[0]);
+    bool own = key[0] == m && m != 0u;
+    const uint32_t cand = own ? (uint32_t)(lane * q + jid[0]) : 0xFFFFFFFFu;
+    const uint32_t best = __reduce_min_sync(0xffffffffu, cand);  // ties: the lower id
+    own = own && cand == best;
+    if (lane == r) my_sel = (best == 0xFFFFFFFFu) ? -1 : (int)best;
+#pragma unroll
+    for (int j = 0; j + 1 < kSelQ; ++j) {  // pop the owner's head
+      key[j] = own ? key[j + 1] : key[j];
+      jid[j] = own ? jid[j + 1] : jid[j];
+    }
+    key[kSelQ - 1] = own ? 0u : key[kSelQ - 1];
+  }
+  return my_sel;
+}
+
 __global__ void __launch_bounds__(1024) select_kernel(
     const double* __restrict__ part, int KS, int T, const float* __restrict__ bias, int E,
-    int n_group, int topk_group, int top_k, float rsf, float top_p,
-    int32_t* __restrict__ idx_out, float* __restrict__ w_out,
+    int n_group, int topk_group, int top_k, float rsf, float top_p, int sel_q, int sel_lgL,
+    int sel_fast, int32_t* __restrict__ idx_out, float* __restrict__ w_out,
     float* __restrict__ scores_out) {
   __shared__ float s_score[1024];
   __shared__ float s_sel[1024];
@@ -145,32 +238,36 @@ __global__ void __launch_bounds__(1024) select_kernel(
   __syncthreads();
   if (warp != 0) return;
 
-  // keep topk_group groups (lane = group)
-  bool kept = false;
-  {
-    ArgMax g{lane < n_group ? s_group[lane] : 0.f, lane < n_group ? lane : -1};
-    for (int r = 0; r < topk_group; ++r) {
-      ArgMax cand = kept ? ArgMax{0.f, -1} : g;
-      const ArgMax best = warp_argmax(cand);
-      if (best.i == lane) kept = true;
+  int my_sel = -1;  // id selected in round == lane
+  if (sel_fast) {
+    my_sel = select_fast_warp(s_sel, E, sel_q, sel_lgL, n_group, topk_group, top_k);
+  } else {
+    // keep topk_group groups (lane = group)
+    bool kept = false;
+    {
+      ArgMax g{lane < n_group ? s_group[lane] : 0.f, lane < n_group ? lane : -1};
+      for (int r = 0; r < topk_group; ++r) {
+        ArgMax cand = kept ? ArgMax{0.f, -1} : g;
+        const ArgMax best = warp_argmax(cand);
+        if (best.i == lane) kept = true;
+      }
     }
-  }
-  const unsigned kept_mask = __ballot_sync(0xffffffffu, kept);
+    const unsigned kept_mask = __ballot_sync(0xffffffffu, kept);
 
-  // top_k over experts of kept groups; lane holds experts lane + 32 * m
-  const int nper = (E + 31) >> 5;
-  unsigned taken = 0;  // bit m: expert lane + 32m already selected
-  int my_sel = -1;     // id selected in round == lane
-  for (int r = 0; r < top_k; ++r) {
-    ArgMax a{0.f, -1};
-    for (int m = 0; m < nper; ++m) {
-      const int e = lane + 32 * m;
-      if (e < E && ((kept_mask >> (e / per)) & 1u) && !((taken >> m) & 1u))
-        a = argmax_merge(a, ArgMax{s_sel[e], e});
+    // top_k over experts of kept groups; lane holds experts lane + 32 * m
+    const int nper = (E + 31) >> 5;
+    unsigned taken = 0;  // bit m: expert lane + 32m already selected
+    for (int r = 0; r < top_k; ++r) {
+      ArgMax a{0.f, -1};
+      for (int m = 0; m < nper; ++m) {
+        const int e = lane + 32 * m;
+        if (e < E && ((kept_mask >> (e / per)) & 1u) && !((taken >> m) & 1u))
+          a = argmax_merge(a, ArgMax{s_sel[e], e});
+      }
+      const ArgMax best = warp_argmax(a);
+      if (best.i >= 0 && (best.i & 31) == lane) taken |= 1u << (best.i >> 5);
+      if (lane == r) my_sel = best.i;
     }
-    const ArgMax best = warp_argmax(a);
-    if (best.i >= 0 && (best.i & 31) == lane) taken |= 1u << (best.i >> 5);
-    if (lane == r) my_sel = best.i;
   }
   const float s_mine = (lane < top_k && my_sel >= 0) ? s_score[my_sel] : 0.f;
   const float denom = warp_sum(s_mine) + 1e-20f;
@@ -287,8 +384,15 @@ cudaError_t launch_router_partial(const float* w, const uint16_t* x, int T, int 
 cudaError_t launch_select(const double* part, int H, const float* bias, int T, int E,
                           int n_group, int topk_group, int top_k, float rsf, float top_p,
                           int32_t* idx, float* w, float* scores_out, cudaStream_t st) {
+  // the one-warp fast selection when the groups align with lanes (as in
+  // the one-token kernel), else the generic rounds
+  const int per = E / n_group, q = (E + 31) / 32;
+  int lgL = 0;
+  while ((1 << lgL) < per / q) ++lgL;
+  const int fast = per % q == 0 && per / q >= 1 && (1 << lgL) == per / q && q <= kSelQ;
   select_kernel<<<T, 32 * n_group, 0, st>>>(part, router_slices(H, T), T, bias, E, n_group,
-                                            topk_group, top_k, rsf, top_p, idx, w, scores_out);
+                                            topk_group, top_k, rsf, top_p, q, lgL, fast, idx, w,
+                                            scores_out);
   return cudaGetLastError();
 }
 
