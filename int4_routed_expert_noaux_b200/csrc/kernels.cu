@@ -32,6 +32,7 @@ __device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, dou
 __global__ void __launch_bounds__(256) router_partial_kernel(
     const float* __restrict__ w, const uint16_t* __restrict__ x, int T, int H, int E, int KS,
     double* __restrict__ part) {
+  pdl_wait();
   const int ks = blockIdx.x, e0 = blockIdx.y * 8;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = warp * 8;
@@ -200,6 +201,7 @@ __global__ void __launch_bounds__(1024) select_kernel(
     int n_group, int topk_group, int top_k, float rsf, float top_p, int sel_q, int sel_lgL,
     int sel_fast, int32_t* __restrict__ idx_out, float* __restrict__ w_out,
     float* __restrict__ scores_out) {
+  pdl_wait();
   __shared__ float s_score[1024];
   __shared__ float s_sel[1024];
   __shared__ float s_group[32];
@@ -376,8 +378,8 @@ cudaError_t launch_router_partial(const float* w, const uint16_t* x, int T, int 
                                   double* part, cudaStream_t st) {
   if (H % 16 != 0 || T < 1 || T > 64) return cudaErrorInvalidValue;
   const int ks = router_slices(H, T);
-  router_partial_kernel<<<dim3(ks, (E + 7) / 8), 32 * ((T + 7) / 8), 0, st>>>(w, x, T, H, E, ks,
-                                                                            part);
+  launch_pdl(router_partial_kernel, dim3(ks, (E + 7) / 8), dim3(32 * ((T + 7) / 8)), 0, st, w, x,
+             T, H, E, ks, part);
   return cudaGetLastError();
 }
 
@@ -390,9 +392,8 @@ cudaError_t launch_select(const double* part, int H, const float* bias, int T, i
   int lgL = 0;
   while ((1 << lgL) < per / q) ++lgL;
   const int fast = per % q == 0 && per / q >= 1 && (1 << lgL) == per / q && q <= kSelQ;
-  select_kernel<<<T, 32 * n_group, 0, st>>>(part, router_slices(H, T), T, bias, E, n_group,
-                                            topk_group, top_k, rsf, top_p, q, lgL, fast, idx, w,
-                                            scores_out);
+  launch_pdl(select_kernel, dim3(T), dim3(32 * n_group), 0, st, part, router_slices(H, T), T, bias,
+             E, n_group, topk_group, top_k, rsf, top_p, q, lgL, fast, idx, w, scores_out);
   return cudaGetLastError();
 }
 

@@ -9,6 +9,29 @@
 
 namespace moe {
 
+// The kernels of a T-token call follow one another on the stream.  Each is a
+// programmatic dependent launch: its blocks may be scheduled while the
+// previous kernel finishes, and the kernel's first statement (pdl_wait)
+// holds it until that kernel's writes are visible.  So only the launch
+// latency overlaps; no kernel touches memory before the wait.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Router logits in K slices: part [router_slices(H, T)][T][E] (fp64), each
 // the sum of W x over a slice of the inputs (1 <= T <= 64, H a multiple of
 // 16).

@@ -232,6 +232,7 @@ struct TcArgs {
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const TcArgs a, const __grid_constant__ CUtensorMap tm_codes,
                    const __grid_constant__ CUtensorMap tm_scales) {
+  pdl_wait();
   extern __shared__ uint8_t tsmem_raw[];
   // 1024-byte alignment for the swizzled code tiles
   TcSmem& S = *reinterpret_cast<TcSmem*>(tsmem_raw + ((1024u - (smem_addr(tsmem_raw) & 1023u)) & 1023u));
@@ -510,6 +511,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 template <bool kF32>
 __global__ void __launch_bounds__(256) tc_rowscale_kernel(const void* in, int K, int rows,
                                                           int* row_exp) {
+  pdl_wait();
   __shared__ float part[8];
   const int r = blockIdx.x;
   if (r >= rows) return;
@@ -567,6 +569,7 @@ template <bool kDown>
 __global__ void __launch_bounds__(256) tc_pack_kernel(const int* lists, int E, int n_list,
                                                       const void* in, int K, int G,
                                                       const int* row_exp, uint8_t* bpack) {
+  pdl_wait();
   const ListsView L = lists_view(lists, E, n_list);
   const int rank = blockIdx.y;
   if (rank >= L.counts[1]) return;
@@ -719,13 +722,13 @@ cudaError_t launch_tc_ffn_step(int mats, const ExpertPtrs* table, const int* lis
                  kGS, (uint32_t)box_rows, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   if (mats == 2) {
-    tc_rowscale_kernel<false><<<in_rows, 256, 0, st>>>(in, K, in_rows, row_exp);
-    tc_pack_kernel<false><<<dim3(16, tcmax), 256, 0, st>>>(lists, E, n_list, in, K, G, row_exp,
-                                                           bpack);
+    launch_pdl(tc_rowscale_kernel<false>, dim3(in_rows), dim3(256), 0, st, in, K, in_rows, row_exp);
+    launch_pdl(tc_pack_kernel<false>, dim3(16, tcmax), dim3(256), 0, st, lists, E, n_list, in, K,
+               G, row_exp, bpack);
   } else {
-    tc_rowscale_kernel<true><<<in_rows, 256, 0, st>>>(in, K, in_rows, row_exp);
-    tc_pack_kernel<true><<<dim3(16, tcmax), 256, 0, st>>>(lists, E, n_list, in, K, G, row_exp,
-                                                          bpack);
+    launch_pdl(tc_rowscale_kernel<true>, dim3(in_rows), dim3(256), 0, st, in, K, in_rows, row_exp);
+    launch_pdl(tc_pack_kernel<true>, dim3(16, tcmax), dim3(256), 0, st, lists, E, n_list, in, K,
+               G, row_exp, bpack);
   }
   TcArgs a;
   a.table = table;
@@ -745,7 +748,8 @@ cudaError_t launch_tc_ffn_step(int mats, const ExpertPtrs* table, const int* lis
   // columns), no more CTAs than the call can have work items
   const int tiles = R / tile_rows;
   const int grid = std::min(std::min(num_sms(), kStreamMaxCtas), tcmax * tiles);
-  tc_gemm_kernel<<<grid, kTcThreads, sizeof(TcSmem) + 1024, st>>>(a, tm_codes, tm_scales);
+  launch_pdl(tc_gemm_kernel, dim3(grid), dim3(kTcThreads), sizeof(TcSmem) + 1024, st, a, tm_codes,
+             tm_scales);
   return cudaGetLastError();
 }
 

@@ -39,6 +39,7 @@ template <bool kBf16>
 __global__ void __launch_bounds__(256) xq_table_kernel(const void* __restrict__ in, int rows,
                                                        int K, uint8_t* __restrict__ words,
                                                        float* __restrict__ fac) {
+  pdl_wait();
   const int G = K >> 5;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= rows * G) return;
@@ -87,6 +88,7 @@ __global__ void __launch_bounds__(256) build_lists_kernel(const int32_t* __restr
                                                           uint64_t slot_mask, int tc_min,
                                                           int* __restrict__ lists,
                                                           uint32_t* __restrict__ err) {
+  pdl_wait();
   __shared__ int cnt[kListMaxE];
   __shared__ int base[kListMaxE];
   __shared__ int sid[kListMaxIds];
@@ -289,6 +291,7 @@ size_t union_smem_bytes(int mats) {
 
 template <int MATS>
 __global__ void __launch_bounds__(kUnionThreads) union_gemm_kernel(const UnionArgs a) {
+  pdl_wait();
   constexpr int RBM = 64 / MATS;  // rows of one matrix per CTA
   extern __shared__ __align__(16) uint8_t usmem[];
   UStage* st = reinterpret_cast<UStage*>(usmem);
@@ -451,6 +454,7 @@ __global__ void __launch_bounds__(kUnionThreads) union_gemm_kernel(const UnionAr
 __global__ void __launch_bounds__(256) union_combine_kernel(
     const int32_t* __restrict__ idx, const float* __restrict__ w, const float* __restrict__ ypart,
     int T, int H, int k, int E, int has_shared, float* __restrict__ y) {
+  pdl_wait();
   const int t = blockIdx.y;
   const int row = blockIdx.x * blockDim.x + threadIdx.x;
   if (row >= H) return;
@@ -485,9 +489,10 @@ cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const 
   const int G = H / 32, GD = I / 32;
   const int n_list = T * slots;
   const int umax = (E < T * k ? E : T * k) + has_shared;
-  xq_table_kernel<true><<<(T * G + 255) / 256, 256, 0, st>>>(x, T, H, xq_words, xq_fac);
-  build_lists_kernel<<<1, 256, 0, st>>>(idx, T, k, E, has_shared, slot_mask, tc ? tc_min : 0,
-                                         lists, err);
+  launch_pdl(xq_table_kernel<true>, dim3((T * G + 255) / 256), dim3(256), 0, st, x, T, H, xq_words,
+             xq_fac);
+  launch_pdl(build_lists_kernel, dim3(1), dim3(256), 0, st, idx, T, k, E, has_shared, slot_mask,
+             tc ? tc_min : 0, lists, err);
   UnionArgs a;
   a.table = table;
   a.lists = lists;
@@ -529,21 +534,21 @@ cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const 
   const int nb2 = (I + 31) / 32, nb1 = (H + 63) / 64;
   const int grid2 = std::min((int)(occ & 0xFFFFu) * sms, umax * nb2);
   const int grid1 = std::min((int)(occ >> 16) * sms, umax * nb1);
-  union_gemm_kernel<2><<<grid2, kUnionThreads, union_smem_bytes(2), st>>>(a);
+  launch_pdl(union_gemm_kernel<2>, dim3(grid2), dim3(kUnionThreads), union_smem_bytes(2), st, a);
   if (tc) {
     const cudaError_t e = launch_tc_ffn_step(2, table, lists, E, n_list, T, k, has_shared, x, H,
                                              I, T, tc_rowexp, tc_bpack, tc_maps, hbuf, err, st);
     if (e != cudaSuccess) return e;
   }
-  xq_table_kernel<false><<<(n_list * GD + 255) / 256, 256, 0, st>>>(hbuf, n_list, I, hq_words,
-                                                                    hq_fac);
+  launch_pdl(xq_table_kernel<false>, dim3((n_list * GD + 255) / 256), dim3(256), 0, st, hbuf,
+             n_list, I, hq_words, hq_fac);
   a.xq_words = hq_words;
   a.xq_fac = hq_fac;
   a.G = GD;
   a.R = H;
   a.in_is_pos = 1;
   a.out = ypart;
-  union_gemm_kernel<1><<<grid1, kUnionThreads, union_smem_bytes(1), st>>>(a);
+  launch_pdl(union_gemm_kernel<1>, dim3(grid1), dim3(kUnionThreads), union_smem_bytes(1), st, a);
   if (tc) {
     const cudaError_t e = launch_tc_ffn_step(1, table, lists, E, n_list, T, k, has_shared, hbuf,
                                              I, H, n_list, tc_rowexp, tc_bpack, tc_maps, ypart,
@@ -551,8 +556,8 @@ cudaError_t launch_union_ffn(const ExpertPtrs* table, const int32_t* idx, const 
     if (e != cudaSuccess) return e;
   }
   if (combine)
-    union_combine_kernel<<<dim3((H + 255) / 256, T), 256, 0, st>>>(idx, w, ypart, T, H, k, E,
-                                                                   has_shared, y);
+    launch_pdl(union_combine_kernel, dim3((H + 255) / 256, T), dim3(256), 0, st, idx, w, ypart, T,
+               H, k, E, has_shared, y);
   return cudaGetLastError();
 }
 
