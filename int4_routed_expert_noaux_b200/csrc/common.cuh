@@ -266,7 +266,8 @@ __device__ __forceinline__ float sigmoid_f64_to_f32(double v) {
 // kept when the weight share of the picks ranked before it (descending
 // score, ties to the lower id) is below p: the kept picks are the shortest
 // weight-ordered prefix whose share reaches p (colibri summary, "--topp":
-// adaptive expert top-p; the rule is reading R16 of the layer's design).
+// adaptive expert top-p; the page gives no formula, so this rule is our
+// plainest reading of it).
 __device__ __forceinline__ bool topp_keep(int id, float s, float denom, int k, float p) {
   const int lane = threadIdx.x & 31;
   float before = 0.f;

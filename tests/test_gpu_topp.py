@@ -1,6 +1,7 @@
-"""Adaptive expert top-p on the GPU against the fp64 oracle (reading R16 of
-the layer's design: keep the fewest selected experts, in descending weight,
-whose weights reach p * rsf; renormalise over the kept ones).
+"""Adaptive expert top-p on the GPU against the fp64 oracle.  The page names
+the option but gives no formula; the reading used: keep the fewest selected
+experts, in descending weight, whose weights reach p * rsf; renormalise over
+the kept ones.
 
 A token is flagged when its noaux_tc decision margin or its top-p margin
 (distance of a cumulative weight share to p at the boundary, or the share
