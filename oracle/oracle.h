@@ -19,7 +19,7 @@
  *    [-8, 7], two per byte, one fp16 scale per 32 consecutive input weights)
  *    and the router constants (n_group, topk_group, routed_scaling_factor).
  *
- * Readings where the pages are silent (each also listed in the design notes):
+ * Readings where the pages are silent:
  *  R1 group score = sum of the two largest bias-corrected scores of a group;
  *  R2 experts of dropped groups are excluded (never selected);
  *  R3 ties go to the lower group index and to the lower expert index;
@@ -30,7 +30,15 @@
  *  R6 the shared expert has the routed experts' format and size and is added
  *     with weight 1;
  *  R9 stacked layers: x_next = x + MoE(bf16(RMSNorm(x))), unit gain,
- *     eps 1e-6.
+ *     eps 1e-6;
+ *  R11 LRU: per token, hits are touched in ascending id, then misses are
+ *     loaded in ascending id, each evicting the least recently used slot not
+ *     used by the current token;
+ *  R16 adaptive expert top-p: of the k selected experts keep the fewest, in
+ *     descending weight (ties: lower id), whose weights reach p * rsf, and
+ *     normalise the kept weights again; p >= 1 keeps all k;
+ *  R19 hot-store: experts pinned per layer are never evicted; the other
+ *     slots follow R11; pin loads count as bytes, not as hits or misses.
  *
  * Parity pins live in the CPU test-suite; no function here is unpinned.
  */
